@@ -1,0 +1,243 @@
+/*
+ * qgemm.h — C ABI of the B200 (sm_100a) quantized linear-layer GEMM library
+ * (libqgemm.so).
+ *
+ * The library computes, on one GPU,
+ *
+ *     y[M, N] = dequant(A_q)[M, K] . dequant(W_q)[N, K]^T      (bf16 out)
+ *
+ * for the 8-bit formats of the vLLM linear backend described in "Helion in
+ * the vLLM backend: one GEMM, tuning per shape" (ai-radar.it; first
+ * paragraph: FP8_Dynamic, W8A8_INT8, Block_FP8) and for NVFP4, the format of
+ * FlashInfer's mm_fp4 GEMM (FlashInfer PR 3948, "perf(gemm): update mm_fp4
+ * cute-dsl tactic heuristic ...", benchmark command with --use_nvfp4 and
+ * --use_128x4_sf_layout).  One kernel family covers the three algorithms of
+ * the same article (second paragraph): Standard, Split-K (power-of-two
+ * splits up to 256, third paragraph) and Swap-AB, computed as
+ * (W_q . A_q^T)^T so that the weight rows fill the 128-row MMA slot.  An
+ * ahead-of-time table maps (format, M, N, K) to a configuration (third and
+ * fourth paragraphs; M is bucketed as in FlashInfer PR 3948, "M bucketing by
+ * floor(log2 M)").
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers unless a parameter says
+ *     otherwise.  The caller owns every buffer, the workspace and the stream;
+ *     the run path (qgemm_quantize_act, qgemm_run, qgemm_dispatch) allocates
+ *     nothing, synchronises nothing and copies nothing between host and
+ *     device, so it may be captured into a CUDA graph.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy stream).
+ *   - Arguments are checked on the host before any launch; a failed check
+ *     returns a status and launches nothing.  Zero-sized M, N or K is
+ *     QG_ERR_INVALID_ARG (FlashInfer PR 3948 review: guard against
+ *     zero-dimension inputs).
+ *   - Row-major everywhere; "K-contiguous" means element (r, k) of a
+ *     [rows, K] operand is at byte r * row_bytes + k * elem_bytes.
+ *   - Device memory alignment: every pointer 16-byte aligned.
+ */
+#ifndef QGEMM_H_
+#define QGEMM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define QGEMM_ABI_VERSION 1
+
+typedef enum {
+  QG_FP8_DYNAMIC = 0, /* e4m3 codes, fp32 scale per token / per channel        */
+  QG_W8A8_INT8 = 1,   /* int8 codes, fp32 scale per token / per channel        */
+  QG_BLOCK_FP8 = 2,   /* e4m3 codes, fp32 scale per 1x128 act group / 128x128 W block */
+  QG_NVFP4 = 3        /* e2m1 codes, e4m3 scale per 16 K elements + fp32 tensor scale */
+} qg_format;
+
+typedef enum {
+  QG_OK = 0,
+  QG_ERR_INVALID_ARG = 1,    /* null pointer, bad size, misaligned pointer, bad enum   */
+  QG_ERR_UNSUPPORTED = 2,    /* shape/config the kernels do not cover, or not sm_100   */
+  QG_ERR_WORKSPACE = 3,      /* workspace missing or smaller than *_workspace_size     */
+  QG_ERR_TABLE_IO = 4,       /* table file missing, corrupt or of another version      */
+  QG_ERR_TABLE_MISS = 5,     /* (reserved) strict dispatch found no entry              */
+  QG_ERR_CUDA = 6,           /* a CUDA runtime/driver call or a launch failed          */
+  QG_ERR_DEVICE_TIMEOUT = 7, /* a bounded in-kernel wait expired (qgemm_device_error)  */
+  QG_ERR_NO_DEVICE = 8       /* no CUDA device visible                                 */
+} qg_status;
+
+/* Output kind of qgemm_run. */
+typedef enum {
+  QG_OUT_BF16 = 0, /* y as bf16 [M, ldy]                                            */
+  QG_OUT_ACC = 1   /* debug: the raw contraction before the scale epilogue, [M, ldy]:
+                      int32 for W8A8_INT8 (exact), fp32 for the other formats (for
+                      Block_FP8 this is the group-promoted sum, i.e. the final y
+                      before bf16 rounding)                                         */
+} qg_out_kind;
+
+/* Kernel configuration: the tunables of the unified kernel. */
+typedef struct {
+  int32_t split_k;     /* 1, 2, 4, ..., 256: K is cut into split_k slices of whole
+                          128-byte K tiles, each reduced by its own CTA            */
+  int32_t swap_ab;     /* 1: weights take the 128-row MMA operand and tokens the
+                          N operand (y^T = W_q A_q^T); 0: tokens take the 128 rows */
+  int32_t tile_n;      /* MMA N extent: tokens per CTA when swap_ab = 1, weight
+                          rows per CTA when swap_ab = 0; one of 16,32,64,128,256   */
+  int32_t stages;      /* shared-memory pipeline depth, 2..12 (capped by smem)     */
+  int32_t reduce_mode; /* split_k > 1 only: 0 = in-kernel (the last CTA of a tile
+                          sums the partials in split order), 1 = second pass      */
+  int32_t reserved[3]; /* must be zero                                             */
+} qg_config;
+
+/* A quantized operand (activations A_q or weights W_q); non-owning views.
+ * Layouts by format, for an operand of `rows` rows and K reduction elements:
+ *   q:     FP8_DYNAMIC, BLOCK_FP8: e4m3 bytes [rows, K]
+ *          W8A8_INT8: int8 [rows, K]
+ *          NVFP4: packed e2m1 [rows, K/2] bytes, element 2j in the low nibble
+ *   scale: FP8_DYNAMIC, W8A8_INT8: fp32 [rows]
+ *          BLOCK_FP8 activations: fp32 [rows, K/128]
+ *          BLOCK_FP8 weights:     fp32 [ceil(rows/128), K/128]
+ *          NVFP4: e4m3 block scales in the 128x4 tiled layout: the
+ *                 [rows, K/16] scale matrix is padded to R = ceil(rows/128)*128
+ *                 rows and C = ceil(K/256)*16 columns and cut into 128x4
+ *                 atoms of 512 bytes; atom (rb, cb) starts at byte
+ *                 (rb * C/4 + cb) * 512 and holds scale (r, c) at
+ *                 (r%32)*16 + ((r%128)/32)*4 + c%4.  Padding bytes are 0.
+ *   global_scale: NVFP4 only — device fp32 scalar g (decode scale of the
+ *                 tensor: x ~= dec(code) * dec(block scale) * g).          */
+typedef struct {
+  void* q;
+  void* scale;
+  float* global_scale;
+  int32_t rows;
+  int32_t K;
+} qg_operand;
+
+/* ---------------------------------------------------------------- sizes -- */
+
+/* Bytes of the `q` and `scale` buffers of an operand (weights when
+ * is_weight != 0).  Returns QG_ERR_INVALID_ARG for an unknown format or
+ * non-positive sizes. */
+qg_status qgemm_operand_bytes(qg_format f, int is_weight, int rows, int K,
+                              size_t* q_bytes, size_t* scale_bytes);
+
+/* Scratch bytes qgemm_quantize_act / qgemm_quantize_weight need (NVFP4 keeps
+ * its per-CTA amax partials there; the 8-bit formats need none: 0). */
+size_t qgemm_quant_workspace_size(qg_format f, int rows, int K);
+
+/* Scratch bytes qgemm_run needs for this configuration: 0 when split_k == 1,
+ * else split_k * M * N * 4 bytes of partial sums plus one 4-byte counter per
+ * output tile (in-kernel reduction).  The counter region must be zero before
+ * the first call (see qgemm_workspace_clear); every completed call leaves it
+ * zero again. */
+size_t qgemm_workspace_size(qg_format f, int M, int N, int K, const qg_config* cfg);
+
+/* Zeroes a run workspace on `stream` (one cudaMemsetAsync). */
+qg_status qgemm_workspace_clear(void* workspace, size_t ws_bytes, void* stream);
+
+/* ----------------------------------------------------------- quantisers -- */
+
+/* Dynamic activation quantisation (the "quantization" auxiliary kernel of
+ * "Helion in the vLLM backend", seventh paragraph), fused in one pass per
+ * row / group: amax over the row (FP8_DYNAMIC, W8A8_INT8), the 1x128 group
+ * (BLOCK_FP8) or the tensor and each 16-element block (NVFP4), then
+ * scale = amax / Qmax (448 for e4m3, 127 for int8) in correctly rounded fp32,
+ * and codes = round-to-nearest-even(x / scale) saturated to the format
+ * (int8 clamped to [-127, 127]).  An all-zero row/group/tensor gets scale 1.
+ * NVFP4: g = amax(tensor) / 2688, block scale = e4m3((amax_b / 6) / g),
+ * code = e2m1(x / (dec(block scale) * g)), code 0 where the block scale is 0.
+ *
+ *   A:   bf16 [M, lda] (lda >= K elements, lda*2 a multiple of 16 bytes)
+ *   static_amax: NVFP4 only, optional device fp32 scalar; when non-NULL it
+ *        replaces the tensor amax (a static activation scale).
+ *   out: caller-allocated q / scale / global_scale of the sizes
+ *        qgemm_operand_bytes(f, 0, M, K) gives; out->rows = M, out->K = K.
+ *   workspace: qgemm_quant_workspace_size(f, M, K) bytes (NULL if 0).
+ * K must be a multiple of 16 (FP8_DYNAMIC, W8A8_INT8), 128 (BLOCK_FP8) or
+ * 32 (NVFP4). */
+qg_status qgemm_quantize_act(qg_format f, const void* A, int M, int K, int lda,
+                             const float* static_amax, qg_operand* out,
+                             void* workspace, size_t ws_bytes, void* stream);
+
+/* Offline weight quantisation of W bf16 [N, K] (contiguous): per-channel
+ * (FP8_DYNAMIC: amax/448, W8A8_INT8: amax/127), per 128x128 block
+ * (BLOCK_FP8) or NVFP4 as above. */
+qg_status qgemm_quantize_weight(qg_format f, const void* W, int N, int K, qg_operand* out,
+                                void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------ GEMM -- */
+
+/* y = dequant(A_q) . dequant(W_q)^T with configuration `cfg`.
+ *   A: activations, A->rows == M, A->K == K;  W: weights, W->rows == N.
+ *   Y: bf16 [M, ldy] (QG_OUT_BF16) or int32/fp32 [M, ldy] (QG_OUT_ACC);
+ *      ldy >= N, ldy * elem a multiple of 16 bytes.
+ *   workspace: qgemm_workspace_size(f, M, N, K, cfg) bytes (NULL if 0).
+ * Epilogue: y = acc * s_a[m] * s_w[n] (FP8_DYNAMIC, W8A8_INT8; int32 acc
+ * converted to fp32 first), per-group promotion acc += (p_g * s_a[m,g]) *
+ * s_w[n/128,g] (BLOCK_FP8), y = acc * (g_a * g_w) (NVFP4); all in fp32, then
+ * bf16 round-to-nearest-even.  Returns QG_ERR_UNSUPPORTED for a config the
+ * kernels do not implement (e.g. split_k larger than the number of 128-byte
+ * K tiles) and QG_ERR_WORKSPACE if ws_bytes is too small.
+ * Weights are read before the kernel waits on the preceding kernel of the
+ * stream (programmatic dependent launch): W_q must not be written by a
+ * kernel that may still run when qgemm_run is enqueued. */
+qg_status qgemm_run(qg_format f, const qg_operand* A, const qg_operand* W, int M, int N, int K,
+                    const qg_config* cfg, void* workspace, size_t ws_bytes, void* Y, int ldy,
+                    int out_kind, void* stream);
+
+/* Default configuration for a shape when no table entry exists: swap_ab = 1
+ * for M < 32 ("Helion in the vLLM backend", second paragraph: vLLM's
+ * Block_FP8 backend swaps A and B below M = 32), split_k chosen so that
+ * output tiles x split_k approaches the SM count. */
+qg_status qgemm_default_config(qg_format f, int M, int N, int K, qg_config* out);
+
+/* ---------------------------------------------------- table and tuning -- */
+
+/* Loads a per-shape table file written by qgemm_tune / qgemm_table_save.
+ * *table receives a library-owned handle, freed by qgemm_table_free. */
+qg_status qgemm_table_load(const char* path, void** table);
+/* Creates an empty table. */
+qg_status qgemm_table_create(void** table);
+/* Inserts or replaces the entry for (f, M, N, K). */
+qg_status qgemm_table_put(void* table, qg_format f, int M, int N, int K, const qg_config* cfg,
+                          double us);
+/* Writes the table (text, versioned, with device name and SM count). */
+qg_status qgemm_table_save(const void* table, const char* path);
+void qgemm_table_free(void* table);
+/* Number of entries. */
+int qgemm_table_size(const void* table);
+
+/* Looks up (f, M, N, K).  *hit = 1 on an exact entry.  On a miss the entry
+ * with the same (f, N, K) and the smallest tuned M' >= M is used (*hit = 2);
+ * failing that, qgemm_default_config (*hit = 0).  Host only, no device
+ * work, capture-safe. */
+qg_status qgemm_dispatch(const void* table, qg_format f, int M, int N, int K, qg_config* out,
+                         int* hit);
+
+/* Ahead-of-time tuner: for each (M, (N, K)) enumerates the valid configs
+ * (split_k, swap_ab, tile_n, stages, reduce_mode), times each with CUDA
+ * events over a graph of back-to-back calls (selection pass), re-times the
+ * winner in an independent pass that is what the table records, and rejects
+ * any config whose output differs from the default config's.  Shapes already
+ * present in `table` are skipped (resume).  Synthetic inputs are generated
+ * on the device; `budget_s_per_shape` bounds the wall time per shape.
+ * NK holds nNK pairs (N, K). */
+qg_status qgemm_tune(void* table, qg_format f, const int* Ms, int nM, const int* NK, int nNK,
+                     double budget_s_per_shape, int verbose);
+
+/* -------------------------------------------------------------- errors -- */
+
+const char* qgemm_status_string(qg_status s);
+/* Reads (and clears) the device error word set by a bounded in-kernel wait
+ * that expired; synchronises the device.  Returns QG_OK or
+ * QG_ERR_DEVICE_TIMEOUT. */
+qg_status qgemm_device_error(void);
+/* Enables (1) or disables (0) programmatic dependent launch for the
+ * library's kernels (default 1). */
+void qgemm_set_pdl(int enable);
+/* ABI version of the loaded library (QGEMM_ABI_VERSION). */
+int qgemm_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QGEMM_H_ */

@@ -1,0 +1,334 @@
+"""Python binding of libqgemm.so — the B200 quantized linear-layer GEMM.
+
+Argument marshalling only: every step of the quantized path (activation
+quantisation, the tcgen05 GEMM, split-K reduction, dispatch, tuning) runs in
+the C-ABI library ``libqgemm.so`` built from ``csrc/``.  PyTorch supplies
+device memory and streams.  If the library is missing this module raises on
+first use; there is no fallback.
+
+The ctypes entry points carry the C names (``qgemm_run`` ...).  ``Operand``,
+``quantize_act``, ``quantize_weight``, ``run`` and ``Linear`` are
+conveniences over them that allocate the caller-owned buffers with torch.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, c_char_p, c_double, c_int, c_int32, c_size_t, c_void_p
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqgemm.so")
+
+# formats
+QG_FP8_DYNAMIC, QG_W8A8_INT8, QG_BLOCK_FP8, QG_NVFP4 = 0, 1, 2, 3
+FORMATS = {"fp8_dynamic": 0, "w8a8_int8": 1, "block_fp8": 2, "nvfp4": 3}
+# statuses
+QG_OK = 0
+QG_ERR_INVALID_ARG = 1
+QG_ERR_UNSUPPORTED = 2
+QG_ERR_WORKSPACE = 3
+QG_ERR_TABLE_IO = 4
+QG_ERR_TABLE_MISS = 5
+QG_ERR_CUDA = 6
+QG_ERR_DEVICE_TIMEOUT = 7
+QG_ERR_NO_DEVICE = 8
+# output kinds
+QG_OUT_BF16, QG_OUT_ACC = 0, 1
+
+EXPORTS = [
+    "qgemm_abi_version", "qgemm_set_pdl", "qgemm_status_string", "qgemm_operand_bytes",
+    "qgemm_quant_workspace_size", "qgemm_workspace_size", "qgemm_workspace_clear",
+    "qgemm_quantize_act", "qgemm_quantize_weight", "qgemm_run", "qgemm_default_config",
+    "qgemm_table_load", "qgemm_table_create", "qgemm_table_put", "qgemm_table_save",
+    "qgemm_table_free", "qgemm_table_size", "qgemm_dispatch", "qgemm_tune", "qgemm_device_error",
+]
+
+
+class qg_config(ctypes.Structure):
+    _fields_ = [("split_k", c_int32), ("swap_ab", c_int32), ("tile_n", c_int32),
+                ("stages", c_int32), ("reduce_mode", c_int32), ("reserved", c_int32 * 3)]
+
+    def as_dict(self):
+        return {k: getattr(self, k) for k in ("split_k", "swap_ab", "tile_n", "stages", "reduce_mode")}
+
+    def __repr__(self):
+        return f"qg_config({self.as_dict()})"
+
+
+def make_config(split_k=1, swap_ab=1, tile_n=16, stages=8, reduce_mode=0) -> qg_config:
+    c = qg_config()
+    c.split_k, c.swap_ab, c.tile_n, c.stages, c.reduce_mode = split_k, swap_ab, tile_n, stages, reduce_mode
+    return c
+
+
+class qg_operand(ctypes.Structure):
+    _fields_ = [("q", c_void_p), ("scale", c_void_p), ("global_scale", c_void_p),
+                ("rows", c_int32), ("K", c_int32)]
+
+
+class QGemmError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libqgemm.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m precision_quantized_gemm_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        sig = {
+            "qgemm_abi_version": (c_int, []),
+            "qgemm_set_pdl": (None, [c_int]),
+            "qgemm_status_string": (c_char_p, [c_int]),
+            "qgemm_operand_bytes": (c_int, [c_int, c_int, c_int, c_int, POINTER(c_size_t), POINTER(c_size_t)]),
+            "qgemm_quant_workspace_size": (c_size_t, [c_int, c_int, c_int]),
+            "qgemm_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int, POINTER(qg_config)]),
+            "qgemm_workspace_clear": (c_int, [c_void_p, c_size_t, c_void_p]),
+            "qgemm_quantize_act": (c_int, [c_int, c_void_p, c_int, c_int, c_int, c_void_p,
+                                           POINTER(qg_operand), c_void_p, c_size_t, c_void_p]),
+            "qgemm_quantize_weight": (c_int, [c_int, c_void_p, c_int, c_int, POINTER(qg_operand),
+                                              c_void_p, c_size_t, c_void_p]),
+            "qgemm_run": (c_int, [c_int, POINTER(qg_operand), POINTER(qg_operand), c_int, c_int, c_int,
+                                  POINTER(qg_config), c_void_p, c_size_t, c_void_p, c_int, c_int, c_void_p]),
+            "qgemm_default_config": (c_int, [c_int, c_int, c_int, c_int, POINTER(qg_config)]),
+            "qgemm_table_load": (c_int, [c_char_p, POINTER(c_void_p)]),
+            "qgemm_table_create": (c_int, [POINTER(c_void_p)]),
+            "qgemm_table_put": (c_int, [c_void_p, c_int, c_int, c_int, c_int, POINTER(qg_config), c_double]),
+            "qgemm_table_save": (c_int, [c_void_p, c_char_p]),
+            "qgemm_table_free": (None, [c_void_p]),
+            "qgemm_table_size": (c_int, [c_void_p]),
+            "qgemm_dispatch": (c_int, [c_void_p, c_int, c_int, c_int, c_int, POINTER(qg_config), POINTER(c_int)]),
+            "qgemm_tune": (c_int, [c_void_p, c_int, POINTER(c_int), c_int, POINTER(c_int), c_int, c_double, c_int]),
+            "qgemm_device_error": (c_int, []),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().qgemm_status_string(status).decode()
+
+
+def check(status: int, what: str = "qgemm") -> None:
+    if status != QG_OK:
+        raise QGemmError(status, what)
+
+
+# ------------------------------------------------------- C-named entry points --
+def qgemm_operand_bytes(fmt, is_weight, rows, K):
+    q, s = c_size_t(), c_size_t()
+    st = lib().qgemm_operand_bytes(fmt, int(is_weight), rows, K, ctypes.byref(q), ctypes.byref(s))
+    check(st, "qgemm_operand_bytes")
+    return q.value, s.value
+
+
+def qgemm_quant_workspace_size(fmt, rows, K):
+    return lib().qgemm_quant_workspace_size(fmt, rows, K)
+
+
+def qgemm_workspace_size(fmt, M, N, K, cfg: qg_config):
+    return lib().qgemm_workspace_size(fmt, M, N, K, ctypes.byref(cfg))
+
+
+def qgemm_workspace_clear(ws_ptr, ws_bytes, stream=None):
+    return lib().qgemm_workspace_clear(ws_ptr, ws_bytes, stream)
+
+
+def qgemm_quantize_act(fmt, A_ptr, M, K, lda, static_amax_ptr, out: qg_operand, ws_ptr, ws_bytes, stream):
+    return lib().qgemm_quantize_act(fmt, A_ptr, M, K, lda, static_amax_ptr, ctypes.byref(out),
+                                    ws_ptr, ws_bytes, stream)
+
+
+def qgemm_quantize_weight(fmt, W_ptr, N, K, out: qg_operand, ws_ptr, ws_bytes, stream):
+    return lib().qgemm_quantize_weight(fmt, W_ptr, N, K, ctypes.byref(out), ws_ptr, ws_bytes, stream)
+
+
+def qgemm_run(fmt, A: qg_operand, W: qg_operand, M, N, K, cfg: qg_config, ws_ptr, ws_bytes,
+              Y_ptr, ldy, out_kind, stream):
+    return lib().qgemm_run(fmt, ctypes.byref(A), ctypes.byref(W), M, N, K, ctypes.byref(cfg),
+                           ws_ptr, ws_bytes, Y_ptr, ldy, out_kind, stream)
+
+
+def qgemm_default_config(fmt, M, N, K) -> qg_config:
+    c = qg_config()
+    check(lib().qgemm_default_config(fmt, M, N, K, ctypes.byref(c)), "qgemm_default_config")
+    return c
+
+
+def qgemm_dispatch(table, fmt, M, N, K):
+    c = qg_config()
+    hit = c_int(0)
+    check(lib().qgemm_dispatch(table, fmt, M, N, K, ctypes.byref(c), ctypes.byref(hit)), "qgemm_dispatch")
+    return c, hit.value
+
+
+def qgemm_device_error():
+    return lib().qgemm_device_error()
+
+
+def qgemm_set_pdl(enable: bool):
+    lib().qgemm_set_pdl(1 if enable else 0)
+
+
+class Table:
+    """Owning wrapper of a qgemm table handle."""
+
+    def __init__(self, path: str | None = None):
+        h = c_void_p()
+        if path is None:
+            check(lib().qgemm_table_create(ctypes.byref(h)), "qgemm_table_create")
+        else:
+            check(lib().qgemm_table_load(path.encode(), ctypes.byref(h)), f"qgemm_table_load({path})")
+        self.handle = h
+
+    def __len__(self):
+        return lib().qgemm_table_size(self.handle)
+
+    def put(self, fmt, M, N, K, cfg: qg_config, us: float = 0.0):
+        check(lib().qgemm_table_put(self.handle, fmt, M, N, K, ctypes.byref(cfg), us), "qgemm_table_put")
+
+    def save(self, path: str):
+        check(lib().qgemm_table_save(self.handle, path.encode()), "qgemm_table_save")
+
+    def dispatch(self, fmt, M, N, K):
+        return qgemm_dispatch(self.handle, fmt, M, N, K)
+
+    def tune(self, fmt, Ms, NK, budget_s_per_shape=30.0, verbose=True):
+        Ms_arr = (c_int * len(Ms))(*Ms)
+        flat = [v for nk in NK for v in nk]
+        NK_arr = (c_int * len(flat))(*flat)
+        check(lib().qgemm_tune(self.handle, fmt, Ms_arr, len(Ms), NK_arr, len(NK),
+                               float(budget_s_per_shape), 1 if verbose else 0), "qgemm_tune")
+
+    def close(self):
+        if getattr(self, "handle", None) is not None and self.handle.value:
+            lib().qgemm_table_free(self.handle)
+            self.handle = c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+# ------------------------------------------------------------ torch helpers --
+def _torch():
+    import torch
+    return torch
+
+
+def _stream(stream=None):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return c_void_p(s.cuda_stream)
+
+
+class Operand:
+    """Caller-owned buffers of a quantized operand, allocated with torch."""
+
+    def __init__(self, fmt: int, is_weight: bool, rows: int, K: int, device="cuda"):
+        torch = _torch()
+        qb, sb = qgemm_operand_bytes(fmt, is_weight, rows, K)
+        self.fmt, self.is_weight, self.rows, self.K = fmt, is_weight, rows, K
+        self.q = torch.empty(qb, dtype=torch.uint8, device=device)
+        self.scale = torch.zeros(max(sb, 16) // 4 * 4 + 16, dtype=torch.uint8, device=device)[:sb]
+        self.global_scale = torch.zeros(4, dtype=torch.float32, device=device)
+        self.c = qg_operand(self.q.data_ptr(), self.scale.data_ptr(), self.global_scale.data_ptr(), rows, K)
+
+
+def quantize_act(fmt: int, A, out: Operand | None = None, static_amax=None, stream=None) -> Operand:
+    """Dynamic activation quantisation of bf16 A [M, K] (row stride A.stride(0))."""
+    torch = _torch()
+    M, K = A.shape
+    out = out or Operand(fmt, False, M, K, A.device)
+    wsb = qgemm_quant_workspace_size(fmt, M, K)
+    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=A.device)
+    sa = static_amax.data_ptr() if static_amax is not None else None
+    check(qgemm_quantize_act(fmt, A.data_ptr(), M, K, A.stride(0), sa, out.c, ws.data_ptr(), wsb,
+                             _stream(stream)), "qgemm_quantize_act")
+    out._ws = ws
+    return out
+
+
+def quantize_weight(fmt: int, W, stream=None) -> Operand:
+    torch = _torch()
+    N, K = W.shape
+    out = Operand(fmt, True, N, K, W.device)
+    wsb = qgemm_quant_workspace_size(fmt, N, K)
+    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=W.device)
+    check(qgemm_quantize_weight(fmt, W.contiguous().data_ptr(), N, K, out.c, ws.data_ptr(), wsb,
+                                _stream(stream)), "qgemm_quantize_weight")
+    out._ws = ws
+    return out
+
+
+class Workspace:
+    """A zeroed run workspace that grows on demand."""
+
+    def __init__(self, device="cuda"):
+        self.device = device
+        self.buf = None
+
+    def get(self, nbytes: int):
+        torch = _torch()
+        if nbytes == 0:
+            return None, 0
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.zeros(nbytes, dtype=torch.uint8, device=self.device)
+        return self.buf.data_ptr(), self.buf.numel()
+
+
+def run(fmt: int, A: Operand, W: Operand, cfg: qg_config | None = None, out=None,
+        out_kind: int = QG_OUT_BF16, workspace: Workspace | None = None, stream=None):
+    """y = dequant(A_q) . dequant(W_q)^T through qgemm_run; returns y [M, N]."""
+    torch = _torch()
+    M, N, K = A.rows, W.rows, A.K
+    cfg = cfg or qgemm_default_config(fmt, M, N, K)
+    if out is None:
+        dt = torch.bfloat16 if out_kind == QG_OUT_BF16 else (torch.int32 if fmt == QG_W8A8_INT8 else torch.float32)
+        out = torch.empty(M, N, dtype=dt, device=A.q.device)
+    workspace = workspace or Workspace(A.q.device)
+    wsp, wsb = workspace.get(qgemm_workspace_size(fmt, M, N, K, cfg))
+    check(qgemm_run(fmt, A.c, W.c, M, N, K, cfg, wsp, wsb, out.data_ptr(), out.stride(0), out_kind,
+                    _stream(stream)), "qgemm_run")
+    return out
+
+
+class Linear:
+    """A quantized linear layer: weights quantised once, activations per call,
+    configuration from a tuned table (or the default), optional CUDA-graph
+    replay per token count (``capture(M)``)."""
+
+    def __init__(self, fmt: int, W, table: Table | None = None):
+        self.fmt = fmt
+        self.N, self.K = W.shape
+        self.Wq = quantize_weight(fmt, W)
+        self.table = table
+        self.ws = Workspace(W.device)
+        self._act = {}
+        self.graphs = {}
+
+    def config(self, M):
+        if self.table is not None:
+            return self.table.dispatch(self.fmt, M, self.N, self.K)[0]
+        return qgemm_default_config(self.fmt, M, self.N, self.K)
+
+    def __call__(self, A, out=None, stream=None):
+        M = A.shape[0]
+        act = self._act.get(M)
+        if act is None:
+            act = self._act[M] = Operand(self.fmt, False, M, self.K, A.device)
+        quantize_act(self.fmt, A, out=act, stream=stream)
+        return run(self.fmt, act, self.Wq, self.config(M), out=out, workspace=self.ws, stream=stream)

@@ -1,0 +1,411 @@
+// api.cu — the C ABI of libqgemm.so: argument checks, buffer sizes, TMA
+// descriptors, launches of the quantisers and of the unified GEMM kernel.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/qgemm.h"
+#include "gemm_kernel.cuh"
+#include "internal.h"
+
+namespace qg {
+// Device error word: set by bounded in-kernel waits that expire.
+__device__ unsigned int g_qg_error = 0;
+}  // namespace qg
+
+namespace {
+
+using qg::GemmParams;
+
+bool g_pdl = true;
+
+constexpr int kMaxDevices = 64;
+struct DeviceInfo {
+  bool probed = false;
+  bool sm100 = false;
+  int sms = 0;
+  unsigned int* err = nullptr;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+qg_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QG_ERR_NO_DEVICE;
+  if (dev < 0 || dev >= kMaxDevices) return QG_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.probed) {
+    cudaDeviceProp p;
+    if (cudaGetDeviceProperties(&p, dev) != cudaSuccess) return QG_ERR_CUDA;
+    d.sm100 = (p.major == 10 && p.minor == 0);
+    d.sms = p.multiProcessorCount;
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, qg::g_qg_error) != cudaSuccess) return QG_ERR_CUDA;
+    d.err = static_cast<unsigned int*>(addr);
+    d.probed = true;
+  }
+  if (!d.sm100) return QG_ERR_UNSUPPORTED;
+  *out = &d;
+  return QG_OK;
+}
+
+// ------------------------------------------------------------- TMA maps --
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2D byte tensor [rows, row_bytes] (row stride row_bytes), box 128 bytes x
+// box_rows, 128-byte swizzle, out-of-range elements read as zero.
+bool make_tmap(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows,
+               uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {row_bytes, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- checks --
+bool valid_format(int f) { return f >= QG_FP8_DYNAMIC && f <= QG_NVFP4; }
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+int k_multiple(qg_format f) {
+  switch (f) {
+    case QG_BLOCK_FP8: return 128;
+    case QG_NVFP4: return 32;
+    default: return 16;
+  }
+}
+size_t row_bytes(qg_format f, int K) { return f == QG_NVFP4 ? (size_t)K / 2 : (size_t)K; }
+int kt_total(qg_format f, int K) { return (int)((row_bytes(f, K) + 127) / 128); }
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+size_t gemm_smem(qg_format f, int tile_n, int stages) {
+  switch (f) {
+    case QG_FP8_DYNAMIC: return qg::launch_gemm_fp8_smem(tile_n, stages);
+    case QG_W8A8_INT8: return qg::launch_gemm_int8_smem(tile_n, stages);
+    case QG_BLOCK_FP8: return qg::launch_gemm_block_smem(tile_n, stages);
+    default: return qg::launch_gemm_nvf4_smem(tile_n, stages);
+  }
+}
+constexpr size_t kSmemLimit = 232448;  // 227 KB opt-in per CTA on sm_100
+
+qg_status check_config(qg_format f, int M, int N, int K, const qg_config* c) {
+  if (!c) return QG_ERR_INVALID_ARG;
+  if (c->reserved[0] || c->reserved[1] || c->reserved[2]) return QG_ERR_INVALID_ARG;
+  if (!is_pow2(c->split_k) || c->split_k > 256) return QG_ERR_UNSUPPORTED;
+  if (c->swap_ab != 0 && c->swap_ab != 1) return QG_ERR_INVALID_ARG;
+  if (c->reduce_mode != 0 && c->reduce_mode != 1) return QG_ERR_INVALID_ARG;
+  const int tn = c->tile_n;
+  if (tn != 16 && tn != 32 && tn != 64 && tn != 128 && tn != 256) return QG_ERR_UNSUPPORTED;
+  if (f == QG_BLOCK_FP8 && tn > 128) return QG_ERR_UNSUPPORTED;
+  // NVFP4 block scales of the N operand sit in 32-lane TMEM words: a 16-row
+  // tile must start at a multiple of 32 rows, i.e. be the only tile.
+  if (f == QG_NVFP4 && tn == 16 && (c->swap_ab ? M : N) > 16) return QG_ERR_UNSUPPORTED;
+  if (c->stages < 2 || c->stages > 12) return QG_ERR_UNSUPPORTED;
+  const int kt = kt_total(f, K);
+  if (c->split_k > kt) return QG_ERR_UNSUPPORTED;
+  if (gemm_smem(f, tn, c->stages) > kSmemLimit) return QG_ERR_UNSUPPORTED;
+  if (f == QG_BLOCK_FP8) {
+    const int nkt_max = (kt + c->split_k - 1) / c->split_k;
+    const int act_rows = c->swap_ab ? tn : 128;
+    if (nkt_max > 64 || act_rows * nkt_max > qg::kMaxScaleStage) return QG_ERR_UNSUPPORTED;
+  }
+  return QG_OK;
+}
+
+size_t ws_partial_bytes(int M, int N, int split) {
+  return split > 1 ? align_up((size_t)split * M * N * 4, 256) : 0;
+}
+void tiles_of(const qg_config* c, int M, int N, int* tp, int* tq) {
+  const int rows_p = c->swap_ab ? N : M;
+  const int rows_q = c->swap_ab ? M : N;
+  *tp = (rows_p + 127) / 128;
+  *tq = (rows_q + c->tile_n - 1) / c->tile_n;
+}
+
+}  // namespace
+
+extern "C" {
+
+int qgemm_abi_version(void) { return QGEMM_ABI_VERSION; }
+
+void qgemm_set_pdl(int enable) { g_pdl = enable != 0; }
+
+const char* qgemm_status_string(qg_status s) {
+  switch (s) {
+    case QG_OK: return "ok";
+    case QG_ERR_INVALID_ARG: return "invalid argument";
+    case QG_ERR_UNSUPPORTED: return "unsupported shape, configuration or device";
+    case QG_ERR_WORKSPACE: return "workspace missing or too small";
+    case QG_ERR_TABLE_IO: return "table file missing, corrupt or of another version";
+    case QG_ERR_TABLE_MISS: return "no table entry";
+    case QG_ERR_CUDA: return "CUDA error";
+    case QG_ERR_DEVICE_TIMEOUT: return "in-kernel wait timed out";
+    case QG_ERR_NO_DEVICE: return "no CUDA device";
+  }
+  return "unknown status";
+}
+
+qg_status qgemm_operand_bytes(qg_format f, int is_weight, int rows, int K, size_t* q_bytes,
+                              size_t* scale_bytes) {
+  if (!valid_format(f) || rows <= 0 || K <= 0 || !q_bytes || !scale_bytes) return QG_ERR_INVALID_ARG;
+  if (K % k_multiple(f) != 0) return QG_ERR_INVALID_ARG;
+  *q_bytes = (size_t)rows * row_bytes(f, K);
+  switch (f) {
+    case QG_FP8_DYNAMIC:
+    case QG_W8A8_INT8: *scale_bytes = (size_t)rows * 4; break;
+    case QG_BLOCK_FP8:
+      *scale_bytes = (is_weight ? (size_t)((rows + 127) / 128) : (size_t)rows) * (K / 128) * 4;
+      break;
+    case QG_NVFP4:
+      *scale_bytes = (size_t)((rows + 127) / 128) * 128 * (size_t)(((K + 255) / 256) * 16);
+      break;
+  }
+  return QG_OK;
+}
+
+size_t qgemm_quant_workspace_size(qg_format f, int rows, int K) {
+  (void)rows;
+  (void)K;
+  return f == QG_NVFP4 ? (size_t)qg::kNvfp4AmaxMaxCtas * 4 : 0;
+}
+
+size_t qgemm_workspace_size(qg_format f, int M, int N, int K, const qg_config* cfg) {
+  if (!valid_format(f) || !cfg || M <= 0 || N <= 0 || K <= 0 || cfg->split_k <= 1) return 0;
+  int tp, tq;
+  tiles_of(cfg, M, N, &tp, &tq);
+  return ws_partial_bytes(M, N, cfg->split_k) + align_up((size_t)tp * tq * 4, 256);
+}
+
+qg_status qgemm_workspace_clear(void* workspace, size_t ws_bytes, void* stream) {
+  if (ws_bytes == 0) return QG_OK;
+  if (!workspace) return QG_ERR_INVALID_ARG;
+  return cudaMemsetAsync(workspace, 0, ws_bytes, (cudaStream_t)stream) == cudaSuccess ? QG_OK
+                                                                                     : QG_ERR_CUDA;
+}
+
+static qg_status check_quant_out(qg_format f, int rows, int K, const qg_operand* out) {
+  if (!out || !out->q || !out->scale) return QG_ERR_INVALID_ARG;
+  if (out->rows != rows || out->K != K) return QG_ERR_INVALID_ARG;
+  if (!aligned(out->q, 16) || !aligned(out->scale, f == QG_NVFP4 ? 16 : 4)) return QG_ERR_INVALID_ARG;
+  if (f == QG_NVFP4 && (!out->global_scale || !aligned(out->global_scale, 4))) return QG_ERR_INVALID_ARG;
+  return QG_OK;
+}
+
+qg_status qgemm_quantize_act(qg_format f, const void* A, int M, int K, int lda,
+                             const float* static_amax, qg_operand* out, void* workspace,
+                             size_t ws_bytes, void* stream) {
+  if (!valid_format(f) || !A || M <= 0 || K <= 0 || lda < K) return QG_ERR_INVALID_ARG;
+  if (K % k_multiple(f) != 0 || (lda * 2) % 16 != 0 || !aligned(A, 16)) return QG_ERR_INVALID_ARG;
+  qg_status s = check_quant_out(f, M, K, out);
+  if (s != QG_OK) return s;
+  const size_t need = qgemm_quant_workspace_size(f, M, K);
+  if (f == QG_NVFP4 && static_amax == nullptr && (ws_bytes < need || !workspace))
+    return QG_ERR_WORKSPACE;
+  DeviceInfo* d;
+  if ((s = device_info(&d)) != QG_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e;
+  switch (f) {
+    case QG_FP8_DYNAMIC:
+    case QG_W8A8_INT8:
+      e = qg::launch_quant_rows(f == QG_W8A8_INT8, A, M, K, lda, out->q, (float*)out->scale, st, g_pdl);
+      break;
+    case QG_BLOCK_FP8:
+      e = qg::launch_quant_act_groups(A, M, K, lda, out->q, (float*)out->scale, st, g_pdl);
+      break;
+    default:
+      e = qg::launch_quant_nvfp4(A, M, K, lda, static_amax, out->q, out->scale, out->global_scale,
+                                 (float*)workspace, st, g_pdl);
+  }
+  return e == cudaSuccess ? QG_OK : QG_ERR_CUDA;
+}
+
+qg_status qgemm_quantize_weight(qg_format f, const void* W, int N, int K, qg_operand* out,
+                                void* workspace, size_t ws_bytes, void* stream) {
+  if (!valid_format(f) || !W || N <= 0 || K <= 0) return QG_ERR_INVALID_ARG;
+  if (K % k_multiple(f) != 0 || !aligned(W, 16)) return QG_ERR_INVALID_ARG;
+  qg_status s = check_quant_out(f, N, K, out);
+  if (s != QG_OK) return s;
+  if (f == QG_NVFP4 && (ws_bytes < qgemm_quant_workspace_size(f, N, K) || !workspace))
+    return QG_ERR_WORKSPACE;
+  DeviceInfo* d;
+  if ((s = device_info(&d)) != QG_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e;
+  switch (f) {
+    case QG_FP8_DYNAMIC:
+    case QG_W8A8_INT8:
+      e = qg::launch_quant_rows(f == QG_W8A8_INT8, W, N, K, K, out->q, (float*)out->scale, st, g_pdl);
+      break;
+    case QG_BLOCK_FP8:
+      e = qg::launch_quant_weight_blocks(W, N, K, out->q, (float*)out->scale, st, g_pdl);
+      break;
+    default:
+      e = qg::launch_quant_nvfp4(W, N, K, K, nullptr, out->q, out->scale, out->global_scale,
+                                 (float*)workspace, st, g_pdl);
+  }
+  return e == cudaSuccess ? QG_OK : QG_ERR_CUDA;
+}
+
+static qg_status check_operand(qg_format f, const qg_operand* o, int rows, int K) {
+  if (!o || !o->q || !o->scale) return QG_ERR_INVALID_ARG;
+  if (o->rows != rows || o->K != K) return QG_ERR_INVALID_ARG;
+  if (!aligned(o->q, 16) || !aligned(o->scale, f == QG_NVFP4 ? 16 : 4)) return QG_ERR_INVALID_ARG;
+  if (f == QG_NVFP4 && (!o->global_scale || !aligned(o->global_scale, 4))) return QG_ERR_INVALID_ARG;
+  return QG_OK;
+}
+
+qg_status qgemm_run(qg_format f, const qg_operand* A, const qg_operand* W, int M, int N, int K,
+                    const qg_config* cfg, void* workspace, size_t ws_bytes, void* Y, int ldy,
+                    int out_kind, void* stream) {
+  if (!valid_format(f) || M <= 0 || N <= 0 || K <= 0 || !Y || ldy < N) return QG_ERR_INVALID_ARG;
+  if (out_kind != QG_OUT_BF16 && out_kind != QG_OUT_ACC) return QG_ERR_INVALID_ARG;
+  if (K % k_multiple(f) != 0 || !aligned(Y, 16)) return QG_ERR_INVALID_ARG;
+  qg_status s;
+  if ((s = check_operand(f, A, M, K)) != QG_OK) return s;
+  if ((s = check_operand(f, W, N, K)) != QG_OK) return s;
+  if ((s = check_config(f, M, N, K, cfg)) != QG_OK) return s;
+  const size_t need = qgemm_workspace_size(f, M, N, K, cfg);
+  if (need > 0 && (!workspace || ws_bytes < need || !aligned(workspace, 256))) return QG_ERR_WORKSPACE;
+  DeviceInfo* d;
+  if ((s = device_info(&d)) != QG_OK) return s;
+
+  const bool swap = cfg->swap_ab != 0;
+  GemmParams prm = {};
+  prm.M = M;
+  prm.N = N;
+  prm.K = K;
+  prm.rows_p = swap ? N : M;
+  prm.rows_q = swap ? M : N;
+  prm.kt_total = kt_total(f, K);
+  prm.split_k = cfg->split_k;
+  prm.stages = cfg->stages;
+  prm.groups = K / 128;
+  prm.scale_a = static_cast<const float*>(A->scale);
+  prm.scale_w = static_cast<const float*>(W->scale);
+  const uint8_t* sfa = static_cast<const uint8_t*>(A->scale);
+  const uint8_t* sfw = static_cast<const uint8_t*>(W->scale);
+  prm.sf_p = swap ? sfw : sfa;
+  prm.sf_q = swap ? sfa : sfw;
+  prm.sf_atoms_per_rb = ((K + 255) / 256) * 4;
+  prm.g_a = A->global_scale;
+  prm.g_w = W->global_scale;
+  prm.Y = Y;
+  prm.ldy = ldy;
+  prm.out_kind = out_kind;
+  int tp, tq;
+  tiles_of(cfg, M, N, &tp, &tq);
+  if (cfg->split_k > 1) {
+    prm.partial = workspace;
+    prm.counters = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(workspace) +
+                                                   ws_partial_bytes(M, N, cfg->split_k));
+  }
+  prm.reduce_mode = cfg->reduce_mode;
+  prm.err = d->err;
+
+  const void* base_p = swap ? W->q : A->q;
+  const void* base_q = swap ? A->q : W->q;
+  CUtensorMap tmp, tmq;
+  const uint64_t rb = row_bytes(f, K);
+  if (!make_tmap(&tmp, base_p, rb, (uint64_t)prm.rows_p, 128) ||
+      !make_tmap(&tmq, base_q, rb, (uint64_t)prm.rows_q, (uint32_t)cfg->tile_n))
+    return QG_ERR_CUDA;
+  if (tq > 65535) return QG_ERR_UNSUPPORTED;
+  const dim3 grid(tp, tq, cfg->split_k);
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e;
+  switch (f) {
+    case QG_FP8_DYNAMIC: e = qg::launch_gemm_fp8(swap, cfg->tile_n, tmp, tmq, prm, grid, st, g_pdl); break;
+    case QG_W8A8_INT8: e = qg::launch_gemm_int8(swap, cfg->tile_n, tmp, tmq, prm, grid, st, g_pdl); break;
+    case QG_BLOCK_FP8: e = qg::launch_gemm_block(swap, cfg->tile_n, tmp, tmq, prm, grid, st, g_pdl); break;
+    default: e = qg::launch_gemm_nvf4(swap, cfg->tile_n, tmp, tmq, prm, grid, st, g_pdl); break;
+  }
+  if (e != cudaSuccess) return e == cudaErrorInvalidValue ? QG_ERR_UNSUPPORTED : QG_ERR_CUDA;
+  if (cfg->split_k > 1 && cfg->reduce_mode == 1) {
+    switch (f) {
+      case QG_FP8_DYNAMIC: e = qg::launch_gemm_fp8_reduce(prm, st, g_pdl); break;
+      case QG_W8A8_INT8: e = qg::launch_gemm_int8_reduce(prm, st, g_pdl); break;
+      case QG_BLOCK_FP8: e = qg::launch_gemm_block_reduce(prm, st, g_pdl); break;
+      default: e = qg::launch_gemm_nvf4_reduce(prm, st, g_pdl); break;
+    }
+    if (e != cudaSuccess) return QG_ERR_CUDA;
+  }
+  return QG_OK;
+}
+
+qg_status qgemm_default_config(qg_format f, int M, int N, int K, qg_config* out) {
+  if (!valid_format(f) || M <= 0 || N <= 0 || K <= 0 || !out) return QG_ERR_INVALID_ARG;
+  if (K % k_multiple(f) != 0) return QG_ERR_INVALID_ARG;
+  qg_config c = {};
+  c.reduce_mode = 0;
+  // Swap-AB below 32 tokens (and up to 64, where tokens still fit the MMA N
+  // slot in one tile); the standard orientation above.
+  c.swap_ab = M <= 64 ? 1 : 0;
+  if (c.swap_ab) {
+    c.tile_n = M <= 16 ? 16 : M <= 32 ? 32 : 64;
+  } else {
+    c.tile_n = f == QG_BLOCK_FP8 ? 128 : 256;
+  }
+  // deepest pipeline that fits, at most 8 stages
+  c.stages = 2;
+  for (int s = 8; s >= 2; --s)
+    if (gemm_smem(f, c.tile_n, s) <= kSmemLimit) { c.stages = s; break; }
+  // split-K: fill the SMs with tiles x split, keeping >= 2 K tiles per split
+  int tp, tq;
+  c.split_k = 1;
+  tiles_of(&c, M, N, &tp, &tq);
+  const int tiles = tp * tq;
+  const int kt = kt_total(f, K);
+  int sms = 148;
+  DeviceInfo* d;
+  if (device_info(&d) == QG_OK) sms = d->sms;
+  while (c.split_k < 256 && tiles * c.split_k * 2 <= sms && kt / (c.split_k * 2) >= 2) c.split_k *= 2;
+  if (f == QG_BLOCK_FP8) {
+    const int act_rows = c.swap_ab ? c.tile_n : 128;
+    while ((kt + c.split_k - 1) / c.split_k > 64 ||
+           act_rows * ((kt + c.split_k - 1) / c.split_k) > qg::kMaxScaleStage)
+      c.split_k *= 2;
+    if (c.split_k > kt) return QG_ERR_UNSUPPORTED;
+  }
+  *out = c;
+  return QG_OK;
+}
+
+qg_status qgemm_device_error(void) {
+  DeviceInfo* d;
+  qg_status s = device_info(&d);
+  if (s != QG_OK) return s;
+  if (cudaDeviceSynchronize() != cudaSuccess) return QG_ERR_CUDA;
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, qg::g_qg_error, sizeof(v)) != cudaSuccess) return QG_ERR_CUDA;
+  if (v != 0 && cudaMemcpyToSymbol(qg::g_qg_error, &zero, sizeof(zero)) != cudaSuccess) return QG_ERR_CUDA;
+  return v ? QG_ERR_DEVICE_TIMEOUT : QG_OK;
+}
+
+}  // extern "C"

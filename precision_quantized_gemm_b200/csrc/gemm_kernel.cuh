@@ -1,0 +1,538 @@
+// gemm_kernel.cuh — the unified quantized GEMM kernel for sm_100a.
+//
+// One CTA computes an output tile D[128 x BN] over a slice of the K tiles:
+//   D[p, q] = sum_k P[p, k] * Q[q, k]
+// P is the 128-row MMA operand and Q the BN-row one, both K-contiguous.
+// Standard orientation: P = A_q (tokens), Q = W_q (channels).
+// Swap-AB ("Helion in the vLLM backend", second paragraph: A@B rewritten as
+// (B^T A^T)^T): P = W_q, Q = A_q, so the weight rows fill the 128-row MMA
+// slot and a handful of tokens fill N = 16 or 32.
+//
+// Warp roles (192 threads):
+//   warp 0      TMA producer: weights first (they do not depend on the
+//               preceding kernel), then griddepcontrol.wait, then activations;
+//               a `stages`-deep ring of 128-byte K tiles in shared memory.
+//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer.
+//   warps 2..5  epilogue: tcgen05.ld of the fp32/int32 accumulator, scales in
+//               fp32, bf16 store (or split-K partials and their reduction).
+// Block_FP8 promotes every 128-wide K group: the MMA writes the group's
+// partial sum into one of NACC TMEM buffers and the epilogue warps fold it
+// into fp32 registers with the group's activation and weight-block scales.
+// NVFP4 uses kind::mxf4nvf4 with the e4m3 block scales copied
+// smem -> TMEM by tcgen05.cp.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace qg {
+
+enum Fmt : int { kFP8 = 0, kINT8 = 1, kBLOCK = 2, kNVF4 = 3 };
+
+constexpr int kThreads = 192;
+constexpr int kKTileBytes = 128;     // bytes of K per pipeline stage (one 128B swizzle row)
+constexpr int kPTileBytes = 128 * kKTileBytes;
+constexpr int kSfAtomBytes = 512;    // one 128x4 atom of e4m3 block scales
+constexpr int kMaxScaleStage = 8192; // floats of Block_FP8 scales staged per CTA
+
+struct GemmParams {
+  int M, N, K;
+  int rows_p, rows_q;          // rows of the P / Q operands
+  int kt_total;                // 128-byte K tiles
+  int split_k;
+  int stages;
+  int groups;                  // Block_FP8: K / 128
+  const float* scale_a;        // activation scales (per token, or [M, groups])
+  const float* scale_w;        // weight scales (per channel, or [ceil(N/128), groups])
+  const uint8_t* sf_p;         // NVFP4 block scales of P / Q (128x4 layout)
+  const uint8_t* sf_q;
+  int sf_atoms_per_rb;         // NVFP4: 128x4 atoms per 128-row block (= ceil(K/256)*4)
+  const float* g_a;            // NVFP4 tensor scales
+  const float* g_w;
+  void* Y;
+  int ldy;
+  int out_kind;                // 0 = bf16, 1 = raw accumulators
+  void* partial;               // split-K partials [split][M][N] (4-byte elements)
+  unsigned int* counters;      // split-K per-tile arrival counters
+  int reduce_mode;             // 0 = in-kernel, 1 = second pass
+  unsigned int* err;           // device error word
+};
+
+template <int FMT, int BN>
+struct Cfg {
+  static constexpr bool kBlock = FMT == kBLOCK;
+  static constexpr bool kNvf4 = FMT == kNVF4;
+  static constexpr int kQTileBytes = BN * kKTileBytes;
+  static constexpr int kSfQAtoms = BN > 128 ? 2 : 1;               // 128-row SF blocks of Q
+  static constexpr int kSfPBytes = kNvf4 ? 4 * kSfAtomBytes : 0;   // 4 K-atoms per 128B tile
+  static constexpr int kSfQBytes = kNvf4 ? 4 * kSfAtomBytes * kSfQAtoms : 0;
+  static constexpr int kStageBytes = kPTileBytes + kQTileBytes + kSfPBytes + kSfQBytes;
+  static constexpr int kNAcc = kBlock ? (BN >= 128 ? 2 : 4) : 1;  // TMEM accumulators
+  static constexpr int kSfaCol = kNAcc * BN;                       // TMEM column of SF A
+  static constexpr int kSfbCol = kSfaCol + 16;                     // 4 steps x 4 words
+  static constexpr int kTmemUsed = kNvf4 ? kSfbCol + 16 * kSfQAtoms : kNAcc * BN;
+  static constexpr int kTmemCols = kTmemUsed <= 32    ? 32
+                                   : kTmemUsed <= 64  ? 64
+                                   : kTmemUsed <= 128 ? 128
+                                   : kTmemUsed <= 256 ? 256
+                                                      : 512;
+  static constexpr uint32_t kIdesc = kNvf4              ? idesc_nvf4(BN)
+                                     : (FMT == kINT8)   ? idesc_i8(BN)
+                                                        : idesc_f8f6f4_e4m3(BN);
+};
+
+// Shared-memory carve-up (offsets from a 1024-byte aligned base).
+struct SmemLayout {
+  uint32_t p, q, sfp, sfq, bars, misc, scales, total;
+};
+template <int FMT, int BN>
+__host__ __device__ inline SmemLayout smem_layout(int stages) {
+  using C = Cfg<FMT, BN>;
+  SmemLayout L;
+  L.p = 0;
+  L.q = L.p + stages * kPTileBytes;
+  L.sfp = L.q + stages * C::kQTileBytes;
+  L.sfq = L.sfp + stages * C::kSfPBytes;
+  L.bars = L.sfq + stages * C::kSfQBytes;
+  // full[stages], empty[stages], acc_full, tfull[4], tempty[4]
+  L.misc = L.bars + 8 * (2 * stages + 1 + 8);
+  L.scales = (L.misc + 16 + 15) & ~15u;
+  L.total = L.scales + (C::kBlock ? 4 * (kMaxScaleStage + 2 * 64) : 0);
+  return L;
+}
+template <int FMT, int BN>
+__host__ inline size_t smem_bytes(int stages) {
+  return smem_layout<FMT, BN>(stages).total + 1024;  // + alignment slack
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_u32_cg(const void* p) {
+  return __ldcg(reinterpret_cast<const unsigned int*>(p));
+}
+
+// Epilogue scale of one output element, before bf16 rounding.
+template <int FMT>
+__device__ __forceinline__ float finish_value(uint32_t acc_bits, float sa, float sw, float alpha) {
+  if constexpr (FMT == kINT8) {
+    return (__int2float_rn(static_cast<int>(acc_bits)) * sa) * sw;
+  } else if constexpr (FMT == kFP8) {
+    return (__uint_as_float(acc_bits) * sa) * sw;
+  } else if constexpr (FMT == kNVF4) {
+    return __uint_as_float(acc_bits) * alpha;
+  } else {
+    return __uint_as_float(acc_bits);   // Block_FP8: already promoted
+  }
+}
+
+template <int FMT, bool SWAP, int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+    qgemm_kernel(const __grid_constant__ CUtensorMap tmap_p,
+                 const __grid_constant__ CUtensorMap tmap_q, const GemmParams prm) {
+  using C = Cfg<FMT, BN>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const SmemLayout L = smem_layout<FMT, BN>(prm.stages);
+  const int S = prm.stages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
+  uint64_t* empty = full + S;
+  uint64_t* acc_full = empty + S;
+  uint64_t* tfull = acc_full + 1;
+  uint64_t* tempty = tfull + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.misc);
+  volatile int* flag_last = reinterpret_cast<volatile int*>(smem + L.misc + 4);
+  volatile int* flag_abort = reinterpret_cast<volatile int*>(smem + L.misc + 8);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int p0 = blockIdx.x * 128;
+  const int q0 = blockIdx.y * BN;
+  const int kz = blockIdx.z;
+  const int kt_begin = (int)(((long long)kz * prm.kt_total) / prm.split_k);
+  const int kt_end = (int)(((long long)(kz + 1) * prm.kt_total) / prm.split_k);
+  const int nkt = kt_end - kt_begin;
+
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tmap_p);
+    prefetch_tmap(&tmap_q);
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(acc_full, 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 4);
+    }
+    *flag_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  // Let the next kernel of the stream start its prologue; it waits on our
+  // completion before touching what we write.
+  if (threadIdx.x == 0) griddep_launch_dependents();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && nkt > 0) {
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_a = policy_evict_last();
+      const CUtensorMap* map_w = SWAP ? &tmap_p : &tmap_q;
+      const CUtensorMap* map_a = SWAP ? &tmap_q : &tmap_p;
+      const uint32_t off_w = SWAP ? L.p : L.q;
+      const uint32_t off_a = SWAP ? L.q : L.p;
+      const uint32_t bytes_w = SWAP ? kPTileBytes : C::kQTileBytes;
+      const uint32_t bytes_a = SWAP ? C::kQTileBytes : kPTileBytes;
+      const int row_w = SWAP ? p0 : q0;
+      const int row_a = SWAP ? q0 : p0;
+      // NVFP4 scale atoms: P rows [p0, p0+128) are one 128-row block; Q has
+      // one or two blocks (the second only if it holds any row).
+      const int sfq_atoms = (C::kSfQAtoms == 2 && q0 + 128 < prm.rows_q) ? 2 : 1;
+      const uint32_t stage_tx = kPTileBytes + C::kQTileBytes +
+                                (C::kNvf4 ? (uint32_t)(4 * kSfAtomBytes * (1 + sfq_atoms)) : 0u);
+      auto load_w = [&](int i) {
+        const int st = i % S;
+        const int kt = kt_begin + i;
+        tma_load_2d(smem + off_w + st * bytes_w, map_w, &full[st], kt * kKTileBytes, row_w, pol_w);
+        if constexpr (C::kNvf4) {
+          const uint8_t* sfw = SWAP ? prm.sf_p : prm.sf_q;
+          const int rb = row_w / 128;
+          if (SWAP) {
+            bulk_load(smem + L.sfp + st * C::kSfPBytes,
+                      sfw + ((size_t)rb * prm.sf_atoms_per_rb + kt * 4) * kSfAtomBytes,
+                      4 * kSfAtomBytes, &full[st]);
+          } else {
+            for (int a = 0; a < sfq_atoms; ++a)
+              bulk_load(smem + L.sfq + st * C::kSfQBytes + a * 4 * kSfAtomBytes,
+                        sfw + ((size_t)(rb + a) * prm.sf_atoms_per_rb + kt * 4) * kSfAtomBytes,
+                        4 * kSfAtomBytes, &full[st]);
+          }
+        }
+      };
+      auto load_a = [&](int i) {
+        const int st = i % S;
+        const int kt = kt_begin + i;
+        tma_load_2d(smem + off_a + st * bytes_a, map_a, &full[st], kt * kKTileBytes, row_a, pol_a);
+        if constexpr (C::kNvf4) {
+          const uint8_t* sfa = SWAP ? prm.sf_q : prm.sf_p;
+          const int rb = row_a / 128;
+          if (SWAP) {
+            for (int a = 0; a < sfq_atoms; ++a)
+              bulk_load(smem + L.sfq + st * C::kSfQBytes + a * 4 * kSfAtomBytes,
+                        sfa + ((size_t)(rb + a) * prm.sf_atoms_per_rb + kt * 4) * kSfAtomBytes,
+                        4 * kSfAtomBytes, &full[st]);
+          } else {
+            bulk_load(smem + L.sfp + st * C::kSfPBytes,
+                      sfa + ((size_t)rb * prm.sf_atoms_per_rb + kt * 4) * kSfAtomBytes,
+                      4 * kSfAtomBytes, &full[st]);
+          }
+        }
+      };
+      const int pre = nkt < S ? nkt : S;
+      for (int i = 0; i < pre; ++i) {
+        mbar_arrive_expect_tx(&full[i], stage_tx);
+        load_w(i);
+      }
+      griddep_wait();
+      for (int i = 0; i < pre; ++i) load_a(i);
+      bool ok = true;
+      int issued = pre;
+      for (int i = pre; i < nkt; ++i) {
+        const int st = i % S;
+        if (!mbar_wait(&empty[st], ((i / S) - 1) & 1, prm.err)) { ok = false; break; }
+        mbar_arrive_expect_tx(&full[st], stage_tx);
+        load_w(i);
+        load_a(i);
+        issued = i + 1;
+      }
+      if (!ok) {
+        *flag_abort = 1;
+        // Drain: wait (bounded) until every issued copy has landed.
+        for (int i = (issued > S ? issued - S : 0); i < issued; ++i)
+          mbar_wait(&full[i % S], (i / S) & 1, prm.err);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0 && nkt > 0) {
+      const uint32_t sp = smem_u32(smem + L.p);
+      const uint32_t sq = smem_u32(smem + L.q);
+      const uint32_t ssfp = smem_u32(smem + L.sfp);
+      const uint32_t ssfq = smem_u32(smem + L.sfq);
+      const uint32_t sfa_t = tmem_base + C::kSfaCol;
+      const uint32_t sfb_t = tmem_base + C::kSfbCol;
+      // word offset of this CTA's first Q row inside its 128-row SF atom
+      const uint32_t sfb_word = (uint32_t)((q0 % 128) / 32);
+      for (int i = 0; i < nkt; ++i) {
+        const int st = i % S;
+        if (*flag_abort || !mbar_wait(&full[st], (i / S) & 1, prm.err)) { *flag_abort = 1; break; }
+        uint32_t d_t = tmem_base;
+        if constexpr (C::kBlock) {
+          const int b = i % C::kNAcc;
+          const int r = i / C::kNAcc;
+          if (r > 0 && !mbar_wait(&tempty[b], (r - 1) & 1, prm.err)) { *flag_abort = 1; break; }
+          d_t = tmem_base + b * BN;
+        }
+        tc_fence_after();
+        if constexpr (C::kNvf4) {
+          for (int s = 0; s < 4; ++s) {
+            tmem_cp_32x128b_x4(sfa_t + 4 * s,
+                               sdesc_plain_32x16(ssfp + st * C::kSfPBytes + s * kSfAtomBytes));
+            for (int a = 0; a < C::kSfQAtoms; ++a)
+              tmem_cp_32x128b_x4(sfb_t + 4 * C::kSfQAtoms * s + 4 * a,
+                                 sdesc_plain_32x16(ssfq + st * C::kSfQBytes + a * 4 * kSfAtomBytes +
+                                                   s * kSfAtomBytes));
+          }
+        }
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+          const uint64_t da = sdesc_sw128(sp + st * kPTileBytes + 32 * s);
+          const uint64_t db = sdesc_sw128(sq + st * C::kQTileBytes + 32 * s);
+          const uint32_t accum = C::kBlock ? (s > 0) : (i > 0 || s > 0);
+          if constexpr (C::kNvf4)
+            mma_nvf4(d_t, da, db, C::kIdesc, sfa_t + 4 * s,
+                     sfb_t + 4 * C::kSfQAtoms * s + sfb_word, accum);
+          else if constexpr (FMT == kINT8)
+            mma_i8(d_t, da, db, C::kIdesc, accum);
+          else
+            mma_f8f6f4(d_t, da, db, C::kIdesc, accum);
+        }
+        mma_commit(&empty[st]);
+        if constexpr (C::kBlock) mma_commit(&tfull[i % C::kNAcc]);
+      }
+      if constexpr (!C::kBlock) mma_commit(acc_full);
+    }
+  } else {
+    // --------------------------------------------------------------- epilogue
+    const int quarter = warp & 3;              // TMEM lanes this warp may access
+    const int row = quarter * 32 + lane;       // row of P in the tile
+    const int etid = threadIdx.x - 64;         // 0..127
+    const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
+    griddep_wait();                            // scales/partials of earlier kernels
+
+    volatile int* flag_epi = reinterpret_cast<volatile int*>(smem + L.misc + 12);
+    bool ok = true;                            // warp-uniform
+    float acc_f[BN];                           // Block_FP8 promoted accumulator
+    int wblocks = 1;
+    if constexpr (C::kBlock) {
+      float* sa_s = reinterpret_cast<float*>(smem + L.scales);          // act scales
+      float* sw_s = sa_s + kMaxScaleStage;                              // weight scales
+      const int G = prm.groups;
+      const int g0 = kt_begin;
+      // Stage this CTA's scales: activations per (row, group), weights per
+      // (128-row block, group).
+      const int act_rows = SWAP ? BN : 128;
+      const int act_base = SWAP ? q0 : p0;
+      for (int idx = etid; idx < act_rows * nkt; idx += 128) {
+        const int r = idx / nkt, gl = idx % nkt;
+        const int m = act_base + r;
+        sa_s[idx] = (m < prm.M) ? __ldg(prm.scale_a + (size_t)m * G + g0 + gl) : 0.f;
+      }
+      wblocks = SWAP ? 1 : (BN > 128 ? 2 : 1);
+      const int wrow0 = (SWAP ? p0 : q0) / 128;
+      const int nblk = (prm.N + 127) / 128;
+      for (int idx = etid; idx < wblocks * nkt; idx += 128) {
+        const int gl = idx / wblocks, jb = idx % wblocks;
+        const int b = wrow0 + jb;
+        sw_s[idx] = (b < nblk) ? __ldg(prm.scale_w + (size_t)b * G + g0 + gl) : 0.f;
+      }
+      named_bar_sync(1, 128);
+#pragma unroll
+      for (int c = 0; c < BN; ++c) acc_f[c] = 0.f;
+      for (int i = 0; i < nkt; ++i) {
+        const int b = i % C::kNAcc;
+        ok = __all_sync(0xffffffffu, mbar_wait(&tfull[b], (i / C::kNAcc) & 1, prm.err));
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld16(lane_addr + b * BN + c0, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int c = c0 + j;
+            float sa, sw;
+            if (SWAP) {
+              sa = sa_s[c * nkt + i];
+              sw = sw_s[i];
+            } else {
+              sa = sa_s[row * nkt + i];
+              sw = sw_s[i * wblocks + (BN > 128 ? c / 128 : 0)];
+            }
+            acc_f[c] += (__uint_as_float(v[j]) * sa) * sw;
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[b]);
+      }
+    } else {
+      if (nkt > 0) ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, prm.err));
+      tc_fence_after();
+    }
+    if (etid == 0) *flag_epi = 0;
+    named_bar_sync(1, 128);
+    if (!ok) *flag_epi = 1;
+    named_bar_sync(1, 128);
+    const bool epi_ok = (*flag_epi == 0);      // uniform over the 128 epilogue threads
+
+    // ---- write out: direct epilogue or split-K partials
+    float alpha = 1.f;
+    if constexpr (C::kNvf4) alpha = __ldg(prm.g_a) * __ldg(prm.g_w);
+    const bool split = prm.split_k > 1;
+    const int prow = p0 + row;                 // global row of P
+    const bool prow_ok = prow < prm.rows_p;
+    float s_row = 1.f;                         // scale of this thread's P row
+    if constexpr (FMT == kFP8 || FMT == kINT8) {
+      if (prow_ok) s_row = __ldg((SWAP ? prm.scale_w : prm.scale_a) + prow);
+    }
+    const float* scale_col = SWAP ? prm.scale_a : prm.scale_w;
+    const size_t MN = (size_t)prm.M * prm.N;
+    uint32_t* part = reinterpret_cast<uint32_t*>(prm.partial);
+
+    auto out_index = [&](int c, int& m, int& n) {
+      if (SWAP) { m = q0 + c; n = prow; } else { m = prow; n = q0 + c; }
+    };
+    auto store_final = [&](int m, int n, uint32_t acc_bits) {
+      if (prm.out_kind == 1) {
+        reinterpret_cast<uint32_t*>(prm.Y)[(size_t)m * prm.ldy + n] = acc_bits;
+      } else {
+        float sa = 1.f, sw = 1.f;
+        if constexpr (FMT == kFP8 || FMT == kINT8) {
+          const float sc = __ldg(scale_col + (SWAP ? m : n));
+          sa = SWAP ? sc : s_row;
+          sw = SWAP ? s_row : sc;
+        }
+        const float y = finish_value<FMT>(acc_bits, sa, sw, alpha);
+        reinterpret_cast<__nv_bfloat16*>(prm.Y)[(size_t)m * prm.ldy + n] = __float2bfloat16_rn(y);
+      }
+    };
+
+    if (epi_ok) {
+#pragma unroll
+      for (int c0 = 0; c0 < BN; c0 += 16) {
+        uint32_t v[16];
+        if constexpr (C::kBlock) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(acc_f[c0 + j]);
+        } else {
+          if (nkt > 0) {
+            tmem_ld16(lane_addr + c0, v);
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = 0u;
+          }
+        }
+        if (prow_ok) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            int m, n;
+            out_index(c0 + j, m, n);
+            if (m < prm.M && n < prm.N) {
+              if (split)
+                part[(size_t)kz * MN + (size_t)m * prm.N + n] = v[j];
+              else
+                store_final(m, n, v[j]);
+            }
+          }
+        }
+      }
+      if (split && prm.reduce_mode == 0) {
+        // Last-arriving CTA of this output tile sums the partials in split
+        // order (deterministic) and applies the epilogue.
+        __threadfence();
+        named_bar_sync(1, 128);
+        const unsigned tile = blockIdx.y * gridDim.x + blockIdx.x;
+        if (etid == 0) {
+          const unsigned prev = atomicAdd(&prm.counters[tile], 1u);
+          *flag_last = (prev == (unsigned)(prm.split_k - 1));
+        }
+        named_bar_sync(1, 128);
+        if (*flag_last) {
+          __threadfence();
+          if (prow_ok) {
+            for (int c = 0; c < BN; ++c) {
+              int m, n;
+              out_index(c, m, n);
+              if (m >= prm.M || n >= prm.N) continue;
+              const size_t o = (size_t)m * prm.N + n;
+              uint32_t sum_bits;
+              if constexpr (FMT == kINT8) {
+                int s = 0;
+                for (int z = 0; z < prm.split_k; ++z) s += (int)ld_u32_cg(part + z * MN + o);
+                sum_bits = (uint32_t)s;
+              } else {
+                float s = 0.f;
+                for (int z = 0; z < prm.split_k; ++z) s += __uint_as_float(ld_u32_cg(part + z * MN + o));
+                sum_bits = __float_as_uint(s);
+              }
+              store_final(m, n, sum_bits);
+            }
+          }
+          if (etid == 0) prm.counters[tile] = 0u;
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// Second-pass split-K reduction: y[m, n] = epilogue(sum_z partial[z, m, n]),
+// summed in split order.
+template <int FMT>
+__global__ void splitk_reduce_kernel(const GemmParams prm) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const size_t MN = (size_t)prm.M * prm.N;
+  const uint32_t* part = reinterpret_cast<const uint32_t*>(prm.partial);
+  float alpha = 1.f;
+  if constexpr (FMT == kNVF4) alpha = __ldg(prm.g_a) * __ldg(prm.g_w);
+  for (size_t o = blockIdx.x * (size_t)blockDim.x + threadIdx.x; o < MN;
+       o += (size_t)gridDim.x * blockDim.x) {
+    const int m = (int)(o / prm.N), n = (int)(o % prm.N);
+    uint32_t bits;
+    if constexpr (FMT == kINT8) {
+      int s = 0;
+      for (int z = 0; z < prm.split_k; ++z) s += (int)__ldcg(part + z * MN + o);
+      bits = (uint32_t)s;
+    } else {
+      float s = 0.f;
+      for (int z = 0; z < prm.split_k; ++z) s += __uint_as_float(__ldcg(part + z * MN + o));
+      bits = __float_as_uint(s);
+    }
+    if (prm.out_kind == 1) {
+      reinterpret_cast<uint32_t*>(prm.Y)[(size_t)m * prm.ldy + n] = bits;
+    } else {
+      float sa = 1.f, sw = 1.f;
+      if constexpr (FMT == kFP8 || FMT == kINT8) {
+        sa = __ldg(prm.scale_a + m);
+        sw = __ldg(prm.scale_w + n);
+      }
+      reinterpret_cast<__nv_bfloat16*>(prm.Y)[(size_t)m * prm.ldy + n] =
+          __float2bfloat16_rn(finish_value<FMT>(bits, sa, sw, alpha));
+    }
+  }
+}
+
+}  // namespace qg

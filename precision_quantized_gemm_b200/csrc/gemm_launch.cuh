@@ -1,0 +1,91 @@
+// gemm_launch.cuh — host-side launch of one format's GEMM instantiations.
+// Included by exactly one translation unit per format with QG_FMT and
+// QG_LAUNCH_NAME defined.
+#pragma once
+#include "gemm_kernel.cuh"
+#include "internal.h"
+
+namespace qg {
+namespace {
+
+template <int FMT, bool SWAP, int BN>
+cudaError_t launch_one(const CUtensorMap& tp, const CUtensorMap& tq, const GemmParams& prm,
+                       dim3 grid, cudaStream_t st, bool pdl) {
+  auto kern = qgemm_kernel<FMT, SWAP, BN>;
+  const size_t smem = smem_bytes<FMT, BN>(prm.stages);
+  static int configured_bytes = 0;
+  if ((int)smem > configured_bytes) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured_bytes = (int)smem;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, tp, tq, prm);
+}
+
+template <int FMT, bool SWAP>
+cudaError_t launch_bn(int bn, const CUtensorMap& tp, const CUtensorMap& tq, const GemmParams& prm,
+                      dim3 grid, cudaStream_t st, bool pdl) {
+  switch (bn) {
+    case 16: return launch_one<FMT, SWAP, 16>(tp, tq, prm, grid, st, pdl);
+    case 32: return launch_one<FMT, SWAP, 32>(tp, tq, prm, grid, st, pdl);
+    case 64: return launch_one<FMT, SWAP, 64>(tp, tq, prm, grid, st, pdl);
+    case 128: return launch_one<FMT, SWAP, 128>(tp, tq, prm, grid, st, pdl);
+    case 256:
+      if constexpr (FMT != kBLOCK) return launch_one<FMT, SWAP, 256>(tp, tq, prm, grid, st, pdl);
+      return cudaErrorInvalidValue;
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int FMT>
+size_t smem_for(int bn, int stages) {
+  switch (bn) {
+    case 16: return smem_bytes<FMT, 16>(stages);
+    case 32: return smem_bytes<FMT, 32>(stages);
+    case 64: return smem_bytes<FMT, 64>(stages);
+    case 128: return smem_bytes<FMT, 128>(stages);
+    case 256: return FMT == kBLOCK ? (size_t)1 << 30 : smem_bytes<FMT, 256>(stages);
+    default: return (size_t)1 << 30;
+  }
+}
+
+}  // namespace
+
+cudaError_t QG_LAUNCH_NAME(bool swap, int tile_n, const CUtensorMap& tp, const CUtensorMap& tq,
+                           const GemmParams& prm, dim3 grid, cudaStream_t st, bool pdl) {
+  return swap ? launch_bn<QG_FMT, true>(tile_n, tp, tq, prm, grid, st, pdl)
+              : launch_bn<QG_FMT, false>(tile_n, tp, tq, prm, grid, st, pdl);
+}
+
+#define QG_CAT2(a, b) a##b
+#define QG_CAT(a, b) QG_CAT2(a, b)
+
+size_t QG_CAT(QG_LAUNCH_NAME, _smem)(int tile_n, int stages) { return smem_for<QG_FMT>(tile_n, stages); }
+
+cudaError_t QG_CAT(QG_LAUNCH_NAME, _reduce)(const GemmParams& prm, cudaStream_t st, bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  const long long mn = (long long)prm.M * prm.N;
+  long long blocks = (mn + 255) / 256;
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  cfg.gridDim = dim3((unsigned)(blocks < 1 ? 1 : blocks));
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, splitk_reduce_kernel<QG_FMT>, prm);
+}
+
+}  // namespace qg

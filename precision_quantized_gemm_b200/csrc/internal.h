@@ -1,0 +1,39 @@
+// internal.h — declarations shared by the library's translation units.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace qg {
+
+struct GemmParams;
+
+constexpr int kNvfp4AmaxMaxCtas = 296;   // partial-amax slots in the NVFP4 quant workspace
+
+cudaError_t launch_quant_rows(bool int8, const void* X, int R, int K, int ldx, void* q,
+                              float* scale, cudaStream_t st, bool pdl);
+cudaError_t launch_quant_act_groups(const void* X, int M, int K, int ldx, void* q, float* scale,
+                                    cudaStream_t st, bool pdl);
+cudaError_t launch_quant_weight_blocks(const void* W, int N, int K, void* q, float* scale,
+                                       cudaStream_t st, bool pdl);
+int nvfp4_amax_ctas(int R, int K);
+cudaError_t launch_quant_nvfp4(const void* X, int R, int K, int ldx, const float* static_amax,
+                               void* q, void* sf, float* gscale, float* partial,
+                               cudaStream_t st, bool pdl);
+
+// GEMM launchers, one per format (each in its own translation unit).
+// Returns cudaErrorInvalidValue for a (swap, tile_n) pair not instantiated.
+#define QG_DECLARE_GEMM_LAUNCH(NAME)                                                      \
+  cudaError_t NAME(bool swap, int tile_n, const CUtensorMap& tp, const CUtensorMap& tq,    \
+                   const GemmParams& prm, dim3 grid, cudaStream_t st, bool pdl);           \
+  size_t NAME##_smem(int tile_n, int stages);                                              \
+  cudaError_t NAME##_reduce(const GemmParams& prm, cudaStream_t st, bool pdl);
+QG_DECLARE_GEMM_LAUNCH(launch_gemm_fp8)
+QG_DECLARE_GEMM_LAUNCH(launch_gemm_int8)
+QG_DECLARE_GEMM_LAUNCH(launch_gemm_block)
+QG_DECLARE_GEMM_LAUNCH(launch_gemm_nvf4)
+#undef QG_DECLARE_GEMM_LAUNCH
+
+}  // namespace qg

@@ -1,0 +1,188 @@
+"""C-ABI boundary tests that need no GPU: the library loads, exports every
+symbol the header declares, sizes its buffers, rejects bad arguments on the
+host before any launch, and round-trips its per-shape table."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import precision_quantized_gemm_b200 as qg
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qgemm.h")
+
+FAKE = 0x100000  # an aligned, never-dereferenced stand-in for a device pointer
+
+
+def _declared():
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"\b(qgemm_[a-z_0-9]+)\s*\(", txt)))
+
+
+def test_every_declared_symbol_is_exported():
+    L = qg.lib()
+    names = _declared()
+    assert len(names) >= 18
+    for n in names:
+        assert hasattr(L, n), n
+    assert sorted(qg.EXPORTS) == names
+
+
+def test_abi_version_and_status_strings():
+    assert qg.lib().qgemm_abi_version() == 1
+    for s in range(9):
+        assert qg.status_string(s)
+    assert qg.status_string(0) == "ok"
+
+
+@pytest.mark.parametrize("fmt,is_w,rows,K,q,s", [
+    (qg.QG_FP8_DYNAMIC, 0, 16, 2048, 16 * 2048, 16 * 4),
+    (qg.QG_W8A8_INT8, 1, 4096, 4096, 4096 * 4096, 4096 * 4),
+    (qg.QG_BLOCK_FP8, 0, 4, 7168, 4 * 7168, 4 * 56 * 4),
+    (qg.QG_BLOCK_FP8, 1, 4608, 7168, 4608 * 7168, 36 * 56 * 4),
+    (qg.QG_BLOCK_FP8, 1, 200, 256, 200 * 256, 2 * 2 * 4),
+    (qg.QG_NVFP4, 0, 8, 1024, 8 * 512, 128 * 64),
+    (qg.QG_NVFP4, 1, 1280, 8192, 1280 * 4096, 1280 * 512),
+    (qg.QG_NVFP4, 1, 130, 96, 130 * 48, 256 * 16),
+])
+def test_operand_bytes(fmt, is_w, rows, K, q, s):
+    assert qg.qgemm_operand_bytes(fmt, is_w, rows, K) == (q, s)
+
+
+@pytest.mark.parametrize("fmt,K", [(qg.QG_FP8_DYNAMIC, 24), (qg.QG_BLOCK_FP8, 192),
+                                   (qg.QG_NVFP4, 48), (7, 128)])
+def test_operand_bytes_rejects_bad_k_or_format(fmt, K):
+    with pytest.raises(qg.QGemmError):
+        qg.qgemm_operand_bytes(fmt, 0, 4, K)
+
+
+def test_workspace_sizes():
+    c = qg.make_config(split_k=1)
+    assert qg.qgemm_workspace_size(qg.QG_FP8_DYNAMIC, 16, 2048, 2048, c) == 0
+    c = qg.make_config(split_k=8, swap_ab=1, tile_n=16)
+    ws = qg.qgemm_workspace_size(qg.QG_FP8_DYNAMIC, 16, 2048, 2048, c)
+    assert ws == 8 * 16 * 2048 * 4 + 256          # partials + 16 tile counters padded to 256
+    assert qg.qgemm_quant_workspace_size(qg.QG_NVFP4, 8, 1024) > 0
+    assert qg.qgemm_quant_workspace_size(qg.QG_W8A8_INT8, 8, 1024) == 0
+
+
+def test_default_config_follows_the_swap_rule_and_fills_sms():
+    c = qg.qgemm_default_config(qg.QG_W8A8_INT8, 8, 4096, 4096)
+    assert c.swap_ab == 1 and c.tile_n == 16
+    assert c.split_k >= 2 and (c.split_k & (c.split_k - 1)) == 0
+    assert 32 * c.split_k <= 148
+    c = qg.qgemm_default_config(qg.QG_BLOCK_FP8, 4096, 5120, 5120)
+    assert c.swap_ab == 0 and c.tile_n == 128
+    c = qg.qgemm_default_config(qg.QG_FP8_DYNAMIC, 32, 2048, 2048)
+    assert c.swap_ab == 1 and c.tile_n == 32
+
+
+def _op(rows, K, q=FAKE, s=FAKE, g=FAKE):
+    return qg.qg_operand(q, s, g, rows, K)
+
+
+def _run(fmt=qg.QG_FP8_DYNAMIC, M=16, N=256, K=512, cfg=None, A=None, W=None, ws=None, wsb=0,
+         Y=FAKE, ldy=None, out_kind=0):
+    cfg = cfg or qg.make_config(split_k=1, swap_ab=1, tile_n=16, stages=4)
+    A = A or _op(M, K)
+    W = W or _op(N, K)
+    return qg.qgemm_run(fmt, A, W, M, N, K, cfg, ws, wsb, Y, ldy if ldy is not None else N, out_kind, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(M=0), qg.QG_ERR_INVALID_ARG),                         # zero dimension
+    (dict(N=0), qg.QG_ERR_INVALID_ARG),
+    (dict(K=0), qg.QG_ERR_INVALID_ARG),
+    (dict(K=520), qg.QG_ERR_INVALID_ARG),                       # K % 16
+    (dict(fmt=qg.QG_BLOCK_FP8, K=384 + 64), qg.QG_ERR_INVALID_ARG),
+    (dict(Y=None), qg.QG_ERR_INVALID_ARG),
+    (dict(Y=FAKE + 8), qg.QG_ERR_INVALID_ARG),                  # misaligned output
+    (dict(ldy=100), qg.QG_ERR_INVALID_ARG),                     # ldy < N
+    (dict(out_kind=5), qg.QG_ERR_INVALID_ARG),
+    (dict(A=_op(16, 512, q=FAKE + 4)), qg.QG_ERR_INVALID_ARG),  # misaligned codes
+    (dict(A=_op(8, 512)), qg.QG_ERR_INVALID_ARG),               # rows != M
+    (dict(W=_op(256, 256)), qg.QG_ERR_INVALID_ARG),             # K mismatch
+    (dict(fmt=qg.QG_NVFP4, A=_op(16, 512, g=0)), qg.QG_ERR_INVALID_ARG),  # no tensor scale
+    (dict(fmt=9), qg.QG_ERR_INVALID_ARG),
+    (dict(cfg=qg.make_config(split_k=3)), qg.QG_ERR_UNSUPPORTED),      # not a power of two
+    (dict(cfg=qg.make_config(split_k=512)), qg.QG_ERR_UNSUPPORTED),    # above 256
+    (dict(cfg=qg.make_config(split_k=8)), qg.QG_ERR_UNSUPPORTED),      # > 4 K tiles of 128 B
+    (dict(cfg=qg.make_config(tile_n=48)), qg.QG_ERR_UNSUPPORTED),
+    (dict(cfg=qg.make_config(stages=1)), qg.QG_ERR_UNSUPPORTED),
+    (dict(cfg=qg.make_config(tile_n=256, stages=12)), qg.QG_ERR_UNSUPPORTED),  # smem
+    (dict(fmt=qg.QG_BLOCK_FP8, cfg=qg.make_config(tile_n=256)), qg.QG_ERR_UNSUPPORTED),
+    (dict(cfg=qg.make_config(swap_ab=2)), qg.QG_ERR_INVALID_ARG),
+    (dict(cfg=qg.make_config(split_k=2, stages=4), ws=None), qg.QG_ERR_WORKSPACE),
+    (dict(cfg=qg.make_config(split_k=2, stages=4), ws=FAKE, wsb=64), qg.QG_ERR_WORKSPACE),
+])
+def test_run_rejects_bad_arguments_before_any_launch(kw, status):
+    assert _run(**kw) == status
+
+
+def test_run_reserved_fields_must_be_zero():
+    c = qg.make_config()
+    c.reserved[1] = 7
+    assert _run(cfg=c) == qg.QG_ERR_INVALID_ARG
+
+
+def test_quantize_rejects_bad_arguments():
+    out = _op(4, 512)
+    assert qg.qgemm_quantize_act(qg.QG_FP8_DYNAMIC, FAKE, 4, 512, 100, None, out, None, 0, None) == qg.QG_ERR_INVALID_ARG
+    assert qg.qgemm_quantize_act(qg.QG_FP8_DYNAMIC, FAKE + 2, 4, 512, 512, None, out, None, 0, None) == qg.QG_ERR_INVALID_ARG
+    assert qg.qgemm_quantize_act(qg.QG_FP8_DYNAMIC, FAKE, 5, 512, 512, None, out, None, 0, None) == qg.QG_ERR_INVALID_ARG
+    assert qg.qgemm_quantize_act(qg.QG_NVFP4, FAKE, 4, 512, 512, None, out, None, 0, None) == qg.QG_ERR_WORKSPACE
+    assert qg.qgemm_quantize_weight(qg.QG_W8A8_INT8, None, 4, 512, out, None, 0, None) == qg.QG_ERR_INVALID_ARG
+
+
+def test_valid_arguments_reach_the_device_check():
+    # Everything is valid on the host: without a GPU the call stops at the
+    # device check (with one, this test does not run: fake pointers).
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("needs a machine without a GPU")
+    assert _run() in (qg.QG_ERR_NO_DEVICE, qg.QG_ERR_UNSUPPORTED)
+
+
+def test_table_roundtrip_and_dispatch(tmp_path):
+    t = qg.Table()
+    c8 = qg.make_config(split_k=4, swap_ab=1, tile_n=16, stages=8)
+    c32 = qg.make_config(split_k=2, swap_ab=1, tile_n=32, stages=6, reduce_mode=1)
+    t.put(qg.QG_W8A8_INT8, 8, 4096, 4096, c8, 3.5)
+    t.put(qg.QG_W8A8_INT8, 32, 4096, 4096, c32, 4.25)
+    assert len(t) == 2
+    p = str(tmp_path / "table.txt")
+    t.save(p)
+    t2 = qg.Table(p)
+    assert len(t2) == 2
+    c, hit = t2.dispatch(qg.QG_W8A8_INT8, 8, 4096, 4096)
+    assert hit == 1 and c.as_dict() == c8.as_dict()
+    c, hit = t2.dispatch(qg.QG_W8A8_INT8, 20, 4096, 4096)         # rounds up to M=32
+    assert hit == 2 and c.as_dict() == c32.as_dict()
+    c, hit = t2.dispatch(qg.QG_W8A8_INT8, 1, 4096, 4096)          # rounds up to M=8
+    assert hit == 2 and c.as_dict() == c8.as_dict()
+    c, hit = t2.dispatch(qg.QG_W8A8_INT8, 64, 4096, 4096)         # beyond the table: default
+    assert hit == 0 and c.as_dict() == qg.qgemm_default_config(qg.QG_W8A8_INT8, 64, 4096, 4096).as_dict()
+    c, hit = t2.dispatch(qg.QG_FP8_DYNAMIC, 8, 4096, 4096)        # other format: default
+    assert hit == 0
+
+
+@pytest.mark.parametrize("content", [
+    "",
+    "qgemm-table 2\ndevice x sms 148\n",
+    "qgemm-table 1\ndevice x sms 148\n1 8 4096 4096 4 1 16 8 0\n",          # missing field
+    "qgemm-table 1\ndevice x sms 148\n1 8 4096 4096 4 3 16 8 0 1.0\n",      # bad swap
+    "not a table\n",
+])
+def test_table_load_rejects_corrupt_files(tmp_path, content):
+    p = tmp_path / "bad.txt"
+    p.write_text(content)
+    with pytest.raises(qg.QGemmError) as e:
+        qg.Table(str(p))
+    assert e.value.status == qg.QG_ERR_TABLE_IO
+
+
+def test_table_load_missing_file():
+    with pytest.raises(qg.QGemmError) as e:
+        qg.Table("/nonexistent/qgemm_table.txt")
+    assert e.value.status == qg.QG_ERR_TABLE_IO
