@@ -1,0 +1,422 @@
+"""Benchmark of the quantized linear-layer GEMM hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pass of the whole decode hot path over one batch: for each
+token count M of the W8A8_INT8 decode workload (M in {1, 8, 32}, N = K = 4096,
+per-token int8 activations, per-channel int8 weights, bf16 out) the dynamic
+activation quantiser and the tcgen05 GEMM run as one CUDA-graph replay with
+the configuration the per-shape table dispatches (or the built-in default).
+Weights are quantised once at set-up; the step rotates over enough weight
+copies (more than twice the L2) that every GEMM streams its weights from HBM.
+
+Printed (rank 0, one JSON line): the metric of the workload as whole-job
+algorithmic HBM throughput (GB/s) of the step, per-shape GEMM microseconds and
+fraction of the HBM roofline, the dominant kernel's roofline object, the CPU
+oracle's throughput on a bounded sample, the end-to-end number through the
+public API with host buffers, clocks sampled during the timed region and the
+count of library kernels launched while timing.
+
+``--impl reference`` times the CPU oracle on the same workload (the only
+"reference" that exists: the pages ship no code).  Multi-GPU (torchrun): every
+rank runs the same replica workload, no collective on the data path.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "µs/shape and geomean % roofline (HBM GB/s or TC TFLOP/s), quantized GEMM M≤32"
+WORKLOAD = ("W8A8_INT8 decode linear layer: A bf16 ~N(0,1) [M,4096] per-token int8 (amax/127), "
+            "W ~N(0,0.02) [4096,4096] per-channel int8, int32 accumulate, fp32 scale epilogue, bf16 out; "
+            "M in {1,8,32}; seed 0 (A) / 1 (W)")
+FMT_INT8 = 1
+MS = (1, 8, 32)
+N = K = 4096
+TABLE = os.path.join(ROOT, "precision_quantized_gemm_b200", "tables", "b200.qgt")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--table", default=TABLE)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------- bytes ---
+def gemm_bytes(M):
+    """Algorithmic bytes of one INT8 GEMM call: W_q + W scales + A_q + A scales + Y (bf16)."""
+    return N * K + 4 * N + M * K + 4 * M + 2 * M * N
+
+
+def quant_bytes(M):
+    """Algorithmic bytes of one activation quantisation: A (bf16) + A_q + scales."""
+    return 2 * M * K + M * K + 4 * M
+
+
+def step_bytes():
+    return sum(gemm_bytes(m) + quant_bytes(m) for m in MS)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------- clocks ---
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) >= 9:
+                rows.append(f)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------ helpers ---
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        backend = "nccl"
+        try:
+            import torch
+            if not torch.cuda.is_available():
+                backend = "gloo"
+        except ImportError:
+            backend = "gloo"
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world, device):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_baseline(sample_steps=6):
+    """The oracle (numpy, as it stands) on a bounded sample of the workload:
+    ``sample_steps`` steps of quantise-3-activations + exact int64 GEMMs +
+    bf16 epilogue; the weights are quantised once outside the timing."""
+    import numpy as np
+    import qg_synth
+    from oracle import gemm as OG
+    from oracle import quant as OQ
+    w = qg_synth.weights(N, K)
+    qw, sw = OQ.per_row_int8(w)
+    acts = {m: qg_synth.activations(m, K) for m in MS}
+    t0 = time.perf_counter()
+    for _ in range(sample_steps):
+        for m in MS:
+            qa, sa = OQ.per_row_int8(acts[m])
+            OG.w8a8_int8(qa, sa, qw, sw)
+    dt = (time.perf_counter() - t0) / sample_steps
+    return {"value": step_bytes() / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{sample_steps} full steps (3 activation quantisations + 3 exact int64 GEMMs "
+                      f"M in {{1,8,32}}, N=K=4096 + bf16 epilogue), weights quantised once; numpy int64 "
+                      f"matmul runs on one thread",
+            "seconds_per_step": dt}
+
+
+# ---------------------------------------------------------- reference ---
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    steps = max(1, min(args.steps, 4))
+    warm = max(0, min(args.warmup, 1))
+    for _ in range(warm):
+        cpu_baseline(1)
+    cb = cpu_baseline(steps)
+    line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": steps, "warmup": warm, "ms_per_step": 1000 * cb["seconds_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "M": list(MS), "N": N, "K": K},
+            "cpu_baseline": {"value": cb["value"], "unit": "GB/s", "cores": cb["cores"], "kind": "oracle",
+                             "sample": cb["sample"]},
+            "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------- ours ---
+def run_ours(args, world, rank, local):
+    import numpy as np
+    import torch
+
+    import precision_quantized_gemm_b200 as qg
+    import qg_synth
+
+    assert torch.cuda.is_available(), "bench.py needs a CUDA device"
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    table = qg.Table(args.table) if os.path.exists(args.table) else None
+
+    def bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    # weights: quantised once, then copied so the rotation exceeds 2 x L2
+    w = bf16(qg_synth.weights(N, K))
+    layer = qg.Linear(FMT_INT8, w, table=table)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    wbytes = layer.Wq.q.numel() + layer.Wq.scale.numel()
+    copies = max(4, min(64, (2 * l2) // wbytes + 2))
+    Ws = [layer.Wq]
+    for _ in range(copies - 1):
+        o = qg.Operand(FMT_INT8, True, N, K, dev)
+        o.q.copy_(layer.Wq.q)
+        o.scale.copy_(layer.Wq.scale)
+        Ws.append(o)
+    cfgs, hits = {}, {}
+    for m in MS:
+        if table is not None:
+            cfgs[m], hits[m] = table.dispatch(FMT_INT8, m, N, K)
+        else:
+            cfgs[m], hits[m] = qg.qgemm_default_config(FMT_INT8, m, N, K), 0
+
+    acts = {m: bf16(qg_synth.activations(m, K)) for m in MS}
+    # one captured step per rotation slot: shape i of step s uses copy (3s+i) % copies
+    nslots = copies
+    steps_g = []
+    for s in range(nslots):
+        per = []
+        for i, m in enumerate(MS):
+            gs = qg.GraphStep(layer, m, W=Ws[(len(MS) * s + i) % copies], cfg=cfgs[m])
+            gs.A.copy_(acts[m])
+            per.append(gs)
+        steps_g.append(per)
+    # a single graph per step slot holding the three shapes back to back
+    step_graphs = []
+    for s in range(nslots):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for gs in steps_g[s]:
+                gs._launch()
+        step_graphs.append(g)
+    launches_per_step = sum(2 + (1 if (cfgs[m].split_k > 1 and cfgs[m].reduce_mode == 1) else 0) for m in MS)
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream()
+    # ---- warm-up
+    for s in range(args.warmup):
+        step_graphs[s % nslots].replay()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K full steps
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for s in range(args.steps):
+        step_graphs[s % nslots].replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms_step = e0.elapsed_time(e1) / args.steps
+
+    # ---- kernel-level timing on the same stream: per shape, graphs of
+    # back-to-back GEMM launches (and activation quantisations) over the rotation
+    per_shape = []
+    gemm_total_us = 0.0
+    gemm_total_bytes = 0
+    for m in MS:
+        gsz = steps_g[0][MS.index(m)]
+        reps = 2 * copies
+        def capture(kind):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for r in range(reps):
+                    gs = gsz
+                    st = qg._stream(None)
+                    if kind == "quant":
+                        qg.check(qg.qgemm_quantize_act(FMT_INT8, gs.A.data_ptr(), m, K, K, None, gs.act.c,
+                                                       gs.qws.data_ptr(), gs.qws.numel(), st))
+                    else:
+                        Wop = Ws[r % copies]
+                        wsp, wsb = gs.ws.get(qg.qgemm_workspace_size(FMT_INT8, m, N, K, gs.cfg))
+                        qg.check(qg.qgemm_run(FMT_INT8, gs.act.c, Wop.c, m, N, K, gs.cfg, wsp, wsb,
+                                              gs.Y.data_ptr(), N, qg.QG_OUT_BF16, st))
+            return g
+        gg = capture("gemm")
+        gq = capture("quant")
+        for g in (gg, gq):
+            g.replay()
+        torch.cuda.synchronize()
+        res = {}
+        for name, g in (("gemm", gg), ("quant", gq)):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(5):
+                g.replay()
+            b.record(stream)
+            torch.cuda.synchronize()
+            res[name] = 1000.0 * a.elapsed_time(b) / (5 * reps)
+        gb = gemm_bytes(m)
+        peak, peak_src = peaks()
+        gbs = gb / (res["gemm"] * 1e-6) / 1e9
+        per_shape.append({"M": m, "N": N, "K": K, "gemm_us": round(res["gemm"], 3),
+                          "quant_us": round(res["quant"], 3), "gemm_bytes": gb,
+                          "gemm_gbs": round(gbs, 1), "frac_hbm": round(gbs / peak, 4),
+                          "config": cfgs[m].as_dict(), "table_hit": hits[m]})
+        gemm_total_us += res["gemm"]
+        gemm_total_bytes += gb
+    clk = clocks.stop()
+
+    # ---- end to end through the public API with host buffers
+    host_in = {m: torch.empty(m, K, dtype=torch.bfloat16, pin_memory=True) for m in MS}
+    host_out = {m: torch.empty(m, N, dtype=torch.bfloat16, pin_memory=True) for m in MS}
+    for m in MS:
+        host_in[m].copy_(acts[m].cpu())
+    def e2e_step(s):
+        for i, m in enumerate(MS):
+            gs = steps_g[s % nslots][i]
+            gs.A.copy_(host_in[m], non_blocking=True)
+        step_graphs[s % nslots].replay()
+        for i, m in enumerate(MS):
+            host_out[m].copy_(steps_g[s % nslots][i].Y, non_blocking=True)
+        stream.synchronize()
+    for s in range(args.warmup):
+        e2e_step(s)
+    barrier(world)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for s in range(args.steps):
+        e2e_step(s)
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms_e2e = a.elapsed_time(b) / args.steps
+
+    ms_step_max = max_over_ranks(ms_step, world, dev)
+    ms_e2e_max = max_over_ranks(ms_e2e, world, dev)
+    peak, peak_src = peaks()
+    value = world * step_bytes() / (ms_step_max * 1e-3) / 1e9
+    achieved = gemm_total_bytes / (gemm_total_us * 1e-6) / 1e9
+    geo = math.exp(sum(math.log(max(p["frac_hbm"], 1e-9)) for p in per_shape) / len(per_shape))
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(prof):
+        t = json.load(open(prof)).get("w8a8_int8_gemm_bytes_per_launch")
+        traffic = t
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step_max, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": list(MS), "N": N, "K": K, "format": "W8A8_INT8",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": f"inputs larger than L2: {copies} rotating weight copies "
+                         f"({copies * wbytes / 1e6:.0f} MB > 2 x {l2 / 1e6:.0f} MB L2)",
+                   "step": "per M: activation quant + GEMM, one CUDA-graph replay per step",
+                   "table": os.path.relpath(args.table, ROOT) if table is not None else "built-in default"},
+        "per_shape": per_shape,
+        "geomean_frac_hbm_roofline": round(geo, 4),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "kernel": "qgemm_kernel<INT8, swap-AB> (all three shapes, launch-weighted)",
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
+                     else "fallback 6650 GB/s"},
+        "e2e": {"value": round(world * step_bytes() / (ms_e2e_max * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": sum(2 * m * K for m in MS),
+                "d2h_bytes_per_step": sum(2 * m * N for m in MS), "ms_per_step": round(ms_e2e_max, 5)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        cb = cpu_baseline()
+        line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+    elif world > 1:
+        line["cpu_baseline"] = None
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

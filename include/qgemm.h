@@ -83,8 +83,14 @@ typedef struct {
   int32_t tile_n;      /* MMA N extent: tokens per CTA when swap_ab = 1, weight
                           rows per CTA when swap_ab = 0; one of 16,32,64,128,256   */
   int32_t stages;      /* shared-memory pipeline depth, 2..12 (capped by smem)     */
-  int32_t reduce_mode; /* split_k > 1 only: 0 = in-kernel (the last CTA of a tile
-                          sums the partials in split order), 1 = second pass      */
+  int32_t reduce_mode; /* split_k > 1 only; every mode sums the partials in split
+                          order, so all three give identical bits:
+                          0 = the split_k CTAs of a tile form a thread-block
+                              cluster and sum through distributed shared memory
+                              (split_k <= 8, no workspace);
+                          1 = partials in the workspace + a second-pass kernel;
+                          2 = partials in the workspace, summed in-kernel by the
+                              last-arriving CTA of each tile (tile counters)    */
   int32_t reserved[3]; /* must be zero                                             */
 } qg_config;
 
@@ -124,11 +130,12 @@ qg_status qgemm_operand_bytes(qg_format f, int is_weight, int rows, int K,
  * its per-CTA amax partials there; the 8-bit formats need none: 0). */
 size_t qgemm_quant_workspace_size(qg_format f, int rows, int K);
 
-/* Scratch bytes qgemm_run needs for this configuration: 0 when split_k == 1,
- * else split_k * M * N * 4 bytes of partial sums plus one 4-byte counter per
- * output tile (in-kernel reduction).  The counter region must be zero before
- * the first call (see qgemm_workspace_clear); every completed call leaves it
- * zero again. */
+/* Scratch bytes qgemm_run needs for this configuration: 0 when split_k == 1
+ * or reduce_mode == 0; split_k * M * N * 4 bytes of partial sums (rounded up
+ * to 256) for reduce_mode 1; the same plus one 4-byte arrival counter per
+ * output tile for reduce_mode 2.  The counter region must be zero before the
+ * first reduce_mode-2 call (see qgemm_workspace_clear); every completed call
+ * leaves it zero again. */
 size_t qgemm_workspace_size(qg_format f, int M, int N, int K, const qg_config* cfg);
 
 /* Zeroes a run workspace on `stream` (one cudaMemsetAsync). */

@@ -243,7 +243,7 @@ class Operand:
         qb, sb = qgemm_operand_bytes(fmt, is_weight, rows, K)
         self.fmt, self.is_weight, self.rows, self.K = fmt, is_weight, rows, K
         self.q = torch.empty(qb, dtype=torch.uint8, device=device)
-        self.scale = torch.zeros(max(sb, 16) // 4 * 4 + 16, dtype=torch.uint8, device=device)[:sb]
+        self.scale = torch.zeros(sb, dtype=torch.uint8, device=device)
         self.global_scale = torch.zeros(4, dtype=torch.float32, device=device)
         self.c = qg_operand(self.q.data_ptr(), self.scale.data_ptr(), self.global_scale.data_ptr(), rows, K)
 
@@ -332,3 +332,56 @@ class Linear:
             act = self._act[M] = Operand(self.fmt, False, M, self.K, A.device)
         quantize_act(self.fmt, A, out=act, stream=stream)
         return run(self.fmt, act, self.Wq, self.config(M), out=out, workspace=self.ws, stream=stream)
+
+
+class GraphStep:
+    """One captured decode step of a quantized linear layer for a fixed token
+    count M: activation quantisation + GEMM replayed as a single CUDA graph
+    ("Helion in the vLLM backend", fourth paragraph: shapes up to
+    max_helion_size run under CUDA-graph replay).  Write the input into
+    ``A`` (bf16 [M, K]), call ``replay()``, read ``Y`` (bf16 [M, N])."""
+
+    def __init__(self, layer: "Linear", M: int, W: Operand | None = None, cfg: qg_config | None = None):
+        torch = _torch()
+        dev = layer.Wq.q.device
+        self.M, self.N, self.K = M, layer.N, layer.K
+        self.fmt = layer.fmt
+        self.W = W or layer.Wq
+        self.cfg = cfg or layer.config(M)
+        self.A = torch.zeros(M, self.K, dtype=torch.bfloat16, device=dev)
+        self.Y = torch.empty(M, self.N, dtype=torch.bfloat16, device=dev)
+        self.act = Operand(self.fmt, False, M, self.K, dev)
+        self.ws = Workspace(dev)
+        self.ws.get(qgemm_workspace_size(self.fmt, M, self.N, self.K, self.cfg))
+        self.qws = torch.zeros(max(qgemm_quant_workspace_size(self.fmt, M, self.K), 16), dtype=torch.uint8,
+                               device=dev)
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self._launch()                     # warm-up: configures kernels before capture
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize(dev)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self._launch()
+
+    def _launch(self):
+        st = _stream(None)
+        check(qgemm_quantize_act(self.fmt, self.A.data_ptr(), self.M, self.K, self.K, None, self.act.c,
+                                 self.qws.data_ptr(), self.qws.numel(), st), "qgemm_quantize_act")
+        wsp, wsb = self.ws.get(qgemm_workspace_size(self.fmt, self.M, self.N, self.K, self.cfg))
+        check(qgemm_run(self.fmt, self.act.c, self.W.c, self.M, self.N, self.K, self.cfg, wsp, wsb,
+                        self.Y.data_ptr(), self.N, QG_OUT_BF16, st), "qgemm_run")
+
+    def replay(self):
+        self.graph.replay()
+        return self.Y
+
+
+def _linear_capture(self, M: int, W: Operand | None = None, cfg: qg_config | None = None) -> GraphStep:
+    g = GraphStep(self, M, W=W, cfg=cfg)
+    self.graphs[M] = g
+    return g
+
+
+Linear.capture = _linear_capture

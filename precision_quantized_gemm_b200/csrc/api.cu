@@ -114,12 +114,21 @@ size_t gemm_smem(qg_format f, int tile_n, int stages) {
 }
 constexpr size_t kSmemLimit = 232448;  // 227 KB opt-in per CTA on sm_100
 
+bool cluster_fits(qg_format f, int tile_n, bool swap, int stages) {
+  switch (f) {
+    case QG_FP8_DYNAMIC: return qg::launch_gemm_fp8_cluster_fits(tile_n, swap, stages);
+    case QG_W8A8_INT8: return qg::launch_gemm_int8_cluster_fits(tile_n, swap, stages);
+    case QG_BLOCK_FP8: return qg::launch_gemm_block_cluster_fits(tile_n, swap, stages);
+    default: return qg::launch_gemm_nvf4_cluster_fits(tile_n, swap, stages);
+  }
+}
+
 qg_status check_config(qg_format f, int M, int N, int K, const qg_config* c) {
   if (!c) return QG_ERR_INVALID_ARG;
   if (c->reserved[0] || c->reserved[1] || c->reserved[2]) return QG_ERR_INVALID_ARG;
   if (!is_pow2(c->split_k) || c->split_k > 256) return QG_ERR_UNSUPPORTED;
   if (c->swap_ab != 0 && c->swap_ab != 1) return QG_ERR_INVALID_ARG;
-  if (c->reduce_mode != 0 && c->reduce_mode != 1) return QG_ERR_INVALID_ARG;
+  if (c->reduce_mode < 0 || c->reduce_mode > 2) return QG_ERR_INVALID_ARG;
   const int tn = c->tile_n;
   if (tn != 16 && tn != 32 && tn != 64 && tn != 128 && tn != 256) return QG_ERR_UNSUPPORTED;
   if (f == QG_BLOCK_FP8 && tn > 128) return QG_ERR_UNSUPPORTED;
@@ -130,6 +139,9 @@ qg_status check_config(qg_format f, int M, int N, int K, const qg_config* c) {
   const int kt = kt_total(f, K);
   if (c->split_k > kt) return QG_ERR_UNSUPPORTED;
   if (gemm_smem(f, tn, c->stages) > kSmemLimit) return QG_ERR_UNSUPPORTED;
+  if (c->split_k > 1 && c->reduce_mode == qg::kReduceCluster &&
+      (c->split_k > qg::kMaxClusterSplit || !cluster_fits(f, tn, c->swap_ab != 0, c->stages)))
+    return QG_ERR_UNSUPPORTED;
   if (f == QG_BLOCK_FP8) {
     const int nkt_max = (kt + c->split_k - 1) / c->split_k;
     const int act_rows = c->swap_ab ? tn : 128;
@@ -197,6 +209,8 @@ size_t qgemm_quant_workspace_size(qg_format f, int rows, int K) {
 
 size_t qgemm_workspace_size(qg_format f, int M, int N, int K, const qg_config* cfg) {
   if (!valid_format(f) || !cfg || M <= 0 || N <= 0 || K <= 0 || cfg->split_k <= 1) return 0;
+  if (cfg->reduce_mode == qg::kReduceCluster) return 0;
+  if (cfg->reduce_mode == qg::kReduceSecondPass) return ws_partial_bytes(M, N, cfg->split_k);
   int tp, tq;
   tiles_of(cfg, M, N, &tp, &tq);
   return ws_partial_bytes(M, N, cfg->split_k) + align_up((size_t)tp * tq * 4, 256);
@@ -321,7 +335,7 @@ qg_status qgemm_run(qg_format f, const qg_operand* A, const qg_operand* W, int M
   prm.out_kind = out_kind;
   int tp, tq;
   tiles_of(cfg, M, N, &tp, &tq);
-  if (cfg->split_k > 1) {
+  if (cfg->split_k > 1 && cfg->reduce_mode != qg::kReduceCluster) {
     prm.partial = workspace;
     prm.counters = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(workspace) +
                                                    ws_partial_bytes(M, N, cfg->split_k));
@@ -347,7 +361,7 @@ qg_status qgemm_run(qg_format f, const qg_operand* A, const qg_operand* W, int M
     default: e = qg::launch_gemm_nvf4(swap, cfg->tile_n, tmp, tmq, prm, grid, st, g_pdl); break;
   }
   if (e != cudaSuccess) return e == cudaErrorInvalidValue ? QG_ERR_UNSUPPORTED : QG_ERR_CUDA;
-  if (cfg->split_k > 1 && cfg->reduce_mode == 1) {
+  if (cfg->split_k > 1 && cfg->reduce_mode == qg::kReduceSecondPass) {
     switch (f) {
       case QG_FP8_DYNAMIC: e = qg::launch_gemm_fp8_reduce(prm, st, g_pdl); break;
       case QG_W8A8_INT8: e = qg::launch_gemm_int8_reduce(prm, st, g_pdl); break;
@@ -393,6 +407,11 @@ qg_status qgemm_default_config(qg_format f, int M, int N, int K, qg_config* out)
       c.split_k *= 2;
     if (c.split_k > kt) return QG_ERR_UNSUPPORTED;
   }
+  // split-K partials meet in distributed shared memory when the cluster
+  // fits, else the last-arriving CTA sums them from the workspace
+  c.reduce_mode = (c.split_k <= qg::kMaxClusterSplit && cluster_fits(f, c.tile_n, c.swap_ab != 0, c.stages))
+                      ? qg::kReduceCluster
+                      : qg::kReduceLastCta;
   *out = c;
   return QG_OK;
 }

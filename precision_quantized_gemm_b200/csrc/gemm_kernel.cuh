@@ -129,6 +129,52 @@ __device__ __forceinline__ float finish_value(uint32_t acc_bits, float sa, float
   }
 }
 
+constexpr int kReduceCluster = 0;   // split-K partials summed through distributed shared memory
+constexpr int kReduceSecondPass = 1;
+constexpr int kReduceLastCta = 2;   // last-arriving CTA sums the partials from the workspace
+constexpr int kMaxClusterSplit = 8;
+
+// Position of accumulator element (row of P, column c) in the cluster
+// reduction buffer: column-major for Swap-AB (rows are output channels, the
+// contiguous dimension of y), row-major with an odd row pitch otherwise.
+template <bool SWAP, int BN>
+__device__ __forceinline__ int red_index(int row, int c) {
+  return SWAP ? c * 128 + row : row * (BN + 1) + c;
+}
+template <bool SWAP, int BN>
+__host__ __device__ constexpr int red_bytes() {
+  return SWAP ? 4 * 128 * BN : 4 * 128 * (BN + 1);
+}
+
+template <int FMT>
+__device__ __forceinline__ uint32_t add_acc(uint32_t a, uint32_t b) {
+  if constexpr (FMT == kINT8) return (uint32_t)((int)a + (int)b);
+  else return __float_as_uint(__uint_as_float(a) + __uint_as_float(b));
+}
+
+template <int FMT>
+__device__ __forceinline__ float alpha_of(const GemmParams& prm) {
+  if constexpr (FMT == kNVF4) return __ldg(prm.g_a) * __ldg(prm.g_w);
+  else return 1.f;
+}
+
+// Final epilogue of output element (m, n) from its accumulator bits.
+template <int FMT>
+__device__ __forceinline__ void emit(const GemmParams& prm, int m, int n, uint32_t acc_bits,
+                                     float alpha) {
+  if (prm.out_kind == 1) {
+    reinterpret_cast<uint32_t*>(prm.Y)[(size_t)m * prm.ldy + n] = acc_bits;
+    return;
+  }
+  float sa = 1.f, sw = 1.f;
+  if constexpr (FMT == kFP8 || FMT == kINT8) {
+    sa = __ldg(prm.scale_a + m);
+    sw = __ldg(prm.scale_w + n);
+  }
+  reinterpret_cast<__nv_bfloat16*>(prm.Y)[(size_t)m * prm.ldy + n] =
+      __float2bfloat16_rn(finish_value<FMT>(acc_bits, sa, sw, alpha));
+}
+
 template <int FMT, bool SWAP, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     qgemm_kernel(const __grid_constant__ CUtensorMap tmap_p,
@@ -389,37 +435,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     named_bar_sync(1, 128);
     const bool epi_ok = (*flag_epi == 0);      // uniform over the 128 epilogue threads
 
-    // ---- write out: direct epilogue or split-K partials
-    float alpha = 1.f;
-    if constexpr (C::kNvf4) alpha = __ldg(prm.g_a) * __ldg(prm.g_w);
+    // ---- write out: direct epilogue, or this CTA's split-K partial
     const bool split = prm.split_k > 1;
     const int prow = p0 + row;                 // global row of P
     const bool prow_ok = prow < prm.rows_p;
-    float s_row = 1.f;                         // scale of this thread's P row
-    if constexpr (FMT == kFP8 || FMT == kINT8) {
-      if (prow_ok) s_row = __ldg((SWAP ? prm.scale_w : prm.scale_a) + prow);
-    }
-    const float* scale_col = SWAP ? prm.scale_a : prm.scale_w;
     const size_t MN = (size_t)prm.M * prm.N;
     uint32_t* part = reinterpret_cast<uint32_t*>(prm.partial);
-
-    auto out_index = [&](int c, int& m, int& n) {
-      if (SWAP) { m = q0 + c; n = prow; } else { m = prow; n = q0 + c; }
-    };
-    auto store_final = [&](int m, int n, uint32_t acc_bits) {
-      if (prm.out_kind == 1) {
-        reinterpret_cast<uint32_t*>(prm.Y)[(size_t)m * prm.ldy + n] = acc_bits;
-      } else {
-        float sa = 1.f, sw = 1.f;
-        if constexpr (FMT == kFP8 || FMT == kINT8) {
-          const float sc = __ldg(scale_col + (SWAP ? m : n));
-          sa = SWAP ? sc : s_row;
-          sw = SWAP ? s_row : sc;
-        }
-        const float y = finish_value<FMT>(acc_bits, sa, sw, alpha);
-        reinterpret_cast<__nv_bfloat16*>(prm.Y)[(size_t)m * prm.ldy + n] = __float2bfloat16_rn(y);
-      }
-    };
+    uint32_t* red = reinterpret_cast<uint32_t*>(smem + L.p);   // cluster reduction buffer
+    const float alpha = alpha_of<FMT>(prm);
 
     if (epi_ok) {
 #pragma unroll
@@ -429,29 +452,27 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(acc_f[c0 + j]);
         } else {
-          if (nkt > 0) {
-            tmem_ld16(lane_addr + c0, v);
-            tmem_ld_wait();
-          } else {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] = 0u;
-          }
+          tmem_ld16(lane_addr + c0, v);
+          tmem_ld_wait();
         }
-        if (prow_ok) {
+        if (split && prm.reduce_mode == kReduceCluster) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) red[red_index<SWAP, BN>(row, c0 + j)] = v[j];
+        } else if (prow_ok) {
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            int m, n;
-            out_index(c0 + j, m, n);
+            const int m = SWAP ? q0 + c0 + j : prow;
+            const int n = SWAP ? prow : q0 + c0 + j;
             if (m < prm.M && n < prm.N) {
               if (split)
                 part[(size_t)kz * MN + (size_t)m * prm.N + n] = v[j];
               else
-                store_final(m, n, v[j]);
+                emit<FMT>(prm, m, n, v[j], alpha);
             }
           }
         }
       }
-      if (split && prm.reduce_mode == 0) {
+      if (split && prm.reduce_mode == kReduceLastCta) {
         // Last-arriving CTA of this output tile sums the partials in split
         // order (deterministic) and applies the epilogue.
         __threadfence();
@@ -465,28 +486,76 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (*flag_last) {
           __threadfence();
           if (prow_ok) {
-            for (int c = 0; c < BN; ++c) {
-              int m, n;
-              out_index(c, m, n);
-              if (m >= prm.M || n >= prm.N) continue;
-              const size_t o = (size_t)m * prm.N + n;
-              uint32_t sum_bits;
-              if constexpr (FMT == kINT8) {
-                int s = 0;
-                for (int z = 0; z < prm.split_k; ++z) s += (int)ld_u32_cg(part + z * MN + o);
-                sum_bits = (uint32_t)s;
-              } else {
-                float s = 0.f;
-                for (int z = 0; z < prm.split_k; ++z) s += __uint_as_float(ld_u32_cg(part + z * MN + o));
-                sum_bits = __float_as_uint(s);
+            // 16 columns at a time: all their loads of one split are issued
+            // before any store, so the L2 round trips overlap.
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 16) {
+              uint32_t acc[16];
+#pragma unroll
+              for (int j = 0; j < 16; ++j) acc[j] = 0u;
+              for (int z = 0; z < prm.split_k; ++z) {
+                uint32_t t[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                  const int m = SWAP ? q0 + c0 + j : prow;
+                  const int n = SWAP ? prow : q0 + c0 + j;
+                  t[j] = (m < prm.M && n < prm.N) ? ld_u32_cg(part + z * MN + (size_t)m * prm.N + n) : 0u;
+                }
+#pragma unroll
+                for (int j = 0; j < 16; ++j) acc[j] = add_acc<FMT>(acc[j], t[j]);
               }
-              store_final(m, n, sum_bits);
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const int m = SWAP ? q0 + c0 + j : prow;
+                const int n = SWAP ? prow : q0 + c0 + j;
+                if (m < prm.M && n < prm.N) emit<FMT>(prm, m, n, acc[j], alpha);
+              }
             }
           }
           if (etid == 0) prm.counters[tile] = 0u;
         }
       }
     }
+  }
+
+  // ------------------------------------------ split-K reduction in the cluster
+  // The split_k CTAs of one output tile form a cluster; after every CTA has
+  // left its partial tile in its own shared memory, CTA r sums rows
+  // [r*128/S, (r+1)*128/S) of all S partials through distributed shared
+  // memory, in split order, and stores them.  Every thread of every CTA takes
+  // both cluster barriers.
+  if (prm.split_k > 1 && prm.reduce_mode == kReduceCluster) {
+    __syncwarp();
+    cluster_sync();
+    if (warp >= 2 && *reinterpret_cast<volatile int*>(smem + L.misc + 12) == 0) {
+      const int etid = threadIdx.x - 64;
+      const int S = prm.split_k;
+      const uint32_t rank = cluster_ctarank();
+      const int rows_per = 128 / S;
+      const int r0 = (int)rank * rows_per;
+      const uint32_t red_s = smem_u32(smem + L.p);
+      const float alpha = alpha_of<FMT>(prm);
+      for (int idx = etid; idx < rows_per * BN; idx += 128) {
+        int r, c;
+        if (SWAP) { r = r0 + idx % rows_per; c = idx / rows_per; }   // consecutive threads: consecutive n
+        else      { r = r0 + idx / BN;       c = idx % BN; }         // consecutive threads: consecutive n
+        const uint32_t off = 4u * (uint32_t)red_index<SWAP, BN>(r, c);
+        uint32_t t[16];
+        uint32_t acc = 0u;
+#pragma unroll
+        for (int z = 0; z < 16; ++z)
+          if (z < S) t[z] = ld_dsmem_u32(mapa_shared(red_s + off, (uint32_t)z));
+#pragma unroll
+        for (int z = 0; z < 16; ++z)
+          if (z < S) acc = add_acc<FMT>(acc, t[z]);
+        const int prow = p0 + r;
+        const int m = SWAP ? q0 + c : prow;
+        const int n = SWAP ? prow : q0 + c;
+        if (m < prm.M && n < prm.N) emit<FMT>(prm, m, n, acc, alpha);
+      }
+    }
+    __syncwarp();
+    cluster_sync();
   }
 
   // ------------------------------------------------------------------ teardown

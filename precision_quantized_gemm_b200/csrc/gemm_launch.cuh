@@ -24,11 +24,23 @@ cudaError_t launch_one(const CUtensorMap& tp, const CUtensorMap& tq, const GemmP
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (prm.split_k > 1 && prm.reduce_mode == kReduceCluster) {
+    // the split_k CTAs of one output tile form one cluster along z
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 1;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = prm.split_k;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = na;
   return cudaLaunchKernelEx(&cfg, kern, tp, tq, prm);
 }
 
@@ -44,6 +56,25 @@ cudaError_t launch_bn(int bn, const CUtensorMap& tp, const CUtensorMap& tq, cons
       if constexpr (FMT != kBLOCK) return launch_one<FMT, SWAP, 256>(tp, tq, prm, grid, st, pdl);
       return cudaErrorInvalidValue;
     default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int FMT, int BN>
+bool cluster_fits(bool swap, int stages) {
+  using C = Cfg<FMT, BN>;
+  const int ring = stages * (kPTileBytes + C::kQTileBytes);
+  return (swap ? red_bytes<true, BN>() : red_bytes<false, BN>()) <= ring;
+}
+
+template <int FMT>
+bool cluster_fits_for(int bn, bool swap, int stages) {
+  switch (bn) {
+    case 16: return cluster_fits<FMT, 16>(swap, stages);
+    case 32: return cluster_fits<FMT, 32>(swap, stages);
+    case 64: return cluster_fits<FMT, 64>(swap, stages);
+    case 128: return cluster_fits<FMT, 128>(swap, stages);
+    case 256: return cluster_fits<FMT, 256>(swap, stages);
+    default: return false;
   }
 }
 
@@ -71,6 +102,10 @@ cudaError_t QG_LAUNCH_NAME(bool swap, int tile_n, const CUtensorMap& tp, const C
 #define QG_CAT(a, b) QG_CAT2(a, b)
 
 size_t QG_CAT(QG_LAUNCH_NAME, _smem)(int tile_n, int stages) { return smem_for<QG_FMT>(tile_n, stages); }
+
+bool QG_CAT(QG_LAUNCH_NAME, _cluster_fits)(int tile_n, bool swap, int stages) {
+  return cluster_fits_for<QG_FMT>(tile_n, swap, stages);
+}
 
 cudaError_t QG_CAT(QG_LAUNCH_NAME, _reduce)(const GemmParams& prm, cudaStream_t st, bool pdl) {
   cudaLaunchConfig_t cfg = {};

@@ -135,7 +135,7 @@ std::vector<qg_config> candidates(qg_format f, int M, int N, int K) {
       if (!swap && (tn < 64 || M < 64)) continue;         // standard needs a real 128-token tile
       for (int sk = 1; sk <= 256 && sk <= kt; sk *= 2) {
         for (int st : stage_opts) {
-          for (int rm = 0; rm <= (sk > 1 ? 1 : 0); ++rm) {
+          for (int rm = 0; rm <= (sk > 1 ? 2 : 0); ++rm) {
             qg_config c = {};
             c.split_k = sk;
             c.swap_ab = swap;

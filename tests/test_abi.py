@@ -60,7 +60,11 @@ def test_operand_bytes_rejects_bad_k_or_format(fmt, K):
 def test_workspace_sizes():
     c = qg.make_config(split_k=1)
     assert qg.qgemm_workspace_size(qg.QG_FP8_DYNAMIC, 16, 2048, 2048, c) == 0
-    c = qg.make_config(split_k=8, swap_ab=1, tile_n=16)
+    c = qg.make_config(split_k=8, swap_ab=1, tile_n=16, reduce_mode=0)
+    assert qg.qgemm_workspace_size(qg.QG_FP8_DYNAMIC, 16, 2048, 2048, c) == 0   # cluster: none
+    c = qg.make_config(split_k=8, swap_ab=1, tile_n=16, reduce_mode=1)
+    assert qg.qgemm_workspace_size(qg.QG_FP8_DYNAMIC, 16, 2048, 2048, c) == 8 * 16 * 2048 * 4
+    c = qg.make_config(split_k=8, swap_ab=1, tile_n=16, reduce_mode=2)
     ws = qg.qgemm_workspace_size(qg.QG_FP8_DYNAMIC, 16, 2048, 2048, c)
     assert ws == 8 * 16 * 2048 * 4 + 256          # partials + 16 tile counters padded to 256
     assert qg.qgemm_quant_workspace_size(qg.QG_NVFP4, 8, 1024) > 0
@@ -72,6 +76,7 @@ def test_default_config_follows_the_swap_rule_and_fills_sms():
     assert c.swap_ab == 1 and c.tile_n == 16
     assert c.split_k >= 2 and (c.split_k & (c.split_k - 1)) == 0
     assert 32 * c.split_k <= 148
+    assert c.reduce_mode == 0                      # cluster reduction: no workspace
     c = qg.qgemm_default_config(qg.QG_BLOCK_FP8, 4096, 5120, 5120)
     assert c.swap_ab == 0 and c.tile_n == 128
     c = qg.qgemm_default_config(qg.QG_FP8_DYNAMIC, 32, 2048, 2048)
@@ -113,8 +118,10 @@ def _run(fmt=qg.QG_FP8_DYNAMIC, M=16, N=256, K=512, cfg=None, A=None, W=None, ws
     (dict(cfg=qg.make_config(tile_n=256, stages=12)), qg.QG_ERR_UNSUPPORTED),  # smem
     (dict(fmt=qg.QG_BLOCK_FP8, cfg=qg.make_config(tile_n=256)), qg.QG_ERR_UNSUPPORTED),
     (dict(cfg=qg.make_config(swap_ab=2)), qg.QG_ERR_INVALID_ARG),
-    (dict(cfg=qg.make_config(split_k=2, stages=4), ws=None), qg.QG_ERR_WORKSPACE),
-    (dict(cfg=qg.make_config(split_k=2, stages=4), ws=FAKE, wsb=64), qg.QG_ERR_WORKSPACE),
+    (dict(cfg=qg.make_config(split_k=2, stages=4, reduce_mode=2), ws=None), qg.QG_ERR_WORKSPACE),
+    (dict(cfg=qg.make_config(split_k=2, stages=4, reduce_mode=1), ws=FAKE, wsb=64), qg.QG_ERR_WORKSPACE),
+    (dict(cfg=qg.make_config(split_k=4, stages=4, reduce_mode=3)), qg.QG_ERR_INVALID_ARG),
+    (dict(K=4096, cfg=qg.make_config(split_k=16, stages=4, reduce_mode=0)), qg.QG_ERR_UNSUPPORTED),
 ])
 def test_run_rejects_bad_arguments_before_any_launch(kw, status):
     assert _run(**kw) == status

@@ -94,20 +94,25 @@ def _setup(fmt, M, N, K, edge_rows=True):
     return A, W, qa, qw
 
 
-SWAP_CASES = [  # (M, N, K, split_k, tile_n, reduce_mode, stages)
+SWAP_CASES = [  # (M, N, K, split_k, tile_n, reduce_mode, stages); reduce 0 cluster, 1 second pass, 2 last CTA
     (1, 256, 512, 1, 16, 0, 4),
     (5, 384, 1024, 2, 16, 0, 4),
-    (16, 300, 1024, 4, 16, 0, 6),
+    (16, 300, 1024, 4, 16, 2, 6),
     (20, 512, 2048, 4, 32, 1, 8),
     (32, 640, 2048, 8, 32, 0, 8),
+    (32, 640, 2048, 8, 32, 2, 8),
     (48, 256, 1024, 2, 64, 0, 4),
     (33, 130, 512, 1, 16, 0, 4),      # two token tiles, ragged N
+    (3, 260, 4096, 16, 16, 2, 4),     # split beyond the cluster limit
 ]
 STD_CASES = [
     (128, 256, 512, 1, 128, 0, 4),
     (200, 384, 1024, 2, 64, 0, 4),
     (256, 512, 1024, 1, 256, 0, 3),
     (130, 300, 2048, 4, 128, 1, 4),
+    (150, 256, 2048, 4, 128, 0, 4),
+    (150, 256, 2048, 2, 256, 0, 3),
+    (140, 200, 1024, 2, 64, 2, 4),
 ]
 
 
@@ -176,13 +181,10 @@ def test_default_config_parity(fmt):
 def test_split_k_deterministic_and_modes_agree():
     fmt = qg.QG_FP8_DYNAMIC
     A, W, _, _ = _setup(fmt, 16, 512, 4096)
-    c0 = qg.make_config(split_k=8, swap_ab=1, tile_n=16, stages=6, reduce_mode=0)
-    c1 = qg.make_config(split_k=8, swap_ab=1, tile_n=16, stages=6, reduce_mode=1)
-    y0 = qg.run(fmt, A, W, c0)
-    y0b = qg.run(fmt, A, W, c0)
-    y1 = qg.run(fmt, A, W, c1)
-    assert torch.equal(y0, y0b)          # fixed summation order: run to run identical
-    assert torch.equal(y0, y1)           # both modes sum partials in split order
+    ys = [qg.run(fmt, A, W, qg.make_config(split_k=8, swap_ab=1, tile_n=16, stages=6, reduce_mode=r))
+          for r in (0, 1, 2, 0, 2)]
+    for y in ys[1:]:
+        assert torch.equal(ys[0], y)     # fixed split order: every mode, every run, same bits
 
 
 def test_swap_and_standard_agree_int8_bitwise():
