@@ -191,6 +191,30 @@ qg_status qgemm_run(qg_format f, const qg_operand* A, const qg_operand* W, int M
                     const qg_config* cfg, void* workspace, size_t ws_bytes, void* Y, int ldy,
                     int out_kind, void* stream);
 
+/* qgemm_run without a caller-provided workspace.  There is no counterpart of
+ * this entry point in the pages the library follows; it exists for callers
+ * that cannot allocate device memory on this path (an engine whose memory
+ * planner reserved all device memory up front and forbids allocation while
+ * serving, a plugin host that passes only input and output buffers).  Inputs
+ * and outputs are still the caller's; the split-K scratch (reduce_mode 1 or
+ * 2) comes from a fixed array inside the library, QGEMM_NOALLOC_SCRATCH_BYTES
+ * bytes on every GPU that loads the library, held until the process exits.
+ *   - A configuration whose qgemm_workspace_size exceeds that maximum is
+ *     rejected with QG_ERR_WORKSPACE before any device work.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - No cudaMalloc, cudaFree or other allocation is made.  For reduce_mode 2
+ *     the tile-counter region is cleared with cudaMemsetAsync on `stream`.
+ *   - Every call shares the one array and it keeps the last call's contents:
+ *     calls that overlap on the GPU (other streams, other threads) race on it
+ *     and must be serialised by the caller.
+ * Other arguments and results are those of qgemm_run. */
+#define QGEMM_NOALLOC_SCRATCH_BYTES (8u << 20)
+qg_status qgemm_run_noalloc(qg_format f, const qg_operand* A, const qg_operand* W, int M, int N,
+                            int K, const qg_config* cfg, void* Y, int ldy, int out_kind,
+                            void* stream);
+
 /* Default configuration for a shape when no table entry exists: swap_ab = 1
  * for M < 32 ("Helion in the vLLM backend", second paragraph: vLLM's
  * Block_FP8 backend swaps A and B below M = 32), split_k chosen so that

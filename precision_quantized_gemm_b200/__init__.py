@@ -41,6 +41,7 @@ EXPORTS = [
     "qgemm_quantize_act", "qgemm_quantize_weight", "qgemm_run", "qgemm_default_config",
     "qgemm_table_load", "qgemm_table_create", "qgemm_table_put", "qgemm_table_save",
     "qgemm_table_free", "qgemm_table_size", "qgemm_dispatch", "qgemm_tune", "qgemm_device_error",
+    "qgemm_run_noalloc",
 ]
 
 
@@ -107,6 +108,8 @@ def lib() -> ctypes.CDLL:
             "qgemm_dispatch": (c_int, [c_void_p, c_int, c_int, c_int, c_int, POINTER(qg_config), POINTER(c_int)]),
             "qgemm_tune": (c_int, [c_void_p, c_int, POINTER(c_int), c_int, POINTER(c_int), c_int, c_double, c_int]),
             "qgemm_device_error": (c_int, []),
+            "qgemm_run_noalloc": (c_int, [c_int, POINTER(qg_operand), POINTER(qg_operand), c_int, c_int, c_int,
+                                          POINTER(qg_config), c_void_p, c_int, c_int, c_void_p]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -158,6 +161,13 @@ def qgemm_run(fmt, A: qg_operand, W: qg_operand, M, N, K, cfg: qg_config, ws_ptr
               Y_ptr, ldy, out_kind, stream):
     return lib().qgemm_run(fmt, ctypes.byref(A), ctypes.byref(W), M, N, K, ctypes.byref(cfg),
                            ws_ptr, ws_bytes, Y_ptr, ldy, out_kind, stream)
+
+
+def qgemm_run_noalloc(fmt, A: qg_operand, W: qg_operand, M, N, K, cfg: qg_config, Y_ptr, ldy, out_kind,
+                      stream):
+    """qgemm_run with the library's own fixed scratch instead of a caller workspace."""
+    return lib().qgemm_run_noalloc(fmt, ctypes.byref(A), ctypes.byref(W), M, N, K, ctypes.byref(cfg),
+                                   Y_ptr, ldy, out_kind, stream)
 
 
 def qgemm_default_config(fmt, M, N, K) -> qg_config:

@@ -287,7 +287,7 @@ qg_status qgemm_quantize_weight(qg_format f, const void* W, int N, int K, qg_ope
   return e == cudaSuccess ? QG_OK : QG_ERR_CUDA;
 }
 
-static qg_status check_operand(qg_format f, const qg_operand* o, int rows, int K) {
+qg_status check_operand_impl(qg_format f, const qg_operand* o, int rows, int K) {
   if (!o || !o->q || !o->scale) return QG_ERR_INVALID_ARG;
   if (o->rows != rows || o->K != K) return QG_ERR_INVALID_ARG;
   if (!aligned(o->q, 16) || !aligned(o->scale, f == QG_NVFP4 ? 16 : 4)) return QG_ERR_INVALID_ARG;
@@ -295,18 +295,33 @@ static qg_status check_operand(qg_format f, const qg_operand* o, int rows, int K
   return QG_OK;
 }
 
-qg_status qgemm_run(qg_format f, const qg_operand* A, const qg_operand* W, int M, int N, int K,
-                    const qg_config* cfg, void* workspace, size_t ws_bytes, void* Y, int ldy,
-                    int out_kind, void* stream) {
+}  // extern "C"
+
+namespace qg {
+// Host-side argument checks of qgemm_run (no device work).
+qg_status check_run_args(qg_format f, const qg_operand* A, const qg_operand* W, int M, int N, int K,
+                         const qg_config* cfg, void* workspace, size_t ws_bytes, void* Y, int ldy,
+                         int out_kind) {
   if (!valid_format(f) || M <= 0 || N <= 0 || K <= 0 || !Y || ldy < N) return QG_ERR_INVALID_ARG;
   if (out_kind != QG_OUT_BF16 && out_kind != QG_OUT_ACC) return QG_ERR_INVALID_ARG;
   if (K % k_multiple(f) != 0 || !aligned(Y, 16)) return QG_ERR_INVALID_ARG;
   qg_status s;
-  if ((s = check_operand(f, A, M, K)) != QG_OK) return s;
-  if ((s = check_operand(f, W, N, K)) != QG_OK) return s;
+  if ((s = check_operand_impl(f, A, M, K)) != QG_OK) return s;
+  if ((s = check_operand_impl(f, W, N, K)) != QG_OK) return s;
   if ((s = check_config(f, M, N, K, cfg)) != QG_OK) return s;
   const size_t need = qgemm_workspace_size(f, M, N, K, cfg);
   if (need > 0 && (!workspace || ws_bytes < need || !aligned(workspace, 256))) return QG_ERR_WORKSPACE;
+  return QG_OK;
+}
+}  // namespace qg
+
+extern "C" {
+
+qg_status qgemm_run(qg_format f, const qg_operand* A, const qg_operand* W, int M, int N, int K,
+                    const qg_config* cfg, void* workspace, size_t ws_bytes, void* Y, int ldy,
+                    int out_kind, void* stream) {
+  qg_status s = qg::check_run_args(f, A, W, M, N, K, cfg, workspace, ws_bytes, Y, ldy, out_kind);
+  if (s != QG_OK) return s;
   DeviceInfo* d;
   if ((s = device_info(&d)) != QG_OK) return s;
 

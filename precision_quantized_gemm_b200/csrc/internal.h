@@ -10,6 +10,14 @@ namespace qg {
 
 struct GemmParams;
 
+}  // namespace qg
+#include "../../include/qgemm.h"
+namespace qg {
+
+qg_status check_run_args(qg_format f, const qg_operand* A, const qg_operand* W, int M, int N, int K,
+                         const qg_config* cfg, void* workspace, size_t ws_bytes, void* Y, int ldy,
+                         int out_kind);
+
 constexpr int kNvfp4AmaxMaxCtas = 296;   // partial-amax slots in the NVFP4 quant workspace
 
 cudaError_t launch_quant_rows(bool int8, const void* X, int R, int K, int ldx, void* q,
