@@ -55,6 +55,9 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--table", default=TABLE)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--suite", default=None,
+                    help="comma list of per-shape suites to time instead of the step: "
+                         "fp8_tiny,int8,block_fp8,nvfp4,sweep,large_m (one JSON line per shape)")
     return ap.parse_args()
 
 
@@ -404,11 +407,133 @@ def run_ours(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------- suites ---
+# (format, M list, (N, K) list) of the workloads the linear backend is measured
+# on; the (N, K) pairs of the sweep are LLM projection shapes of the FlashInfer
+# mm_fp4 benchmark list.
+SWEEP_NK = [(896, 5120), (1024, 7168), (1280, 8192), (1792, 5120), (2560, 8192), (4096, 4096),
+            (4608, 7168), (5120, 640), (5120, 2048), (6144, 4096), (7168, 2048), (8192, 8192)]
+SUITES = {
+    "fp8_tiny": [(0, [16], [(2048, 2048)])],
+    "int8": [(1, [1, 8, 32], [(4096, 4096)])],
+    "block_fp8": [(2, [1, 4, 16, 32], [(512, 7168), (4608, 7168), (5120, 640), (2560, 8192)])],
+    "nvfp4": [(3, [1, 8, 64, 512], [(896, 1024), (1792, 5120), (5120, 2048), (1280, 8192)])],
+    "sweep": [(0, [1, 2, 4, 8, 16, 32], SWEEP_NK), (2, [1, 2, 4, 8, 16, 32], SWEEP_NK)],
+    "large_m": [(2, [4096, 16384], [(5120, 5120)])],
+}
+FMT_NAME = {0: "FP8_Dynamic", 1: "W8A8_INT8", 2: "Block_FP8", 3: "NVFP4"}
+
+
+def shape_bytes(fmt, M, N, K):
+    """Algorithmic bytes of one GEMM call: codes + scales of A and W, bf16 Y."""
+    if fmt == 3:
+        return N * K // 2 + M * K // 2 + (N + M) * K // 16 + 8 + 2 * M * N
+    if fmt == 2:
+        return N * K + 4 * ((N + 127) // 128) * (K // 128) + M * K + 4 * M * (K // 128) + 2 * M * N
+    return N * K + 4 * N + M * K + 4 * M + 2 * M * N
+
+
+def tensor_peak(fmt, bf16_tflops):
+    """Dense tensor peak for the format: the measured bf16 peak times the
+    nominal ratio (fp8 and int8 2x, fp4 4x)."""
+    return bf16_tflops * (4.0 if fmt == 3 else 2.0)
+
+
+def run_suite(args, names, local):
+    import numpy as np
+    import torch
+
+    import precision_quantized_gemm_b200 as qg
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    table = qg.Table(args.table) if os.path.exists(args.table) else None
+    pk = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
+        os.path.join(ROOT, "MEASURED_PEAKS.json")) else {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+    hbm, bf16 = float(pk["hbm_gbs"]), float(pk["bf16_tflops"])
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0)
+    results = []
+    for name in names:
+        for fmt, Ms, NKs in SUITES[name]:
+            for (N, K) in NKs:
+                w = (torch.randn(N, K, device=dev, generator=gen) * 0.02).to(torch.bfloat16)
+                Wq = qg.quantize_weight(fmt, w)
+                del w
+                wbytes = Wq.q.numel() + Wq.scale.numel()
+                for M in Ms:
+                    flops = 2.0 * M * N * K
+                    byts = shape_bytes(fmt, M, N, K)
+                    # inputs larger than L2: rotate weight copies (and
+                    # activations for large M) past 2 x L2
+                    per_call = wbytes + (M * K if fmt != 3 else M * K // 2)
+                    copies = int(max(1, min(64, (2 * l2) // max(per_call, 1) + 2)))
+                    Ws = [Wq]
+                    for _ in range(copies - 1):
+                        o = qg.Operand(fmt, True, N, K, dev)
+                        o.q.copy_(Wq.q)
+                        o.scale.copy_(Wq.scale)
+                        o.global_scale.copy_(Wq.global_scale)
+                        Ws.append(o)
+                    a = torch.randn(M, K, device=dev, generator=gen).to(torch.bfloat16)
+                    As = [qg.quantize_act(fmt, a) for _ in range(copies if M >= 4096 else 1)]
+                    cfg, hit = (table.dispatch(fmt, M, N, K) if table is not None
+                                else (qg.qgemm_default_config(fmt, M, N, K), 0))
+                    ws = qg.Workspace(dev)
+                    wsp, wsb = ws.get(qg.qgemm_workspace_size(fmt, M, N, K, cfg))
+                    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+                    reps = max(2 * copies, 8) if M < 4096 else 2 * copies
+                    st = qg._stream(None)
+                    qg.check(qg.qgemm_run(fmt, As[0].c, Ws[0].c, M, N, K, cfg, wsp, wsb, Y.data_ptr(), N, 0, st))
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g):
+                        st = qg._stream(None)
+                        for r in range(reps):
+                            qg.check(qg.qgemm_run(fmt, As[r % len(As)].c, Ws[r % copies].c, M, N, K, cfg,
+                                                  wsp, wsb, Y.data_ptr(), N, 0, st))
+                    g.replay()
+                    torch.cuda.synchronize()
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    n_rep = 5 if M < 4096 else 2
+                    e0.record()
+                    for _ in range(n_rep):
+                        g.replay()
+                    e1.record()
+                    torch.cuda.synchronize()
+                    us = 1000.0 * e0.elapsed_time(e1) / (n_rep * reps)
+                    t_hbm = byts / (hbm * 1e9) * 1e6
+                    t_tc = flops / (tensor_peak(fmt, bf16) * 1e12) * 1e6
+                    bound = "hbm" if t_hbm >= t_tc else "tensor"
+                    frac = max(t_hbm, t_tc) / us
+                    rec = {"suite": name, "format": FMT_NAME[fmt], "M": M, "N": N, "K": K, "us": round(us, 3),
+                           "GB/s": round(byts / us / 1e3, 1), "TFLOP/s": round(flops / us / 1e6, 2),
+                           "bound": bound, "roofline_us": round(max(t_hbm, t_tc), 3),
+                           "frac_roofline": round(frac, 4), "config": cfg.as_dict(), "table_hit": hit,
+                           "rotating_copies": copies}
+                    print(json.dumps(rec), flush=True)
+                    results.append(rec)
+                    del g, As, Ws[1:], Y
+                    torch.cuda.empty_cache()
+    def geo(xs):
+        return math.exp(sum(math.log(max(x, 1e-9)) for x in xs) / len(xs)) if xs else None
+    small = [r["frac_roofline"] for r in results if r["M"] <= 32]
+    large = [r["frac_roofline"] for r in results if r["M"] >= 4096]
+    print(json.dumps({"summary": True, "shapes": len(results), "geomean_frac_roofline_M_le_32": geo(small),
+                      "geomean_frac_roofline_M_ge_4096": geo(large),
+                      "geomean_frac_roofline_all": geo([r["frac_roofline"] for r in results]),
+                      "peaks": {"hbm_gbs": hbm, "bf16_tflops": bf16,
+                                "note": "fp8/int8 tensor peak = 2 x measured bf16, fp4 = 4 x"}}), flush=True)
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup()
     try:
-        if args.impl == "reference":
+        if args.suite:
+            run_suite(args, [s.strip() for s in args.suite.split(",") if s.strip()], local)
+        elif args.impl == "reference":
             run_reference(args, world, rank)
         else:
             run_ours(args, world, rank, local)

@@ -14,12 +14,19 @@
 //               a `stages`-deep ring of 128-byte K tiles in shared memory.
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer.
 //   warps 2..5  epilogue: tcgen05.ld of the fp32/int32 accumulator, scales in
-//               fp32, bf16 store (or split-K partials and their reduction).
+//               fp32, bf16 store, or this CTA's split-K partial.
 // Block_FP8 promotes every 128-wide K group: the MMA writes the group's
 // partial sum into one of NACC TMEM buffers and the epilogue warps fold it
 // into fp32 registers with the group's activation and weight-block scales.
 // NVFP4 uses kind::mxf4nvf4 with the e4m3 block scales copied
 // smem -> TMEM by tcgen05.cp.
+//
+// Split-K ("Helion in the vLLM backend", second and third paragraphs): the
+// split_k CTAs of one output tile either form a thread-block cluster and
+// meet in distributed shared memory (no global scratch), or leave partials
+// in a workspace that the last-arriving CTA or a second kernel sums.  Every
+// mode adds the partials in split order, so results are deterministic and
+// identical across modes.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -36,6 +43,11 @@ constexpr int kKTileBytes = 128;     // bytes of K per pipeline stage (one 128B 
 constexpr int kPTileBytes = 128 * kKTileBytes;
 constexpr int kSfAtomBytes = 512;    // one 128x4 atom of e4m3 block scales
 constexpr int kMaxScaleStage = 8192; // floats of Block_FP8 scales staged per CTA
+
+constexpr int kReduceCluster = 0;    // split-K partials summed through distributed shared memory
+constexpr int kReduceSecondPass = 1; // partials in the workspace, summed by a second kernel
+constexpr int kReduceLastCta = 2;    // partials in the workspace, summed by the last-arriving CTA
+constexpr int kMaxClusterSplit = 8;
 
 struct GemmParams {
   int M, N, K;
@@ -56,7 +68,7 @@ struct GemmParams {
   int out_kind;                // 0 = bf16, 1 = raw accumulators
   void* partial;               // split-K partials [split][M][N] (4-byte elements)
   unsigned int* counters;      // split-K per-tile arrival counters
-  int reduce_mode;             // 0 = in-kernel, 1 = second pass
+  int reduce_mode;             // kReduce*
   unsigned int* err;           // device error word
 };
 
@@ -64,11 +76,11 @@ template <int FMT, int BN>
 struct Cfg {
   static constexpr bool kBlock = FMT == kBLOCK;
   static constexpr bool kNvf4 = FMT == kNVF4;
+  static constexpr bool kRowColScales = FMT == kFP8 || FMT == kINT8;
   static constexpr int kQTileBytes = BN * kKTileBytes;
   static constexpr int kSfQAtoms = BN > 128 ? 2 : 1;               // 128-row SF blocks of Q
   static constexpr int kSfPBytes = kNvf4 ? 4 * kSfAtomBytes : 0;   // 4 K-atoms per 128B tile
   static constexpr int kSfQBytes = kNvf4 ? 4 * kSfAtomBytes * kSfQAtoms : 0;
-  static constexpr int kStageBytes = kPTileBytes + kQTileBytes + kSfPBytes + kSfQBytes;
   static constexpr int kNAcc = kBlock ? (BN >= 128 ? 2 : 4) : 1;  // TMEM accumulators
   static constexpr int kSfaCol = kNAcc * BN;                       // TMEM column of SF A
   static constexpr int kSfbCol = kSfaCol + 16;                     // 4 steps x 4 words
@@ -81,11 +93,15 @@ struct Cfg {
   static constexpr uint32_t kIdesc = kNvf4              ? idesc_nvf4(BN)
                                      : (FMT == kINT8)   ? idesc_i8(BN)
                                                         : idesc_f8f6f4_e4m3(BN);
+  // Cluster split-K for narrow tiles pushes partial slices into a dedicated
+  // receive buffer of the owning CTA; wide tiles pull from the ring instead.
+  static constexpr bool kPush = BN <= 64;
+  static constexpr int kRecvBytes = kPush ? 4 * 128 * BN : 0;
 };
 
 // Shared-memory carve-up (offsets from a 1024-byte aligned base).
 struct SmemLayout {
-  uint32_t p, q, sfp, sfq, bars, misc, scales, total;
+  uint32_t p, q, sfp, sfq, recv, bars, misc, epis, scales, total;
 };
 template <int FMT, int BN>
 __host__ __device__ inline SmemLayout smem_layout(int stages) {
@@ -95,16 +111,38 @@ __host__ __device__ inline SmemLayout smem_layout(int stages) {
   L.q = L.p + stages * kPTileBytes;
   L.sfp = L.q + stages * C::kQTileBytes;
   L.sfq = L.sfp + stages * C::kSfPBytes;
-  L.bars = L.sfq + stages * C::kSfQBytes;
-  // full[stages], empty[stages], acc_full, tfull[4], tempty[4]
-  L.misc = L.bars + 8 * (2 * stages + 1 + 8);
-  L.scales = (L.misc + 16 + 15) & ~15u;
+  L.recv = L.sfq + stages * C::kSfQBytes;
+  L.bars = L.recv + C::kRecvBytes;
+  // full[stages], empty[stages], acc_full, tfull[4], tempty[4], recv_full
+  L.misc = L.bars + 8 * (2 * stages + 1 + 8 + 1);
+  L.epis = (L.misc + 16 + 15) & ~15u;          // row / column scales (FP8, INT8)
+  L.scales = L.epis + (C::kRowColScales ? 4 * (128 + BN) : 0);
   L.total = L.scales + (C::kBlock ? 4 * (kMaxScaleStage + 2 * 64) : 0);
   return L;
 }
 template <int FMT, int BN>
 __host__ inline size_t smem_bytes(int stages) {
   return smem_layout<FMT, BN>(stages).total + 1024;  // + alignment slack
+}
+
+// Bytes a pull-mode cluster reduction stages in the (then idle) ring.
+template <bool SWAP, int BN>
+__host__ __device__ constexpr int red_bytes() {
+  return SWAP ? 4 * 128 * BN : 4 * 128 * (BN + 1);
+}
+// Position of accumulator element (row of P, column c) in the pull-mode
+// buffer: column-major for Swap-AB (rows are output channels, the contiguous
+// dimension of y), row-major with an odd row pitch otherwise.
+template <bool SWAP, int BN>
+__device__ __forceinline__ int red_index(int row, int c) {
+  return SWAP ? c * 128 + row : row * (BN + 1) + c;
+}
+// Push mode: CTA `owner` receives rows [owner*rows_per, (owner+1)*rows_per)
+// of every split's partial; slot z holds split z's slice, laid out so the
+// owner's final stores are coalesced.
+template <bool SWAP, int BN>
+__device__ __forceinline__ int slice_index(int rl, int c, int rows_per) {
+  return SWAP ? c * rows_per + rl : rl * BN + c;
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
@@ -129,23 +167,6 @@ __device__ __forceinline__ float finish_value(uint32_t acc_bits, float sa, float
   }
 }
 
-constexpr int kReduceCluster = 0;   // split-K partials summed through distributed shared memory
-constexpr int kReduceSecondPass = 1;
-constexpr int kReduceLastCta = 2;   // last-arriving CTA sums the partials from the workspace
-constexpr int kMaxClusterSplit = 8;
-
-// Position of accumulator element (row of P, column c) in the cluster
-// reduction buffer: column-major for Swap-AB (rows are output channels, the
-// contiguous dimension of y), row-major with an odd row pitch otherwise.
-template <bool SWAP, int BN>
-__device__ __forceinline__ int red_index(int row, int c) {
-  return SWAP ? c * 128 + row : row * (BN + 1) + c;
-}
-template <bool SWAP, int BN>
-__host__ __device__ constexpr int red_bytes() {
-  return SWAP ? 4 * 128 * BN : 4 * 128 * (BN + 1);
-}
-
 template <int FMT>
 __device__ __forceinline__ uint32_t add_acc(uint32_t a, uint32_t b) {
   if constexpr (FMT == kINT8) return (uint32_t)((int)a + (int)b);
@@ -158,18 +179,21 @@ __device__ __forceinline__ float alpha_of(const GemmParams& prm) {
   else return 1.f;
 }
 
-// Final epilogue of output element (m, n) from its accumulator bits.
-template <int FMT>
-__device__ __forceinline__ void emit(const GemmParams& prm, int m, int n, uint32_t acc_bits,
-                                     float alpha) {
+// Final epilogue of tile element (r, c) = output (m, n).  FP8 / INT8 take
+// their per-row scales from the staged copies: row_s[r] is the scale of P row
+// r and col_s[c] that of Q row c.
+template <int FMT, bool SWAP>
+__device__ __forceinline__ void emit(const GemmParams& prm, int r, int c, int m, int n,
+                                     uint32_t acc_bits, float alpha, const float* row_s,
+                                     const float* col_s) {
   if (prm.out_kind == 1) {
     reinterpret_cast<uint32_t*>(prm.Y)[(size_t)m * prm.ldy + n] = acc_bits;
     return;
   }
   float sa = 1.f, sw = 1.f;
   if constexpr (FMT == kFP8 || FMT == kINT8) {
-    sa = __ldg(prm.scale_a + m);
-    sw = __ldg(prm.scale_w + n);
+    sa = SWAP ? col_s[c] : row_s[r];
+    sw = SWAP ? row_s[r] : col_s[c];
   }
   reinterpret_cast<__nv_bfloat16*>(prm.Y)[(size_t)m * prm.ldy + n] =
       __float2bfloat16_rn(finish_value<FMT>(acc_bits, sa, sw, alpha));
@@ -190,9 +214,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_full = empty + S;
   uint64_t* tfull = acc_full + 1;
   uint64_t* tempty = tfull + 4;
+  uint64_t* recv_full = tempty + 4;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.misc);
   volatile int* flag_last = reinterpret_cast<volatile int*>(smem + L.misc + 4);
   volatile int* flag_abort = reinterpret_cast<volatile int*>(smem + L.misc + 8);
+  volatile int* flag_epi = reinterpret_cast<volatile int*>(smem + L.misc + 12);
+  float* row_s = reinterpret_cast<float*>(smem + L.epis);
+  float* col_s = row_s + 128;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -202,6 +230,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kt_begin = (int)(((long long)kz * prm.kt_total) / prm.split_k);
   const int kt_end = (int)(((long long)(kz + 1) * prm.kt_total) / prm.split_k);
   const int nkt = kt_end - kt_begin;
+  const bool cluster_red = prm.split_k > 1 && prm.reduce_mode == kReduceCluster;
+  const int rows_per = 128 / prm.split_k;                  // cluster mode: rows owned per CTA
+  const uint32_t slot_bytes = 4u * (uint32_t)(rows_per * BN);
 
   if (threadIdx.x == 0) {
     prefetch_tmap(&tmap_p);
@@ -215,8 +246,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], 4);
     }
+    mbar_init(recv_full, 1);
     *flag_abort = 0;
     fence_barrier_init();
+    if (C::kPush && cluster_red) mbar_arrive_expect_tx(recv_full, (uint32_t)prm.split_k * slot_bytes);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::kTmemCols);
@@ -226,6 +259,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Cluster phase 1 (arrive now, wait before the first remote access): the
+  // barriers of every CTA in the cluster are initialised.
+  if (cluster_red) cluster_arrive();
   // Let the next kernel of the stream start its prologue; it waits on our
   // completion before touching what we write.
   if (threadIdx.x == 0) griddep_launch_dependents();
@@ -367,8 +403,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int etid = threadIdx.x - 64;         // 0..127
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
     griddep_wait();                            // scales/partials of earlier kernels
-
-    volatile int* flag_epi = reinterpret_cast<volatile int*>(smem + L.misc + 12);
+    // FP8 / INT8: stage the per-row scales of this tile while the mainloop runs
+    if constexpr (C::kRowColScales) {
+      const float* sp = SWAP ? prm.scale_w : prm.scale_a;
+      const float* sq = SWAP ? prm.scale_a : prm.scale_w;
+      row_s[etid] = (p0 + etid < prm.rows_p) ? __ldg(sp + p0 + etid) : 0.f;
+      for (int c = etid; c < BN; c += 128) col_s[c] = (q0 + c < prm.rows_q) ? __ldg(sq + q0 + c) : 0.f;
+    }
     bool ok = true;                            // warp-uniform
     float acc_f[BN];                           // Block_FP8 promoted accumulator
     int wblocks = 1;
@@ -426,53 +467,124 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&tempty[b]);
       }
     } else {
-      if (nkt > 0) ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, prm.err));
+      ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, prm.err));
       tc_fence_after();
     }
     if (etid == 0) *flag_epi = 0;
-    named_bar_sync(1, 128);
+    named_bar_sync(1, 128);                    // also publishes the staged scales
     if (!ok) *flag_epi = 1;
     named_bar_sync(1, 128);
     const bool epi_ok = (*flag_epi == 0);      // uniform over the 128 epilogue threads
 
-    // ---- write out: direct epilogue, or this CTA's split-K partial
     const bool split = prm.split_k > 1;
     const int prow = p0 + row;                 // global row of P
     const bool prow_ok = prow < prm.rows_p;
     const size_t MN = (size_t)prm.M * prm.N;
     uint32_t* part = reinterpret_cast<uint32_t*>(prm.partial);
-    uint32_t* red = reinterpret_cast<uint32_t*>(smem + L.p);   // cluster reduction buffer
+    uint32_t* stage_buf = reinterpret_cast<uint32_t*>(smem + L.p);   // ring, idle now
     const float alpha = alpha_of<FMT>(prm);
+    // Accumulator chunk c0..c0+15 of this thread's row.
+    auto load_chunk = [&](int c0, uint32_t (&v)[16]) {
+      if constexpr (C::kBlock) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(acc_f[c0 + j]);
+      } else {
+        tmem_ld16(lane_addr + c0, v);
+        tmem_ld_wait();
+      }
+    };
 
-    if (epi_ok) {
+    if (!split) {
+      // ---- direct epilogue
+      if (epi_ok) {
 #pragma unroll
-      for (int c0 = 0; c0 < BN; c0 += 16) {
-        uint32_t v[16];
-        if constexpr (C::kBlock) {
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          uint32_t v[16];
+          load_chunk(c0, v);
+          if (prow_ok) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(acc_f[c0 + j]);
-        } else {
-          tmem_ld16(lane_addr + c0, v);
-          tmem_ld_wait();
-        }
-        if (split && prm.reduce_mode == kReduceCluster) {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) red[red_index<SWAP, BN>(row, c0 + j)] = v[j];
-        } else if (prow_ok) {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int m = SWAP ? q0 + c0 + j : prow;
-            const int n = SWAP ? prow : q0 + c0 + j;
-            if (m < prm.M && n < prm.N) {
-              if (split)
-                part[(size_t)kz * MN + (size_t)m * prm.N + n] = v[j];
-              else
-                emit<FMT>(prm, m, n, v[j], alpha);
+            for (int j = 0; j < 16; ++j) {
+              const int c = c0 + j;
+              const int m = SWAP ? q0 + c : prow;
+              const int n = SWAP ? prow : q0 + c;
+              if (m < prm.M && n < prm.N) emit<FMT, SWAP>(prm, row, c, m, n, v[j], alpha, row_s, col_s);
             }
           }
         }
       }
-      if (split && prm.reduce_mode == kReduceLastCta) {
+    } else if (cluster_red && C::kPush) {
+      // ---- cluster split-K, push: slice this partial by owner, bulk-copy
+      // each slice into its owner's receive slot `kz`, then reduce the slices
+      // this CTA owns.
+      const int owner = row / rows_per, rl = row % rows_per;
+      uint32_t* my_slice = stage_buf + owner * (rows_per * BN);
+      if (epi_ok) {
+#pragma unroll
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          uint32_t v[16];
+          load_chunk(c0, v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) my_slice[slice_index<SWAP, BN>(rl, c0 + j, rows_per)] = v[j];
+        }
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      cluster_wait();                          // phase 1: every receiver is initialised
+      if (etid == 0) {
+        const uint32_t recv_s = smem_u32(smem + L.recv) + (uint32_t)kz * slot_bytes;
+        const uint32_t stage_s = smem_u32(stage_buf);
+        const uint32_t bar_s = smem_u32(recv_full);
+        for (int o = 0; o < prm.split_k; ++o)
+          bulk_s2s_cluster(mapa_shared(recv_s, (uint32_t)o), stage_s + (uint32_t)o * slot_bytes,
+                           slot_bytes, mapa_shared(bar_s, (uint32_t)o));
+        bulk_commit();
+      }
+      const bool got = __all_sync(0xffffffffu, mbar_wait(recv_full, 0, prm.err));
+      const uint32_t* recv = reinterpret_cast<const uint32_t*>(smem + L.recv);
+      const int r0 = (int)cluster_ctarank() * rows_per;
+      if (epi_ok && got) {
+        for (int idx = etid; idx < rows_per * BN; idx += 128) {
+          int rl2, c;
+          if (SWAP) { rl2 = idx % rows_per; c = idx / rows_per; }
+          else      { rl2 = idx / BN;       c = idx % BN; }
+          uint32_t acc = 0u;
+          for (int z = 0; z < prm.split_k; ++z)
+            acc = add_acc<FMT>(acc, recv[z * rows_per * BN + slice_index<SWAP, BN>(rl2, c, rows_per)]);
+          const int r = r0 + rl2;
+          const int m = SWAP ? q0 + c : p0 + r;
+          const int n = SWAP ? p0 + r : q0 + c;
+          if (m < prm.M && n < prm.N) emit<FMT, SWAP>(prm, r, c, m, n, acc, alpha, row_s, col_s);
+        }
+      }
+      if (etid == 0) bulk_wait_read_all();     // our slices have left shared memory
+    } else if (cluster_red) {
+      // ---- cluster split-K, pull: stage the partial in the idle ring; the
+      // reduction runs after the cluster barrier below
+      if (epi_ok) {
+#pragma unroll
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          uint32_t v[16];
+          load_chunk(c0, v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) stage_buf[red_index<SWAP, BN>(row, c0 + j)] = v[j];
+        }
+      }
+    } else if (epi_ok) {
+      // ---- workspace split-K: partial to global memory
+#pragma unroll
+      for (int c0 = 0; c0 < BN; c0 += 16) {
+        uint32_t v[16];
+        load_chunk(c0, v);
+        if (prow_ok) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int m = SWAP ? q0 + c0 + j : prow;
+            const int n = SWAP ? prow : q0 + c0 + j;
+            if (m < prm.M && n < prm.N) part[(size_t)kz * MN + (size_t)m * prm.N + n] = v[j];
+          }
+        }
+      }
+      if (prm.reduce_mode == kReduceLastCta) {
         // Last-arriving CTA of this output tile sums the partials in split
         // order (deterministic) and applies the epilogue.
         __threadfence();
@@ -506,9 +618,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
 #pragma unroll
               for (int j = 0; j < 16; ++j) {
-                const int m = SWAP ? q0 + c0 + j : prow;
-                const int n = SWAP ? prow : q0 + c0 + j;
-                if (m < prm.M && n < prm.N) emit<FMT>(prm, m, n, acc[j], alpha);
+                const int c = c0 + j;
+                const int m = SWAP ? q0 + c : prow;
+                const int n = SWAP ? prow : q0 + c;
+                if (m < prm.M && n < prm.N) emit<FMT, SWAP>(prm, row, c, m, n, acc[j], alpha, row_s, col_s);
               }
             }
           }
@@ -518,44 +631,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  // ------------------------------------------ split-K reduction in the cluster
-  // The split_k CTAs of one output tile form a cluster; after every CTA has
-  // left its partial tile in its own shared memory, CTA r sums rows
-  // [r*128/S, (r+1)*128/S) of all S partials through distributed shared
-  // memory, in split order, and stores them.  Every thread of every CTA takes
-  // both cluster barriers.
-  if (prm.split_k > 1 && prm.reduce_mode == kReduceCluster) {
+  // ------------------------------------------------ cluster barrier phases
+  // Phase 1 was arrived at after set-up; push-mode epilogue warps have
+  // already waited on it.  Pull mode adds phase 2 (every partial staged) and
+  // phase 3 (every remote read done) around the reduction.
+  if (cluster_red) {
     __syncwarp();
-    cluster_sync();
-    if (warp >= 2 && *reinterpret_cast<volatile int*>(smem + L.misc + 12) == 0) {
-      const int etid = threadIdx.x - 64;
-      const int S = prm.split_k;
-      const uint32_t rank = cluster_ctarank();
-      const int rows_per = 128 / S;
-      const int r0 = (int)rank * rows_per;
-      const uint32_t red_s = smem_u32(smem + L.p);
-      const float alpha = alpha_of<FMT>(prm);
-      for (int idx = etid; idx < rows_per * BN; idx += 128) {
-        int r, c;
-        if (SWAP) { r = r0 + idx % rows_per; c = idx / rows_per; }   // consecutive threads: consecutive n
-        else      { r = r0 + idx / BN;       c = idx % BN; }         // consecutive threads: consecutive n
-        const uint32_t off = 4u * (uint32_t)red_index<SWAP, BN>(r, c);
-        uint32_t t[16];
-        uint32_t acc = 0u;
+    if (!(C::kPush && warp >= 2)) cluster_wait();
+    if constexpr (!C::kPush) {
+      cluster_sync();
+      if (warp >= 2 && *flag_epi == 0) {
+        const int etid = threadIdx.x - 64;
+        const int Sk = prm.split_k;
+        const uint32_t rank = cluster_ctarank();
+        const int r0 = (int)rank * rows_per;
+        const uint32_t red_s = smem_u32(smem + L.p);
+        const float alpha = alpha_of<FMT>(prm);
+        for (int idx = etid; idx < rows_per * BN; idx += 128) {
+          int r, c;
+          if (SWAP) { r = r0 + idx % rows_per; c = idx / rows_per; }
+          else      { r = r0 + idx / BN;       c = idx % BN; }
+          const uint32_t off = 4u * (uint32_t)red_index<SWAP, BN>(r, c);
+          uint32_t t[kMaxClusterSplit];
+          uint32_t acc = 0u;
 #pragma unroll
-        for (int z = 0; z < 16; ++z)
-          if (z < S) t[z] = ld_dsmem_u32(mapa_shared(red_s + off, (uint32_t)z));
+          for (int z = 0; z < kMaxClusterSplit; ++z)
+            if (z < Sk) t[z] = ld_dsmem_u32(mapa_shared(red_s + off, (uint32_t)z));
 #pragma unroll
-        for (int z = 0; z < 16; ++z)
-          if (z < S) acc = add_acc<FMT>(acc, t[z]);
-        const int prow = p0 + r;
-        const int m = SWAP ? q0 + c : prow;
-        const int n = SWAP ? prow : q0 + c;
-        if (m < prm.M && n < prm.N) emit<FMT>(prm, m, n, acc, alpha);
+          for (int z = 0; z < kMaxClusterSplit; ++z)
+            if (z < Sk) acc = add_acc<FMT>(acc, t[z]);
+          const int m = SWAP ? q0 + c : p0 + r;
+          const int n = SWAP ? p0 + r : q0 + c;
+          if (m < prm.M && n < prm.N) emit<FMT, SWAP>(prm, r, c, m, n, acc, alpha, row_s, col_s);
+        }
       }
+      __syncwarp();
+      cluster_sync();
     }
-    __syncwarp();
-    cluster_sync();
   }
 
   // ------------------------------------------------------------------ teardown

@@ -121,8 +121,10 @@ __global__ void __launch_bounds__(kQThreads) quant_rows_kernel(const __nv_bfloat
                                                                int K, int ldx, uint8_t* __restrict__ q,
                                                                float* __restrict__ scale) {
   __shared__ float red[32];
-  griddep_wait();
+  // let the next kernel (the GEMM) start streaming its weights now; it
+  // waits for this kernel's completion before it reads what we write
   griddep_launch_dependents();
+  griddep_wait();
   const int r = blockIdx.x;
   const uint4* row = reinterpret_cast<const uint4*>(X + (size_t)r * ldx);
   const int nch = K / 8;
@@ -168,8 +170,10 @@ __global__ void __launch_bounds__(kQThreads) quant_rows_kernel(const __nv_bfloat
 __global__ void __launch_bounds__(kQThreads) quant_act_groups_kernel(
     const __nv_bfloat16* __restrict__ X, int M, int K, int ldx, uint8_t* __restrict__ q,
     float* __restrict__ scale) {
-  griddep_wait();
+  // let the next kernel (the GEMM) start streaming its weights now; it
+  // waits for this kernel's completion before it reads what we write
   griddep_launch_dependents();
+  griddep_wait();
   const int G = K / 128;
   const long long gid = (long long)blockIdx.x * (kQThreads / 16) + (threadIdx.x >> 4);
   const int sub = threadIdx.x & 15;
@@ -200,8 +204,10 @@ __global__ void __launch_bounds__(kQThreads) quant_weight_blocks_kernel(
     const __nv_bfloat16* __restrict__ W, int N, int K, uint8_t* __restrict__ q,
     float* __restrict__ scale) {
   __shared__ float red[32];
-  griddep_wait();
+  // let the next kernel (the GEMM) start streaming its weights now; it
+  // waits for this kernel's completion before it reads what we write
   griddep_launch_dependents();
+  griddep_wait();
   const int G = K / 128;
   const int nb = blockIdx.x / G, g = blockIdx.x % G;
   float x[8][8];
@@ -237,6 +243,7 @@ __global__ void __launch_bounds__(kQThreads) nvfp4_amax_kernel(const __nv_bfloat
                                                                int R, int K, int ldx,
                                                                float* __restrict__ partial) {
   __shared__ float red[32];
+  griddep_launch_dependents();
   griddep_wait();
   const int nch = K / 8;
   const long long total = (long long)R * nch;
@@ -250,7 +257,6 @@ __global__ void __launch_bounds__(kQThreads) nvfp4_amax_kernel(const __nv_bfloat
   }
   amax = block_max(amax, red);
   if (threadIdx.x == 0) partial[blockIdx.x] = amax;
-  griddep_launch_dependents();
 }
 
 // Phase 2: one thread per 16-element block (r, c) of the padded scale
@@ -261,8 +267,10 @@ __global__ void __launch_bounds__(kQThreads) nvfp4_quant_kernel(
     int npartial, const float* __restrict__ static_amax, uint8_t* __restrict__ q,
     uint8_t* __restrict__ sf, float* __restrict__ gscale, int R_pad, int C) {
   __shared__ float red[32];
-  griddep_wait();
+  // let the next kernel (the GEMM) start streaming its weights now; it
+  // waits for this kernel's completion before it reads what we write
   griddep_launch_dependents();
+  griddep_wait();
   float amax_t = 0.f;
   if (static_amax != nullptr) {
     amax_t = __ldg(static_amax);

@@ -22,6 +22,8 @@ channel) explicitly.
 """
 from __future__ import annotations
 
+import os
+
 import numpy as np
 
 _GAMMA = np.uint64(0x9E3779B97F4A7C15)
@@ -74,9 +76,27 @@ def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
 
 
 def bf16_matrix(seed: int, rows: int, cols: int, std: float) -> np.ndarray:
-    """A [rows, cols] matrix of bf16 values, returned as uint16 bit patterns."""
-    z = normal_fp64(seed, rows * cols) * std
-    return f32_to_bf16_bits(z.astype(np.float32)).reshape(rows, cols)
+    """A [rows, cols] matrix of bf16 values, returned as uint16 bit patterns.
+    Large matrices are drawn in independent chunks on a thread pool; element
+    i is always normal i of the stream, so the result does not depend on the
+    chunking."""
+    n = rows * cols
+    out = np.empty(n, dtype=np.uint16)
+    chunk = 1 << 22
+
+    def fill(start):
+        cnt = min(chunk, n - start)
+        z = normal_fp64(seed, cnt, start) * std
+        out[start:start + cnt] = f32_to_bf16_bits(z.astype(np.float32))
+
+    starts = range(0, n, chunk)
+    if n <= chunk:
+        fill(0)
+    else:
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 4)) as ex:
+            list(ex.map(fill, starts))
+    return out.reshape(rows, cols)
 
 
 def activations(M: int, K: int, seed: int = SEED_A) -> np.ndarray:
