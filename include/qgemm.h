@@ -179,8 +179,9 @@ qg_status qgemm_quantize_weight(qg_format f, const void* W, int N, int K, qg_ope
  *      ldy >= N, ldy * elem a multiple of 16 bytes.
  *   workspace: qgemm_workspace_size(f, M, N, K, cfg) bytes (NULL if 0).
  * Epilogue: y = acc * s_a[m] * s_w[n] (FP8_DYNAMIC, W8A8_INT8; int32 acc
- * converted to fp32 first), per-group promotion acc += (p_g * s_a[m,g]) *
- * s_w[n/128,g] (BLOCK_FP8), y = acc * (g_a * g_w) (NVFP4); all in fp32, then
+ * converted to fp32 first), per-group promotion acc += p_g
+ * (s_a[m,g] * s_w[n/128,g]) as one fp32 FMA per element (BLOCK_FP8),
+ * y = acc * (g_a * g_w) (NVFP4); all in fp32, then
  * bf16 round-to-nearest-even.  Returns QG_ERR_UNSUPPORTED for a config the
  * kernels do not implement (e.g. split_k larger than the number of 128-byte
  * K tiles) and QG_ERR_WORKSPACE if ws_bytes is too small.
@@ -265,6 +266,17 @@ qg_status qgemm_device_error(void);
 /* Enables (1) or disables (0) programmatic dependent launch for the
  * library's kernels (default 1). */
 void qgemm_set_pdl(int enable);
+/* Tracing (debug): while set, every qgemm_run whose grid fits records, per
+ * CTA, 12 GPU-clock timestamps (%globaltimer, ns, 64-bit) into the device
+ * buffer: entry, set-up done, first weight tile issued, dependency wait
+ * returned, first stage landed, last MMA committed, accumulator ready, stores
+ * done, and for cluster split-K: partial pushed, owned slices received,
+ * owned rows reduced (word 11 unused); CTA c = (z * gridDim.y + y) *
+ * gridDim.x + x writes words [12c, 12c+12).
+ * Launches whose grid needs more than `bytes` are not traced.  NULL turns
+ * tracing off.  Not thread-safe; meant for profiling runs. */
+void qgemm_set_trace(void* device_buffer, size_t bytes);
+
 /* ABI version of the loaded library (QGEMM_ABI_VERSION). */
 int qgemm_abi_version(void);
 

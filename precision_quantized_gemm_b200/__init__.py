@@ -41,7 +41,7 @@ EXPORTS = [
     "qgemm_quantize_act", "qgemm_quantize_weight", "qgemm_run", "qgemm_default_config",
     "qgemm_table_load", "qgemm_table_create", "qgemm_table_put", "qgemm_table_save",
     "qgemm_table_free", "qgemm_table_size", "qgemm_dispatch", "qgemm_tune", "qgemm_device_error",
-    "qgemm_run_noalloc",
+    "qgemm_run_noalloc", "qgemm_set_trace",
 ]
 
 
@@ -108,6 +108,7 @@ def lib() -> ctypes.CDLL:
             "qgemm_dispatch": (c_int, [c_void_p, c_int, c_int, c_int, c_int, POINTER(qg_config), POINTER(c_int)]),
             "qgemm_tune": (c_int, [c_void_p, c_int, POINTER(c_int), c_int, POINTER(c_int), c_int, c_double, c_int]),
             "qgemm_device_error": (c_int, []),
+            "qgemm_set_trace": (None, [c_void_p, c_size_t]),
             "qgemm_run_noalloc": (c_int, [c_int, POINTER(qg_operand), POINTER(qg_operand), c_int, c_int, c_int,
                                           POINTER(qg_config), c_void_p, c_int, c_int, c_void_p]),
         }
@@ -185,6 +186,11 @@ def qgemm_dispatch(table, fmt, M, N, K):
 
 def qgemm_device_error():
     return lib().qgemm_device_error()
+
+
+def qgemm_set_trace(buf_ptr, nbytes):
+    """Debug: record per-CTA phase timestamps of later launches into a device buffer."""
+    lib().qgemm_set_trace(buf_ptr, nbytes)
 
 
 def qgemm_set_pdl(enable: bool):

@@ -21,6 +21,8 @@ namespace {
 using qg::GemmParams;
 
 bool g_pdl = true;
+unsigned long long* g_trace = nullptr;   // debug phase trace buffer (device)
+size_t g_trace_bytes = 0;
 
 constexpr int kMaxDevices = 64;
 struct DeviceInfo {
@@ -131,10 +133,11 @@ qg_status check_config(qg_format f, int M, int N, int K, const qg_config* c) {
   if (c->reduce_mode < 0 || c->reduce_mode > 2) return QG_ERR_INVALID_ARG;
   const int tn = c->tile_n;
   if (tn != 16 && tn != 32 && tn != 64 && tn != 128 && tn != 256) return QG_ERR_UNSUPPORTED;
-  if (f == QG_BLOCK_FP8 && tn > 128) return QG_ERR_UNSUPPORTED;
-  // NVFP4 block scales of the N operand sit in 32-lane TMEM words: a 16-row
-  // tile must start at a multiple of 32 rows, i.e. be the only tile.
-  if (f == QG_NVFP4 && tn == 16 && (c->swap_ab ? M : N) > 16) return QG_ERR_UNSUPPORTED;
+  // NVFP4 block scales of the N operand sit in TMEM words of 32 rows, and the
+  // scale address an MMA takes must be an even word: a tile narrower than 64
+  // rows must be the only tile (a 16-row tile at row 16, or a 32-row tile at
+  // row 32, would start inside a word or at an odd one).
+  if (f == QG_NVFP4 && tn < 64 && (c->swap_ab ? M : N) > tn) return QG_ERR_UNSUPPORTED;
   if (c->stages < 2 || c->stages > 12) return QG_ERR_UNSUPPORTED;
   const int kt = kt_total(f, K);
   if (c->split_k > kt) return QG_ERR_UNSUPPORTED;
@@ -167,6 +170,11 @@ extern "C" {
 int qgemm_abi_version(void) { return QGEMM_ABI_VERSION; }
 
 void qgemm_set_pdl(int enable) { g_pdl = enable != 0; }
+
+void qgemm_set_trace(void* device_buffer, size_t bytes) {
+  g_trace = static_cast<unsigned long long*>(device_buffer);
+  g_trace_bytes = device_buffer ? bytes : 0;
+}
 
 const char* qgemm_status_string(qg_status s) {
   switch (s) {
@@ -357,6 +365,9 @@ qg_status qgemm_run(qg_format f, const qg_operand* A, const qg_operand* W, int M
   }
   prm.reduce_mode = cfg->reduce_mode;
   prm.err = d->err;
+  if (g_trace != nullptr &&
+      (size_t)tp * tq * cfg->split_k * qg::kTraceEvents * sizeof(unsigned long long) <= g_trace_bytes)
+    prm.trace = g_trace;
 
   const void* base_p = swap ? W->q : A->q;
   const void* base_q = swap ? A->q : W->q;
@@ -399,7 +410,7 @@ qg_status qgemm_default_config(qg_format f, int M, int N, int K, qg_config* out)
   if (c.swap_ab) {
     c.tile_n = M <= 16 ? 16 : M <= 32 ? 32 : 64;
   } else {
-    c.tile_n = f == QG_BLOCK_FP8 ? 128 : 256;
+    c.tile_n = 256;
   }
   // deepest pipeline that fits, at most 8 stages
   c.stages = 2;

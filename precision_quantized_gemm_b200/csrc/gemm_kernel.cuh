@@ -38,7 +38,6 @@ namespace qg {
 
 enum Fmt : int { kFP8 = 0, kINT8 = 1, kBLOCK = 2, kNVF4 = 3 };
 
-constexpr int kThreads = 192;
 constexpr int kKTileBytes = 128;     // bytes of K per pipeline stage (one 128B swizzle row)
 constexpr int kPTileBytes = 128 * kKTileBytes;
 constexpr int kSfAtomBytes = 512;    // one 128x4 atom of e4m3 block scales
@@ -70,7 +69,31 @@ struct GemmParams {
   unsigned int* counters;      // split-K per-tile arrival counters
   int reduce_mode;             // kReduce*
   unsigned int* err;           // device error word
+  unsigned long long* trace;   // optional: kTraceEvents timestamps per CTA (ns)
 };
+
+// Phase timestamps (%globaltimer, ns) a traced launch records per CTA.
+enum TraceEvent : int {
+  kTrEntry = 0,        // kernel entry
+  kTrReady = 1,        // barriers initialised, TMEM allocated
+  kTrFirstLoad = 2,    // producer issued its first weight tile
+  kTrDepWait = 3,      // producer returned from griddepcontrol.wait
+  kTrFirstFull = 4,    // MMA issuer saw the first full stage
+  kTrLastMma = 5,      // MMA issuer committed its last MMA
+  kTrAccReady = 6,     // epilogue has the (promoted) accumulator
+  kTrDone = 7,         // epilogue finished its stores
+  kTrSent = 8,         // cluster split-K: partial rows pushed to their owners
+  kTrRecv = 9,         // cluster split-K: owned slices received
+  kTrReduced = 10,     // cluster split-K: owned rows summed into the output tile
+  kTrSpare = 11,
+  kTraceEvents = 12
+};
+__device__ __forceinline__ void trace_at(const GemmParams& prm, int ev) {
+  if (prm.trace != nullptr) {
+    const size_t cta = ((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+    prm.trace[cta * kTraceEvents + ev] = globaltimer();
+  }
+}
 
 template <int FMT, int BN>
 struct Cfg {
@@ -82,6 +105,15 @@ struct Cfg {
   static constexpr int kSfPBytes = kNvf4 ? 4 * kSfAtomBytes : 0;   // 4 K-atoms per 128B tile
   static constexpr int kSfQBytes = kNvf4 ? 4 * kSfAtomBytes * kSfQAtoms : 0;
   static constexpr int kNAcc = kBlock ? (BN >= 128 ? 2 : 4) : 1;  // TMEM accumulators
+  // Wide Block_FP8 tiles promote with 8 epilogue warps: two per 32-lane TMEM
+  // quarter, each owning half of the columns.
+  static constexpr int kEpiWarps = (kBlock && BN >= 128) ? 8 : 4;
+  static constexpr int kEpiThreads = 32 * kEpiWarps;
+  static constexpr int kThreads = 64 + kEpiThreads;
+  static constexpr int kCols = BN / (kEpiWarps / 4);               // columns per epilogue thread
+  // CTAs per SM the register budget must allow: narrow (decode) tiles keep
+  // room for the next launch's CTAs to start streaming weights early.
+  static constexpr int kMinBlocks = (!kBlock && BN <= 64) ? 3 : (kBlock && BN <= 32) ? 2 : 1;
   static constexpr int kSfaCol = kNAcc * BN;                       // TMEM column of SF A
   static constexpr int kSfbCol = kSfaCol + 16;                     // 4 steps x 4 words
   static constexpr int kTmemUsed = kNvf4 ? kSfbCol + 16 * kSfQAtoms : kNAcc * BN;
@@ -128,16 +160,28 @@ __host__ inline size_t smem_bytes(int stages) {
 // Bytes a pull-mode cluster reduction stages in the (then idle) ring.
 template <bool SWAP, int BN>
 __host__ __device__ constexpr int red_bytes() {
-  return SWAP ? 4 * 128 * BN : 4 * 128 * (BN + 1);
+  return SWAP ? 4 * 128 * BN : 4 * 128 * (BN + 4);
 }
 // Position of accumulator element (row of P, column c) in the pull-mode
-// buffer: column-major for Swap-AB (rows are output channels, the contiguous
-// dimension of y), row-major with an odd row pitch otherwise.
+// buffer: the output-tile layout (channels contiguous, 16-byte aligned
+// groups of 8 along them).
 template <bool SWAP, int BN>
 __device__ __forceinline__ int red_index(int row, int c) {
-  return SWAP ? c * 128 + row : row * (BN + 1) + c;
+  return SWAP ? c * 128 + row : row * (BN + 4) + c;
 }
-// Push mode: CTA `owner` receives rows [owner*rows_per, (owner+1)*rows_per)
+// Output tile: element (row r of P, column c) of the raw accumulator tile.
+// Swap-AB keeps channels (r) contiguous, the standard orientation keeps
+// channels (c) contiguous with a padded row pitch; both are 16-byte aligned
+// for every 8-element group along the contiguous dimension.
+template <bool SWAP, int BN>
+__device__ __forceinline__ int tile_index(int r, int c) {
+  return SWAP ? c * 128 + r : r * (BN + 4) + c;
+}
+template <bool SWAP, int BN>
+__host__ __device__ constexpr int tile_bytes() {
+  return SWAP ? 4 * 128 * BN : 4 * 128 * (BN + 4);
+}
+// Push mode (standard orientation): CTA `owner` receives rows [owner*rows_per, (owner+1)*rows_per)
 // of every split's partial; slot z holds split z's slice, laid out so the
 // owner's final stores are coalesced.
 template <bool SWAP, int BN>
@@ -200,7 +244,7 @@ __device__ __forceinline__ void emit(const GemmParams& prm, int r, int c, int m,
 }
 
 template <int FMT, bool SWAP, int BN>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBlocks)
     qgemm_kernel(const __grid_constant__ CUtensorMap tmap_p,
                  const __grid_constant__ CUtensorMap tmap_q, const GemmParams prm) {
   using C = Cfg<FMT, BN>;
@@ -230,6 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kt_begin = (int)(((long long)kz * prm.kt_total) / prm.split_k);
   const int kt_end = (int)(((long long)(kz + 1) * prm.kt_total) / prm.split_k);
   const int nkt = kt_end - kt_begin;
+  if (threadIdx.x == 0) trace_at(prm, kTrEntry);
   const bool cluster_red = prm.split_k > 1 && prm.reduce_mode == kReduceCluster;
   const int rows_per = 128 / prm.split_k;                  // cluster mode: rows owned per CTA
   const uint32_t slot_bytes = 4u * (uint32_t)(rows_per * BN);
@@ -244,12 +289,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(acc_full, 1);
     for (int i = 0; i < 4; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 4);
+      mbar_init(&tempty[i], C::kEpiWarps);
     }
-    mbar_init(recv_full, 1);
+    // push mode: each of the 128 rows of the owned slices arrives once, from
+    // whichever CTA computed it (split_k CTAs x 128/split_k rows)
+    mbar_init(recv_full, 128);
     *flag_abort = 0;
     fence_barrier_init();
-    if (C::kPush && cluster_red) mbar_arrive_expect_tx(recv_full, (uint32_t)prm.split_k * slot_bytes);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::kTmemCols);
@@ -259,6 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  if (threadIdx.x == 0) trace_at(prm, kTrReady);
   // Cluster phase 1 (arrive now, wait before the first remote access): the
   // barriers of every CTA in the cluster are initialised.
   if (cluster_red) cluster_arrive();
@@ -326,8 +373,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < pre; ++i) {
         mbar_arrive_expect_tx(&full[i], stage_tx);
         load_w(i);
+        if (i == 0) trace_at(prm, kTrFirstLoad);
       }
       griddep_wait();
+      trace_at(prm, kTrDepWait);
       for (int i = 0; i < pre; ++i) load_a(i);
       bool ok = true;
       int issued = pre;
@@ -360,6 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < nkt; ++i) {
         const int st = i % S;
         if (*flag_abort || !mbar_wait(&full[st], (i / S) & 1, prm.err)) { *flag_abort = 1; break; }
+        if (i == 0) trace_at(prm, kTrFirstFull);
         uint32_t d_t = tmem_base;
         if constexpr (C::kBlock) {
           const int b = i % C::kNAcc;
@@ -395,24 +445,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (C::kBlock) mma_commit(&tfull[i % C::kNAcc]);
       }
       if constexpr (!C::kBlock) mma_commit(acc_full);
+      trace_at(prm, kTrLastMma);
     }
   } else {
     // --------------------------------------------------------------- epilogue
+    constexpr int EW = C::kEpiWarps;
+    constexpr int ET = C::kEpiThreads;
+    constexpr int NC = C::kCols;
+    constexpr int CW = NC >= 32 ? 32 : NC;     // accumulator columns per TMEM load
     const int quarter = warp & 3;              // TMEM lanes this warp may access
     const int row = quarter * 32 + lane;       // row of P in the tile
-    const int etid = threadIdx.x - 64;         // 0..127
+    const int etid = threadIdx.x - 64;         // 0..ET-1
+    const int cbeg = ((warp - 2) / 4) * NC;    // this thread's columns [cbeg, cbeg + NC)
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
     griddep_wait();                            // scales/partials of earlier kernels
     // FP8 / INT8: stage the per-row scales of this tile while the mainloop runs
     if constexpr (C::kRowColScales) {
       const float* sp = SWAP ? prm.scale_w : prm.scale_a;
       const float* sq = SWAP ? prm.scale_a : prm.scale_w;
-      row_s[etid] = (p0 + etid < prm.rows_p) ? __ldg(sp + p0 + etid) : 0.f;
-      for (int c = etid; c < BN; c += 128) col_s[c] = (q0 + c < prm.rows_q) ? __ldg(sq + q0 + c) : 0.f;
+      for (int r = etid; r < 128; r += ET) row_s[r] = (p0 + r < prm.rows_p) ? __ldg(sp + p0 + r) : 0.f;
+      for (int c = etid; c < BN; c += ET) col_s[c] = (q0 + c < prm.rows_q) ? __ldg(sq + q0 + c) : 0.f;
     }
     bool ok = true;                            // warp-uniform
-    float acc_f[BN];                           // Block_FP8 promoted accumulator
-    int wblocks = 1;
+    float acc_f[NC];                           // Block_FP8 promoted accumulator
     if constexpr (C::kBlock) {
       float* sa_s = reinterpret_cast<float*>(smem + L.scales);          // act scales
       float* sw_s = sa_s + kMaxScaleStage;                              // weight scales
@@ -422,44 +477,53 @@ __global__ void __launch_bounds__(kThreads, 1)
       // (128-row block, group).
       const int act_rows = SWAP ? BN : 128;
       const int act_base = SWAP ? q0 : p0;
-      for (int idx = etid; idx < act_rows * nkt; idx += 128) {
+      for (int idx = etid; idx < act_rows * nkt; idx += ET) {
         const int r = idx / nkt, gl = idx % nkt;
         const int m = act_base + r;
         sa_s[idx] = (m < prm.M) ? __ldg(prm.scale_a + (size_t)m * G + g0 + gl) : 0.f;
       }
-      wblocks = SWAP ? 1 : (BN > 128 ? 2 : 1);
+      constexpr int WB = (!SWAP && BN > 128) ? 2 : 1;                   // weight blocks per tile
       const int wrow0 = (SWAP ? p0 : q0) / 128;
       const int nblk = (prm.N + 127) / 128;
-      for (int idx = etid; idx < wblocks * nkt; idx += 128) {
-        const int gl = idx / wblocks, jb = idx % wblocks;
+      for (int idx = etid; idx < WB * nkt; idx += ET) {
+        const int gl = idx / WB, jb = idx % WB;
         const int b = wrow0 + jb;
         sw_s[idx] = (b < nblk) ? __ldg(prm.scale_w + (size_t)b * G + g0 + gl) : 0.f;
       }
-      named_bar_sync(1, 128);
+      named_bar_sync(1, ET);
 #pragma unroll
-      for (int c = 0; c < BN; ++c) acc_f[c] = 0.f;
+      for (int c = 0; c < NC; ++c) acc_f[c] = 0.f;
       for (int i = 0; i < nkt; ++i) {
         const int b = i % C::kNAcc;
         ok = __all_sync(0xffffffffu, mbar_wait(&tfull[b], (i / C::kNAcc) & 1, prm.err));
         if (!ok) break;
         tc_fence_after();
+        // acc += p_g * (s_a * s_w): one FMA per element
+        float f_row = 0.f;
+        if (!SWAP) f_row = sa_s[row * nkt + i];
+        // 64 columns per TMEM round trip (two 32-column loads, one wait)
 #pragma unroll
-        for (int c0 = 0; c0 < BN; c0 += 16) {
-          uint32_t v[16];
-          tmem_ld16(lane_addr + b * BN + c0, v);
+        for (int c0 = 0; c0 < NC; c0 += 64) {
+          uint32_t v[64];
+          if constexpr (NC % 32 == 0) {
+            tmem_ld32(lane_addr + b * BN + cbeg + c0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+            if (c0 + 32 < NC)
+              tmem_ld32(lane_addr + b * BN + cbeg + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+          } else {                             // 16-column tiles: stay inside the buffer
+            tmem_ld16(lane_addr + b * BN + cbeg + c0, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
+          }
           tmem_ld_wait();
+          if (SWAP) {
+            const float sw = sw_s[i];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int c = c0 + j;
-            float sa, sw;
-            if (SWAP) {
-              sa = sa_s[c * nkt + i];
-              sw = sw_s[i];
-            } else {
-              sa = sa_s[row * nkt + i];
-              sw = sw_s[i * wblocks + (BN > 128 ? c / 128 : 0)];
+            for (int j = 0; j < 64 && c0 + j < NC; ++j)
+              acc_f[c0 + j] = fmaf(__uint_as_float(v[j]), sa_s[(cbeg + c0 + j) * nkt + i] * sw, acc_f[c0 + j]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 64 && c0 + j < NC; ++j) {
+              const float f = f_row * sw_s[i * WB + (WB == 2 ? (cbeg + c0 + j) / 128 : 0)];
+              acc_f[c0 + j] = fmaf(__uint_as_float(v[j]), f, acc_f[c0 + j]);
             }
-            acc_f[c] += (__uint_as_float(v[j]) * sa) * sw;
           }
         }
         tc_fence_before();
@@ -470,11 +534,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, prm.err));
       tc_fence_after();
     }
-    if (etid == 0) *flag_epi = 0;
-    named_bar_sync(1, 128);                    // also publishes the staged scales
+    if (etid == 0) {
+      *flag_epi = 0;
+      trace_at(prm, kTrAccReady);
+    }
+    named_bar_sync(1, ET);                     // also publishes the staged scales
     if (!ok) *flag_epi = 1;
-    named_bar_sync(1, 128);
-    const bool epi_ok = (*flag_epi == 0);      // uniform over the 128 epilogue threads
+    named_bar_sync(1, ET);
+    const bool epi_ok = (*flag_epi == 0);      // uniform over the epilogue threads
 
     const bool split = prm.split_k > 1;
     const int prow = p0 + row;                 // global row of P
@@ -483,103 +550,191 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t* part = reinterpret_cast<uint32_t*>(prm.partial);
     uint32_t* stage_buf = reinterpret_cast<uint32_t*>(smem + L.p);   // ring, idle now
     const float alpha = alpha_of<FMT>(prm);
-    // Accumulator chunk c0..c0+15 of this thread's row.
-    auto load_chunk = [&](int c0, uint32_t (&v)[16]) {
+    // Accumulator columns [cbeg + c0, cbeg + c0 + CW) of this thread's row.
+    auto load_chunk = [&](int c0, uint32_t (&v)[CW]) {
       if constexpr (C::kBlock) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(acc_f[c0 + j]);
+        for (int j = 0; j < CW; ++j) v[j] = __float_as_uint(acc_f[c0 + j]);
+      } else if constexpr (CW == 32) {
+        tmem_ld32(lane_addr + cbeg + c0, v);
+        tmem_ld_wait();
       } else {
-        tmem_ld16(lane_addr + c0, v);
+        tmem_ld16(lane_addr + cbeg + c0, v);
         tmem_ld_wait();
       }
     };
 
+    // Output tile in the idle ring: raw accumulator bits of tile element
+    // (r, c) at otile[tile_index(r, c)], written out by one compact loop that
+    // scales, converts and stores 16-byte vectors along the contiguous
+    // dimension of y (channels: r under Swap-AB, c otherwise).
+    uint32_t* otile = stage_buf;
+    auto write_out = [&](int r_begin, int r_count, int c_begin, int c_count) {
+      const int units = SWAP ? c_count * (r_count / 8) : r_count * (c_count / 8);
+      const bool vec = (prm.ldy % 8) == 0;
+#pragma unroll 1
+      for (int u = etid; u < units; u += ET) {
+        int r, c;                              // first of 8 consecutive output channels
+        if (SWAP) { c = c_begin + u / (r_count / 8); r = r_begin + (u % (r_count / 8)) * 8; }
+        else      { r = r_begin + u / (c_count / 8); c = c_begin + (u % (c_count / 8)) * 8; }
+        const int m = SWAP ? q0 + c : p0 + r;
+        const int n0 = SWAP ? p0 + r : q0 + c;
+        if (m >= prm.M || n0 >= prm.N) continue;
+        const uint4* src = reinterpret_cast<const uint4*>(otile + tile_index<SWAP, BN>(r, c));
+        const uint4 w0 = src[0], w1 = src[1];
+        const uint32_t acc8[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        if (prm.out_kind == 1) {
+          uint32_t* Yu = reinterpret_cast<uint32_t*>(prm.Y) + (size_t)m * prm.ldy;
+          for (int j = 0; j < 8 && n0 + j < prm.N; ++j) Yu[n0 + j] = acc8[j];
+          continue;
+        }
+        float y8[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float sa = 1.f, sw = 1.f;
+          if constexpr (FMT == kFP8 || FMT == kINT8) {
+            sa = SWAP ? col_s[c] : row_s[r];
+            sw = SWAP ? row_s[r + j] : col_s[c + j];
+          }
+          y8[j] = finish_value<FMT>(acc8[j], sa, sw, alpha);
+        }
+        __nv_bfloat16* Yb = reinterpret_cast<__nv_bfloat16*>(prm.Y) + (size_t)m * prm.ldy;
+        if (vec && n0 + 8 <= prm.N) {
+          uint32_t p[4];
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(y8[2 * h], y8[2 * h + 1]);
+            p[h] = *reinterpret_cast<const uint32_t*>(&b2);
+          }
+          *reinterpret_cast<uint4*>(Yb + n0) = make_uint4(p[0], p[1], p[2], p[3]);
+        } else {
+          for (int j = 0; j < 8 && n0 + j < prm.N; ++j) Yb[n0 + j] = __float2bfloat16_rn(y8[j]);
+        }
+      }
+    };
+
     if (!split) {
-      // ---- direct epilogue
+      // ---- direct: accumulator -> tile -> y
       if (epi_ok) {
 #pragma unroll
-        for (int c0 = 0; c0 < BN; c0 += 16) {
-          uint32_t v[16];
+        for (int c0 = 0; c0 < NC; c0 += CW) {
+          uint32_t v[CW];
           load_chunk(c0, v);
-          if (prow_ok) {
+          if constexpr (SWAP) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int c = c0 + j;
-              const int m = SWAP ? q0 + c : prow;
-              const int n = SWAP ? prow : q0 + c;
-              if (m < prm.M && n < prm.N) emit<FMT, SWAP>(prm, row, c, m, n, v[j], alpha, row_s, col_s);
-            }
+            for (int j = 0; j < CW; ++j) otile[tile_index<SWAP, BN>(row, cbeg + c0 + j)] = v[j];
+          } else {                             // row pitch BN+4: 16-byte stores
+#pragma unroll
+            for (int j = 0; j < CW; j += 4)
+              *reinterpret_cast<uint4*>(otile + tile_index<SWAP, BN>(row, cbeg + c0 + j)) =
+                  make_uint4(v[j], v[j + 1], v[j + 2], v[j + 3]);
           }
         }
       }
+      named_bar_sync(1, ET);
+      if (epi_ok) write_out(0, 128, 0, BN);
     } else if (cluster_red && C::kPush) {
-      // ---- cluster split-K, push: slice this partial by owner, bulk-copy
-      // each slice into its owner's receive slot `kz`, then reduce the slices
-      // this CTA owns.
+      // ---- cluster split-K, push: every thread stores its row of this
+      // partial straight from registers into the owning CTA's receive slot
+      // `kz` and arrives (release) on that CTA's barrier; each CTA sums the
+      // rows it owns, in split order, into the output tile.  Only real
+      // outputs cross the cluster: token columns < M under Swap-AB (decode
+      // tiles are mostly padding), token rows < M otherwise.
+      const int Sk = prm.split_k;
       const int owner = row / rows_per, rl = row % rows_per;
-      uint32_t* my_slice = stage_buf + owner * (rows_per * BN);
-      if (epi_ok) {
-#pragma unroll
-        for (int c0 = 0; c0 < BN; c0 += 16) {
-          uint32_t v[16];
-          load_chunk(c0, v);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) my_slice[slice_index<SWAP, BN>(rl, c0 + j, rows_per)] = v[j];
-        }
-      }
-      fence_proxy_async_smem();
-      named_bar_sync(1, 128);
+      const int cvalid = SWAP ? min(BN, prm.M - q0) : BN;
+      const bool rvalid = SWAP || (p0 + row < prm.M);
       cluster_wait();                          // phase 1: every receiver is initialised
-      if (etid == 0) {
-        const uint32_t recv_s = smem_u32(smem + L.recv) + (uint32_t)kz * slot_bytes;
-        const uint32_t stage_s = smem_u32(stage_buf);
-        const uint32_t bar_s = smem_u32(recv_full);
-        for (int o = 0; o < prm.split_k; ++o)
-          bulk_s2s_cluster(mapa_shared(recv_s, (uint32_t)o), stage_s + (uint32_t)o * slot_bytes,
-                           slot_bytes, mapa_shared(bar_s, (uint32_t)o));
-        bulk_commit();
-      }
-      const bool got = __all_sync(0xffffffffu, mbar_wait(recv_full, 0, prm.err));
-      const uint32_t* recv = reinterpret_cast<const uint32_t*>(smem + L.recv);
-      const int r0 = (int)cluster_ctarank() * rows_per;
-      if (epi_ok && got) {
-        for (int idx = etid; idx < rows_per * BN; idx += 128) {
-          int rl2, c;
-          if (SWAP) { rl2 = idx % rows_per; c = idx / rows_per; }
-          else      { rl2 = idx / BN;       c = idx % BN; }
-          uint32_t acc = 0u;
-          for (int z = 0; z < prm.split_k; ++z)
-            acc = add_acc<FMT>(acc, recv[z * rows_per * BN + slice_index<SWAP, BN>(rl2, c, rows_per)]);
-          const int r = r0 + rl2;
-          const int m = SWAP ? q0 + c : p0 + r;
-          const int n = SWAP ? p0 + r : q0 + c;
-          if (m < prm.M && n < prm.N) emit<FMT, SWAP>(prm, r, c, m, n, acc, alpha, row_s, col_s);
+      const uint32_t dst = mapa_shared(smem_u32(smem + L.recv) + (uint32_t)kz * slot_bytes, (uint32_t)owner);
+#pragma unroll
+      for (int c0 = 0; c0 < NC; c0 += CW) {
+        if (cbeg + c0 >= cvalid) break;
+        uint32_t v[CW];
+        if (epi_ok) {
+          load_chunk(c0, v);
+        } else {
+#pragma unroll
+          for (int j = 0; j < CW; ++j) v[j] = 0u;
+        }
+        if (SWAP) {                            // slice [c][rl]: one word per lane, lanes contiguous
+#pragma unroll
+          for (int j = 0; j < CW; ++j)
+            if (cbeg + c0 + j < cvalid)
+              st_dsmem_b32(dst + 4u * (uint32_t)slice_index<SWAP, BN>(rl, cbeg + c0 + j, rows_per), v[j]);
+        } else if (rvalid) {                   // slice [rl][c]: 16 bytes per store
+#pragma unroll
+          for (int j = 0; j < CW; j += 4)
+            st_dsmem_v4(dst + 4u * (uint32_t)slice_index<SWAP, BN>(rl, cbeg + c0 + j, rows_per), v[j], v[j + 1],
+                        v[j + 2], v[j + 3]);
         }
       }
-      if (etid == 0) bulk_wait_read_all();     // our slices have left shared memory
+      mbar_arrive_remote(mapa_shared(smem_u32(recv_full), (uint32_t)owner));
+      if (etid == 0) trace_at(prm, kTrSent);
+      const bool got = __all_sync(0xffffffffu, mbar_wait_cluster(recv_full, 0, prm.err));
+      if (etid == 0) trace_at(prm, kTrRecv);
+      const uint32_t* __restrict__ recv = reinterpret_cast<const uint32_t*>(smem + L.recv);
+      uint32_t* __restrict__ ot = otile;
+      const int r0 = (int)cluster_ctarank() * rows_per;
+      const int zstride = rows_per * BN;
+      if (epi_ok && got) {
+        // fixed per-thread row (Swap-AB) or column (standard), stepping over
+        // the other index: no divisions in the loop, loads of later
+        // iterations overlap
+        if (SWAP) {
+          const int rl2 = etid % rows_per, cstep = ET / rows_per;
+          const uint32_t recv_s = smem_u32(smem + L.recv);
+#pragma unroll 4
+          for (int c = etid / rows_per; c < cvalid; c += cstep) {
+            uint32_t acc = 0u;
+            for (int z = 0; z < Sk; ++z)
+              acc = add_acc<FMT>(acc, lds_u32(recv_s + 4u * (uint32_t)(z * zstride + c * rows_per + rl2)));
+            ot[tile_index<SWAP, BN>(r0 + rl2, c)] = acc;
+          }
+        } else {
+          const int nrow = max(0, min(rows_per, prm.M - p0 - r0));
+          const int c = etid % BN, rstep = ET / BN;
+#pragma unroll 4
+          for (int rl2 = etid / BN; rl2 < nrow; rl2 += rstep) {
+            uint32_t acc = 0u;
+            for (int z = 0; z < Sk; ++z) acc = add_acc<FMT>(acc, recv[z * zstride + rl2 * BN + c]);
+            ot[tile_index<SWAP, BN>(r0 + rl2, c)] = acc;
+          }
+        }
+      }
+      named_bar_sync(1, ET);
+      if (etid == 0) trace_at(prm, kTrReduced);
+      if (epi_ok && got) write_out(r0, rows_per, 0, BN);
     } else if (cluster_red) {
       // ---- cluster split-K, pull: stage the partial in the idle ring; the
       // reduction runs after the cluster barrier below
       if (epi_ok) {
 #pragma unroll
-        for (int c0 = 0; c0 < BN; c0 += 16) {
-          uint32_t v[16];
+        for (int c0 = 0; c0 < NC; c0 += CW) {
+          uint32_t v[CW];
           load_chunk(c0, v);
+          if constexpr (SWAP) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) stage_buf[red_index<SWAP, BN>(row, c0 + j)] = v[j];
+            for (int j = 0; j < CW; ++j) stage_buf[red_index<SWAP, BN>(row, cbeg + c0 + j)] = v[j];
+          } else {
+#pragma unroll
+            for (int j = 0; j < CW; j += 4)
+              *reinterpret_cast<uint4*>(stage_buf + red_index<SWAP, BN>(row, cbeg + c0 + j)) =
+                  make_uint4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+          }
         }
       }
     } else if (epi_ok) {
       // ---- workspace split-K: partial to global memory
 #pragma unroll
-      for (int c0 = 0; c0 < BN; c0 += 16) {
-        uint32_t v[16];
+      for (int c0 = 0; c0 < NC; c0 += CW) {
+        uint32_t v[CW];
         load_chunk(c0, v);
         if (prow_ok) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int m = SWAP ? q0 + c0 + j : prow;
-            const int n = SWAP ? prow : q0 + c0 + j;
+          for (int j = 0; j < CW; ++j) {
+            const int c = cbeg + c0 + j;
+            const int m = SWAP ? q0 + c : prow;
+            const int n = SWAP ? prow : q0 + c;
             if (m < prm.M && n < prm.N) part[(size_t)kz * MN + (size_t)m * prm.N + n] = v[j];
           }
         }
@@ -588,37 +743,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Last-arriving CTA of this output tile sums the partials in split
         // order (deterministic) and applies the epilogue.
         __threadfence();
-        named_bar_sync(1, 128);
+        named_bar_sync(1, ET);
         const unsigned tile = blockIdx.y * gridDim.x + blockIdx.x;
         if (etid == 0) {
           const unsigned prev = atomicAdd(&prm.counters[tile], 1u);
           *flag_last = (prev == (unsigned)(prm.split_k - 1));
         }
-        named_bar_sync(1, 128);
+        named_bar_sync(1, ET);
         if (*flag_last) {
           __threadfence();
           if (prow_ok) {
             // 16 columns at a time: all their loads of one split are issued
             // before any store, so the L2 round trips overlap.
 #pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 16) {
+            for (int c0 = 0; c0 < NC; c0 += 16) {
               uint32_t acc[16];
 #pragma unroll
               for (int j = 0; j < 16; ++j) acc[j] = 0u;
-              for (int z = 0; z < prm.split_k; ++z) {
-                uint32_t t[16];
+              // two splits per round: 32 loads in flight, summed in split order
+              for (int z0 = 0; z0 < prm.split_k; z0 += 2) {
+                uint32_t t[2][16];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                  const int m = SWAP ? q0 + c0 + j : prow;
-                  const int n = SWAP ? prow : q0 + c0 + j;
-                  t[j] = (m < prm.M && n < prm.N) ? ld_u32_cg(part + z * MN + (size_t)m * prm.N + n) : 0u;
+                for (int dz = 0; dz < 2; ++dz) {
+#pragma unroll
+                  for (int j = 0; j < 16; ++j) {
+                    const int c = cbeg + c0 + j;
+                    const int m = SWAP ? q0 + c : prow;
+                    const int n = SWAP ? prow : q0 + c;
+                    t[dz][j] = (z0 + dz < prm.split_k && m < prm.M && n < prm.N)
+                                   ? ld_u32_cg(part + (z0 + dz) * MN + (size_t)m * prm.N + n)
+                                   : 0u;
+                  }
                 }
 #pragma unroll
-                for (int j = 0; j < 16; ++j) acc[j] = add_acc<FMT>(acc[j], t[j]);
+                for (int dz = 0; dz < 2; ++dz)
+#pragma unroll
+                  for (int j = 0; j < 16; ++j)
+                    if (z0 + dz < prm.split_k) acc[j] = add_acc<FMT>(acc[j], t[dz][j]);
               }
 #pragma unroll
               for (int j = 0; j < 16; ++j) {
-                const int c = c0 + j;
+                const int c = cbeg + c0 + j;
                 const int m = SWAP ? q0 + c : prow;
                 const int n = SWAP ? prow : q0 + c;
                 if (m < prm.M && n < prm.N) emit<FMT, SWAP>(prm, row, c, m, n, acc[j], alpha, row_s, col_s);
@@ -647,22 +812,64 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r0 = (int)rank * rows_per;
         const uint32_t red_s = smem_u32(smem + L.p);
         const float alpha = alpha_of<FMT>(prm);
-        for (int idx = etid; idx < rows_per * BN; idx += 128) {
+        // units of 8 consecutive output channels: 2 x 16-byte remote loads per
+        // split, summed in split order, scaled and stored as one 16-byte vector
+        const int units = rows_per * BN / 8;
+        const bool vec = (prm.ldy % 8) == 0;
+#pragma unroll 1
+        for (int u = etid; u < units; u += C::kEpiThreads) {
           int r, c;
-          if (SWAP) { r = r0 + idx % rows_per; c = idx / rows_per; }
-          else      { r = r0 + idx / BN;       c = idx % BN; }
+          if (SWAP) { c = u / (rows_per / 8); r = r0 + (u % (rows_per / 8)) * 8; }
+          else      { r = r0 + u / (BN / 8); c = (u % (BN / 8)) * 8; }
           const uint32_t off = 4u * (uint32_t)red_index<SWAP, BN>(r, c);
-          uint32_t t[kMaxClusterSplit];
-          uint32_t acc = 0u;
+          uint4 t[kMaxClusterSplit][2];
 #pragma unroll
-          for (int z = 0; z < kMaxClusterSplit; ++z)
-            if (z < Sk) t[z] = ld_dsmem_u32(mapa_shared(red_s + off, (uint32_t)z));
+          for (int z = 0; z < kMaxClusterSplit; ++z) {
+            if (z < Sk) {
+              t[z][0] = ld_dsmem_v4(mapa_shared(red_s + off, (uint32_t)z));
+              t[z][1] = ld_dsmem_v4(mapa_shared(red_s + off + 16u, (uint32_t)z));
+            }
+          }
+          uint32_t acc8[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
 #pragma unroll
-          for (int z = 0; z < kMaxClusterSplit; ++z)
-            if (z < Sk) acc = add_acc<FMT>(acc, t[z]);
+          for (int z = 0; z < kMaxClusterSplit; ++z) {
+            if (z < Sk) {
+              const uint32_t w[8] = {t[z][0].x, t[z][0].y, t[z][0].z, t[z][0].w,
+                                     t[z][1].x, t[z][1].y, t[z][1].z, t[z][1].w};
+#pragma unroll
+              for (int j = 0; j < 8; ++j) acc8[j] = add_acc<FMT>(acc8[j], w[j]);
+            }
+          }
           const int m = SWAP ? q0 + c : p0 + r;
-          const int n = SWAP ? p0 + r : q0 + c;
-          if (m < prm.M && n < prm.N) emit<FMT, SWAP>(prm, r, c, m, n, acc, alpha, row_s, col_s);
+          const int n0 = SWAP ? p0 + r : q0 + c;
+          if (m >= prm.M || n0 >= prm.N) continue;
+          if (prm.out_kind == 1) {
+            uint32_t* Yu = reinterpret_cast<uint32_t*>(prm.Y) + (size_t)m * prm.ldy;
+            for (int j = 0; j < 8 && n0 + j < prm.N; ++j) Yu[n0 + j] = acc8[j];
+            continue;
+          }
+          float y8[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            float sa = 1.f, sw = 1.f;
+            if constexpr (FMT == kFP8 || FMT == kINT8) {
+              sa = SWAP ? col_s[c] : row_s[r];
+              sw = SWAP ? row_s[r + j] : col_s[c + j];
+            }
+            y8[j] = finish_value<FMT>(acc8[j], sa, sw, alpha);
+          }
+          __nv_bfloat16* Yb = reinterpret_cast<__nv_bfloat16*>(prm.Y) + (size_t)m * prm.ldy;
+          if (vec && n0 + 8 <= prm.N) {
+            uint32_t p[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const __nv_bfloat162 b2 = __floats2bfloat162_rn(y8[2 * h], y8[2 * h + 1]);
+              p[h] = *reinterpret_cast<const uint32_t*>(&b2);
+            }
+            *reinterpret_cast<uint4*>(Yb + n0) = make_uint4(p[0], p[1], p[2], p[3]);
+          } else {
+            for (int j = 0; j < 8 && n0 + j < prm.N; ++j) Yb[n0 + j] = __float2bfloat16_rn(y8[j]);
+          }
         }
       }
       __syncwarp();
@@ -673,6 +880,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ------------------------------------------------------------------ teardown
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) trace_at(prm, kTrDone);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);

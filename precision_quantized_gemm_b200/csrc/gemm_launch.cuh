@@ -21,7 +21,7 @@ cudaError_t launch_one(const CUtensorMap& tp, const CUtensorMap& tq, const GemmP
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(Cfg<FMT, BN>::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
@@ -52,9 +52,7 @@ cudaError_t launch_bn(int bn, const CUtensorMap& tp, const CUtensorMap& tq, cons
     case 32: return launch_one<FMT, SWAP, 32>(tp, tq, prm, grid, st, pdl);
     case 64: return launch_one<FMT, SWAP, 64>(tp, tq, prm, grid, st, pdl);
     case 128: return launch_one<FMT, SWAP, 128>(tp, tq, prm, grid, st, pdl);
-    case 256:
-      if constexpr (FMT != kBLOCK) return launch_one<FMT, SWAP, 256>(tp, tq, prm, grid, st, pdl);
-      return cudaErrorInvalidValue;
+    case 256: return launch_one<FMT, SWAP, 256>(tp, tq, prm, grid, st, pdl);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -78,14 +76,24 @@ bool cluster_fits_for(int bn, bool swap, int stages) {
   }
 }
 
+// Shared memory of a configuration; configurations whose output tile does
+// not fit the pipeline ring (reused by the epilogue) report an impossible size.
+template <int FMT, int BN>
+size_t smem_checked(int stages) {
+  using C = Cfg<FMT, BN>;
+  const size_t ring = (size_t)stages * (kPTileBytes + C::kQTileBytes);
+  if ((size_t)tile_bytes<false, BN>() > ring) return (size_t)1 << 30;
+  return smem_bytes<FMT, BN>(stages);
+}
+
 template <int FMT>
 size_t smem_for(int bn, int stages) {
   switch (bn) {
-    case 16: return smem_bytes<FMT, 16>(stages);
-    case 32: return smem_bytes<FMT, 32>(stages);
-    case 64: return smem_bytes<FMT, 64>(stages);
-    case 128: return smem_bytes<FMT, 128>(stages);
-    case 256: return FMT == kBLOCK ? (size_t)1 << 30 : smem_bytes<FMT, 256>(stages);
+    case 16: return smem_checked<FMT, 16>(stages);
+    case 32: return smem_checked<FMT, 32>(stages);
+    case 64: return smem_checked<FMT, 64>(stages);
+    case 128: return smem_checked<FMT, 128>(stages);
+    case 256: return smem_checked<FMT, 256>(stages);
     default: return (size_t)1 << 30;
   }
 }

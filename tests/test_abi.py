@@ -78,7 +78,7 @@ def test_default_config_follows_the_swap_rule_and_fills_sms():
     assert 32 * c.split_k <= 148
     assert c.reduce_mode == 0                      # cluster reduction: no workspace
     c = qg.qgemm_default_config(qg.QG_BLOCK_FP8, 4096, 5120, 5120)
-    assert c.swap_ab == 0 and c.tile_n == 128
+    assert c.swap_ab == 0 and c.tile_n == 256
     c = qg.qgemm_default_config(qg.QG_FP8_DYNAMIC, 32, 2048, 2048)
     assert c.swap_ab == 1 and c.tile_n == 32
 
@@ -109,6 +109,10 @@ def _run(fmt=qg.QG_FP8_DYNAMIC, M=16, N=256, K=512, cfg=None, A=None, W=None, ws
     (dict(A=_op(8, 512)), qg.QG_ERR_INVALID_ARG),               # rows != M
     (dict(W=_op(256, 256)), qg.QG_ERR_INVALID_ARG),             # K mismatch
     (dict(fmt=qg.QG_NVFP4, A=_op(16, 512, g=0)), qg.QG_ERR_INVALID_ARG),  # no tensor scale
+    (dict(fmt=qg.QG_NVFP4, M=64, A=_op(64, 512), cfg=qg.make_config(tile_n=32, stages=4)),
+     qg.QG_ERR_UNSUPPORTED),                                    # second 32-token tile: odd SF word
+    (dict(fmt=qg.QG_NVFP4, M=20, A=_op(20, 512), cfg=qg.make_config(tile_n=16, stages=4)),
+     qg.QG_ERR_UNSUPPORTED),
     (dict(fmt=9), qg.QG_ERR_INVALID_ARG),
     (dict(cfg=qg.make_config(split_k=3)), qg.QG_ERR_UNSUPPORTED),      # not a power of two
     (dict(cfg=qg.make_config(split_k=512)), qg.QG_ERR_UNSUPPORTED),    # above 256
@@ -116,7 +120,7 @@ def _run(fmt=qg.QG_FP8_DYNAMIC, M=16, N=256, K=512, cfg=None, A=None, W=None, ws
     (dict(cfg=qg.make_config(tile_n=48)), qg.QG_ERR_UNSUPPORTED),
     (dict(cfg=qg.make_config(stages=1)), qg.QG_ERR_UNSUPPORTED),
     (dict(cfg=qg.make_config(tile_n=256, stages=12)), qg.QG_ERR_UNSUPPORTED),  # smem
-    (dict(fmt=qg.QG_BLOCK_FP8, cfg=qg.make_config(tile_n=256)), qg.QG_ERR_UNSUPPORTED),
+    (dict(fmt=qg.QG_BLOCK_FP8, K=8192 * 2, cfg=qg.make_config(tile_n=256, stages=3)), qg.QG_ERR_UNSUPPORTED),
     (dict(cfg=qg.make_config(swap_ab=2)), qg.QG_ERR_INVALID_ARG),
     (dict(cfg=qg.make_config(split_k=2, stages=4, reduce_mode=2), ws=None), qg.QG_ERR_WORKSPACE),
     (dict(cfg=qg.make_config(split_k=2, stages=4, reduce_mode=1), ws=FAKE, wsb=64), qg.QG_ERR_WORKSPACE),
