@@ -84,6 +84,28 @@ def peaks():
     return 6650.0, "fallback"
 
 
+def kernel_source_hash():
+    """sha1 of the GEMM kernel sources: ties an ncu traffic figure to the code it measured."""
+    import hashlib
+    h = hashlib.sha1()
+    for f in ("gemm_kernel.cuh", "ptx.cuh"):
+        h.update(open(os.path.join(ROOT, "precision_quantized_gemm_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:12]
+
+
+def measured_traffic():
+    """DRAM bytes per GEMM launch of this workload (read + write, averaged over its
+    three shapes) from the committed ncu summary, or None when the kernel has
+    changed since it was captured."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    kv = dict(line.split(None, 1) for line in open(p) if line.strip() and not line.startswith("#"))
+    if kv.get("kernel_sources", "").strip() != kernel_source_hash():
+        return None
+    return float(kv["w8a8_int8_decode_dram_bytes_per_launch"])
+
+
 # ------------------------------------------------------------- clocks ---
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -368,11 +390,7 @@ def run_ours(args, world, rank, local):
     value = world * step_bytes() / (ms_step_max * 1e-3) / 1e9
     achieved = gemm_total_bytes / (gemm_total_us * 1e-6) / 1e9
     geo = math.exp(sum(math.log(max(p["frac_hbm"], 1e-9)) for p in per_shape) / len(per_shape))
-    traffic = None
-    prof = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(prof):
-        t = json.load(open(prof)).get("w8a8_int8_gemm_bytes_per_launch")
-        traffic = t
+    traffic = measured_traffic()
     if rank != 0:
         return
     line = {

@@ -104,7 +104,7 @@ struct Cfg {
   static constexpr int kSfQAtoms = BN > 128 ? 2 : 1;               // 128-row SF blocks of Q
   static constexpr int kSfPBytes = kNvf4 ? 4 * kSfAtomBytes : 0;   // 4 K-atoms per 128B tile
   static constexpr int kSfQBytes = kNvf4 ? 4 * kSfAtomBytes * kSfQAtoms : 0;
-  static constexpr int kNAcc = kBlock ? (BN >= 128 ? 2 : 4) : 1;  // TMEM accumulators
+  static constexpr int kNAcc = kBlock ? (BN >= 256 ? 2 : 4) : 1;  // TMEM accumulators
   // Wide Block_FP8 tiles promote with 8 epilogue warps: two per 32-lane TMEM
   // quarter, each owning half of the columns.
   static constexpr int kEpiWarps = (kBlock && BN >= 128) ? 8 : 4;
@@ -501,14 +501,17 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
         // acc += p_g * (s_a * s_w): one FMA per element
         float f_row = 0.f;
         if (!SWAP) f_row = sa_s[row * nkt + i];
-        // 64 columns per TMEM round trip (two 32-column loads, one wait)
+        // columns per TMEM round trip: 64 (two loads, one wait) while the
+        // accumulator is small, 32 when it already holds 128 registers
+        constexpr int PB = NC >= 128 ? 32 : 64;
 #pragma unroll
-        for (int c0 = 0; c0 < NC; c0 += 64) {
-          uint32_t v[64];
+        for (int c0 = 0; c0 < NC; c0 += PB) {
+          uint32_t v[PB];
           if constexpr (NC % 32 == 0) {
             tmem_ld32(lane_addr + b * BN + cbeg + c0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-            if (c0 + 32 < NC)
-              tmem_ld32(lane_addr + b * BN + cbeg + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+            if constexpr (PB == 64)
+              if (c0 + 32 < NC)
+                tmem_ld32(lane_addr + b * BN + cbeg + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
           } else {                             // 16-column tiles: stay inside the buffer
             tmem_ld16(lane_addr + b * BN + cbeg + c0, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
           }
@@ -516,11 +519,11 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
           if (SWAP) {
             const float sw = sw_s[i];
 #pragma unroll
-            for (int j = 0; j < 64 && c0 + j < NC; ++j)
+            for (int j = 0; j < PB && c0 + j < NC; ++j)
               acc_f[c0 + j] = fmaf(__uint_as_float(v[j]), sa_s[(cbeg + c0 + j) * nkt + i] * sw, acc_f[c0 + j]);
           } else {
 #pragma unroll
-            for (int j = 0; j < 64 && c0 + j < NC; ++j) {
+            for (int j = 0; j < PB && c0 + j < NC; ++j) {
               const float f = f_row * sw_s[i * WB + (WB == 2 ? (cbeg + c0 + j) / 128 : 0)];
               acc_f[c0 + j] = fmaf(__uint_as_float(v[j]), f, acc_f[c0 + j]);
             }

@@ -12,7 +12,7 @@
 // File format (text, one entry per line):
 //   qgemm-table 1
 //   device <name with spaces replaced by _> sms <count>
-//   <fmt> <M> <N> <K> <split_k> <swap_ab> <tile_n> <stages> <reduce_mode> <us>
+//   <fmt> <M> <N> <K> <split_k> <swap_ab> <tile_n> <stages> <reduce_mode 0..2> <us>
 #include <algorithm>
 #include <cstdio>
 #include <cstring>
@@ -44,7 +44,7 @@ constexpr int kVersion = 1;
 bool valid_cfg_fields(const qg_config& c) {
   return c.split_k >= 1 && c.split_k <= 256 && (c.swap_ab == 0 || c.swap_ab == 1) &&
          c.tile_n >= 16 && c.tile_n <= 256 && c.stages >= 2 && c.stages <= 12 &&
-         (c.reduce_mode == 0 || c.reduce_mode == 1);
+         c.reduce_mode >= 0 && c.reduce_mode <= 2;
 }
 
 }  // namespace

@@ -228,18 +228,25 @@ extern "C" qg_status qgemm_tune(void* table, qg_format f, const int* Ms, int nM,
       for (const auto& c : cands) {
         const double el = std::chrono::duration<double>(std::chrono::steady_clock::now() - t0).count();
         if (el > budget_s_per_shape) break;
+        // every candidate starts from a zeroed workspace (tile counters) and
+        // a NaN-poisoned output, so a launch that skips its reduction or
+        // its stores cannot pass validation on an earlier candidate's y
+        if (wsb) cudaMemsetAsync(ws.p, 0, wsb, st);
+        cudaMemsetAsync(Y.p, 0xFF, (size_t)M * N * 2, st);
         if (qgemm_run(f, &A.op, &W0.op, M, N, K, &c, ws.p, wsb, Y.p, N, QG_OUT_BF16, st) != QG_OK) continue;
         cudaMemcpyAsync(got.data(), Y.p, got.size() * 2, cudaMemcpyDeviceToHost, st);
         if (cudaStreamSynchronize(st) != cudaSuccess) { status = QG_ERR_CUDA; break; }
         ++tried;
         if (!close_enough(got, ref, M, N)) { ++rejected; continue; }
+        if (wsb) cudaMemsetAsync(ws.p, 0, wsb, st);
         const double us = time_config(f, Ws, A, M, N, K, c, ws.p, wsb, Y.p, st, calls, 3);
         if (us > 0 && us < best_us) { best_us = us; best = c; }
       }
       if (status != QG_OK) break;
       // independent second timing pass of the winner
+      if (wsb) cudaMemsetAsync(ws.p, 0, wsb, st);
       const double us2 = time_config(f, Ws, A, M, N, K, best, ws.p, wsb, Y.p, st, calls, 10);
-      qgemm_table_put(table, f, M, N, K, &best, us2 > 0 ? us2 : best_us);
+      if ((status = qgemm_table_put(table, f, M, N, K, &best, us2 > 0 ? us2 : best_us)) != QG_OK) break;
       if (verbose)
         std::printf("[qgemm_tune] fmt %d M %d N %d K %d: split %d swap %d tile_n %d stages %d reduce %d "
                     "-> %.3f us (pass1 %.3f, %d tried, %d rejected)\n",

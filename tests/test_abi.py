@@ -159,19 +159,23 @@ def test_table_roundtrip_and_dispatch(tmp_path):
     t = qg.Table()
     c8 = qg.make_config(split_k=4, swap_ab=1, tile_n=16, stages=8)
     c32 = qg.make_config(split_k=2, swap_ab=1, tile_n=32, stages=6, reduce_mode=1)
+    c2 = qg.make_config(split_k=8, swap_ab=1, tile_n=16, stages=4, reduce_mode=2)
+    t.put(qg.QG_W8A8_INT8, 2, 4096, 4096, c2, 3.0)           # every reduce mode is storable
     t.put(qg.QG_W8A8_INT8, 8, 4096, 4096, c8, 3.5)
     t.put(qg.QG_W8A8_INT8, 32, 4096, 4096, c32, 4.25)
-    assert len(t) == 2
+    assert len(t) == 3
     p = str(tmp_path / "table.txt")
     t.save(p)
     t2 = qg.Table(p)
-    assert len(t2) == 2
+    assert len(t2) == 3
+    c, hit = t2.dispatch(qg.QG_W8A8_INT8, 2, 4096, 4096)
+    assert hit == 1 and c.as_dict() == c2.as_dict()
     c, hit = t2.dispatch(qg.QG_W8A8_INT8, 8, 4096, 4096)
     assert hit == 1 and c.as_dict() == c8.as_dict()
     c, hit = t2.dispatch(qg.QG_W8A8_INT8, 20, 4096, 4096)         # rounds up to M=32
     assert hit == 2 and c.as_dict() == c32.as_dict()
-    c, hit = t2.dispatch(qg.QG_W8A8_INT8, 1, 4096, 4096)          # rounds up to M=8
-    assert hit == 2 and c.as_dict() == c8.as_dict()
+    c, hit = t2.dispatch(qg.QG_W8A8_INT8, 1, 4096, 4096)          # rounds up to M=2
+    assert hit == 2 and c.as_dict() == c2.as_dict()
     c, hit = t2.dispatch(qg.QG_W8A8_INT8, 64, 4096, 4096)         # beyond the table: default
     assert hit == 0 and c.as_dict() == qg.qgemm_default_config(qg.QG_W8A8_INT8, 64, 4096, 4096).as_dict()
     c, hit = t2.dispatch(qg.QG_FP8_DYNAMIC, 8, 4096, 4096)        # other format: default
@@ -183,6 +187,7 @@ def test_table_roundtrip_and_dispatch(tmp_path):
     "qgemm-table 2\ndevice x sms 148\n",
     "qgemm-table 1\ndevice x sms 148\n1 8 4096 4096 4 1 16 8 0\n",          # missing field
     "qgemm-table 1\ndevice x sms 148\n1 8 4096 4096 4 3 16 8 0 1.0\n",      # bad swap
+    "qgemm-table 1\ndevice x sms 148\n1 8 4096 4096 4 1 16 8 3 1.0\n",      # bad reduce mode
     "not a table\n",
 ])
 def test_table_load_rejects_corrupt_files(tmp_path, content):
