@@ -106,12 +106,30 @@ int kt_total(qg_format f, int K) { return (int)((row_bytes(f, K) + 127) / 128); 
 bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-size_t gemm_smem(qg_format f, int tile_n, int stages) {
+// Launch-dependent parts of the shared-memory carve-up: the K tiles of the
+// longest split slice (Block_FP8 stages that many scale columns) and the token
+// columns of a push-mode cluster receive slot (only real tokens are pushed).
+struct LaunchShape {
+  int nkt_max;
+  int recv_cols;
+};
+LaunchShape launch_shape(qg_format f, int M, int K, const qg_config* c) {
+  LaunchShape ls;
+  const int kt = kt_total(f, K);
+  ls.nkt_max = (kt + c->split_k - 1) / c->split_k;
+  const bool push = c->split_k > 1 && c->reduce_mode == qg::kReduceCluster && c->tile_n <= 64;
+  ls.recv_cols = push ? (c->swap_ab ? (M < c->tile_n ? M : c->tile_n) : c->tile_n) : 0;
+  return ls;
+}
+
+size_t gemm_smem(qg_format f, int M, int K, const qg_config* c) {
+  const LaunchShape ls = launch_shape(f, M, K, c);
+  const bool swap = c->swap_ab != 0;
   switch (f) {
-    case QG_FP8_DYNAMIC: return qg::launch_gemm_fp8_smem(tile_n, stages);
-    case QG_W8A8_INT8: return qg::launch_gemm_int8_smem(tile_n, stages);
-    case QG_BLOCK_FP8: return qg::launch_gemm_block_smem(tile_n, stages);
-    default: return qg::launch_gemm_nvf4_smem(tile_n, stages);
+    case QG_FP8_DYNAMIC: return qg::launch_gemm_fp8_smem(c->tile_n, swap, c->stages, ls.nkt_max, ls.recv_cols);
+    case QG_W8A8_INT8: return qg::launch_gemm_int8_smem(c->tile_n, swap, c->stages, ls.nkt_max, ls.recv_cols);
+    case QG_BLOCK_FP8: return qg::launch_gemm_block_smem(c->tile_n, swap, c->stages, ls.nkt_max, ls.recv_cols);
+    default: return qg::launch_gemm_nvf4_smem(c->tile_n, swap, c->stages, ls.nkt_max, ls.recv_cols);
   }
 }
 constexpr size_t kSmemLimit = 232448;  // 227 KB opt-in per CTA on sm_100
@@ -141,15 +159,11 @@ qg_status check_config(qg_format f, int M, int N, int K, const qg_config* c) {
   if (c->stages < 2 || c->stages > 12) return QG_ERR_UNSUPPORTED;
   const int kt = kt_total(f, K);
   if (c->split_k > kt) return QG_ERR_UNSUPPORTED;
-  if (gemm_smem(f, tn, c->stages) > kSmemLimit) return QG_ERR_UNSUPPORTED;
+  // covers the Block_FP8 scale columns of the longest slice as well
+  if (gemm_smem(f, M, K, c) > kSmemLimit) return QG_ERR_UNSUPPORTED;
   if (c->split_k > 1 && c->reduce_mode == qg::kReduceCluster &&
       (c->split_k > qg::kMaxClusterSplit || !cluster_fits(f, tn, c->swap_ab != 0, c->stages)))
     return QG_ERR_UNSUPPORTED;
-  if (f == QG_BLOCK_FP8) {
-    const int nkt_max = (kt + c->split_k - 1) / c->split_k;
-    const int act_rows = c->swap_ab ? tn : 128;
-    if (nkt_max > 64 || act_rows * nkt_max > qg::kMaxScaleStage) return QG_ERR_UNSUPPORTED;
-  }
   return QG_OK;
 }
 
@@ -364,6 +378,9 @@ qg_status qgemm_run(qg_format f, const qg_operand* A, const qg_operand* W, int M
                                                    ws_partial_bytes(M, N, cfg->split_k));
   }
   prm.reduce_mode = cfg->reduce_mode;
+  const LaunchShape ls = launch_shape(f, M, K, cfg);
+  prm.nkt_max = ls.nkt_max;
+  prm.recv_cols = ls.recv_cols;
   prm.err = d->err;
   if (g_trace != nullptr &&
       (size_t)tp * tq * cfg->split_k * qg::kTraceEvents * sizeof(unsigned long long) <= g_trace_bytes)
@@ -412,10 +429,6 @@ qg_status qgemm_default_config(qg_format f, int M, int N, int K, qg_config* out)
   } else {
     c.tile_n = 256;
   }
-  // deepest pipeline that fits, at most 8 stages
-  c.stages = 2;
-  for (int s = 8; s >= 2; --s)
-    if (gemm_smem(f, c.tile_n, s) <= kSmemLimit) { c.stages = s; break; }
   // split-K: fill the SMs with tiles x split, keeping >= 2 K tiles per split
   int tp, tq;
   c.split_k = 1;
@@ -426,12 +439,18 @@ qg_status qgemm_default_config(qg_format f, int M, int N, int K, qg_config* out)
   DeviceInfo* d;
   if (device_info(&d) == QG_OK) sms = d->sms;
   while (c.split_k < 256 && tiles * c.split_k * 2 <= sms && kt / (c.split_k * 2) >= 2) c.split_k *= 2;
-  if (f == QG_BLOCK_FP8) {
-    const int act_rows = c.swap_ab ? c.tile_n : 128;
-    while ((kt + c.split_k - 1) / c.split_k > 64 ||
-           act_rows * ((kt + c.split_k - 1) / c.split_k) > qg::kMaxScaleStage)
-      c.split_k *= 2;
-    if (c.split_k > kt) return QG_ERR_UNSUPPORTED;
+  // deepest pipeline that fits, at most 8 stages; a Block_FP8 slice whose
+  // scale columns leave no room for two stages is split further
+  for (;;) {
+    c.stages = 0;
+    for (int s = 8; s >= 2; --s) {
+      c.stages = s;
+      if (gemm_smem(f, M, K, &c) <= kSmemLimit) break;
+      c.stages = 0;
+    }
+    if (c.stages != 0) break;
+    if (c.split_k >= 256 || c.split_k * 2 > kt) return QG_ERR_UNSUPPORTED;
+    c.split_k *= 2;
   }
   // split-K partials meet in distributed shared memory when the cluster
   // fits, else the last-arriving CTA sums them from the workspace

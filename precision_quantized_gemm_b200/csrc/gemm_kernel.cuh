@@ -41,7 +41,6 @@ enum Fmt : int { kFP8 = 0, kINT8 = 1, kBLOCK = 2, kNVF4 = 3 };
 constexpr int kKTileBytes = 128;     // bytes of K per pipeline stage (one 128B swizzle row)
 constexpr int kPTileBytes = 128 * kKTileBytes;
 constexpr int kSfAtomBytes = 512;    // one 128x4 atom of e4m3 block scales
-constexpr int kMaxScaleStage = 8192; // floats of Block_FP8 scales staged per CTA
 
 constexpr int kReduceCluster = 0;    // split-K partials summed through distributed shared memory
 constexpr int kReduceSecondPass = 1; // partials in the workspace, summed by a second kernel
@@ -70,6 +69,8 @@ struct GemmParams {
   int reduce_mode;             // kReduce*
   unsigned int* err;           // device error word
   unsigned long long* trace;   // optional: kTraceEvents timestamps per CTA (ns)
+  int nkt_max;                 // most K tiles any split slice holds: ceil(kt_total / split_k)
+  int recv_cols;               // cluster push: token columns per receive slot (0: no receive buffer)
 };
 
 // Phase timestamps (%globaltimer, ns) a traced launch records per CTA.
@@ -128,15 +129,24 @@ struct Cfg {
   // Cluster split-K for narrow tiles pushes partial slices into a dedicated
   // receive buffer of the owning CTA; wide tiles pull from the ring instead.
   static constexpr bool kPush = BN <= 64;
-  static constexpr int kRecvBytes = kPush ? 4 * 128 * BN : 0;
 };
 
-// Shared-memory carve-up (offsets from a 1024-byte aligned base).
+// Block_FP8 scales staged per CTA: activation rows x K tiles, then weight
+// blocks x K tiles.
+template <bool SWAP, int BN>
+__host__ __device__ constexpr int block_act_rows() { return SWAP ? BN : 128; }
+template <bool SWAP, int BN>
+__host__ __device__ constexpr int block_weight_blocks() { return (!SWAP && BN > 128) ? 2 : 1; }
+
+// Shared-memory carve-up (offsets from a 1024-byte aligned base).  The
+// receive buffer and the Block_FP8 scale area are sized by the launch (its
+// token count and K slice), so decode launches stay small enough for several
+// CTAs per SM: the next launch's CTAs then stream weights while this one ends.
 struct SmemLayout {
   uint32_t p, q, sfp, sfq, recv, bars, misc, epis, scales, total;
 };
-template <int FMT, int BN>
-__host__ __device__ inline SmemLayout smem_layout(int stages) {
+template <int FMT, bool SWAP, int BN>
+__host__ __device__ inline SmemLayout smem_layout(int stages, int nkt_max, int recv_cols) {
   using C = Cfg<FMT, BN>;
   SmemLayout L;
   L.p = 0;
@@ -144,17 +154,19 @@ __host__ __device__ inline SmemLayout smem_layout(int stages) {
   L.sfp = L.q + stages * C::kQTileBytes;
   L.sfq = L.sfp + stages * C::kSfPBytes;
   L.recv = L.sfq + stages * C::kSfQBytes;
-  L.bars = L.recv + C::kRecvBytes;
+  L.bars = L.recv + (C::kPush ? 4u * 128u * (uint32_t)recv_cols : 0u);
   // full[stages], empty[stages], acc_full, tfull[4], tempty[4], recv_full
   L.misc = L.bars + 8 * (2 * stages + 1 + 8 + 1);
   L.epis = (L.misc + 16 + 15) & ~15u;          // row / column scales (FP8, INT8)
   L.scales = L.epis + (C::kRowColScales ? 4 * (128 + BN) : 0);
-  L.total = L.scales + (C::kBlock ? 4 * (kMaxScaleStage + 2 * 64) : 0);
+  L.total = L.scales + (C::kBlock ? 4u * (uint32_t)((block_act_rows<SWAP, BN>() +
+                                                     block_weight_blocks<SWAP, BN>()) * nkt_max)
+                                  : 0u);
   return L;
 }
-template <int FMT, int BN>
-__host__ inline size_t smem_bytes(int stages) {
-  return smem_layout<FMT, BN>(stages).total + 1024;  // + alignment slack
+template <int FMT, bool SWAP, int BN>
+__host__ inline size_t smem_bytes(int stages, int nkt_max, int recv_cols) {
+  return smem_layout<FMT, SWAP, BN>(stages, nkt_max, recv_cols).total + 1024;  // + alignment slack
 }
 
 // Bytes a pull-mode cluster reduction stages in the (then idle) ring.
@@ -251,7 +263,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const SmemLayout L = smem_layout<FMT, BN>(prm.stages);
+  const SmemLayout L = smem_layout<FMT, SWAP, BN>(prm.stages, prm.nkt_max, prm.recv_cols);
   const int S = prm.stages;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* empty = full + S;
@@ -277,7 +289,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
   if (threadIdx.x == 0) trace_at(prm, kTrEntry);
   const bool cluster_red = prm.split_k > 1 && prm.reduce_mode == kReduceCluster;
   const int rows_per = 128 / prm.split_k;                  // cluster mode: rows owned per CTA
-  const uint32_t slot_bytes = 4u * (uint32_t)(rows_per * BN);
+  const uint32_t slot_bytes = 4u * (uint32_t)(rows_per * prm.recv_cols);
 
   if (threadIdx.x == 0) {
     prefetch_tmap(&tmap_p);
@@ -470,19 +482,19 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
     float acc_f[NC];                           // Block_FP8 promoted accumulator
     if constexpr (C::kBlock) {
       float* sa_s = reinterpret_cast<float*>(smem + L.scales);          // act scales
-      float* sw_s = sa_s + kMaxScaleStage;                              // weight scales
+      constexpr int act_rows = block_act_rows<SWAP, BN>();
+      float* sw_s = sa_s + act_rows * prm.nkt_max;                      // weight scales
       const int G = prm.groups;
       const int g0 = kt_begin;
       // Stage this CTA's scales: activations per (row, group), weights per
       // (128-row block, group).
-      const int act_rows = SWAP ? BN : 128;
       const int act_base = SWAP ? q0 : p0;
       for (int idx = etid; idx < act_rows * nkt; idx += ET) {
         const int r = idx / nkt, gl = idx % nkt;
         const int m = act_base + r;
         sa_s[idx] = (m < prm.M) ? __ldg(prm.scale_a + (size_t)m * G + g0 + gl) : 0.f;
       }
-      constexpr int WB = (!SWAP && BN > 128) ? 2 : 1;                   // weight blocks per tile
+      constexpr int WB = block_weight_blocks<SWAP, BN>();              // weight blocks per tile
       const int wrow0 = (SWAP ? p0 : q0) / 128;
       const int nblk = (prm.N + 127) / 128;
       for (int idx = etid; idx < WB * nkt; idx += ET) {
@@ -678,7 +690,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
       const uint32_t* __restrict__ recv = reinterpret_cast<const uint32_t*>(smem + L.recv);
       uint32_t* __restrict__ ot = otile;
       const int r0 = (int)cluster_ctarank() * rows_per;
-      const int zstride = rows_per * BN;
+      const int zstride = rows_per * prm.recv_cols;
       if (epi_ok && got) {
         // fixed per-thread row (Swap-AB) or column (standard), stepping over
         // the other index: no divisions in the loop, loads of later

@@ -12,7 +12,7 @@ template <int FMT, bool SWAP, int BN>
 cudaError_t launch_one(const CUtensorMap& tp, const CUtensorMap& tq, const GemmParams& prm,
                        dim3 grid, cudaStream_t st, bool pdl) {
   auto kern = qgemm_kernel<FMT, SWAP, BN>;
-  const size_t smem = smem_bytes<FMT, BN>(prm.stages);
+  const size_t smem = smem_bytes<FMT, SWAP, BN>(prm.stages, prm.nkt_max, prm.recv_cols);
   static int configured_bytes = 0;
   if ((int)smem > configured_bytes) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -76,24 +76,24 @@ bool cluster_fits_for(int bn, bool swap, int stages) {
   }
 }
 
-// Shared memory of a configuration; configurations whose output tile does
-// not fit the pipeline ring (reused by the epilogue) report an impossible size.
-template <int FMT, int BN>
-size_t smem_checked(int stages) {
+// Shared memory of a launch; configurations whose output tile does not fit
+// the pipeline ring (reused by the epilogue) report an impossible size.
+template <int FMT, bool SWAP, int BN>
+size_t smem_checked(int stages, int nkt_max, int recv_cols) {
   using C = Cfg<FMT, BN>;
   const size_t ring = (size_t)stages * (kPTileBytes + C::kQTileBytes);
-  if ((size_t)tile_bytes<false, BN>() > ring) return (size_t)1 << 30;
-  return smem_bytes<FMT, BN>(stages);
+  if ((size_t)tile_bytes<SWAP, BN>() > ring) return (size_t)1 << 30;
+  return smem_bytes<FMT, SWAP, BN>(stages, nkt_max, recv_cols);
 }
 
-template <int FMT>
-size_t smem_for(int bn, int stages) {
+template <int FMT, bool SWAP>
+size_t smem_for(int bn, int stages, int nkt_max, int recv_cols) {
   switch (bn) {
-    case 16: return smem_checked<FMT, 16>(stages);
-    case 32: return smem_checked<FMT, 32>(stages);
-    case 64: return smem_checked<FMT, 64>(stages);
-    case 128: return smem_checked<FMT, 128>(stages);
-    case 256: return smem_checked<FMT, 256>(stages);
+    case 16: return smem_checked<FMT, SWAP, 16>(stages, nkt_max, recv_cols);
+    case 32: return smem_checked<FMT, SWAP, 32>(stages, nkt_max, recv_cols);
+    case 64: return smem_checked<FMT, SWAP, 64>(stages, nkt_max, recv_cols);
+    case 128: return smem_checked<FMT, SWAP, 128>(stages, nkt_max, recv_cols);
+    case 256: return smem_checked<FMT, SWAP, 256>(stages, nkt_max, recv_cols);
     default: return (size_t)1 << 30;
   }
 }
@@ -109,7 +109,10 @@ cudaError_t QG_LAUNCH_NAME(bool swap, int tile_n, const CUtensorMap& tp, const C
 #define QG_CAT2(a, b) a##b
 #define QG_CAT(a, b) QG_CAT2(a, b)
 
-size_t QG_CAT(QG_LAUNCH_NAME, _smem)(int tile_n, int stages) { return smem_for<QG_FMT>(tile_n, stages); }
+size_t QG_CAT(QG_LAUNCH_NAME, _smem)(int tile_n, bool swap, int stages, int nkt_max, int recv_cols) {
+  return swap ? smem_for<QG_FMT, true>(tile_n, stages, nkt_max, recv_cols)
+              : smem_for<QG_FMT, false>(tile_n, stages, nkt_max, recv_cols);
+}
 
 bool QG_CAT(QG_LAUNCH_NAME, _cluster_fits)(int tile_n, bool swap, int stages) {
   return cluster_fits_for<QG_FMT>(tile_n, swap, stages);

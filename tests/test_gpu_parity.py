@@ -104,6 +104,8 @@ SWAP_CASES = [  # (M, N, K, split_k, tile_n, reduce_mode, stages); reduce 0 clus
     (48, 256, 1024, 2, 64, 0, 4),
     (33, 130, 512, 1, 16, 0, 4),      # two token tiles, ragged N
     (3, 260, 4096, 16, 16, 2, 4),     # split beyond the cluster limit
+    (8, 512, 2048, 4, 16, 0, 2),      # two-stage ring, wrapping twice per CTA
+    (1, 384, 4096, 2, 16, 0, 3),      # three-stage ring, ragged wrap
 ]
 STD_CASES = [
     (128, 256, 512, 1, 128, 0, 4),
