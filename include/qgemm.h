@@ -192,6 +192,33 @@ qg_status qgemm_run(qg_format f, const qg_operand* A, const qg_operand* W, int M
                     const qg_config* cfg, void* workspace, size_t ws_bytes, void* Y, int ldy,
                     int out_kind, void* stream);
 
+/* Activation quantisation fused into the GEMM: y = dequant(quant(A)) .
+ * dequant(W_q)^T for bf16 activations A, in one kernel.  The pages name the
+ * dynamic activation quantisation among the auxiliary kernels around the
+ * linear-layer GEMM ("Helion in the vLLM backend", seventh paragraph); here
+ * the GEMM's epilogue warps, idle during the mainloop, quantise the
+ * activation slice of their CTA into the shared-memory ring themselves, so a
+ * decode step makes one launch instead of two and the quantised activations
+ * never go through HBM.  The codes and scales are those qgemm_quantize_act
+ * computes (same arithmetic, bit for bit), so y is bitwise equal to
+ * qgemm_quantize_act followed by qgemm_run with the same configuration.
+ *   A:   bf16 [M, lda], 16-byte aligned, lda >= K, lda*2 a multiple of 16.
+ *   W, M, N, K, cfg, workspace, Y, ldy, out_kind: as for qgemm_run.
+ *   act_scale_out: optional fp32 output of the activation scales the kernel
+ *        used: [M] (FP8_DYNAMIC, W8A8_INT8) or [M, K/128] (BLOCK_FP8).
+ * Supported: FP8_DYNAMIC, W8A8_INT8 and BLOCK_FP8 with swap_ab = 1 (the
+ * decode orientation).  A per-token scale spans all of K, so FP8_DYNAMIC and
+ * W8A8_INT8 need split_k = 1 or reduce_mode 0 (the split-K CTAs of a tile
+ * form a cluster and exchange partial amaxes through distributed shared
+ * memory); BLOCK_FP8 groups are local to a K tile and take any split.
+ * NVFP4 (whose tensor scale needs the amax of all of A) and swap_ab = 0
+ * return QG_ERR_UNSUPPORTED; bad pointers, strides or sizes
+ * QG_ERR_INVALID_ARG; all checks happen on the host before any launch.
+ * The caller owns every buffer; nothing is allocated. */
+qg_status qgemm_run_fused_act(qg_format f, const void* A, int lda, const qg_operand* W, int M, int N,
+                              int K, const qg_config* cfg, void* workspace, size_t ws_bytes, void* Y,
+                              int ldy, int out_kind, float* act_scale_out, void* stream);
+
 /* qgemm_run without a caller-provided workspace.  There is no counterpart of
  * this entry point in the pages the library follows; it exists for callers
  * that cannot allocate device memory on this path (an engine whose memory
@@ -247,9 +274,11 @@ qg_status qgemm_dispatch(const void* table, qg_format f, int M, int N, int K, qg
 
 /* Ahead-of-time tuner: for each (M, (N, K)) enumerates the valid configs
  * (split_k, swap_ab, tile_n, stages, reduce_mode), times each with CUDA
- * events over a graph of back-to-back calls (selection pass), re-times the
- * winner in an independent pass that is what the table records, and rejects
- * any config whose output differs from the default config's.  Shapes already
+ * events over a graph of back-to-back layer steps -- qgemm_quantize_act then
+ * qgemm_run, as a layer with dynamic activations runs them (selection pass),
+ * re-times the winner in an independent pass whose step time is what the
+ * table records, and rejects any config whose output differs from the
+ * default config's.  Shapes already
  * present in `table` are skipped (resume).  Synthetic inputs are generated
  * on the device; `budget_s_per_shape` bounds the wall time per shape.
  * NK holds nNK pairs (N, K). */
@@ -271,7 +300,9 @@ void qgemm_set_pdl(int enable);
  * buffer: entry, set-up done, first weight tile issued, dependency wait
  * returned, first stage landed, last MMA committed, accumulator ready, stores
  * done, and for cluster split-K: partial pushed, owned slices received,
- * owned rows reduced (word 11 unused); CTA c = (z * gridDim.y + y) *
+ * owned rows reduced; word 11: the MMA issuer saw the last full stage.  In a
+ * fused launch (qgemm_run_fused_act) word 3 is the epilogue warps' dependency
+ * wait.  CTA c = (z * gridDim.y + y) *
  * gridDim.x + x writes words [12c, 12c+12).
  * Launches whose grid needs more than `bytes` are not traced.  NULL turns
  * tracing off.  Not thread-safe; meant for profiling runs. */

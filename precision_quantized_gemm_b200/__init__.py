@@ -41,7 +41,7 @@ EXPORTS = [
     "qgemm_quantize_act", "qgemm_quantize_weight", "qgemm_run", "qgemm_default_config",
     "qgemm_table_load", "qgemm_table_create", "qgemm_table_put", "qgemm_table_save",
     "qgemm_table_free", "qgemm_table_size", "qgemm_dispatch", "qgemm_tune", "qgemm_device_error",
-    "qgemm_run_noalloc", "qgemm_set_trace",
+    "qgemm_run_noalloc", "qgemm_set_trace", "qgemm_run_fused_act",
 ]
 
 
@@ -111,6 +111,9 @@ def lib() -> ctypes.CDLL:
             "qgemm_set_trace": (None, [c_void_p, c_size_t]),
             "qgemm_run_noalloc": (c_int, [c_int, POINTER(qg_operand), POINTER(qg_operand), c_int, c_int, c_int,
                                           POINTER(qg_config), c_void_p, c_int, c_int, c_void_p]),
+            "qgemm_run_fused_act": (c_int, [c_int, c_void_p, c_int, POINTER(qg_operand), c_int, c_int, c_int,
+                                            POINTER(qg_config), c_void_p, c_size_t, c_void_p, c_int, c_int,
+                                            c_void_p, c_void_p]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -169,6 +172,13 @@ def qgemm_run_noalloc(fmt, A: qg_operand, W: qg_operand, M, N, K, cfg: qg_config
     """qgemm_run with the library's own fixed scratch instead of a caller workspace."""
     return lib().qgemm_run_noalloc(fmt, ctypes.byref(A), ctypes.byref(W), M, N, K, ctypes.byref(cfg),
                                    Y_ptr, ldy, out_kind, stream)
+
+
+def qgemm_run_fused_act(fmt, A_ptr, lda, W: qg_operand, M, N, K, cfg: qg_config, ws_ptr, ws_bytes,
+                        Y_ptr, ldy, out_kind, act_scale_ptr, stream):
+    """GEMM on bf16 activations, quantised inside the kernel (Swap-AB decode path)."""
+    return lib().qgemm_run_fused_act(fmt, A_ptr, lda, ctypes.byref(W), M, N, K, ctypes.byref(cfg), ws_ptr,
+                                     ws_bytes, Y_ptr, ldy, out_kind, act_scale_ptr, stream)
 
 
 def qgemm_default_config(fmt, M, N, K) -> qg_config:
@@ -322,6 +332,26 @@ def run(fmt: int, A: Operand, W: Operand, cfg: qg_config | None = None, out=None
     return out
 
 
+def run_fused(fmt: int, A, W: Operand, cfg: qg_config | None = None, out=None,
+              out_kind: int = QG_OUT_BF16, workspace: Workspace | None = None, act_scale_out=None,
+              stream=None):
+    """y = dequant(quant(A)) . dequant(W_q)^T for bf16 A [M, K] through
+    qgemm_run_fused_act (activation quantisation inside the GEMM); returns y."""
+    torch = _torch()
+    M, K = A.shape
+    N = W.rows
+    cfg = cfg or qgemm_default_config(fmt, M, N, K)
+    if out is None:
+        dt = torch.bfloat16 if out_kind == QG_OUT_BF16 else (torch.int32 if fmt == QG_W8A8_INT8 else torch.float32)
+        out = torch.empty(M, N, dtype=dt, device=A.device)
+    workspace = workspace or Workspace(A.device)
+    wsp, wsb = workspace.get(qgemm_workspace_size(fmt, M, N, K, cfg))
+    sp = act_scale_out.data_ptr() if act_scale_out is not None else None
+    check(qgemm_run_fused_act(fmt, A.data_ptr(), A.stride(0), W.c, M, N, K, cfg, wsp, wsb, out.data_ptr(),
+                              out.stride(0), out_kind, sp, _stream(stream)), "qgemm_run_fused_act")
+    return out
+
+
 class Linear:
     """A quantized linear layer: weights quantised once, activations per call,
     configuration from a tuned table (or the default), optional CUDA-graph
@@ -355,10 +385,13 @@ class GraphStep:
     count M: activation quantisation + GEMM replayed as a single CUDA graph
     ("Helion in the vLLM backend", fourth paragraph: shapes up to
     max_helion_size run under CUDA-graph replay).  Write the input into
-    ``A`` (bf16 [M, K]), call ``replay()``, read ``Y`` (bf16 [M, N])."""
+    ``A`` (bf16 [M, K]), call ``replay()``, read ``Y`` (bf16 [M, N]).
+    ``fused=True`` captures the one-launch path (qgemm_run_fused_act)."""
 
-    def __init__(self, layer: "Linear", M: int, W: Operand | None = None, cfg: qg_config | None = None):
+    def __init__(self, layer: "Linear", M: int, W: Operand | None = None, cfg: qg_config | None = None,
+                 fused: bool = False):
         torch = _torch()
+        self.fused = fused
         dev = layer.Wq.q.device
         self.M, self.N, self.K = M, layer.N, layer.K
         self.fmt = layer.fmt
@@ -383,6 +416,12 @@ class GraphStep:
 
     def _launch(self):
         st = _stream(None)
+        if self.fused:
+            wsp, wsb = self.ws.get(qgemm_workspace_size(self.fmt, self.M, self.N, self.K, self.cfg))
+            check(qgemm_run_fused_act(self.fmt, self.A.data_ptr(), self.K, self.W.c, self.M, self.N, self.K,
+                                      self.cfg, wsp, wsb, self.Y.data_ptr(), self.N, QG_OUT_BF16, None, st),
+                  "qgemm_run_fused_act")
+            return
         check(qgemm_quantize_act(self.fmt, self.A.data_ptr(), self.M, self.K, self.K, None, self.act.c,
                                  self.qws.data_ptr(), self.qws.numel(), st), "qgemm_quantize_act")
         wsp, wsb = self.ws.get(qgemm_workspace_size(self.fmt, self.M, self.N, self.K, self.cfg))
@@ -394,8 +433,9 @@ class GraphStep:
         return self.Y
 
 
-def _linear_capture(self, M: int, W: Operand | None = None, cfg: qg_config | None = None) -> GraphStep:
-    g = GraphStep(self, M, W=W, cfg=cfg)
+def _linear_capture(self, M: int, W: Operand | None = None, cfg: qg_config | None = None,
+                    fused: bool = False) -> GraphStep:
+    g = GraphStep(self, M, W=W, cfg=cfg, fused=fused)
     self.graphs[M] = g
     return g
 

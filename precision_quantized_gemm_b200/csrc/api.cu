@@ -1,6 +1,7 @@
 // api.cu — the C ABI of libqgemm.so: argument checks, buffer sizes, TMA
 // descriptors, launches of the quantisers and of the unified GEMM kernel.
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -106,41 +107,64 @@ int kt_total(qg_format f, int K) { return (int)((row_bytes(f, K) + 127) / 128); 
 bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// How the activation tiles of a launch fill (qg::kAct*): fused launches
+// quantise the bf16 activations in the kernel; every other launch streams the
+// quantised codes through the ring by TMA.
+int act_mode(bool fused) { return fused ? qg::kActFused : qg::kActTma; }
+
 // Launch-dependent parts of the shared-memory carve-up: the K tiles of the
-// longest split slice (Block_FP8 stages that many scale columns) and the token
-// columns of a push-mode cluster receive slot (only real tokens are pushed).
+// longest split slice (Block_FP8 stages that many scale columns; a fused
+// launch's activation slice that many tiles) and the token columns of a
+// push-mode cluster receive slot (only real tokens are pushed).
 struct LaunchShape {
   int nkt_max;
   int recv_cols;
+  int a_mode;
+  int act_tiles;
 };
-LaunchShape launch_shape(qg_format f, int M, int K, const qg_config* c) {
+LaunchShape launch_shape(qg_format f, int M, int K, const qg_config* c, bool fused) {
   LaunchShape ls;
   const int kt = kt_total(f, K);
   ls.nkt_max = (kt + c->split_k - 1) / c->split_k;
   const bool push = c->split_k > 1 && c->reduce_mode == qg::kReduceCluster && c->tile_n <= 64;
   ls.recv_cols = push ? (c->swap_ab ? (M < c->tile_n ? M : c->tile_n) : c->tile_n) : 0;
+  ls.a_mode = act_mode(fused);
+  ls.act_tiles = ls.a_mode != qg::kActTma ? ls.nkt_max : 0;
   return ls;
 }
 
-size_t gemm_smem(qg_format f, int M, int K, const qg_config* c) {
-  const LaunchShape ls = launch_shape(f, M, K, c);
+size_t gemm_smem(qg_format f, int M, int K, const qg_config* c, bool fused) {
+  const LaunchShape ls = launch_shape(f, M, K, c, fused);
   const bool swap = c->swap_ab != 0;
+  const int tn = c->tile_n, st = c->stages;
   switch (f) {
-    case QG_FP8_DYNAMIC: return qg::launch_gemm_fp8_smem(c->tile_n, swap, c->stages, ls.nkt_max, ls.recv_cols);
-    case QG_W8A8_INT8: return qg::launch_gemm_int8_smem(c->tile_n, swap, c->stages, ls.nkt_max, ls.recv_cols);
-    case QG_BLOCK_FP8: return qg::launch_gemm_block_smem(c->tile_n, swap, c->stages, ls.nkt_max, ls.recv_cols);
-    default: return qg::launch_gemm_nvf4_smem(c->tile_n, swap, c->stages, ls.nkt_max, ls.recv_cols);
+    case QG_FP8_DYNAMIC: return qg::launch_gemm_fp8_smem(tn, swap, st, ls.nkt_max, ls.recv_cols, ls.act_tiles);
+    case QG_W8A8_INT8: return qg::launch_gemm_int8_smem(tn, swap, st, ls.nkt_max, ls.recv_cols, ls.act_tiles);
+    case QG_BLOCK_FP8: return qg::launch_gemm_block_smem(tn, swap, st, ls.nkt_max, ls.recv_cols, ls.act_tiles);
+    default: return qg::launch_gemm_nvf4_smem(tn, swap, st, ls.nkt_max, ls.recv_cols, ls.act_tiles);
   }
 }
 constexpr size_t kSmemLimit = 232448;  // 227 KB opt-in per CTA on sm_100
 
-bool cluster_fits(qg_format f, int tile_n, bool swap, int stages) {
+bool cluster_fits(qg_format f, int M, int K, const qg_config* c, bool fused) {
+  const int act_tiles = launch_shape(f, M, K, c, fused).act_tiles;
+  const bool swap = c->swap_ab != 0;
   switch (f) {
-    case QG_FP8_DYNAMIC: return qg::launch_gemm_fp8_cluster_fits(tile_n, swap, stages);
-    case QG_W8A8_INT8: return qg::launch_gemm_int8_cluster_fits(tile_n, swap, stages);
-    case QG_BLOCK_FP8: return qg::launch_gemm_block_cluster_fits(tile_n, swap, stages);
-    default: return qg::launch_gemm_nvf4_cluster_fits(tile_n, swap, stages);
+    case QG_FP8_DYNAMIC: return qg::launch_gemm_fp8_cluster_fits(c->tile_n, swap, c->stages, act_tiles);
+    case QG_W8A8_INT8: return qg::launch_gemm_int8_cluster_fits(c->tile_n, swap, c->stages, act_tiles);
+    case QG_BLOCK_FP8: return qg::launch_gemm_block_cluster_fits(c->tile_n, swap, c->stages, act_tiles);
+    default: return qg::launch_gemm_nvf4_cluster_fits(c->tile_n, swap, c->stages, act_tiles);
   }
+}
+
+// Shared-memory and cluster feasibility of a launch (fused or not).
+qg_status check_launch_fit(qg_format f, int M, int K, const qg_config* c, bool fused) {
+  // covers the Block_FP8 scale columns and the activation slice as well
+  if (gemm_smem(f, M, K, c, fused) > kSmemLimit) return QG_ERR_UNSUPPORTED;
+  if (c->split_k > 1 && c->reduce_mode == qg::kReduceCluster &&
+      (c->split_k > qg::kMaxClusterSplit || !cluster_fits(f, M, K, c, fused)))
+    return QG_ERR_UNSUPPORTED;
+  return QG_OK;
 }
 
 qg_status check_config(qg_format f, int M, int N, int K, const qg_config* c) {
@@ -159,12 +183,7 @@ qg_status check_config(qg_format f, int M, int N, int K, const qg_config* c) {
   if (c->stages < 2 || c->stages > 12) return QG_ERR_UNSUPPORTED;
   const int kt = kt_total(f, K);
   if (c->split_k > kt) return QG_ERR_UNSUPPORTED;
-  // covers the Block_FP8 scale columns of the longest slice as well
-  if (gemm_smem(f, M, K, c) > kSmemLimit) return QG_ERR_UNSUPPORTED;
-  if (c->split_k > 1 && c->reduce_mode == qg::kReduceCluster &&
-      (c->split_k > qg::kMaxClusterSplit || !cluster_fits(f, tn, c->swap_ab != 0, c->stages)))
-    return QG_ERR_UNSUPPORTED;
-  return QG_OK;
+  return check_launch_fit(f, M, K, c, false);
 }
 
 size_t ws_partial_bytes(int M, int N, int split) {
@@ -335,16 +354,43 @@ qg_status check_run_args(qg_format f, const qg_operand* A, const qg_operand* W, 
   if (need > 0 && (!workspace || ws_bytes < need || !aligned(workspace, 256))) return QG_ERR_WORKSPACE;
   return QG_OK;
 }
+
+// Host-side argument checks of qgemm_run_fused_act (no device work).
+qg_status check_fused_args(qg_format f, const void* A, int lda, const qg_operand* W, int M, int N, int K,
+                           const qg_config* cfg, void* workspace, size_t ws_bytes, void* Y, int ldy,
+                           int out_kind, const float* act_scale_out) {
+  if (!valid_format(f) || M <= 0 || N <= 0 || K <= 0 || !Y || ldy < N || !A || lda < K)
+    return QG_ERR_INVALID_ARG;
+  if (out_kind != QG_OUT_BF16 && out_kind != QG_OUT_ACC) return QG_ERR_INVALID_ARG;
+  if (K % k_multiple(f) != 0 || !aligned(Y, 16) || !aligned(A, 16) || (lda * 2) % 16 != 0)
+    return QG_ERR_INVALID_ARG;
+  if (act_scale_out != nullptr && !aligned(act_scale_out, 4)) return QG_ERR_INVALID_ARG;
+  // NVFP4's tensor scale needs the amax of the whole activation tensor
+  if (f == QG_NVFP4) return QG_ERR_UNSUPPORTED;
+  qg_status s;
+  if ((s = check_operand_impl(f, W, N, K)) != QG_OK) return s;
+  if ((s = check_config(f, M, N, K, cfg)) != QG_OK) return s;
+  if (cfg->swap_ab != 1) return QG_ERR_UNSUPPORTED;
+  // the whole activation slice of a CTA is held in shared memory
+  if ((s = check_launch_fit(f, M, K, cfg, true)) != QG_OK) return s;
+  // a per-token scale spans all of K: split-K slices must meet in a cluster
+  if (f != QG_BLOCK_FP8 && cfg->split_k > 1 && cfg->reduce_mode != kReduceCluster)
+    return QG_ERR_UNSUPPORTED;
+  const size_t need = qgemm_workspace_size(f, M, N, K, cfg);
+  if (need > 0 && (!workspace || ws_bytes < need || !aligned(workspace, 256))) return QG_ERR_WORKSPACE;
+  return QG_OK;
+}
 }  // namespace qg
 
-extern "C" {
-
-qg_status qgemm_run(qg_format f, const qg_operand* A, const qg_operand* W, int M, int N, int K,
-                    const qg_config* cfg, void* workspace, size_t ws_bytes, void* Y, int ldy,
-                    int out_kind, void* stream) {
-  qg_status s = qg::check_run_args(f, A, W, M, N, K, cfg, workspace, ws_bytes, Y, ldy, out_kind);
-  if (s != QG_OK) return s;
+namespace {
+// Launch of the GEMM (and, for reduce_mode 1, its second pass) after the
+// arguments were checked.  `A` is the quantised activation operand, or null
+// when the kernel quantises the bf16 activations `act` itself (fused).
+qg_status launch_run(qg_format f, const qg_operand* A, const void* act, int lda, float* act_scale_out,
+                     const qg_operand* W, int M, int N, int K, const qg_config* cfg, void* workspace,
+                     void* Y, int ldy, int out_kind, void* stream) {
   DeviceInfo* d;
+  qg_status s;
   if ((s = device_info(&d)) != QG_OK) return s;
 
   const bool swap = cfg->swap_ab != 0;
@@ -358,18 +404,21 @@ qg_status qgemm_run(qg_format f, const qg_operand* A, const qg_operand* W, int M
   prm.split_k = cfg->split_k;
   prm.stages = cfg->stages;
   prm.groups = K / 128;
-  prm.scale_a = static_cast<const float*>(A->scale);
+  prm.scale_a = A ? static_cast<const float*>(A->scale) : nullptr;
   prm.scale_w = static_cast<const float*>(W->scale);
-  const uint8_t* sfa = static_cast<const uint8_t*>(A->scale);
+  const uint8_t* sfa = A ? static_cast<const uint8_t*>(A->scale) : nullptr;
   const uint8_t* sfw = static_cast<const uint8_t*>(W->scale);
   prm.sf_p = swap ? sfw : sfa;
   prm.sf_q = swap ? sfa : sfw;
   prm.sf_atoms_per_rb = ((K + 255) / 256) * 4;
-  prm.g_a = A->global_scale;
+  prm.g_a = A ? A->global_scale : nullptr;
   prm.g_w = W->global_scale;
   prm.Y = Y;
   prm.ldy = ldy;
   prm.out_kind = out_kind;
+  prm.act = static_cast<const __nv_bfloat16*>(act);
+  prm.lda = lda;
+  prm.act_scale_out = act_scale_out;
   int tp, tq;
   tiles_of(cfg, M, N, &tp, &tq);
   if (cfg->split_k > 1 && cfg->reduce_mode != qg::kReduceCluster) {
@@ -378,21 +427,24 @@ qg_status qgemm_run(qg_format f, const qg_operand* A, const qg_operand* W, int M
                                                    ws_partial_bytes(M, N, cfg->split_k));
   }
   prm.reduce_mode = cfg->reduce_mode;
-  const LaunchShape ls = launch_shape(f, M, K, cfg);
+  const LaunchShape ls = launch_shape(f, M, K, cfg, act != nullptr);
   prm.nkt_max = ls.nkt_max;
   prm.recv_cols = ls.recv_cols;
+  prm.a_mode = ls.a_mode;
   prm.err = d->err;
   if (g_trace != nullptr &&
       (size_t)tp * tq * cfg->split_k * qg::kTraceEvents * sizeof(unsigned long long) <= g_trace_bytes)
     prm.trace = g_trace;
 
-  const void* base_p = swap ? W->q : A->q;
-  const void* base_q = swap ? A->q : W->q;
   CUtensorMap tmp, tmq;
   const uint64_t rb = row_bytes(f, K);
-  if (!make_tmap(&tmp, base_p, rb, (uint64_t)prm.rows_p, 128) ||
-      !make_tmap(&tmq, base_q, rb, (uint64_t)prm.rows_q, (uint32_t)cfg->tile_n))
-    return QG_ERR_CUDA;
+  if (!make_tmap(&tmp, swap ? W->q : A->q, rb, (uint64_t)prm.rows_p, 128)) return QG_ERR_CUDA;
+  if (A != nullptr) {
+    if (!make_tmap(&tmq, swap ? A->q : W->q, rb, (uint64_t)prm.rows_q, (uint32_t)cfg->tile_n))
+      return QG_ERR_CUDA;
+  } else {
+    tmq = tmp;                                 // fused: the kernel writes the Q tiles itself
+  }
   if (tq > 65535) return QG_ERR_UNSUPPORTED;
   const dim3 grid(tp, tq, cfg->split_k);
   cudaStream_t st = (cudaStream_t)stream;
@@ -414,6 +466,27 @@ qg_status qgemm_run(qg_format f, const qg_operand* A, const qg_operand* W, int M
     if (e != cudaSuccess) return QG_ERR_CUDA;
   }
   return QG_OK;
+}
+}  // namespace
+
+extern "C" {
+
+qg_status qgemm_run(qg_format f, const qg_operand* A, const qg_operand* W, int M, int N, int K,
+                    const qg_config* cfg, void* workspace, size_t ws_bytes, void* Y, int ldy,
+                    int out_kind, void* stream) {
+  qg_status s = qg::check_run_args(f, A, W, M, N, K, cfg, workspace, ws_bytes, Y, ldy, out_kind);
+  if (s != QG_OK) return s;
+  return launch_run(f, A, nullptr, 0, nullptr, W, M, N, K, cfg, workspace, Y, ldy, out_kind, stream);
+}
+
+qg_status qgemm_run_fused_act(qg_format f, const void* A, int lda, const qg_operand* W, int M, int N,
+                              int K, const qg_config* cfg, void* workspace, size_t ws_bytes, void* Y,
+                              int ldy, int out_kind, float* act_scale_out, void* stream) {
+  qg_status s = qg::check_fused_args(f, A, lda, W, M, N, K, cfg, workspace, ws_bytes, Y, ldy, out_kind,
+                                     act_scale_out);
+  if (s != QG_OK) return s;
+  return launch_run(f, nullptr, A, lda, act_scale_out, W, M, N, K, cfg, workspace, Y, ldy, out_kind,
+                    stream);
 }
 
 qg_status qgemm_default_config(qg_format f, int M, int N, int K, qg_config* out) {
@@ -445,7 +518,7 @@ qg_status qgemm_default_config(qg_format f, int M, int N, int K, qg_config* out)
     c.stages = 0;
     for (int s = 8; s >= 2; --s) {
       c.stages = s;
-      if (gemm_smem(f, M, K, &c) <= kSmemLimit) break;
+      if (gemm_smem(f, M, K, &c, false) <= kSmemLimit) break;
       c.stages = 0;
     }
     if (c.stages != 0) break;
@@ -454,7 +527,7 @@ qg_status qgemm_default_config(qg_format f, int M, int N, int K, qg_config* out)
   }
   // split-K partials meet in distributed shared memory when the cluster
   // fits, else the last-arriving CTA sums them from the workspace
-  c.reduce_mode = (c.split_k <= qg::kMaxClusterSplit && cluster_fits(f, c.tile_n, c.swap_ab != 0, c.stages))
+  c.reduce_mode = (c.split_k <= qg::kMaxClusterSplit && cluster_fits(f, M, K, &c, false))
                       ? qg::kReduceCluster
                       : qg::kReduceLastCta;
   *out = c;

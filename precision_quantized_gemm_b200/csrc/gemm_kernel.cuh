@@ -33,6 +33,7 @@
 #include <cstdint>
 
 #include "ptx.cuh"
+#include "quant_math.cuh"
 
 namespace qg {
 
@@ -46,6 +47,15 @@ constexpr int kReduceCluster = 0;    // split-K partials summed through distribu
 constexpr int kReduceSecondPass = 1; // partials in the workspace, summed by a second kernel
 constexpr int kReduceLastCta = 2;    // partials in the workspace, summed by the last-arriving CTA
 constexpr int kMaxClusterSplit = 8;
+
+// How the activation (Q) tiles of a Swap-AB launch reach shared memory.
+// TMA: the quantised codes stream through the ring, one box per stage next to
+// the weight tile.  Fused: the epilogue warps (idle until the accumulator is
+// ready) quantise this CTA's bf16 activation slice, K tiles [kt_begin,
+// kt_end), into a dedicated region once and publish it through one barrier;
+// the ring then carries only weights.
+constexpr int kActTma = 0;
+constexpr int kActFused = 1;
 
 struct GemmParams {
   int M, N, K;
@@ -71,6 +81,14 @@ struct GemmParams {
   unsigned long long* trace;   // optional: kTraceEvents timestamps per CTA (ns)
   int nkt_max;                 // most K tiles any split slice holds: ceil(kt_total / split_k)
   int recv_cols;               // cluster push: token columns per receive slot (0: no receive buffer)
+  // Fused activation quantisation (Swap-AB; FP8_Dynamic, W8A8_INT8,
+  // Block_FP8): with `act` set, the epilogue warps read the bf16 activations,
+  // quantise them exactly as the standalone quantiser does and write the
+  // codes into the ring's Q tiles; `act` null selects the TMA-fed A_q path.
+  const __nv_bfloat16* act;    // bf16 A [M, lda]
+  int lda;
+  float* act_scale_out;        // optional: the activation scales (per token, or [M, K/128])
+  int a_mode;                  // kActTma / kActFused: how the Q (activation) tiles fill
 };
 
 // Phase timestamps (%globaltimer, ns) a traced launch records per CTA.
@@ -86,7 +104,7 @@ enum TraceEvent : int {
   kTrSent = 8,         // cluster split-K: partial rows pushed to their owners
   kTrRecv = 9,         // cluster split-K: owned slices received
   kTrReduced = 10,     // cluster split-K: owned rows summed into the output tile
-  kTrSpare = 11,
+  kTrLastFull = 11,    // MMA issuer saw the last full stage
   kTraceEvents = 12
 };
 __device__ __forceinline__ void trace_at(const GemmParams& prm, int ev) {
@@ -105,7 +123,7 @@ struct Cfg {
   static constexpr int kSfQAtoms = BN > 128 ? 2 : 1;               // 128-row SF blocks of Q
   static constexpr int kSfPBytes = kNvf4 ? 4 * kSfAtomBytes : 0;   // 4 K-atoms per 128B tile
   static constexpr int kSfQBytes = kNvf4 ? 4 * kSfAtomBytes * kSfQAtoms : 0;
-  static constexpr int kNAcc = kBlock ? (BN >= 256 ? 2 : 4) : 1;  // TMEM accumulators
+  static constexpr int kNAcc = kBlock ? (BN >= 256 ? 2 : 4) : 1;  // Block_FP8 group buffers
   // Wide Block_FP8 tiles promote with 8 epilogue warps: two per 32-lane TMEM
   // quarter, each owning half of the columns.
   static constexpr int kEpiWarps = (kBlock && BN >= 128) ? 8 : 4;
@@ -115,9 +133,10 @@ struct Cfg {
   // CTAs per SM the register budget must allow: narrow (decode) tiles keep
   // room for the next launch's CTAs to start streaming weights early.
   static constexpr int kMinBlocks = (!kBlock && BN <= 64) ? 3 : (kBlock && BN <= 32) ? 2 : 1;
-  static constexpr int kSfaCol = kNAcc * BN;                       // TMEM column of SF A
+  static constexpr int kAccCols = kNAcc * BN;                      // accumulator columns
+  static constexpr int kSfaCol = kAccCols;                         // TMEM column of SF A
   static constexpr int kSfbCol = kSfaCol + 16;                     // 4 steps x 4 words
-  static constexpr int kTmemUsed = kNvf4 ? kSfbCol + 16 * kSfQAtoms : kNAcc * BN;
+  static constexpr int kTmemUsed = kNvf4 ? kSfbCol + 16 * kSfQAtoms : kAccCols;
   static constexpr int kTmemCols = kTmemUsed <= 32    ? 32
                                    : kTmemUsed <= 64  ? 64
                                    : kTmemUsed <= 128 ? 128
@@ -143,30 +162,39 @@ __host__ __device__ constexpr int block_weight_blocks() { return (!SWAP && BN > 
 // token count and K slice), so decode launches stay small enough for several
 // CTAs per SM: the next launch's CTAs then stream weights while this one ends.
 struct SmemLayout {
-  uint32_t p, q, sfp, sfq, recv, bars, misc, epis, scales, total;
+  uint32_t p, q, sfp, sfq, recv, bars, misc, epis, scales, fuse, total;
 };
+// Fused activation prologue: this CTA's per-token amax, then one slot of
+// partial amaxes per split-K peer of the cluster.
 template <int FMT, bool SWAP, int BN>
-__host__ __device__ inline SmemLayout smem_layout(int stages, int nkt_max, int recv_cols) {
+__host__ __device__ constexpr uint32_t fuse_bytes() {
+  return (SWAP && FMT != kNVF4) ? 4u * (uint32_t)((1 + kMaxClusterSplit) * BN) : 0u;
+}
+template <int FMT, bool SWAP, int BN>
+__host__ __device__ inline SmemLayout smem_layout(int stages, int nkt_max, int recv_cols, int act_tiles) {
   using C = Cfg<FMT, BN>;
   SmemLayout L;
   L.p = 0;
   L.q = L.p + stages * kPTileBytes;
-  L.sfp = L.q + stages * C::kQTileBytes;
+  // Q tiles: one per stage in the ring, or (act_tiles > 0) the activation
+  // slice of the whole K range, one tile per K tile
+  L.sfp = L.q + (act_tiles > 0 ? act_tiles : stages) * C::kQTileBytes;
   L.sfq = L.sfp + stages * C::kSfPBytes;
   L.recv = L.sfq + stages * C::kSfQBytes;
   L.bars = L.recv + (C::kPush ? 4u * 128u * (uint32_t)recv_cols : 0u);
-  // full[stages], empty[stages], acc_full, tfull[4], tempty[4], recv_full
-  L.misc = L.bars + 8 * (2 * stages + 1 + 8 + 1);
+  // full[stages], empty[stages], acc_full, tfull[4], tempty[4], recv_full, amax_full, act_ready
+  L.misc = L.bars + 8 * (2 * stages + 1 + 8 + 3);
   L.epis = (L.misc + 16 + 15) & ~15u;          // row / column scales (FP8, INT8)
   L.scales = L.epis + (C::kRowColScales ? 4 * (128 + BN) : 0);
-  L.total = L.scales + (C::kBlock ? 4u * (uint32_t)((block_act_rows<SWAP, BN>() +
-                                                     block_weight_blocks<SWAP, BN>()) * nkt_max)
-                                  : 0u);
+  L.fuse = L.scales + (C::kBlock ? 4u * (uint32_t)((block_act_rows<SWAP, BN>() +
+                                                    block_weight_blocks<SWAP, BN>()) * nkt_max)
+                                 : 0u);
+  L.total = L.fuse + fuse_bytes<FMT, SWAP, BN>();
   return L;
 }
 template <int FMT, bool SWAP, int BN>
-__host__ inline size_t smem_bytes(int stages, int nkt_max, int recv_cols) {
-  return smem_layout<FMT, SWAP, BN>(stages, nkt_max, recv_cols).total + 1024;  // + alignment slack
+__host__ inline size_t smem_bytes(int stages, int nkt_max, int recv_cols, int act_tiles) {
+  return smem_layout<FMT, SWAP, BN>(stages, nkt_max, recv_cols, act_tiles).total + 1024;  // + alignment slack
 }
 
 // Bytes a pull-mode cluster reduction stages in the (then idle) ring.
@@ -255,7 +283,7 @@ __device__ __forceinline__ void emit(const GemmParams& prm, int r, int c, int m,
       __float2bfloat16_rn(finish_value<FMT>(acc_bits, sa, sw, alpha));
 }
 
-template <int FMT, bool SWAP, int BN>
+template <int FMT, bool SWAP, int BN, bool FUSED>
 __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBlocks)
     qgemm_kernel(const __grid_constant__ CUtensorMap tmap_p,
                  const __grid_constant__ CUtensorMap tmap_q, const GemmParams prm) {
@@ -263,7 +291,13 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const SmemLayout L = smem_layout<FMT, SWAP, BN>(prm.stages, prm.nkt_max, prm.recv_cols);
+  // Fused activation quantisation is its own instantiation, so the TMA-fed
+  // kernel carries none of its code.
+  constexpr bool kFusable = FUSED && SWAP && FMT != kNVF4;
+  constexpr bool fused = kFusable;
+  constexpr bool a_threads = fused;                    // Q tiles written by the epilogue warps
+  const SmemLayout L =
+      smem_layout<FMT, SWAP, BN>(prm.stages, prm.nkt_max, prm.recv_cols, a_threads ? prm.nkt_max : 0);
   const int S = prm.stages;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* empty = full + S;
@@ -271,6 +305,8 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
   uint64_t* tfull = acc_full + 1;
   uint64_t* tempty = tfull + 4;
   uint64_t* recv_full = tempty + 4;
+  uint64_t* amax_full = recv_full + 1;
+  uint64_t* act_ready = amax_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.misc);
   volatile int* flag_last = reinterpret_cast<volatile int*>(smem + L.misc + 4);
   volatile int* flag_abort = reinterpret_cast<volatile int*>(smem + L.misc + 8);
@@ -288,6 +324,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
   const int nkt = kt_end - kt_begin;
   if (threadIdx.x == 0) trace_at(prm, kTrEntry);
   const bool cluster_red = prm.split_k > 1 && prm.reduce_mode == kReduceCluster;
+  bool epi_phase1 = false;                                 // epilogue warps waited cluster phase 1
   const int rows_per = 128 / prm.split_k;                  // cluster mode: rows owned per CTA
   const uint32_t slot_bytes = 4u * (uint32_t)(rows_per * prm.recv_cols);
 
@@ -306,6 +343,10 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
     // push mode: each of the 128 rows of the owned slices arrives once, from
     // whichever CTA computed it (split_k CTAs x 128/split_k rows)
     mbar_init(recv_full, 128);
+    // fused per-token amax exchange: one arrival per epilogue thread of the cluster
+    mbar_init(amax_full, C::kEpiThreads);
+    // thread-written activation slice: one arrival per epilogue thread
+    mbar_init(act_ready, C::kEpiThreads);
     *flag_abort = 0;
     fence_barrier_init();
   }
@@ -341,10 +382,10 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
       // NVFP4 scale atoms: P rows [p0, p0+128) are one 128-row block; Q has
       // one or two blocks (the second only if it holds any row).
       const int sfq_atoms = (C::kSfQAtoms == 2 && q0 + 128 < prm.rows_q) ? 2 : 1;
-      const uint32_t stage_tx = kPTileBytes + C::kQTileBytes +
-                                (C::kNvf4 ? (uint32_t)(4 * kSfAtomBytes * (1 + sfq_atoms)) : 0u);
-      auto load_w = [&](int i) {
-        const int st = i % S;
+      const uint32_t stage_tx = a_threads ? bytes_w
+                                      : kPTileBytes + C::kQTileBytes +
+                                            (C::kNvf4 ? (uint32_t)(4 * kSfAtomBytes * (1 + sfq_atoms)) : 0u);
+      auto load_w = [&](int i, int st) {
         const int kt = kt_begin + i;
         tma_load_2d(smem + off_w + st * bytes_w, map_w, &full[st], kt * kKTileBytes, row_w, pol_w);
         if constexpr (C::kNvf4) {
@@ -362,8 +403,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
           }
         }
       };
-      auto load_a = [&](int i) {
-        const int st = i % S;
+      auto load_a = [&](int i, int st) {
         const int kt = kt_begin + i;
         tma_load_2d(smem + off_a + st * bytes_a, map_a, &full[st], kt * kKTileBytes, row_a, pol_a);
         if constexpr (C::kNvf4) {
@@ -384,21 +424,25 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
       const int pre = nkt < S ? nkt : S;
       for (int i = 0; i < pre; ++i) {
         mbar_arrive_expect_tx(&full[i], stage_tx);
-        load_w(i);
+        load_w(i, i);
         if (i == 0) trace_at(prm, kTrFirstLoad);
       }
-      griddep_wait();
-      trace_at(prm, kTrDepWait);
-      for (int i = 0; i < pre; ++i) load_a(i);
+      if (!a_threads) {                        // activations come from the preceding kernel
+        griddep_wait();
+        trace_at(prm, kTrDepWait);
+        for (int i = 0; i < pre; ++i) load_a(i, i);
+      }
       bool ok = true;
       int issued = pre;
+      int st = 0;                              // stage of K tile i; its previous use's phase
+      uint32_t ph = 0;
       for (int i = pre; i < nkt; ++i) {
-        const int st = i % S;
-        if (!mbar_wait(&empty[st], ((i / S) - 1) & 1, prm.err)) { ok = false; break; }
+        if (!mbar_wait(&empty[st], ph, prm.err)) { ok = false; break; }
         mbar_arrive_expect_tx(&full[st], stage_tx);
-        load_w(i);
-        load_a(i);
+        load_w(i, st);
+        if (!a_threads) load_a(i, st);
         issued = i + 1;
+        if (++st == S) { st = 0; ph ^= 1u; }
       }
       if (!ok) {
         *flag_abort = 1;
@@ -410,40 +454,54 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0 && nkt > 0) {
-      const uint32_t sp = smem_u32(smem + L.p);
-      const uint32_t sq = smem_u32(smem + L.q);
-      const uint32_t ssfp = smem_u32(smem + L.sfp);
-      const uint32_t ssfq = smem_u32(smem + L.sfq);
+      // One k tile costs this thread a barrier test, four MMA issues and a
+      // commit; everything else is kept out of the loop.  Descriptors are
+      // built once for stage 0 / K step 0: a stage or K step adds its byte
+      // offset / 16 to the start-address field (bits 0-13, which shared
+      // addresses below 256 KB never carry out of).
+      const uint64_t dp0 = sdesc_sw128(smem_u32(smem + L.p));
+      const uint64_t dq0 = sdesc_sw128(smem_u32(smem + L.q));
+      const uint64_t dsfp0 = sdesc_plain_32x16(smem_u32(smem + L.sfp));
+      const uint64_t dsfq0 = sdesc_plain_32x16(smem_u32(smem + L.sfq));
       const uint32_t sfa_t = tmem_base + C::kSfaCol;
       const uint32_t sfb_t = tmem_base + C::kSfbCol;
       // word offset of this CTA's first Q row inside its 128-row SF atom
       const uint32_t sfb_word = (uint32_t)((q0 % 128) / 32);
+      int st = 0;                              // stage of K tile i, and its full-barrier phase
+      uint32_t ph = 0;
+      int gb = 0, gr = 0;                      // Block_FP8: group buffer of K tile i, and its round
+      bool abort = false;
       for (int i = 0; i < nkt; ++i) {
-        const int st = i % S;
-        if (*flag_abort || !mbar_wait(&full[st], (i / S) & 1, prm.err)) { *flag_abort = 1; break; }
-        if (i == 0) trace_at(prm, kTrFirstFull);
+        if (!mbar_wait(&full[st], ph, prm.err)) { abort = true; break; }
+        if (i == 0) {
+          if (a_threads && !mbar_wait(act_ready, 0, prm.err)) { abort = true; break; }
+          trace_at(prm, kTrFirstFull);
+        }
+        if (i == nkt - 1) trace_at(prm, kTrLastFull);
         uint32_t d_t = tmem_base;
         if constexpr (C::kBlock) {
-          const int b = i % C::kNAcc;
-          const int r = i / C::kNAcc;
-          if (r > 0 && !mbar_wait(&tempty[b], (r - 1) & 1, prm.err)) { *flag_abort = 1; break; }
-          d_t = tmem_base + b * BN;
+          if (gr > 0 && !mbar_wait(&tempty[gb], (uint32_t)(gr - 1) & 1u, prm.err)) { abort = true; break; }
+          d_t = tmem_base + (uint32_t)(gb * BN);
         }
         tc_fence_after();
+        const uint64_t dp = dp0 + (uint64_t)((st * kPTileBytes) >> 4);
+        const uint64_t dq = dq0 + (uint64_t)(((a_threads ? i : st) * C::kQTileBytes) >> 4);
         if constexpr (C::kNvf4) {
+          const uint64_t sfp = dsfp0 + (uint64_t)((st * C::kSfPBytes) >> 4);
+          const uint64_t sfq = dsfq0 + (uint64_t)((st * C::kSfQBytes) >> 4);
+#pragma unroll
           for (int s = 0; s < 4; ++s) {
-            tmem_cp_32x128b_x4(sfa_t + 4 * s,
-                               sdesc_plain_32x16(ssfp + st * C::kSfPBytes + s * kSfAtomBytes));
+            tmem_cp_32x128b_x4(sfa_t + 4 * s, sfp + (uint64_t)((s * kSfAtomBytes) >> 4));
+#pragma unroll
             for (int a = 0; a < C::kSfQAtoms; ++a)
               tmem_cp_32x128b_x4(sfb_t + 4 * C::kSfQAtoms * s + 4 * a,
-                                 sdesc_plain_32x16(ssfq + st * C::kSfQBytes + a * 4 * kSfAtomBytes +
-                                                   s * kSfAtomBytes));
+                                 sfq + (uint64_t)((a * 4 * kSfAtomBytes + s * kSfAtomBytes) >> 4));
           }
         }
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
-          const uint64_t da = sdesc_sw128(sp + st * kPTileBytes + 32 * s);
-          const uint64_t db = sdesc_sw128(sq + st * C::kQTileBytes + 32 * s);
+          const uint64_t da = dp + (uint64_t)(2 * s);   // 32 bytes further along K
+          const uint64_t db = dq + (uint64_t)(2 * s);
           const uint32_t accum = C::kBlock ? (s > 0) : (i > 0 || s > 0);
           if constexpr (C::kNvf4)
             mma_nvf4(d_t, da, db, C::kIdesc, sfa_t + 4 * s,
@@ -454,14 +512,18 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
             mma_f8f6f4(d_t, da, db, C::kIdesc, accum);
         }
         mma_commit(&empty[st]);
-        if constexpr (C::kBlock) mma_commit(&tfull[i % C::kNAcc]);
+        if constexpr (C::kBlock) {
+          mma_commit(&tfull[gb]);
+          if (++gb == C::kNAcc) { gb = 0; ++gr; }
+        }
+        if (++st == S) { st = 0; ph ^= 1u; }
       }
+      if (abort) *flag_abort = 1;
       if constexpr (!C::kBlock) mma_commit(acc_full);
       trace_at(prm, kTrLastMma);
     }
   } else {
     // --------------------------------------------------------------- epilogue
-    constexpr int EW = C::kEpiWarps;
     constexpr int ET = C::kEpiThreads;
     constexpr int NC = C::kCols;
     constexpr int CW = NC >= 32 ? 32 : NC;     // accumulator columns per TMEM load
@@ -470,13 +532,208 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
     const int etid = threadIdx.x - 64;         // 0..ET-1
     const int cbeg = ((warp - 2) / 4) * NC;    // this thread's columns [cbeg, cbeg + NC)
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
-    griddep_wait();                            // scales/partials of earlier kernels
-    // FP8 / INT8: stage the per-row scales of this tile while the mainloop runs
+
+    // ---- fused activation slice (Swap-AB): the bf16 activations of tokens
+    // [q0, q0 + Mt) x K tiles [kt_begin, kt_begin + nkt), quantised into the
+    // dedicated Q region, K tile j at L.q + j * BN * 128, every byte where a TMA copy
+    // with the 128-byte swizzle would have put it (16-byte chunk index XOR
+    // row % 8).  The loads of a batch are all in flight together (L2 only:
+    // the preceding kernel wrote them); each epilogue thread then arrives
+    // once on act_ready, after a proxy fence that makes its writes visible
+    // to the tensor core.
+    const int Mt = min(BN, prm.M - q0);                      // real tokens of this tile
+    uint8_t* const qtiles = smem + L.q;
+    uint32_t* const amax_u = reinterpret_cast<uint32_t*>(smem + L.fuse);   // [BN]
+    float* const exch = reinterpret_cast<float*>(smem + L.fuse) + BN;      // [split][BN]
+    float* const sa_blk = reinterpret_cast<float*>(smem + L.scales);       // Block_FP8 act scales
+    const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
+    // fused units: 8 elements = 16 bytes of bf16 -> 8 code bytes; unit u is
+    // K tile u / (Mt*16), token row (u % (Mt*16)) / 16, elements 8*(u % 16)..
+    const int UT = Mt * 16;
+    auto unit_load = [&](int u) -> uint4 {
+      const int j = u / UT, rem = u - j * UT;
+      const int k = (kt_begin + j) * kKTileBytes + (rem & 15) * 8;
+      if (k >= prm.K) return zero4;
+      return __ldcg(reinterpret_cast<const uint4*>(prm.act + (size_t)(q0 + (rem >> 4)) * prm.lda + k));
+    };
+    auto unit_store = [&](int u, uint2 codes) {
+      const int j = u / UT, rem = u - j * UT;
+      const int r = rem >> 4, c8 = rem & 15;
+      const uint32_t off = (uint32_t)(j * C::kQTileBytes + r * kKTileBytes) +
+                           ((uint32_t)(((c8 >> 1) ^ (r & 7)) << 4) | (uint32_t)((c8 & 1) << 3));
+      *reinterpret_cast<uint2*>(qtiles + off) = codes;
+    };
+    auto publish_act = [&]() {
+      fence_proxy_async_smem();
+      mbar_arrive(act_ready);
+    };
+    if constexpr (kFusable) {
+      if (a_threads) {
+        // independent of the preceding kernel: the padding token rows of
+        // every K tile are zero, the amax slots start at zero
+        const int pad = BN - Mt;
+        for (int idx = etid; idx < nkt * pad * 8; idx += ET) {
+          const int j = idx / (pad * 8), rem = idx % (pad * 8);
+          *reinterpret_cast<uint4*>(qtiles + j * C::kQTileBytes + (Mt + rem / 8) * kKTileBytes +
+                                    (rem % 8) * 16) = zero4;
+        }
+        if (fused && etid < BN) amax_u[etid] = 0u;
+        if (fused) named_bar_sync(1, ET);
+      }
+    }
+    // FP8 / INT8 Swap-AB: the weight (row) scales do not depend on the
+    // preceding kernel, so they are staged while it still runs
+    if constexpr (C::kRowColScales && SWAP)
+      for (int r = etid; r < 128; r += ET) row_s[r] = (p0 + r < prm.rows_p) ? __ldg(prm.scale_w + p0 + r) : 0.f;
+    griddep_wait();                            // scales/partials/activations of earlier kernels
+    if (a_threads && etid == 0) trace_at(prm, kTrDepWait);
+    bool fz_ok = true;
+    // FP8 / INT8: the remaining per-row scales of this tile (activation
+    // scales come from the preceding kernel unless the kernel quantises)
     if constexpr (C::kRowColScales) {
-      const float* sp = SWAP ? prm.scale_w : prm.scale_a;
+      if constexpr (!SWAP)
+        for (int r = etid; r < 128; r += ET) row_s[r] = (p0 + r < prm.rows_p) ? __ldg(prm.scale_a + p0 + r) : 0.f;
       const float* sq = SWAP ? prm.scale_a : prm.scale_w;
-      for (int r = etid; r < 128; r += ET) row_s[r] = (p0 + r < prm.rows_p) ? __ldg(sp + p0 + r) : 0.f;
-      for (int c = etid; c < BN; c += ET) col_s[c] = (q0 + c < prm.rows_q) ? __ldg(sq + q0 + c) : 0.f;
+      if (!fused)
+        for (int c = etid; c < BN; c += ET) col_s[c] = (q0 + c < prm.rows_q) ? __ldg(sq + q0 + c) : 0.f;
+    }
+    if constexpr (kFusable && C::kRowColScales) {
+      if (fused) {
+        // ---- per-token FP8 / INT8.  Pass 1: amax of every token row over
+        // this slice (the first kCache units of a thread stay in registers).
+        constexpr bool kI8 = FMT == kINT8;
+        constexpr int kCache = 8;
+        const int U = nkt * UT;
+        uint4 cache[kCache];
+#pragma unroll
+        for (int b = 0; b < kCache; ++b) {
+          const int u = b * ET + etid;
+          cache[b] = u < U ? unit_load(u) : zero4;
+        }
+#pragma unroll
+        for (int b = 0; b < kCache; ++b) {
+          const int u = b * ET + etid;
+          if (u < U) {
+            float x[8];
+            unpack8(cache[b], x);
+            atomicMax(&amax_u[(u % UT) >> 4], __float_as_uint(absmax8(x)));
+          }
+        }
+        for (int u0 = kCache * ET; u0 < U; u0 += 4 * ET) {     // beyond the cache: 4 loads in flight
+          uint4 v[4];
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const int u = u0 + b * ET + etid;
+            v[b] = u < U ? unit_load(u) : zero4;
+          }
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const int u = u0 + b * ET + etid;
+            if (u < U) {
+              float x[8];
+              unpack8(v[b], x);
+              atomicMax(&amax_u[(u % UT) >> 4], __float_as_uint(absmax8(x)));
+            }
+          }
+        }
+        named_bar_sync(1, ET);
+        // the row amax spans the whole K: the split-K CTAs of the cluster
+        // swap their partial maxima (thread etid serves peer etid % split)
+        if (cluster_red) {
+          cluster_wait();                      // phase 1: every peer is initialised
+          epi_phase1 = true;
+          const int Sk = prm.split_k;
+          const uint32_t z = (uint32_t)(etid % Sk);
+          const uint32_t dst = mapa_shared(smem_u32(exch + kz * BN), z);
+          for (int r = etid / Sk; r < Mt; r += ET / Sk) st_dsmem_b32(dst + 4u * (uint32_t)r, amax_u[r]);
+          mbar_arrive_remote(mapa_shared(smem_u32(amax_full), z));
+          fz_ok = mbar_wait_cluster(amax_full, 0, prm.err);
+        }
+        if (etid < BN) {
+          float am = 0.f;
+          if (etid < Mt) {
+            if (cluster_red) {
+              for (int zz = 0; zz < prm.split_k; ++zz) am = fmaxf(am, exch[zz * BN + etid]);
+            } else {
+              am = __uint_as_float(amax_u[etid]);
+            }
+          }
+          const float sc = scale_of_amax<kI8>(am);
+          col_s[etid] = etid < Mt ? sc : 0.f;
+          if (etid < Mt && prm.act_scale_out != nullptr && blockIdx.x == 0 && kz == 0)
+            prm.act_scale_out[q0 + etid] = sc;
+        }
+        named_bar_sync(1, ET);
+        // pass 2: the codes of every unit
+#pragma unroll
+        for (int b = 0; b < kCache; ++b) {
+          const int u = b * ET + etid;
+          if (u < U) {
+            float x[8];
+            unpack8(cache[b], x);
+            const float sc = col_s[(u % UT) >> 4];
+            unit_store(u, quant8<kI8>(x, sc));
+          }
+        }
+        for (int u0 = kCache * ET; u0 < U; u0 += 4 * ET) {
+          uint4 v[4];
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const int u = u0 + b * ET + etid;
+            v[b] = u < U ? unit_load(u) : zero4;
+          }
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const int u = u0 + b * ET + etid;
+            if (u < U) {
+              float x[8];
+              unpack8(v[b], x);
+              unit_store(u, quant8<kI8>(x, col_s[(u % UT) >> 4]));
+            }
+          }
+        }
+        publish_act();
+      }
+    }
+    if constexpr (kFusable && C::kBlock) {
+      if (fused) {
+        // ---- Block_FP8: 1x128 groups are local to a K tile; a group is 16
+        // consecutive units on 16 consecutive lanes (ET and UT are multiples
+        // of 16), its amax a max over shuffles.  Rounds are uniform over the
+        // epilogue threads, four units of loads in flight per thread.
+        const int U = nkt * UT;
+        const int rounds = (U + ET - 1) / ET;
+        for (int b0 = 0; b0 < rounds; b0 += 4) {
+          uint4 v[4];
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const int u = (b0 + b) * ET + etid;
+            v[b] = (b0 + b < rounds && u < U) ? unit_load(u) : zero4;
+          }
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            if (b0 + b < rounds) {
+              const int u = (b0 + b) * ET + etid;
+              float x[8];
+              unpack8(v[b], x);
+              float a = absmax8(x);
+#pragma unroll
+              for (int o = 8; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+              const float sc = scale_of_amax<false>(a);
+              if (u < U) {
+                unit_store(u, quant8<false>(x, sc));
+                const int j = u / UT, rem = u - j * UT;
+                if ((rem & 15) == 0) {
+                  sa_blk[(rem >> 4) * nkt + j] = sc;
+                  if (prm.act_scale_out != nullptr && blockIdx.x == 0)
+                    prm.act_scale_out[(size_t)(q0 + (rem >> 4)) * prm.groups + kt_begin + j] = sc;
+                }
+              }
+            }
+          }
+        }
+        publish_act();
+      }
     }
     bool ok = true;                            // warp-uniform
     float acc_f[NC];                           // Block_FP8 promoted accumulator
@@ -489,10 +746,16 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
       // Stage this CTA's scales: activations per (row, group), weights per
       // (128-row block, group).
       const int act_base = SWAP ? q0 : p0;
-      for (int idx = etid; idx < act_rows * nkt; idx += ET) {
-        const int r = idx / nkt, gl = idx % nkt;
-        const int m = act_base + r;
-        sa_s[idx] = (m < prm.M) ? __ldg(prm.scale_a + (size_t)m * G + g0 + gl) : 0.f;
+      if (!fused) {
+        for (int idx = etid; idx < act_rows * nkt; idx += ET) {
+          const int r = idx / nkt, gl = idx % nkt;
+          const int m = act_base + r;
+          sa_s[idx] = (m < prm.M) ? __ldg(prm.scale_a + (size_t)m * G + g0 + gl) : 0.f;
+        }
+      } else {
+        // fused: rows of real tokens were written above; padding tokens
+        // scale to zero
+        for (int idx = Mt * nkt + etid; idx < act_rows * nkt; idx += ET) sa_s[idx] = 0.f;
       }
       constexpr int WB = block_weight_blocks<SWAP, BN>();              // weight blocks per tile
       const int wrow0 = (SWAP ? p0 : q0) / 128;
@@ -505,7 +768,8 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
       named_bar_sync(1, ET);
 #pragma unroll
       for (int c = 0; c < NC; ++c) acc_f[c] = 0.f;
-      for (int i = 0; i < nkt; ++i) {
+      ok = __all_sync(0xffffffffu, fz_ok);
+      for (int i = 0; i < nkt && ok; ++i) {
         const int b = i % C::kNAcc;
         ok = __all_sync(0xffffffffu, mbar_wait(&tfull[b], (i / C::kNAcc) & 1, prm.err));
         if (!ok) break;
@@ -534,11 +798,12 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
             for (int j = 0; j < PB && c0 + j < NC; ++j)
               acc_f[c0 + j] = fmaf(__uint_as_float(v[j]), sa_s[(cbeg + c0 + j) * nkt + i] * sw, acc_f[c0 + j]);
           } else {
+            // one weight block per chunk (chunks start on multiples of PB
+            // and never cross a 128-column block): one FFMA per element
+            const float f = f_row * sw_s[i * WB + (WB == 2 ? (cbeg + c0) / 128 : 0)];
 #pragma unroll
-            for (int j = 0; j < PB && c0 + j < NC; ++j) {
-              const float f = f_row * sw_s[i * WB + (WB == 2 ? (cbeg + c0 + j) / 128 : 0)];
+            for (int j = 0; j < PB && c0 + j < NC; ++j)
               acc_f[c0 + j] = fmaf(__uint_as_float(v[j]), f, acc_f[c0 + j]);
-            }
           }
         }
         tc_fence_before();
@@ -546,7 +811,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
         if (lane == 0) mbar_arrive(&tempty[b]);
       }
     } else {
-      ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, prm.err));
+      ok = __all_sync(0xffffffffu, fz_ok && mbar_wait(acc_full, 0, prm.err));
       tc_fence_after();
     }
     if (etid == 0) {
@@ -659,7 +924,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
       const int owner = row / rows_per, rl = row % rows_per;
       const int cvalid = SWAP ? min(BN, prm.M - q0) : BN;
       const bool rvalid = SWAP || (p0 + row < prm.M);
-      cluster_wait();                          // phase 1: every receiver is initialised
+      if (!epi_phase1) cluster_wait();         // phase 1: every receiver is initialised
       const uint32_t dst = mapa_shared(smem_u32(smem + L.recv) + (uint32_t)kz * slot_bytes, (uint32_t)owner);
 #pragma unroll
       for (int c0 = 0; c0 < NC; c0 += CW) {
@@ -817,7 +1082,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
   // phase 3 (every remote read done) around the reduction.
   if (cluster_red) {
     __syncwarp();
-    if (!(C::kPush && warp >= 2)) cluster_wait();
+    if (!(warp >= 2 && (C::kPush || epi_phase1))) cluster_wait();
     if constexpr (!C::kPush) {
       cluster_sync();
       if (warp >= 2 && *flag_epi == 0) {

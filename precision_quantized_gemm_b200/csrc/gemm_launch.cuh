@@ -8,11 +8,20 @@
 namespace qg {
 namespace {
 
-template <int FMT, bool SWAP, int BN>
+template <int FMT, bool SWAP, int BN, bool FUSED>
 cudaError_t launch_one(const CUtensorMap& tp, const CUtensorMap& tq, const GemmParams& prm,
                        dim3 grid, cudaStream_t st, bool pdl) {
-  auto kern = qgemm_kernel<FMT, SWAP, BN>;
-  const size_t smem = smem_bytes<FMT, SWAP, BN>(prm.stages, prm.nkt_max, prm.recv_cols);
+  auto kern = qgemm_kernel<FMT, SWAP, BN, FUSED>;
+  const int act_tiles = FUSED ? prm.nkt_max : 0;
+  size_t smem = smem_bytes<FMT, SWAP, BN>(prm.stages, prm.nkt_max, prm.recv_cols, act_tiles);
+  // Every CTA of this kernel that fits on an SM must also fit in its 512 TMEM
+  // columns: a CTA whose tcgen05.alloc waited on another CTA of the same
+  // (clustered) grid could wait for good.  At most 512 / kTmemCols CTAs may
+  // share an SM, so the shared memory of one is raised to at least
+  // 228 KB / (that count + 1).
+  constexpr int kTmemCtas = 512 / Cfg<FMT, BN>::kTmemCols;
+  const size_t smem_floor = (size_t)233472 / (kTmemCtas + 1);
+  if (smem < smem_floor) smem = smem_floor;
   static int configured_bytes = 0;
   if ((int)smem > configured_bytes) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -44,56 +53,61 @@ cudaError_t launch_one(const CUtensorMap& tp, const CUtensorMap& tq, const GemmP
   return cudaLaunchKernelEx(&cfg, kern, tp, tq, prm);
 }
 
-template <int FMT, bool SWAP>
+template <int FMT, bool SWAP, bool FUSED>
 cudaError_t launch_bn(int bn, const CUtensorMap& tp, const CUtensorMap& tq, const GemmParams& prm,
                       dim3 grid, cudaStream_t st, bool pdl) {
   switch (bn) {
-    case 16: return launch_one<FMT, SWAP, 16>(tp, tq, prm, grid, st, pdl);
-    case 32: return launch_one<FMT, SWAP, 32>(tp, tq, prm, grid, st, pdl);
-    case 64: return launch_one<FMT, SWAP, 64>(tp, tq, prm, grid, st, pdl);
-    case 128: return launch_one<FMT, SWAP, 128>(tp, tq, prm, grid, st, pdl);
-    case 256: return launch_one<FMT, SWAP, 256>(tp, tq, prm, grid, st, pdl);
+    case 16: return launch_one<FMT, SWAP, 16, FUSED>(tp, tq, prm, grid, st, pdl);
+    case 32: return launch_one<FMT, SWAP, 32, FUSED>(tp, tq, prm, grid, st, pdl);
+    case 64: return launch_one<FMT, SWAP, 64, FUSED>(tp, tq, prm, grid, st, pdl);
+    case 128: return launch_one<FMT, SWAP, 128, FUSED>(tp, tq, prm, grid, st, pdl);
+    case 256: return launch_one<FMT, SWAP, 256, FUSED>(tp, tq, prm, grid, st, pdl);
     default: return cudaErrorInvalidValue;
   }
 }
 
+// Bytes from the ring's start to the end of the Q tiles: the region the
+// epilogue reuses once the mainloop is done (act_tiles > 0: the Q tiles are
+// the thread-written activation slice instead of one per stage).
 template <int FMT, int BN>
-bool cluster_fits(bool swap, int stages) {
+size_t ring_bytes(int stages, int act_tiles) {
   using C = Cfg<FMT, BN>;
-  const int ring = stages * (kPTileBytes + C::kQTileBytes);
-  return (swap ? red_bytes<true, BN>() : red_bytes<false, BN>()) <= ring;
+  return (size_t)stages * kPTileBytes + (size_t)(act_tiles > 0 ? act_tiles : stages) * C::kQTileBytes;
+}
+
+template <int FMT, int BN>
+bool cluster_fits(bool swap, int stages, int act_tiles) {
+  return (size_t)(swap ? red_bytes<true, BN>() : red_bytes<false, BN>()) <= ring_bytes<FMT, BN>(stages, act_tiles);
 }
 
 template <int FMT>
-bool cluster_fits_for(int bn, bool swap, int stages) {
+bool cluster_fits_for(int bn, bool swap, int stages, int act_tiles) {
   switch (bn) {
-    case 16: return cluster_fits<FMT, 16>(swap, stages);
-    case 32: return cluster_fits<FMT, 32>(swap, stages);
-    case 64: return cluster_fits<FMT, 64>(swap, stages);
-    case 128: return cluster_fits<FMT, 128>(swap, stages);
-    case 256: return cluster_fits<FMT, 256>(swap, stages);
+    case 16: return cluster_fits<FMT, 16>(swap, stages, act_tiles);
+    case 32: return cluster_fits<FMT, 32>(swap, stages, act_tiles);
+    case 64: return cluster_fits<FMT, 64>(swap, stages, act_tiles);
+    case 128: return cluster_fits<FMT, 128>(swap, stages, act_tiles);
+    case 256: return cluster_fits<FMT, 256>(swap, stages, act_tiles);
     default: return false;
   }
 }
 
 // Shared memory of a launch; configurations whose output tile does not fit
-// the pipeline ring (reused by the epilogue) report an impossible size.
+// the ring region (reused by the epilogue) report an impossible size.
 template <int FMT, bool SWAP, int BN>
-size_t smem_checked(int stages, int nkt_max, int recv_cols) {
-  using C = Cfg<FMT, BN>;
-  const size_t ring = (size_t)stages * (kPTileBytes + C::kQTileBytes);
-  if ((size_t)tile_bytes<SWAP, BN>() > ring) return (size_t)1 << 30;
-  return smem_bytes<FMT, SWAP, BN>(stages, nkt_max, recv_cols);
+size_t smem_checked(int stages, int nkt_max, int recv_cols, int act_tiles) {
+  if ((size_t)tile_bytes<SWAP, BN>() > ring_bytes<FMT, BN>(stages, act_tiles)) return (size_t)1 << 30;
+  return smem_bytes<FMT, SWAP, BN>(stages, nkt_max, recv_cols, act_tiles);
 }
 
 template <int FMT, bool SWAP>
-size_t smem_for(int bn, int stages, int nkt_max, int recv_cols) {
+size_t smem_for(int bn, int stages, int nkt_max, int recv_cols, int act_tiles) {
   switch (bn) {
-    case 16: return smem_checked<FMT, SWAP, 16>(stages, nkt_max, recv_cols);
-    case 32: return smem_checked<FMT, SWAP, 32>(stages, nkt_max, recv_cols);
-    case 64: return smem_checked<FMT, SWAP, 64>(stages, nkt_max, recv_cols);
-    case 128: return smem_checked<FMT, SWAP, 128>(stages, nkt_max, recv_cols);
-    case 256: return smem_checked<FMT, SWAP, 256>(stages, nkt_max, recv_cols);
+    case 16: return smem_checked<FMT, SWAP, 16>(stages, nkt_max, recv_cols, act_tiles);
+    case 32: return smem_checked<FMT, SWAP, 32>(stages, nkt_max, recv_cols, act_tiles);
+    case 64: return smem_checked<FMT, SWAP, 64>(stages, nkt_max, recv_cols, act_tiles);
+    case 128: return smem_checked<FMT, SWAP, 128>(stages, nkt_max, recv_cols, act_tiles);
+    case 256: return smem_checked<FMT, SWAP, 256>(stages, nkt_max, recv_cols, act_tiles);
     default: return (size_t)1 << 30;
   }
 }
@@ -102,20 +116,28 @@ size_t smem_for(int bn, int stages, int nkt_max, int recv_cols) {
 
 cudaError_t QG_LAUNCH_NAME(bool swap, int tile_n, const CUtensorMap& tp, const CUtensorMap& tq,
                            const GemmParams& prm, dim3 grid, cudaStream_t st, bool pdl) {
-  return swap ? launch_bn<QG_FMT, true>(tile_n, tp, tq, prm, grid, st, pdl)
-              : launch_bn<QG_FMT, false>(tile_n, tp, tq, prm, grid, st, pdl);
+  if (prm.a_mode == kActFused) {
+    // fused activation quantisation: Swap-AB, 8-bit formats only
+    if constexpr (QG_FMT != kNVF4) {
+      if (swap) return launch_bn<QG_FMT, true, true>(tile_n, tp, tq, prm, grid, st, pdl);
+    }
+    return cudaErrorInvalidValue;
+  }
+  return swap ? launch_bn<QG_FMT, true, false>(tile_n, tp, tq, prm, grid, st, pdl)
+              : launch_bn<QG_FMT, false, false>(tile_n, tp, tq, prm, grid, st, pdl);
 }
 
 #define QG_CAT2(a, b) a##b
 #define QG_CAT(a, b) QG_CAT2(a, b)
 
-size_t QG_CAT(QG_LAUNCH_NAME, _smem)(int tile_n, bool swap, int stages, int nkt_max, int recv_cols) {
-  return swap ? smem_for<QG_FMT, true>(tile_n, stages, nkt_max, recv_cols)
-              : smem_for<QG_FMT, false>(tile_n, stages, nkt_max, recv_cols);
+size_t QG_CAT(QG_LAUNCH_NAME, _smem)(int tile_n, bool swap, int stages, int nkt_max, int recv_cols,
+                                     int act_tiles) {
+  return swap ? smem_for<QG_FMT, true>(tile_n, stages, nkt_max, recv_cols, act_tiles)
+              : smem_for<QG_FMT, false>(tile_n, stages, nkt_max, recv_cols, act_tiles);
 }
 
-bool QG_CAT(QG_LAUNCH_NAME, _cluster_fits)(int tile_n, bool swap, int stages) {
-  return cluster_fits_for<QG_FMT>(tile_n, swap, stages);
+bool QG_CAT(QG_LAUNCH_NAME, _cluster_fits)(int tile_n, bool swap, int stages, int act_tiles) {
+  return cluster_fits_for<QG_FMT>(tile_n, swap, stages, act_tiles);
 }
 
 cudaError_t QG_CAT(QG_LAUNCH_NAME, _reduce)(const GemmParams& prm, cudaStream_t st, bool pdl) {

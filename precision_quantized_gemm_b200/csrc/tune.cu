@@ -8,9 +8,10 @@
 // and the winner's recorded time comes from an independent second pass.  A
 // candidate whose output disagrees with the default configuration's is
 // rejected (the "correctness validation failure" fallback of TensorRT-LLM
-// issue 16363).  Timing replays a CUDA graph of back-to-back calls that
-// rotate over enough weight copies to exceed twice the L2, so every call
-// streams its weights from HBM.
+// issue 16363).  Timing replays a CUDA graph of back-to-back layer steps
+// (dynamic activation quantisation, then the GEMM) that rotate over enough
+// weight copies to exceed twice the L2, so every GEMM streams its weights
+// from HBM.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -89,17 +90,25 @@ bool close_enough(const std::vector<uint16_t>& got, const std::vector<uint16_t>&
   return true;
 }
 
-// Median-free timing: mean µs per call over `reps` launches of a graph that
-// holds `calls` back-to-back GEMMs rotating over the weight copies.
-double time_config(qg_format f, const std::vector<Operand*>& Ws, const Operand& A, int M, int N,
-                   int K, const qg_config& c, void* ws, size_t wsb, void* Y, cudaStream_t st,
-                   int calls, int reps) {
+// Median-free timing: mean µs per step over `reps` launches of a graph that
+// holds `calls` back-to-back steps rotating over the weight copies.  A step is
+// what a linear layer with dynamic activations runs: the activation
+// quantisation of `act` (bf16 [M, K]) into A, then the GEMM.  The GEMM's
+// weight prefetch overlaps the quantiser through programmatic dependent
+// launch, and how well depends on the configuration, so the pair is timed.
+double time_config(qg_format f, const std::vector<Operand*>& Ws, const Operand& A, const void* act,
+                   void* qws, size_t qwsb, int M, int N, int K, const qg_config& c, void* ws,
+                   size_t wsb, void* Y, cudaStream_t st, int calls, int reps) {
   cudaGraph_t g = nullptr;
   cudaGraphExec_t ge = nullptr;
   if (cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal) != cudaSuccess) return -1;
   qg_status s = QG_OK;
-  for (int i = 0; i < calls && s == QG_OK; ++i)
-    s = qgemm_run(f, &A.op, &Ws[i % Ws.size()]->op, M, N, K, &c, ws, wsb, Y, N, QG_OUT_BF16, st);
+  qg_operand aop = A.op;
+  for (int i = 0; i < calls && s == QG_OK; ++i) {
+    s = qgemm_quantize_act(f, act, M, K, K, nullptr, &aop, qws, qwsb, st);
+    if (s == QG_OK)
+      s = qgemm_run(f, &A.op, &Ws[i % Ws.size()]->op, M, N, K, &c, ws, wsb, Y, N, QG_OUT_BF16, st);
+  }
   if (cudaStreamEndCapture(st, &g) != cudaSuccess || s != QG_OK) {
     if (g) cudaGraphDestroy(g);
     return -1;
@@ -127,10 +136,16 @@ double time_config(qg_format f, const std::vector<Operand*>& Ws, const Operand& 
 std::vector<qg_config> candidates(qg_format f, int M, int N, int K) {
   std::vector<qg_config> out;
   const int kt = (int)(((f == QG_NVFP4 ? K / 2 : K) + 127) / 128);
-  const int tiles_n[] = {16, 32, 64, 128, 256};
-  const int stage_opts[] = {4, 6, 8, 10};
+  // Swap-AB tiles narrow first, standard tiles wide first: within the time
+  // budget the likelier winners are timed before the others.
+  const int tiles_swap[] = {16, 32, 64, 128, 256};
+  const int tiles_std[] = {256, 128, 64};
+  const int stage_opts[] = {3, 4, 6, 8};
   for (int swap = 0; swap <= 1; ++swap) {
-    for (int tn : tiles_n) {
+    const int* tiles = swap ? tiles_swap : tiles_std;
+    const int ntiles = swap ? 5 : 3;
+    for (int ti = 0; ti < ntiles; ++ti) {
+      const int tn = tiles[ti];
       if (swap && tn > 2 * std::max(16, M)) continue;     // tokens would mostly be padding
       if (!swap && (tn < 64 || M < 64)) continue;         // standard needs a real 128-token tile
       for (int sk = 1; sk <= 256 && sk <= kt; sk *= 2) {
@@ -239,13 +254,13 @@ extern "C" qg_status qgemm_tune(void* table, qg_format f, const int* Ms, int nM,
         ++tried;
         if (!close_enough(got, ref, M, N)) { ++rejected; continue; }
         if (wsb) cudaMemsetAsync(ws.p, 0, wsb, st);
-        const double us = time_config(f, Ws, A, M, N, K, c, ws.p, wsb, Y.p, st, calls, 3);
+        const double us = time_config(f, Ws, A, asrc.p, qas.p, qasb, M, N, K, c, ws.p, wsb, Y.p, st, calls, 3);
         if (us > 0 && us < best_us) { best_us = us; best = c; }
       }
       if (status != QG_OK) break;
       // independent second timing pass of the winner
       if (wsb) cudaMemsetAsync(ws.p, 0, wsb, st);
-      const double us2 = time_config(f, Ws, A, M, N, K, best, ws.p, wsb, Y.p, st, calls, 10);
+      const double us2 = time_config(f, Ws, A, asrc.p, qas.p, qasb, M, N, K, best, ws.p, wsb, Y.p, st, calls, 10);
       if ((status = qgemm_table_put(table, f, M, N, K, &best, us2 > 0 ? us2 : best_us)) != QG_OK) break;
       if (verbose)
         std::printf("[qgemm_tune] fmt %d M %d N %d K %d: split %d swap %d tile_n %d stages %d reduce %d "

@@ -202,3 +202,48 @@ def test_table_load_missing_file():
     with pytest.raises(qg.QGemmError) as e:
         qg.Table("/nonexistent/qgemm_table.txt")
     assert e.value.status == qg.QG_ERR_TABLE_IO
+
+
+def _fused(fmt=qg.QG_W8A8_INT8, M=8, N=256, K=512, cfg=None, A=FAKE, lda=None, W=None, ws=None, wsb=0,
+           Y=FAKE, ldy=None, out_kind=0, scales=None):
+    cfg = cfg or qg.make_config(split_k=2, swap_ab=1, tile_n=16, stages=4, reduce_mode=0)
+    W = W or _op(N, K)
+    return qg.qgemm_run_fused_act(fmt, A, lda if lda is not None else K, W, M, N, K, cfg, ws, wsb, Y,
+                                  ldy if ldy is not None else N, out_kind, scales, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(M=0), qg.QG_ERR_INVALID_ARG),
+    (dict(A=None), qg.QG_ERR_INVALID_ARG),
+    (dict(A=FAKE + 8), qg.QG_ERR_INVALID_ARG),                  # activations not 16-byte aligned
+    (dict(lda=500), qg.QG_ERR_INVALID_ARG),                     # lda < K
+    (dict(lda=516), qg.QG_ERR_INVALID_ARG),                     # row stride not a multiple of 16 bytes
+    (dict(K=520), qg.QG_ERR_INVALID_ARG),
+    (dict(scales=FAKE + 2), qg.QG_ERR_INVALID_ARG),             # misaligned scale output
+    (dict(W=_op(128, 512)), qg.QG_ERR_INVALID_ARG),             # W rows != N
+    (dict(fmt=qg.QG_NVFP4), qg.QG_ERR_UNSUPPORTED),             # tensor amax spans all of A
+    (dict(cfg=qg.make_config(split_k=1, swap_ab=0, tile_n=128, stages=4)), qg.QG_ERR_UNSUPPORTED),
+    (dict(cfg=qg.make_config(split_k=2, swap_ab=1, tile_n=16, stages=4, reduce_mode=1), ws=FAKE,
+          wsb=1 << 20), qg.QG_ERR_UNSUPPORTED),                 # per-token amax needs a cluster
+    (dict(fmt=qg.QG_FP8_DYNAMIC, cfg=qg.make_config(split_k=2, swap_ab=1, tile_n=16, stages=4,
+                                                     reduce_mode=2), ws=FAKE, wsb=1 << 20),
+     qg.QG_ERR_UNSUPPORTED),
+    (dict(fmt=qg.QG_BLOCK_FP8, cfg=qg.make_config(split_k=2, swap_ab=1, tile_n=16, stages=4,
+                                                   reduce_mode=1)), qg.QG_ERR_WORKSPACE),
+    (dict(cfg=qg.make_config(split_k=3, swap_ab=1, tile_n=16, stages=4)), qg.QG_ERR_UNSUPPORTED),
+])
+def test_fused_rejects_bad_arguments_before_any_launch(kw, status):
+    assert _fused(**kw) == status
+
+
+def test_fused_valid_arguments_reach_the_device_check():
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("needs a machine without a GPU")
+    # Block_FP8 groups are local to a K tile: any split and reduce mode
+    ok = [dict(),
+          dict(fmt=qg.QG_BLOCK_FP8, cfg=qg.make_config(split_k=2, swap_ab=1, tile_n=16, stages=4,
+                                                        reduce_mode=1), ws=FAKE, wsb=1 << 20),
+          dict(fmt=qg.QG_FP8_DYNAMIC, cfg=qg.make_config(split_k=1, swap_ab=1, tile_n=32, stages=4))]
+    for kw in ok:
+        assert _fused(**kw) in (qg.QG_ERR_NO_DEVICE, qg.QG_ERR_UNSUPPORTED)
