@@ -133,9 +133,12 @@ double time_config(qg_format f, const std::vector<Operand*>& Ws, const Operand& 
   return ms < 0 ? -1 : 1000.0 * ms / ((double)reps * calls);
 }
 
+// 128-byte K tiles of a row.
+int kt_of(qg_format f, int K) { return (int)(((f == QG_NVFP4 ? K / 2 : K) + 127) / 128); }
+
 std::vector<qg_config> candidates(qg_format f, int M, int N, int K) {
   std::vector<qg_config> out;
-  const int kt = (int)(((f == QG_NVFP4 ? K / 2 : K) + 127) / 128);
+  const int kt = kt_of(f, K);
   // Swap-AB tiles narrow first, standard tiles wide first: within the time
   // budget the likelier winners are timed before the others.
   const int tiles_swap[] = {16, 32, 64, 128, 256};
@@ -240,6 +243,7 @@ extern "C" qg_status qgemm_tune(void* table, qg_format f, const int* Ms, int nM,
       double best_us = 1e30;
       qg_config best = dflt;
       int tried = 0, rejected = 0;
+      std::vector<std::pair<double, qg_config>> timed;
       for (const auto& c : cands) {
         const double el = std::chrono::duration<double>(std::chrono::steady_clock::now() - t0).count();
         if (el > budget_s_per_shape) break;
@@ -255,9 +259,26 @@ extern "C" qg_status qgemm_tune(void* table, qg_format f, const int* Ms, int nM,
         if (!close_enough(got, ref, M, N)) { ++rejected; continue; }
         if (wsb) cudaMemsetAsync(ws.p, 0, wsb, st);
         const double us = time_config(f, Ws, A, asrc.p, qas.p, qasb, M, N, K, c, ws.p, wsb, Y.p, st, calls, 3);
+        if (us > 0) timed.emplace_back(us, c);
         if (us > 0 && us < best_us) { best_us = us; best = c; }
       }
       if (status != QG_OK) break;
+      // Near-ties (within 3%) go to a configuration whose ring holds every
+      // K tile of its slice: all of its weights are requested at launch, so
+      // it also keeps its time after a graph boundary or a host sync, where
+      // no earlier kernel's tail hides the reload of a stage (steady-state
+      // timing does not see that case).
+      {
+        double tie_us = 1e30;
+        for (const auto& t : timed) {
+          const int nkt = (kt_of(f, K) + t.second.split_k - 1) / t.second.split_k;
+          if (t.first <= 1.03 * best_us && t.second.stages >= nkt && t.first < tie_us) {
+            tie_us = t.first;
+            best = t.second;
+          }
+        }
+        if (tie_us < 1e30) best_us = tie_us;
+      }
       // independent second timing pass of the winner
       if (wsb) cudaMemsetAsync(ws.p, 0, wsb, st);
       const double us2 = time_config(f, Ws, A, asrc.p, qas.p, qasb, M, N, K, best, ws.p, wsb, Y.p, st, calls, 10);
