@@ -124,9 +124,11 @@ struct Cfg {
   static constexpr int kSfPBytes = kNvf4 ? 4 * kSfAtomBytes : 0;   // 4 K-atoms per 128B tile
   static constexpr int kSfQBytes = kNvf4 ? 4 * kSfAtomBytes * kSfQAtoms : 0;
   static constexpr int kNAcc = kBlock ? (BN >= 256 ? 2 : 4) : 1;  // Block_FP8 group buffers
-  // Wide Block_FP8 tiles promote with 8 epilogue warps: two per 32-lane TMEM
-  // quarter, each owning half of the columns.
-  static constexpr int kEpiWarps = (kBlock && BN >= 128) ? 8 : 4;
+  // Wide Block_FP8 tiles promote with more epilogue warps: two (BN = 128) or
+  // four (BN = 256) per 32-lane TMEM quarter, each owning a share of the
+  // columns, so that while some warps wait on their TMEM loads others run
+  // their FMAs (a warp's promotion is a chain of load -> wait -> FMA).
+  static constexpr int kEpiWarps = (kBlock && BN >= 256) ? 16 : (kBlock && BN >= 128) ? 8 : 4;
   static constexpr int kEpiThreads = 32 * kEpiWarps;
   static constexpr int kThreads = 64 + kEpiThreads;
   static constexpr int kCols = BN / (kEpiWarps / 4);               // columns per epilogue thread
@@ -736,7 +738,10 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
       }
     }
     bool ok = true;                            // warp-uniform
-    float acc_f[NC];                           // Block_FP8 promoted accumulator
+    // Block_FP8 promoted accumulator, as packed fp32 pairs: the promotion is
+    // one fma.rn.f32x2 per two elements (two independent round-to-nearest
+    // FMAs, the same bits as fmaf), halving the FMA issue slots it takes
+    uint64_t acc2[NC / 2];
     if constexpr (C::kBlock) {
       float* sa_s = reinterpret_cast<float*>(smem + L.scales);          // act scales
       constexpr int act_rows = block_act_rows<SWAP, BN>();
@@ -767,7 +772,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
       }
       named_bar_sync(1, ET);
 #pragma unroll
-      for (int c = 0; c < NC; ++c) acc_f[c] = 0.f;
+      for (int c = 0; c < NC / 2; ++c) acc2[c] = 0ull;
       ok = __all_sync(0xffffffffu, fz_ok);
       for (int i = 0; i < nkt && ok; ++i) {
         const int b = i % C::kNAcc;
@@ -779,11 +784,12 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
         if (!SWAP) f_row = sa_s[row * nkt + i];
         // columns per TMEM round trip: 64 (two loads, one wait) while the
         // accumulator is small, 32 when it already holds 128 registers
-        constexpr int PB = NC >= 128 ? 32 : 64;
+        // (16 columns when 16 warps share the register file)
+        constexpr int PB = C::kEpiWarps >= 16 ? 16 : NC >= 128 ? 32 : 64;
 #pragma unroll
         for (int c0 = 0; c0 < NC; c0 += PB) {
           uint32_t v[PB];
-          if constexpr (NC % 32 == 0) {
+          if constexpr (NC % 32 == 0 && PB >= 32) {
             tmem_ld32(lane_addr + b * BN + cbeg + c0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
             if constexpr (PB == 64)
               if (c0 + 32 < NC)
@@ -795,15 +801,16 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
           if (SWAP) {
             const float sw = sw_s[i];
 #pragma unroll
-            for (int j = 0; j < PB && c0 + j < NC; ++j)
-              acc_f[c0 + j] = fmaf(__uint_as_float(v[j]), sa_s[(cbeg + c0 + j) * nkt + i] * sw, acc_f[c0 + j]);
+            for (int j = 0; j < PB && c0 + j < NC; j += 2)
+              ffma2(acc2[(c0 + j) / 2], v[j], v[j + 1],
+                    pack_f32x2(sa_s[(cbeg + c0 + j) * nkt + i] * sw, sa_s[(cbeg + c0 + j + 1) * nkt + i] * sw));
           } else {
             // one weight block per chunk (chunks start on multiples of PB
-            // and never cross a 128-column block): one FFMA per element
+            // and never cross a 128-column block): one scale for all of it
             const float f = f_row * sw_s[i * WB + (WB == 2 ? (cbeg + c0) / 128 : 0)];
+            const uint64_t f2 = pack_f32x2(f, f);
 #pragma unroll
-            for (int j = 0; j < PB && c0 + j < NC; ++j)
-              acc_f[c0 + j] = fmaf(__uint_as_float(v[j]), f, acc_f[c0 + j]);
+            for (int j = 0; j < PB && c0 + j < NC; j += 2) ffma2(acc2[(c0 + j) / 2], v[j], v[j + 1], f2);
           }
         }
         tc_fence_before();
@@ -834,7 +841,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
     auto load_chunk = [&](int c0, uint32_t (&v)[CW]) {
       if constexpr (C::kBlock) {
 #pragma unroll
-        for (int j = 0; j < CW; ++j) v[j] = __float_as_uint(acc_f[c0 + j]);
+        for (int j = 0; j < CW; j += 2) unpack_u32x2(acc2[(c0 + j) / 2], v[j], v[j + 1]);
       } else if constexpr (CW == 32) {
         tmem_ld32(lane_addr + cbeg + c0, v);
         tmem_ld_wait();

@@ -282,6 +282,22 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
           smem_u32(bar))
       : "memory");
 }
+// Packed fp32 pairs (low word = first element) and the two-wide FMA of
+// sm_100: acc.{lo,hi} = fma(x0, f.lo, acc.lo), fma(x1, f.hi, acc.hi), each
+// rounded to nearest like fmaf.
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpack_u32x2(uint64_t p, uint32_t& lo, uint32_t& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(p));
+}
+__device__ __forceinline__ void ffma2(uint64_t& acc, uint32_t x0, uint32_t x1, uint64_t f) {
+  asm("{\n\t.reg .b64 x;\n\tmov.b64 x, {%1, %2};\n\tfma.rn.f32x2 %0, x, %3, %0;\n\t}"
+      : "+l"(acc)
+      : "r"(x0), "r"(x1), "l"(f));
+}
 // smem (32 rows x 16 bytes) -> TMEM 32 lanes x 4 columns, replicated to all
 // four 32-lane sub-partitions.
 __device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
