@@ -243,11 +243,32 @@ qg_status qgemm_run_noalloc(qg_format f, const qg_operand* A, const qg_operand* 
                             int K, const qg_config* cfg, void* Y, int ldy, int out_kind,
                             void* stream);
 
-/* Default configuration for a shape when no table entry exists: swap_ab = 1
- * for M < 32 ("Helion in the vLLM backend", second paragraph: vLLM's
- * Block_FP8 backend swaps A and B below M = 32), split_k chosen so that
- * output tiles x split_k approaches the SM count. */
+/* Default configuration for a shape when no table entry exists: the
+ * configuration qgemm_rank_configs ranks first (the zero-tune default of
+ * FlashInfer PR 3948's tactic heuristic).  If no candidate of the scorer's
+ * grid is feasible, a fixed rule: swap_ab = 1 up to 64 tokens ("Helion in
+ * the vLLM backend", second paragraph: vLLM's Block_FP8 backend swaps A and
+ * B below M = 32), split_k chosen so that output tiles x split_k approaches
+ * the SM count, the deepest ring that fits. */
 qg_status qgemm_default_config(qg_format f, int M, int N, int K, qg_config* out);
+
+/* Analytic tactic scorer (FlashInfer PR 3948: rank tactics with a heuristic
+ * from the shape -- wave quantisation, efficiency, feasibility -- and tune
+ * only the top N).  The model estimates a launch's time from the bytes each
+ * CTA streams through its ring (Little's law: in-flight bytes / latency, per-SM
+ * and HBM caps), the MMA loop's cycles per K tile (plus Block_FP8
+ * promotion), waves over the SMs (shared memory, registers and TMEM columns
+ * per CTA) and the split-K reduction of each mode; its constants were fitted
+ * to the tuner's measurements of every candidate on one B200.  Host only, no
+ * device work, capture-safe.
+ *   qgemm_score_config: *est_us = the estimate for one configuration;
+ *     returns the qgemm_run status of the configuration if it is invalid.
+ *   qgemm_rank_configs: the feasible configurations of the tuner's candidate
+ *     grid, best estimate first, written to out[0 .. *n_out) (at most
+ *     max_out; est_us, if not NULL, receives the estimates).  Deterministic. */
+qg_status qgemm_score_config(qg_format f, int M, int N, int K, const qg_config* cfg, double* est_us);
+qg_status qgemm_rank_configs(qg_format f, int M, int N, int K, qg_config* out, int max_out, double* est_us,
+                             int* n_out);
 
 /* ---------------------------------------------------- table and tuning -- */
 
@@ -284,6 +305,17 @@ qg_status qgemm_dispatch(const void* table, qg_format f, int M, int N, int K, qg
  * NK holds nNK pairs (N, K). */
 qg_status qgemm_tune(void* table, qg_format f, const int* Ms, int nM, const int* NK, int nNK,
                      double budget_s_per_shape, int verbose);
+/* qgemm_tune over the top_n configurations qgemm_rank_configs ranks first
+ * instead of the whole grid (top-N pruned tuning, FlashInfer PR 3948's
+ * "autotune over a top-N ranked list"); the other arguments and the table
+ * entries are those of qgemm_tune. */
+qg_status qgemm_tune_ranked(void* table, qg_format f, const int* Ms, int nM, const int* NK, int nNK,
+                            int top_n, double budget_s_per_shape, int verbose);
+/* Tuning instrumentation: while `path` is set (NULL clears it), qgemm_tune
+ * appends one text line per timed candidate to that file:
+ *   <fmt> <M> <N> <K> <split_k> <swap_ab> <tile_n> <stages> <reduce_mode> <us>
+ * (the selection-pass step time).  Host only; not thread-safe. */
+void qgemm_set_tune_log(const char* path);
 
 /* -------------------------------------------------------------- errors -- */
 

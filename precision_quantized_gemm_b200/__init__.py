@@ -41,7 +41,8 @@ EXPORTS = [
     "qgemm_quantize_act", "qgemm_quantize_weight", "qgemm_run", "qgemm_default_config",
     "qgemm_table_load", "qgemm_table_create", "qgemm_table_put", "qgemm_table_save",
     "qgemm_table_free", "qgemm_table_size", "qgemm_dispatch", "qgemm_tune", "qgemm_device_error",
-    "qgemm_run_noalloc", "qgemm_set_trace", "qgemm_run_fused_act",
+    "qgemm_run_noalloc", "qgemm_set_trace", "qgemm_run_fused_act", "qgemm_set_tune_log",
+    "qgemm_score_config", "qgemm_rank_configs", "qgemm_tune_ranked",
 ]
 
 
@@ -109,6 +110,12 @@ def lib() -> ctypes.CDLL:
             "qgemm_tune": (c_int, [c_void_p, c_int, POINTER(c_int), c_int, POINTER(c_int), c_int, c_double, c_int]),
             "qgemm_device_error": (c_int, []),
             "qgemm_set_trace": (None, [c_void_p, c_size_t]),
+            "qgemm_set_tune_log": (None, [c_char_p]),
+            "qgemm_score_config": (c_int, [c_int, c_int, c_int, c_int, POINTER(qg_config), POINTER(c_double)]),
+            "qgemm_rank_configs": (c_int, [c_int, c_int, c_int, c_int, POINTER(qg_config), c_int,
+                                           POINTER(c_double), POINTER(c_int)]),
+            "qgemm_tune_ranked": (c_int, [c_void_p, c_int, POINTER(c_int), c_int, POINTER(c_int), c_int, c_int,
+                                          c_double, c_int]),
             "qgemm_run_noalloc": (c_int, [c_int, POINTER(qg_operand), POINTER(qg_operand), c_int, c_int, c_int,
                                           POINTER(qg_config), c_void_p, c_int, c_int, c_void_p]),
             "qgemm_run_fused_act": (c_int, [c_int, c_void_p, c_int, POINTER(qg_operand), c_int, c_int, c_int,
@@ -187,6 +194,22 @@ def qgemm_default_config(fmt, M, N, K) -> qg_config:
     return c
 
 
+def qgemm_score_config(fmt, M, N, K, cfg: qg_config) -> float:
+    """The analytic scorer's estimated µs for one configuration (raises if it is invalid)."""
+    est = c_double()
+    check(lib().qgemm_score_config(fmt, M, N, K, ctypes.byref(cfg), ctypes.byref(est)), "qgemm_score_config")
+    return est.value
+
+
+def qgemm_rank_configs(fmt, M, N, K, max_out=16):
+    """The scorer's ranking: [(qg_config, estimated µs)], best first."""
+    out = (qg_config * max(max_out, 1))()
+    est = (c_double * max(max_out, 1))()
+    n = c_int(0)
+    check(lib().qgemm_rank_configs(fmt, M, N, K, out, max_out, est, ctypes.byref(n)), "qgemm_rank_configs")
+    return [(out[i], est[i]) for i in range(n.value)]
+
+
 def qgemm_dispatch(table, fmt, M, N, K):
     c = qg_config()
     hit = c_int(0)
@@ -201,6 +224,11 @@ def qgemm_device_error():
 def qgemm_set_trace(buf_ptr, nbytes):
     """Debug: record per-CTA phase timestamps of later launches into a device buffer."""
     lib().qgemm_set_trace(buf_ptr, nbytes)
+
+
+def qgemm_set_tune_log(path):
+    """Tuning instrumentation: log every timed candidate of qgemm_tune to `path` (None: off)."""
+    lib().qgemm_set_tune_log(path.encode() if path else None)
 
 
 def qgemm_set_pdl(enable: bool):
@@ -230,10 +258,16 @@ class Table:
     def dispatch(self, fmt, M, N, K):
         return qgemm_dispatch(self.handle, fmt, M, N, K)
 
-    def tune(self, fmt, Ms, NK, budget_s_per_shape=30.0, verbose=True):
+    def tune(self, fmt, Ms, NK, budget_s_per_shape=30.0, verbose=True, top_n=0):
+        """qgemm_tune over the whole candidate grid, or (top_n > 0) qgemm_tune_ranked
+        over the scorer's top_n configurations."""
         Ms_arr = (c_int * len(Ms))(*Ms)
         flat = [v for nk in NK for v in nk]
         NK_arr = (c_int * len(flat))(*flat)
+        if top_n > 0:
+            check(lib().qgemm_tune_ranked(self.handle, fmt, Ms_arr, len(Ms), NK_arr, len(NK), int(top_n),
+                                          float(budget_s_per_shape), 1 if verbose else 0), "qgemm_tune_ranked")
+            return
         check(lib().qgemm_tune(self.handle, fmt, Ms_arr, len(Ms), NK_arr, len(NK),
                                float(budget_s_per_shape), 1 if verbose else 0), "qgemm_tune")
 

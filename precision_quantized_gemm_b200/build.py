@@ -24,7 +24,7 @@ LIB = os.path.join(PKG, "libqgemm.so")
 INCLUDE = os.path.join(ROOT, "include")
 
 SOURCES = ["api.cu", "quant.cu", "gemm_fp8.cu", "gemm_int8.cu", "gemm_block.cu", "gemm_nvf4.cu",
-           "tune.cu", "table.cpp", "noalloc.cu"]
+           "tune.cu", "table.cpp", "noalloc.cu", "scorer.cu"]
 HEADERS = ["ptx.cuh", "gemm_kernel.cuh", "gemm_launch.cuh", "internal.h", "quant_math.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -492,6 +492,29 @@ qg_status qgemm_run_fused_act(qg_format f, const void* A, int lda, const qg_oper
 qg_status qgemm_default_config(qg_format f, int M, int N, int K, qg_config* out) {
   if (!valid_format(f) || M <= 0 || N <= 0 || K <= 0 || !out) return QG_ERR_INVALID_ARG;
   if (K % k_multiple(f) != 0) return QG_ERR_INVALID_ARG;
+  // the analytic scorer's best-ranked configuration; the fixed rule below
+  // only if no candidate of the scorer's grid is feasible
+  int n = 0;
+  if (qgemm_rank_configs(f, M, N, K, out, 1, nullptr, &n) == QG_OK && n == 1) return QG_OK;
+  return qg::rule_default_config(f, M, N, K, out);
+}
+
+}  // extern "C"
+
+namespace qg {
+// Feasibility and shared memory of a configuration, for the scorer.
+qg_status config_check(qg_format f, int M, int N, int K, const qg_config* c) {
+  return check_config(f, M, N, K, c);
+}
+size_t config_smem(qg_format f, int M, int K, const qg_config* c) { return gemm_smem(f, M, K, c, false); }
+int device_sm_count() {
+  DeviceInfo* d;
+  return device_info(&d) == QG_OK ? d->sms : 148;
+}
+
+// The fixed-rule default (before the analytic scorer): Swap-AB up to 64
+// tokens, split-K filling the SMs, the deepest ring that fits.
+qg_status rule_default_config(qg_format f, int M, int N, int K, qg_config* out) {
   qg_config c = {};
   c.reduce_mode = 0;
   // Swap-AB below 32 tokens (and up to 64, where tokens still fit the MMA N
@@ -533,6 +556,9 @@ qg_status qgemm_default_config(qg_format f, int M, int N, int K, qg_config* out)
   *out = c;
   return QG_OK;
 }
+}  // namespace qg
+
+extern "C" {
 
 qg_status qgemm_device_error(void) {
   DeviceInfo* d;

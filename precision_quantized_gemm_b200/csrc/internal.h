@@ -20,6 +20,17 @@ qg_status check_run_args(qg_format f, const qg_operand* A, const qg_operand* W, 
 
 constexpr int kNvfp4AmaxMaxCtas = 296;   // partial-amax slots in the NVFP4 quant workspace
 
+// Configuration feasibility (the checks of qgemm_run), the shared memory a
+// launch takes, the SM count of the current device (148 without one), the
+// fixed-rule default configuration (api.cu).
+qg_status config_check(qg_format f, int M, int N, int K, const qg_config* c);
+size_t config_smem(qg_format f, int M, int K, const qg_config* c);
+int device_sm_count();
+qg_status rule_default_config(qg_format f, int M, int N, int K, qg_config* out);
+// The candidate grid the scorer ranks and the tuner times (scorer.cu), before
+// feasibility checks.
+void candidate_grid(qg_format f, int M, int N, int K, qg_config* out, int max_out, int* n_out);
+
 cudaError_t launch_quant_rows(bool int8, const void* X, int R, int K, int ldx, void* q,
                               float* scale, cudaStream_t st, bool pdl);
 cudaError_t launch_quant_act_groups(const void* X, int M, int K, int ldx, void* q, float* scale,

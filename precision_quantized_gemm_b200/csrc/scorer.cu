@@ -1,0 +1,187 @@
+// scorer.cu — the analytic tactic scorer: estimated time of a configuration,
+// used to rank candidates without running them.
+//
+// FlashInfer PR 3948 ("perf(gemm): update mm_fp4 cute-dsl tactic heuristic and
+// autotune over a top-N ranked list") replaces exhaustive tactic search with a
+// heuristic that ranks tactics from the shape (wave quantisation, efficiency,
+// feasibility) and tunes only the top N.  Here the ranking model is written
+// from how this kernel spends its time, with its constants fitted (least
+// squares on log time, per-shape offsets) to the tuner's measurements of
+// every candidate on one B200 (precision_quantized_gemm_b200/fit_scorer.py,
+// data in tables/b200_candidates.txt).  For one launch of configuration c:
+//
+//   rate   = min(in-flight bytes / L, per-SM bandwidth / CTAs per SM)
+//            in-flight bytes = min(stages, K tiles of the slice) x stage bytes
+//            (Little's law: a CTA keeps its ring's requests outstanding)
+//   stream = bytes one CTA loads / rate
+//   mma    = K tiles of the slice x (a0 + a1 tile_n [+ Block_FP8 promotion
+//            a2 x columns one thread promotes + a3]) cycles / clock
+//   body   = max(weight bytes / HBM bandwidth, waves x max(stream, mma))
+//   epi    = e0 x pushed token columns / 16
+//          + split-K: cluster: waves x (e1 + exchanged bytes / e2),
+//                     second pass: e3, last CTA: e4,
+//                     workspace modes: + 2 x split x M x N x 4 bytes / e5
+//   time   = body + epi   (+ a per-shape constant that ranking ignores)
+//
+// Waves and CTAs per SM follow the launch's shared memory, register budget
+// and TMEM columns.  On the 170 tuned shapes the top-ranked configuration is
+// within 1.07x of the measured best (geomean), the best of the top 8 within
+// 1.013x and of the top 16 within 1.004x; the previous fixed rule was 1.32x.
+#include <algorithm>
+#include <cmath>
+#include <vector>
+
+#include "../../include/qgemm.h"
+#include "internal.h"
+
+namespace {
+
+// Fitted constants (B200, 1965 MHz boost, measured HBM 6450.9 GB/s).
+struct Model {
+  double hbm_gbs = 6450.9;   // HBM bandwidth (measured copy bandwidth, held fixed)
+  double lat_us = 1.37010;   // load latency under load seen by one CTA's ring
+  double sm_gbs = 267.235;   // per-SM load bandwidth
+  double a0 = 524.357, a1 = 2.61095;   // MMA-loop cycles per K tile: fixed, per tile_n column
+  double a2 = 8.11785, a3 = 0.0464;    // Block_FP8 promotion cycles per K tile: per promoted column
+  double clock_mhz = 1900.0;
+  double e0 = 0.321420;      // epilogue per 16 pushed token columns, µs
+  double e1 = 2.55770;       // cluster split-K exchange, fixed, µs per wave
+  double e2 = 59.3979;       // cluster exchange bandwidth, GB/s per tile
+  double e3 = 2.72842;       // second-pass launch, µs
+  double e4 = 8.94439;       // last-CTA reduction, µs
+  double e5 = 920.860;       // workspace traffic bandwidth, GB/s
+};
+const Model kModel;
+
+constexpr int kSmemPerSm = 233472;   // 228 KB of shared memory per SM
+
+int tmem_columns(qg_format f, int tn) {
+  int used;
+  if (f == QG_BLOCK_FP8) used = (tn >= 256 ? 2 : 4) * tn;
+  else if (f == QG_NVFP4) used = tn + 16 + 16 * (tn > 128 ? 2 : 1);
+  else used = tn;
+  int cols = 32;
+  while (cols < used) cols *= 2;
+  return cols;
+}
+
+int ctas_per_sm(qg_format f, int M, int K, const qg_config& c) {
+  const bool blk = f == QG_BLOCK_FP8;
+  const int regcap = (!blk && c.tile_n <= 64) ? 3 : ((!blk || c.tile_n <= 64) ? 2 : 1);
+  const int tmemcap = 512 / tmem_columns(f, c.tile_n);
+  const size_t smem = qg::config_smem(f, M, K, &c);
+  const int smemcap = (int)(kSmemPerSm / (smem + 1024));
+  return std::max(1, std::min(std::min(regcap, tmemcap), smemcap));
+}
+
+double estimate_us(qg_format f, int M, int N, int K, const qg_config& c, int sms) {
+  const Model& m = kModel;
+  const double rb = f == QG_NVFP4 ? K / 2.0 : (double)K;
+  const int kt = (int)((rb + 127) / 128);
+  const int nkt = (kt + c.split_k - 1) / c.split_k;
+  const int rows_p = c.swap_ab ? N : M, rows_q = c.swap_ab ? M : N;
+  const double tiles = (double)((rows_p + 127) / 128) * ((rows_q + c.tile_n - 1) / c.tile_n);
+  const double ctas = tiles * c.split_k;
+  const int cps = ctas_per_sm(f, M, K, c);
+  const double waves = std::ceil(ctas / ((double)sms * cps));
+  const double stage_bytes = (128.0 + c.tile_n) * 128.0;
+  const double inflight = std::min(c.stages, nkt) * stage_bytes;
+  const double rate = std::min(inflight / m.lat_us, m.sm_gbs * 1e3 / cps);   // bytes per µs
+  const double t_stream = (128.0 + c.tile_n) * nkt * 128.0 / rate;
+  // Block_FP8 promotes on 4, 8 or 16 epilogue warps (tile_n < 128, 128,
+  // 256): the columns one thread promotes per K tile set its cost
+  const int pcols = c.tile_n / (c.tile_n >= 256 ? 4 : c.tile_n >= 128 ? 2 : 1);
+  const double kcyc = m.a0 + m.a1 * c.tile_n + (f == QG_BLOCK_FP8 ? m.a2 * pcols + m.a3 : 0.0);
+  const double t_mma = nkt * kcyc / m.clock_mhz;
+  const double hbm_bytes = (double)N * rb + (M >= 1024 ? (double)M * rb : 0.0);
+  const double body = std::max(hbm_bytes / (m.hbm_gbs * 1e3), waves * std::max(t_stream, t_mma));
+  const double mt = c.swap_ab ? std::min(M, c.tile_n) : std::min(M, 128);
+  const double pushed = c.swap_ab ? mt : c.tile_n;
+  double epi = m.e0 * pushed / 16.0;
+  if (c.split_k > 1) {
+    if (c.reduce_mode == 0) {
+      epi += waves * (m.e1 + c.split_k * 128.0 * pushed * 4.0 / (m.e2 * 1e3));
+    } else {
+      epi += (c.reduce_mode == 1 ? m.e3 : m.e4) + 2.0 * c.split_k * M * (double)N * 4.0 / (m.e5 * 1e3);
+    }
+  }
+  return body + epi;
+}
+
+}  // namespace
+
+namespace qg {
+// The candidate grid: split_k over powers of two up to the K tiles (and 256),
+// Swap-AB tiles no wider than twice the token count, standard tiles for at
+// least 64 tokens, rings of 3, 4, 6 or 8 stages, every reduction mode.
+void candidate_grid(qg_format f, int M, int N, int K, qg_config* out, int max_out, int* n_out) {
+  (void)N;
+  const int kt = (int)(((f == QG_NVFP4 ? K / 2 : K) + 127) / 128);
+  const int tiles_swap[] = {16, 32, 64, 128, 256};
+  const int tiles_std[] = {256, 128, 64};
+  const int stage_opts[] = {3, 4, 6, 8};
+  int n = 0;
+  for (int swap = 0; swap <= 1; ++swap) {
+    const int* tiles = swap ? tiles_swap : tiles_std;
+    const int ntiles = swap ? 5 : 3;
+    for (int ti = 0; ti < ntiles; ++ti) {
+      const int tn = tiles[ti];
+      if (swap && tn > 2 * std::max(16, M)) continue;     // tokens would mostly be padding
+      if (!swap && (tn < 64 || M < 64)) continue;         // standard needs a real 128-token tile
+      for (int sk = 1; sk <= 256 && sk <= kt; sk *= 2)
+        for (int st : stage_opts)
+          for (int rm = 0; rm <= (sk > 1 ? 2 : 0); ++rm) {
+            if (n < max_out) {
+              qg_config c = {};
+              c.split_k = sk;
+              c.swap_ab = swap;
+              c.tile_n = tn;
+              c.stages = st;
+              c.reduce_mode = rm;
+              out[n] = c;
+            }
+            ++n;
+          }
+    }
+  }
+  *n_out = n;
+}
+}  // namespace qg
+
+extern "C" {
+
+qg_status qgemm_score_config(qg_format f, int M, int N, int K, const qg_config* cfg, double* est_us) {
+  if (!cfg || !est_us || (int)f < 0 || (int)f > 3 || M <= 0 || N <= 0 || K <= 0) return QG_ERR_INVALID_ARG;
+  const qg_status s = qg::config_check(f, M, N, K, cfg);
+  if (s != QG_OK) return s;
+  *est_us = estimate_us(f, M, N, K, *cfg, qg::device_sm_count());
+  return QG_OK;
+}
+
+qg_status qgemm_rank_configs(qg_format f, int M, int N, int K, qg_config* out, int max_out, double* est_us,
+                             int* n_out) {
+  if (!n_out || (max_out > 0 && !out) || max_out < 0 || (int)f < 0 || (int)f > 3 || M <= 0 || N <= 0 ||
+      K <= 0)
+    return QG_ERR_INVALID_ARG;
+  int total = 0;
+  qg::candidate_grid(f, M, N, K, nullptr, 0, &total);
+  std::vector<qg_config> grid((size_t)total);
+  qg::candidate_grid(f, M, N, K, grid.data(), total, &total);
+  const int sms = qg::device_sm_count();
+  std::vector<std::pair<double, int>> scored;
+  for (int i = 0; i < total; ++i)
+    if (qg::config_check(f, M, N, K, &grid[i]) == QG_OK)
+      scored.emplace_back(estimate_us(f, M, N, K, grid[i], sms), i);
+  // ties keep grid order, so the ranking is deterministic
+  std::stable_sort(scored.begin(), scored.end(),
+                   [](const std::pair<double, int>& a, const std::pair<double, int>& b) { return a.first < b.first; });
+  const int n = std::min((int)scored.size(), max_out);
+  for (int i = 0; i < n; ++i) {
+    out[i] = grid[scored[i].second];
+    if (est_us) est_us[i] = scored[i].first;
+  }
+  *n_out = n;
+  return QG_OK;
+}
+
+}  // extern "C"

@@ -20,13 +20,18 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <string>
 #include <vector>
 
 #include "../../include/qgemm.h"
+#include "internal.h"
 
 void qg_table_set_device(void* table, const char* name, int sms);
 
 namespace {
+
+// Optional log of every timed candidate (qgemm_set_tune_log).
+std::string g_tune_log;
 
 __global__ void fill_bf16_kernel(__nv_bfloat16* p, size_t n, unsigned long long seed, float amp) {
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
@@ -136,43 +141,47 @@ double time_config(qg_format f, const std::vector<Operand*>& Ws, const Operand& 
 // 128-byte K tiles of a row.
 int kt_of(qg_format f, int K) { return (int)(((f == QG_NVFP4 ? K / 2 : K) + 127) / 128); }
 
-std::vector<qg_config> candidates(qg_format f, int M, int N, int K) {
-  std::vector<qg_config> out;
-  const int kt = kt_of(f, K);
-  // Swap-AB tiles narrow first, standard tiles wide first: within the time
-  // budget the likelier winners are timed before the others.
-  const int tiles_swap[] = {16, 32, 64, 128, 256};
-  const int tiles_std[] = {256, 128, 64};
-  const int stage_opts[] = {3, 4, 6, 8};
-  for (int swap = 0; swap <= 1; ++swap) {
-    const int* tiles = swap ? tiles_swap : tiles_std;
-    const int ntiles = swap ? 5 : 3;
-    for (int ti = 0; ti < ntiles; ++ti) {
-      const int tn = tiles[ti];
-      if (swap && tn > 2 * std::max(16, M)) continue;     // tokens would mostly be padding
-      if (!swap && (tn < 64 || M < 64)) continue;         // standard needs a real 128-token tile
-      for (int sk = 1; sk <= 256 && sk <= kt; sk *= 2) {
-        for (int st : stage_opts) {
-          for (int rm = 0; rm <= (sk > 1 ? 2 : 0); ++rm) {
-            qg_config c = {};
-            c.split_k = sk;
-            c.swap_ab = swap;
-            c.tile_n = tn;
-            c.stages = st;
-            c.reduce_mode = rm;
-            out.push_back(c);
-          }
-        }
-      }
-    }
+// The candidates timed for a shape: the scorer's whole grid (top_n <= 0), or
+// its top_n ranked configurations.  Swap-AB tiles come narrow first and
+// standard tiles wide first, so within the time budget the likelier winners
+// are timed before the others.
+std::vector<qg_config> candidates(qg_format f, int M, int N, int K, int top_n) {
+  int n = 0;
+  if (top_n > 0) {
+    std::vector<qg_config> out((size_t)top_n);
+    if (qgemm_rank_configs(f, M, N, K, out.data(), top_n, nullptr, &n) != QG_OK) n = 0;
+    out.resize((size_t)n);
+    return out;
   }
+  qg::candidate_grid(f, M, N, K, nullptr, 0, &n);
+  std::vector<qg_config> out((size_t)n);
+  qg::candidate_grid(f, M, N, K, out.data(), n, &n);
   return out;
 }
 
 }  // namespace
 
+extern "C" void qgemm_set_tune_log(const char* path) { g_tune_log = path ? path : ""; }
+
+namespace {
+qg_status tune_impl(void* table, qg_format f, const int* Ms, int nM, const int* NK, int nNK, int top_n,
+                    double budget_s_per_shape, int verbose);
+}  // namespace
+
 extern "C" qg_status qgemm_tune(void* table, qg_format f, const int* Ms, int nM, const int* NK,
                                 int nNK, double budget_s_per_shape, int verbose) {
+  return tune_impl(table, f, Ms, nM, NK, nNK, 0, budget_s_per_shape, verbose);
+}
+
+extern "C" qg_status qgemm_tune_ranked(void* table, qg_format f, const int* Ms, int nM, const int* NK,
+                                       int nNK, int top_n, double budget_s_per_shape, int verbose) {
+  if (top_n <= 0) return QG_ERR_INVALID_ARG;
+  return tune_impl(table, f, Ms, nM, NK, nNK, top_n, budget_s_per_shape, verbose);
+}
+
+namespace {
+qg_status tune_impl(void* table, qg_format f, const int* Ms, int nM, const int* NK, int nNK, int top_n,
+                    double budget_s_per_shape, int verbose) {
   if (!table || !Ms || !NK || nM <= 0 || nNK <= 0 || (int)f < 0 || (int)f > 3) return QG_ERR_INVALID_ARG;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return QG_ERR_NO_DEVICE;
@@ -228,7 +237,7 @@ extern "C" qg_status qgemm_tune(void* table, qg_format f, const int* Ms, int nM,
       if ((status = qgemm_quantize_act(f, asrc.p, M, K, K, nullptr, &A.op, qas.p, qasb, st)) != QG_OK) break;
       // workspace for the largest split
       size_t wsb = 0;
-      const auto cands = candidates(f, M, N, K);
+      const auto cands = candidates(f, M, N, K, top_n);
       for (const auto& c : cands) wsb = std::max(wsb, qgemm_workspace_size(f, M, N, K, &c));
       if (!ws.alloc(wsb)) { status = QG_ERR_CUDA; break; }
       if (wsb) cudaMemsetAsync(ws.p, 0, wsb, st);
@@ -263,6 +272,14 @@ extern "C" qg_status qgemm_tune(void* table, qg_format f, const int* Ms, int nM,
         if (us > 0 && us < best_us) { best_us = us; best = c; }
       }
       if (status != QG_OK) break;
+      if (!g_tune_log.empty()) {
+        if (FILE* lf = std::fopen(g_tune_log.c_str(), "a")) {
+          for (const auto& t : timed)
+            std::fprintf(lf, "%d %d %d %d %d %d %d %d %d %.4f\n", (int)f, M, N, K, t.second.split_k,
+                         t.second.swap_ab, t.second.tile_n, t.second.stages, t.second.reduce_mode, t.first);
+          std::fclose(lf);
+        }
+      }
       // Near-ties (within 3%) go to a configuration whose ring holds every
       // K tile of its slice: all of its weights are requested at launch, so
       // it also keeps its time after a graph boundary or a host sync, where
@@ -293,3 +310,4 @@ extern "C" qg_status qgemm_tune(void* table, qg_format f, const int* Ms, int nM,
   cudaStreamDestroy(st);
   return status;
 }
+}  // namespace

@@ -8,7 +8,10 @@ stages / reduce_mode, reject candidates whose output disagrees with the
 default configuration, select on one graph-timed pass, record an
 independent second pass) over the decode and prefill shapes of the
 quantized linear layers this library serves, and writes the table that
-qgemm_dispatch reads.  Needs a B200.
+qgemm_dispatch reads.  ``--top-n N`` times only the analytic scorer's N
+best-ranked configurations per shape (qgemm_tune_ranked); ``--log`` keeps
+every candidate's time (the data fit_scorer.py fits the scorer to).
+Needs a B200.
 """
 from __future__ import annotations
 
@@ -41,11 +44,16 @@ def main(argv=None):
     ap.add_argument("--suites", default="fp8_tiny,int8,block_fp8,nvfp4,large_m,sweep")
     ap.add_argument("--budget", type=float, default=20.0, help="seconds per shape")
     ap.add_argument("--resume", action="store_true", help="start from the existing table, skip tuned shapes")
+    ap.add_argument("--log", default=None, help="append every timed candidate to this file")
+    ap.add_argument("--top-n", type=int, default=0,
+                    help="time only the analytic scorer's top-N configurations per shape (0: the whole grid)")
     a = ap.parse_args(argv)
+    if a.log:
+        qg.qgemm_set_tune_log(a.log)
     table = qg.Table(a.out) if (a.resume and os.path.exists(a.out)) else qg.Table()
     for name in [s.strip() for s in a.suites.split(",") if s.strip()]:
         for fmt, Ms, NK in SHAPES[name]:
-            table.tune(fmt, Ms, NK, budget_s_per_shape=a.budget, verbose=True)
+            table.tune(fmt, Ms, NK, budget_s_per_shape=a.budget, verbose=True, top_n=a.top_n)
             table.save(a.out)            # checkpoint after every family
     print(f"wrote {len(table)} entries to {a.out}", flush=True)
     return 0

@@ -72,15 +72,17 @@ def test_workspace_sizes():
 
 
 def test_default_config_follows_the_swap_rule_and_fills_sms():
-    c = qg.qgemm_default_config(qg.QG_W8A8_INT8, 8, 4096, 4096)
-    assert c.swap_ab == 1 and c.tile_n == 16
-    assert c.split_k >= 2 and (c.split_k & (c.split_k - 1)) == 0
-    assert 32 * c.split_k <= 148
-    assert c.reduce_mode == 0                      # cluster reduction: no workspace
+    # the scored default (qgemm_rank_configs' first): decode shapes swap A and
+    # B and split K over a cluster until tiles x split covers most SMs; large
+    # M keeps the standard orientation with wide tiles and no split
+    for fmt, M in ((qg.QG_W8A8_INT8, 8), (qg.QG_FP8_DYNAMIC, 1), (qg.QG_BLOCK_FP8, 16)):
+        c = qg.qgemm_default_config(fmt, M, 4096, 4096)
+        assert c.swap_ab == 1 and c.tile_n <= 32
+        assert c.split_k >= 2 and (c.split_k & (c.split_k - 1)) == 0
+        assert 74 <= 32 * c.split_k * ((M + c.tile_n - 1) // c.tile_n) <= 2 * 148
+        assert c.reduce_mode == 0                      # cluster reduction: no workspace
     c = qg.qgemm_default_config(qg.QG_BLOCK_FP8, 4096, 5120, 5120)
-    assert c.swap_ab == 0 and c.tile_n == 256
-    c = qg.qgemm_default_config(qg.QG_FP8_DYNAMIC, 32, 2048, 2048)
-    assert c.swap_ab == 1 and c.tile_n == 32
+    assert c.swap_ab == 0 and c.tile_n == 256 and c.split_k == 1
 
 
 def _op(rows, K, q=FAKE, s=FAKE, g=FAKE):
