@@ -57,7 +57,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--suite", default=None,
                     help="comma list of per-shape suites to time instead of the step: "
-                         "fp8_tiny,int8,block_fp8,nvfp4,sweep,large_m (one JSON line per shape)")
+                         "fp8_tiny,int8,block_fp8,nvfp4,sweep,large_m,medium_m (one JSON line per shape)")
     return ap.parse_args()
 
 
@@ -438,6 +438,8 @@ SUITES = {
     "nvfp4": [(3, [1, 8, 64, 512], [(896, 1024), (1792, 5120), (5120, 2048), (1280, 8192)])],
     "sweep": [(0, [1, 2, 4, 8, 16, 32], SWEEP_NK), (2, [1, 2, 4, 8, 16, 32], SWEEP_NK)],
     "large_m": [(2, [4096, 16384], [(5120, 5120)])],
+    "medium_m": [(0, [64, 128, 256, 512, 1024, 2048], [(1792, 5120), (4096, 4096), (5120, 2048), (8192, 8192)]),
+                 (2, [64, 128, 256, 512, 1024, 2048], [(1792, 5120), (4096, 4096), (5120, 2048), (8192, 8192)])],
 }
 FMT_NAME = {0: "FP8_Dynamic", 1: "W8A8_INT8", 2: "Block_FP8", 3: "NVFP4"}
 
@@ -537,8 +539,10 @@ def run_suite(args, names, local):
     def geo(xs):
         return math.exp(sum(math.log(max(x, 1e-9)) for x in xs) / len(xs)) if xs else None
     small = [r["frac_roofline"] for r in results if r["M"] <= 32]
+    medium = [r["frac_roofline"] for r in results if 32 < r["M"] < 4096]
     large = [r["frac_roofline"] for r in results if r["M"] >= 4096]
     print(json.dumps({"summary": True, "shapes": len(results), "geomean_frac_roofline_M_le_32": geo(small),
+                      "geomean_frac_roofline_M_33_to_4095": geo(medium),
                       "geomean_frac_roofline_M_ge_4096": geo(large),
                       "geomean_frac_roofline_all": geo([r["frac_roofline"] for r in results]),
                       "peaks": {"hbm_gbs": hbm, "bf16_tflops": bf16,

@@ -287,9 +287,14 @@ void qgemm_table_free(void* table);
 int qgemm_table_size(const void* table);
 
 /* Looks up (f, M, N, K).  *hit = 1 on an exact entry.  On a miss the entry
- * with the same (f, N, K) and the smallest tuned M' >= M is used (*hit = 2);
- * failing that, qgemm_default_config (*hit = 0).  Host only, no device
- * work, capture-safe. */
+ * with the same (f, N, K) and the smallest tuned M' >= M is used (*hit = 2):
+ * tuned token counts act as buckets -- decode (M <= 32), medium (64 ... 2048)
+ * and large -- as in TensorRT-LLM issue 16363's policy buckets.  Failing
+ * that, qgemm_default_config (*hit = 0).  Identity gate: a table whose
+ * recorded device name or SM count differs from the current device's is not
+ * used at all (*hit = -1, qgemm_default_config); without a device, or for a
+ * table that records none ("unknown" / 0 SMs), no gate applies.  Host only,
+ * no device work beyond reading the device's properties, capture-safe. */
 qg_status qgemm_dispatch(const void* table, qg_format f, int M, int N, int K, qg_config* out,
                          int* hit);
 
@@ -305,6 +310,17 @@ qg_status qgemm_dispatch(const void* table, qg_format f, int M, int N, int K, qg
  * NK holds nNK pairs (N, K). */
 qg_status qgemm_tune(void* table, qg_format f, const int* Ms, int nM, const int* NK, int nNK,
                      double budget_s_per_shape, int verbose);
+/* Validation gate of a table (TensorRT-LLM issue 16363's shape-gated policy:
+ * a configuration that fails validation falls back to a known-good one).
+ * Runs every entry on synthetic inputs of its shape next to the scored
+ * default configuration (qgemm_default_config) and removes the entries that
+ * the kernels refuse on this device or whose bf16 output leaves
+ * |y - y_default| <= 0.01 |y_default| + 0.01 rms(y_default row); dispatch
+ * then answers those shapes with the default.  *checked / *rejected receive
+ * the counts.  Allocates device memory and synchronises: an offline step (at
+ * table load), not a run-path call.  verbose != 0 prints each rejection. */
+qg_status qgemm_table_validate(void* table, int* checked, int* rejected, int verbose);
+
 /* qgemm_tune over the top_n configurations qgemm_rank_configs ranks first
  * instead of the whole grid (top-N pruned tuning, FlashInfer PR 3948's
  * "autotune over a top-N ranked list"); the other arguments and the table

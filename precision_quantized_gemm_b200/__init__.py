@@ -42,7 +42,7 @@ EXPORTS = [
     "qgemm_table_load", "qgemm_table_create", "qgemm_table_put", "qgemm_table_save",
     "qgemm_table_free", "qgemm_table_size", "qgemm_dispatch", "qgemm_tune", "qgemm_device_error",
     "qgemm_run_noalloc", "qgemm_set_trace", "qgemm_run_fused_act", "qgemm_set_tune_log",
-    "qgemm_score_config", "qgemm_rank_configs", "qgemm_tune_ranked",
+    "qgemm_score_config", "qgemm_rank_configs", "qgemm_tune_ranked", "qgemm_table_validate",
 ]
 
 
@@ -116,6 +116,7 @@ def lib() -> ctypes.CDLL:
                                            POINTER(c_double), POINTER(c_int)]),
             "qgemm_tune_ranked": (c_int, [c_void_p, c_int, POINTER(c_int), c_int, POINTER(c_int), c_int, c_int,
                                           c_double, c_int]),
+            "qgemm_table_validate": (c_int, [c_void_p, POINTER(c_int), POINTER(c_int), c_int]),
             "qgemm_run_noalloc": (c_int, [c_int, POINTER(qg_operand), POINTER(qg_operand), c_int, c_int, c_int,
                                           POINTER(qg_config), c_void_p, c_int, c_int, c_void_p]),
             "qgemm_run_fused_act": (c_int, [c_int, c_void_p, c_int, POINTER(qg_operand), c_int, c_int, c_int,
@@ -270,6 +271,14 @@ class Table:
             return
         check(lib().qgemm_tune(self.handle, fmt, Ms_arr, len(Ms), NK_arr, len(NK),
                                float(budget_s_per_shape), 1 if verbose else 0), "qgemm_tune")
+
+    def validate(self, verbose=False):
+        """qgemm_table_validate: run every entry next to the scored default and drop
+        the ones refused or out of tolerance; returns (checked, rejected)."""
+        checked, rejected = c_int(0), c_int(0)
+        check(lib().qgemm_table_validate(self.handle, ctypes.byref(checked), ctypes.byref(rejected),
+                                         1 if verbose else 0), "qgemm_table_validate")
+        return checked.value, rejected.value
 
     def close(self):
         if getattr(self, "handle", None) is not None and self.handle.value:

@@ -501,6 +501,22 @@ qg_status qgemm_default_config(qg_format f, int M, int N, int K, qg_config* out)
 
 }  // extern "C"
 
+// Name (spaces as '_') and SM count of the current device, for the table's
+// identity gate; false without a device.
+bool qg_current_device(char* name, size_t cap, int* sms) {
+  int dev = 0;
+  cudaDeviceProp p;
+  if (cap == 0 || cudaGetDevice(&dev) != cudaSuccess || cudaGetDeviceProperties(&p, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  std::snprintf(name, cap, "%s", p.name);
+  for (char* c = name; *c; ++c)
+    if (*c == ' ') *c = '_';
+  *sms = p.multiProcessorCount;
+  return true;
+}
+
 namespace qg {
 // Feasibility and shared memory of a configuration, for the scorer.
 qg_status config_check(qg_format f, int M, int N, int K, const qg_config* c) {

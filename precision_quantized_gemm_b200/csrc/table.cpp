@@ -24,6 +24,9 @@
 
 #include "../../include/qgemm.h"
 
+// Name (spaces as '_') and SM count of the current device; false without one.
+bool qg_current_device(char* name, size_t cap, int* sms);
+
 namespace {
 
 struct Entry {
@@ -134,6 +137,16 @@ qg_status qgemm_dispatch(const void* table, qg_format f, int M, int N, int K, qg
   if (!out || !hit || M <= 0 || N <= 0 || K <= 0 || (int)f < 0 || (int)f > 3) return QG_ERR_INVALID_ARG;
   if (table) {
     const Table* t = static_cast<const Table*>(table);
+    // identity gate: a table tuned on another device (name or SM count) is
+    // not used; the scored default stands in (hit = -1)
+    if (t->sms > 0 && t->device != "unknown") {
+      char name[256];
+      int sms = 0;
+      if (qg_current_device(name, sizeof(name), &sms) && (sms != t->sms || t->device != name)) {
+        *hit = -1;
+        return qgemm_default_config(f, M, N, K, out);
+      }
+    }
     auto it = t->entries.lower_bound(Key((int)f, N, K, M));
     if (it != t->entries.end()) {
       int ef, eN, eK, eM;
@@ -151,9 +164,25 @@ qg_status qgemm_dispatch(const void* table, qg_format f, int M, int N, int K, qg
 
 }  // extern "C"
 
-// Used by the tuner to stamp the table with the device it was tuned on.
+// Used by the tuner to stamp the table with the device it was tuned on
+// (spaces in the name become '_', as in the file).
 void qg_table_set_device(void* table, const char* name, int sms) {
   Table* t = static_cast<Table*>(table);
   t->device = name ? name : "unknown";
+  std::replace(t->device.begin(), t->device.end(), ' ', '_');
   t->sms = sms;
+}
+
+// Entries in key order, for the validation gate; and their removal.
+int qg_table_entry(const void* table, int i, int* f, int* M, int* N, int* K, qg_config* cfg) {
+  const Table* t = static_cast<const Table*>(table);
+  if (i < 0 || i >= (int)t->entries.size()) return 0;
+  auto it = t->entries.begin();
+  std::advance(it, i);
+  std::tie(*f, *N, *K, *M) = it->first;
+  *cfg = it->second.cfg;
+  return 1;
+}
+void qg_table_erase(void* table, int f, int M, int N, int K) {
+  static_cast<Table*>(table)->entries.erase(Key(f, N, K, M));
 }

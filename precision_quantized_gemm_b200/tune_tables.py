@@ -27,6 +27,8 @@ DEFAULT_OUT = os.path.join(HERE, "tables", "b200.qgt")
 # (format, token counts, (N, K) pairs): LLM projection shapes.
 SWEEP_NK = [(896, 5120), (1024, 7168), (1280, 8192), (1792, 5120), (2560, 8192), (4096, 4096),
             (4608, 7168), (5120, 640), (5120, 2048), (6144, 4096), (7168, 2048), (8192, 8192)]
+MEDIUM_M = [64, 128, 256, 512, 1024, 2048]
+MEDIUM_NK = [(1792, 5120), (4096, 4096), (5120, 2048), (8192, 8192)]
 SHAPES = {
     "fp8_tiny": [(qg.QG_FP8_DYNAMIC, [16], [(2048, 2048)])],
     "int8": [(qg.QG_W8A8_INT8, [1, 8, 32], [(4096, 4096)])],
@@ -35,13 +37,16 @@ SHAPES = {
     "sweep": [(qg.QG_FP8_DYNAMIC, [1, 2, 4, 8, 16, 32], SWEEP_NK),
               (qg.QG_BLOCK_FP8, [1, 2, 4, 8, 16, 32], SWEEP_NK)],
     "large_m": [(qg.QG_BLOCK_FP8, [4096, 16384], [(5120, 5120)])],
+    # medium token counts (prefill chunks, batched decode): the buckets between
+    # decode and large M
+    "medium_m": [(qg.QG_FP8_DYNAMIC, MEDIUM_M, MEDIUM_NK), (qg.QG_BLOCK_FP8, MEDIUM_M, MEDIUM_NK)],
 }
 
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--out", default=DEFAULT_OUT)
-    ap.add_argument("--suites", default="fp8_tiny,int8,block_fp8,nvfp4,large_m,sweep")
+    ap.add_argument("--suites", default="fp8_tiny,int8,block_fp8,nvfp4,large_m,sweep,medium_m")
     ap.add_argument("--budget", type=float, default=20.0, help="seconds per shape")
     ap.add_argument("--resume", action="store_true", help="start from the existing table, skip tuned shapes")
     ap.add_argument("--log", default=None, help="append every timed candidate to this file")
