@@ -57,7 +57,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--suite", default=None,
                     help="comma list of per-shape suites to time instead of the step: "
-                         "fp8_tiny,int8,block_fp8,nvfp4,sweep,large_m,medium_m (one JSON line per shape)")
+                         "fp8_tiny,int8,block_fp8,nvfp4,sweep,large_m,medium_m,moe (one JSON line per shape)")
     return ap.parse_args()
 
 
@@ -459,6 +459,130 @@ def tensor_peak(fmt, bf16_tflops):
     return bf16_tflops * (4.0 if fmt == 3 else 2.0)
 
 
+# Mixture-of-experts layer of 128 experts, top-8 routing, hidden size 2048
+# and expert intermediate size 768 (gate and up projections stacked: N = 1536,
+# K = 2048; down projection: N = 2048, K = 768), at decode token counts.
+MOE_EXPERTS, MOE_TOPK = 128, 8
+MOE_NK = [(1536, 2048), (2048, 768)]
+MOE_TOKENS = [1, 4, 16, 64]
+MOE_FMTS = [0, 1, 2]
+
+
+def moe_routing(T, seed):
+    """Seeded top-k routing: each token picks MOE_TOPK distinct experts
+    uniformly.  Returns tokens per expert (assignments sorted by expert)."""
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    picks = np.stack([rng.permutation(MOE_EXPERTS)[:MOE_TOPK] for _ in range(T)])
+    return np.bincount(picks.ravel(), minlength=MOE_EXPERTS)
+
+
+def run_moe_suite(args, local):
+    import numpy as np
+    import torch
+
+    import precision_quantized_gemm_b200 as qg
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pk = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
+        os.path.join(ROOT, "MEASURED_PEAKS.json")) else {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+    hbm = float(pk["hbm_gbs"])
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0)
+    E = MOE_EXPERTS
+    results = []
+    for fmt in MOE_FMTS:
+        for (N, K) in MOE_NK:
+            w = (torch.randn(E * N, K, device=dev, generator=gen) * 0.02).to(torch.bfloat16)
+            Wq = qg.quantize_weight(fmt, w)
+            del w
+            for T in MOE_TOKENS:
+                counts = moe_routing(T, seed=1000 + T)
+                rows = int(counts.sum())
+                offs = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+                offsets = torch.from_numpy(offs).to(dev)
+                active = [e for e in range(E) if counts[e] > 0]
+                sb_row = 4 * (K // 128) if fmt == 2 else 4
+                w_bytes = len(active) * (N * K + (4 * (N // 128) * (K // 128) if fmt == 2 else 4 * N))
+                byts = w_bytes + rows * (K + sb_row) + 2 * rows * N
+                # rotate weight copies past 2 x L2 so each call streams from HBM
+                copies = int(max(1, min(32, (2 * l2) // max(w_bytes, 1) + 2)))
+                Ws = [Wq]
+                for _ in range(copies - 1):
+                    o = qg.Operand(fmt, True, E * N, K, dev)
+                    o.q.copy_(Wq.q)
+                    o.scale.copy_(Wq.scale)
+                    o.global_scale.copy_(Wq.global_scale)
+                    Ws.append(o)
+                a = torch.randn(rows, K, device=dev, generator=gen).to(torch.bfloat16)
+                A = qg.quantize_act(fmt, a)
+                cfg = qg.qgemm_grouped_default_config(fmt, E, rows, N, K)
+                ws = qg.Workspace(dev)
+                wsp, wsb = ws.get(qg.qgemm_workspace_size(fmt, rows, N, K, cfg))
+                Y = torch.empty(rows, N, dtype=torch.bfloat16, device=dev)
+                reps = max(2 * copies, 8)
+
+                def grouped(Wo, st):
+                    qg.check(qg.qgemm_run_grouped(fmt, E, offsets.data_ptr(), A.c, Wo.c, N, K, cfg, wsp, wsb,
+                                                  Y.data_ptr(), N, 0, st))
+
+                # the baseline: one qgemm_run per active expert on its slices
+                ecfg = {e: qg.qgemm_default_config(fmt, int(counts[e]), N, K) for e in active}
+                ews = qg.Workspace(dev)
+                ewsp, ewsb = ews.get(max(qg.qgemm_workspace_size(fmt, int(counts[e]), N, K, ecfg[e])
+                                         for e in active))
+
+                def per_expert(Wo, st):
+                    for e in active:
+                        m0, m = int(offs[e]), int(counts[e])
+                        s_a = A.scale.data_ptr() + m0 * sb_row
+                        s_w = Wo.scale.data_ptr() + (e * N // 128 * (K // 128) * 4 if fmt == 2 else e * N * 4)
+                        Ae = qg.qg_operand(A.q.data_ptr() + m0 * K, s_a, A.global_scale.data_ptr(), m, K)
+                        We = qg.qg_operand(Wo.q.data_ptr() + e * N * K, s_w, Wo.global_scale.data_ptr(), N, K)
+                        qg.check(qg.qgemm_run(fmt, Ae, We, m, N, K, ecfg[e], ewsp, ewsb,
+                                              Y.data_ptr() + m0 * N * 2, N, 0, st))
+
+                times = {}
+                for name, fn in (("grouped", grouped), ("per_expert", per_expert)):
+                    fn(Ws[0], qg._stream(None))
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g):
+                        st = qg._stream(None)
+                        for r in range(reps):
+                            fn(Ws[r % copies], st)
+                    g.replay()
+                    torch.cuda.synchronize()
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    for _ in range(5):
+                        g.replay()
+                    e1.record()
+                    torch.cuda.synchronize()
+                    times[name] = 1000.0 * e0.elapsed_time(e1) / (5 * reps)
+                    del g
+                us = times["grouped"]
+                t_hbm = byts / (hbm * 1e9) * 1e6
+                rec = {"suite": "moe", "format": FMT_NAME[fmt], "experts": E, "top_k": MOE_TOPK, "tokens": T,
+                       "assignments": rows, "active_experts": len(active), "N": N, "K": K, "us": round(us, 3),
+                       "GB/s": round(byts / us / 1e3, 1), "bound": "hbm", "roofline_us": round(t_hbm, 3),
+                       "frac_roofline": round(t_hbm / us, 4), "per_expert_launches_us": round(times["per_expert"], 3),
+                       "speedup_vs_per_expert": round(times["per_expert"] / us, 2), "config": cfg.as_dict(),
+                       "rotating_copies": copies}
+                print(json.dumps(rec), flush=True)
+                results.append(rec)
+                del Ws[1:], Y, A
+                torch.cuda.empty_cache()
+    fr = [r["frac_roofline"] for r in results]
+    sp = [r["speedup_vs_per_expert"] for r in results]
+    print(json.dumps({"summary": True, "suite": "moe", "shapes": len(results),
+                      "geomean_frac_roofline": math.exp(sum(math.log(x) for x in fr) / len(fr)),
+                      "geomean_speedup_vs_per_expert": math.exp(sum(math.log(x) for x in sp) / len(sp)),
+                      "peaks": {"hbm_gbs": hbm}}), flush=True)
+
+
 def run_suite(args, names, local):
     import numpy as np
     import torch
@@ -554,7 +678,12 @@ def main():
     world, rank, local = dist_setup()
     try:
         if args.suite:
-            run_suite(args, [s.strip() for s in args.suite.split(",") if s.strip()], local)
+            names = [s.strip() for s in args.suite.split(",") if s.strip()]
+            if "moe" in names:
+                run_moe_suite(args, local)
+                names.remove("moe")
+            if names:
+                run_suite(args, names, local)
         elif args.impl == "reference":
             run_reference(args, world, rank)
         else:

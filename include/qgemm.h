@@ -192,6 +192,45 @@ qg_status qgemm_run(qg_format f, const qg_operand* A, const qg_operand* W, int M
                     const qg_config* cfg, void* workspace, size_t ws_bytes, void* Y, int ldy,
                     int out_kind, void* stream);
 
+/* Grouped GEMM for a mixture-of-experts layer ("Helion in the vLLM
+ * backend", last paragraph: an MoE backend is the next target): for every
+ * expert e and every token t routed to it,
+ *     y[t, :] = dequant(A_q)[t, :] . dequant(W_q[e])^T,
+ * in one launch.  Tokens are sorted by expert: expert e owns rows
+ * [expert_offsets[e], expert_offsets[e + 1]) of A and y.
+ *   experts:        1 ... 256.
+ *   expert_offsets: DEVICE int32 [experts + 1], nondecreasing, [0] = 0,
+ *                   [experts] = A->rows; read by the kernel after it waits on
+ *                   the preceding kernel of the stream (the routing), so the
+ *                   call needs no host copy and can be captured.  Offsets
+ *                   outside [0, A->rows] are clamped on the device.
+ *   A:  activations of all T = A->rows tokens (quantised as one operand).
+ *   W:  all experts' weights stacked, W->rows = experts * N, expert e's rows
+ *       at [e * N, (e + 1) * N); per-channel scales [experts * N] or 128x128
+ *       block scales [experts * N / 128, K / 128].  N must be a multiple of
+ *       128 (no 128-row block straddles two experts).
+ *   Y:  [T, ldy]; cfg: swap_ab = 1 (a decode expert sees few tokens), any
+ *       split_k with reduce_mode 0 or 1 (workspace as qgemm_workspace_size(f,
+ *       T, N, K, cfg)); tile_n is the token tile.
+ * The grid covers floor((T - a) / tile_n) + a token tiles, a = min(experts,
+ * T): the most that any routing of T tokens over the experts needs.  A CTA
+ * finds its expert and tokens with a warp scan over the offsets and exits if
+ * it has none.  Weights are loaded after that lookup (which experts run depends on
+ * the routing).  FP8_DYNAMIC, W8A8_INT8 and BLOCK_FP8; NVFP4 returns
+ * QG_ERR_UNSUPPORTED (its scale atoms need 128-aligned token tiles). */
+qg_status qgemm_run_grouped(qg_format f, int experts, const int* expert_offsets, const qg_operand* A,
+                            const qg_operand* W, int N, int K, const qg_config* cfg, void* workspace,
+                            size_t ws_bytes, void* Y, int ldy, int out_kind, void* stream);
+
+/* Default configuration of a grouped launch of T tokens over `experts`
+ * experts, without the routing: at most min(experts, T) experts are active
+ * and the launch streams their weights, so the configuration is the
+ * scorer's first-ranked one for min(experts, T) * N weight rows and
+ * ceil(T / active) tokens among those qgemm_run_grouped accepts (swap_ab = 1,
+ * reduce_mode 0 or 1); else split_k 1, tile_n 16, 4 stages.  NVFP4 returns
+ * QG_ERR_UNSUPPORTED. */
+qg_status qgemm_grouped_default_config(qg_format f, int experts, int T, int N, int K, qg_config* out);
+
 /* Activation quantisation fused into the GEMM: y = dequant(quant(A)) .
  * dequant(W_q)^T for bf16 activations A, in one kernel.  The pages name the
  * dynamic activation quantisation among the auxiliary kernels around the

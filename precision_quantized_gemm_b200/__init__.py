@@ -43,6 +43,7 @@ EXPORTS = [
     "qgemm_table_free", "qgemm_table_size", "qgemm_dispatch", "qgemm_tune", "qgemm_device_error",
     "qgemm_run_noalloc", "qgemm_set_trace", "qgemm_run_fused_act", "qgemm_set_tune_log",
     "qgemm_score_config", "qgemm_rank_configs", "qgemm_tune_ranked", "qgemm_table_validate",
+    "qgemm_run_grouped", "qgemm_grouped_default_config",
 ]
 
 
@@ -117,6 +118,10 @@ def lib() -> ctypes.CDLL:
             "qgemm_tune_ranked": (c_int, [c_void_p, c_int, POINTER(c_int), c_int, POINTER(c_int), c_int, c_int,
                                           c_double, c_int]),
             "qgemm_table_validate": (c_int, [c_void_p, POINTER(c_int), POINTER(c_int), c_int]),
+            "qgemm_grouped_default_config": (c_int, [c_int, c_int, c_int, c_int, c_int, POINTER(qg_config)]),
+            "qgemm_run_grouped": (c_int, [c_int, c_int, c_void_p, POINTER(qg_operand), POINTER(qg_operand), c_int,
+                                          c_int, POINTER(qg_config), c_void_p, c_size_t, c_void_p, c_int, c_int,
+                                          c_void_p]),
             "qgemm_run_noalloc": (c_int, [c_int, POINTER(qg_operand), POINTER(qg_operand), c_int, c_int, c_int,
                                           POINTER(qg_config), c_void_p, c_int, c_int, c_void_p]),
             "qgemm_run_fused_act": (c_int, [c_int, c_void_p, c_int, POINTER(qg_operand), c_int, c_int, c_int,
@@ -189,9 +194,22 @@ def qgemm_run_fused_act(fmt, A_ptr, lda, W: qg_operand, M, N, K, cfg: qg_config,
                                      ws_bytes, Y_ptr, ldy, out_kind, act_scale_ptr, stream)
 
 
+def qgemm_run_grouped(fmt, experts, offsets_ptr, A: qg_operand, W: qg_operand, N, K, cfg: qg_config, ws_ptr,
+                      ws_bytes, Y_ptr, ldy, out_kind, stream):
+    """Grouped (mixture-of-experts) GEMM over tokens sorted by expert."""
+    return lib().qgemm_run_grouped(fmt, experts, offsets_ptr, ctypes.byref(A), ctypes.byref(W), N, K,
+                                   ctypes.byref(cfg), ws_ptr, ws_bytes, Y_ptr, ldy, out_kind, stream)
+
+
 def qgemm_default_config(fmt, M, N, K) -> qg_config:
     c = qg_config()
     check(lib().qgemm_default_config(fmt, M, N, K, ctypes.byref(c)), "qgemm_default_config")
+    return c
+
+
+def qgemm_grouped_default_config(fmt, experts, T, N, K) -> qg_config:
+    c = qg_config()
+    check(lib().qgemm_grouped_default_config(fmt, experts, T, N, K, ctypes.byref(c)), "qgemm_grouped_default_config")
     return c
 
 
@@ -392,6 +410,25 @@ def run_fused(fmt: int, A, W: Operand, cfg: qg_config | None = None, out=None,
     sp = act_scale_out.data_ptr() if act_scale_out is not None else None
     check(qgemm_run_fused_act(fmt, A.data_ptr(), A.stride(0), W.c, M, N, K, cfg, wsp, wsb, out.data_ptr(),
                               out.stride(0), out_kind, sp, _stream(stream)), "qgemm_run_fused_act")
+    return out
+
+
+def run_grouped(fmt: int, A: Operand, W: Operand, offsets, N: int, cfg: qg_config | None = None, out=None,
+                out_kind: int = QG_OUT_BF16, workspace: Workspace | None = None, stream=None):
+    """y = per-expert dequant(A_q) . dequant(W_q[e])^T through qgemm_run_grouped.
+    ``offsets``: device int32 [experts + 1] token offsets (tokens sorted by
+    expert); W: the experts' weights stacked, W.rows = experts * N."""
+    torch = _torch()
+    T, K = A.rows, A.K
+    experts = offsets.numel() - 1
+    cfg = cfg or qgemm_grouped_default_config(fmt, experts, T, N, K)
+    if out is None:
+        dt = torch.bfloat16 if out_kind == QG_OUT_BF16 else (torch.int32 if fmt == QG_W8A8_INT8 else torch.float32)
+        out = torch.empty(T, N, dtype=dt, device=A.q.device)
+    workspace = workspace or Workspace(A.q.device)
+    wsp, wsb = workspace.get(qgemm_workspace_size(fmt, T, N, K, cfg))
+    check(qgemm_run_grouped(fmt, experts, offsets.data_ptr(), A.c, W.c, N, K, cfg, wsp, wsb, out.data_ptr(),
+                            out.stride(0), out_kind, _stream(stream)), "qgemm_run_grouped")
     return out
 
 

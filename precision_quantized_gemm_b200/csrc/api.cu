@@ -4,6 +4,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
+#include <cstdint>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -388,7 +390,8 @@ namespace {
 // when the kernel quantises the bf16 activations `act` itself (fused).
 qg_status launch_run(qg_format f, const qg_operand* A, const void* act, int lda, float* act_scale_out,
                      const qg_operand* W, int M, int N, int K, const qg_config* cfg, void* workspace,
-                     void* Y, int ldy, int out_kind, void* stream) {
+                     void* Y, int ldy, int out_kind, void* stream, int experts = 0,
+                     const int* expert_offsets = nullptr) {
   DeviceInfo* d;
   qg_status s;
   if ((s = device_info(&d)) != QG_OK) return s;
@@ -431,6 +434,8 @@ qg_status launch_run(qg_format f, const qg_operand* A, const void* act, int lda,
   prm.nkt_max = ls.nkt_max;
   prm.recv_cols = ls.recv_cols;
   prm.a_mode = ls.a_mode;
+  prm.experts = experts;
+  prm.expert_offsets = expert_offsets;
   prm.err = d->err;
   if (g_trace != nullptr &&
       (size_t)tp * tq * cfg->split_k * qg::kTraceEvents * sizeof(unsigned long long) <= g_trace_bytes)
@@ -438,12 +443,24 @@ qg_status launch_run(qg_format f, const qg_operand* A, const void* act, int lda,
 
   CUtensorMap tmp, tmq;
   const uint64_t rb = row_bytes(f, K);
-  if (!make_tmap(&tmp, swap ? W->q : A->q, rb, (uint64_t)prm.rows_p, 128)) return QG_ERR_CUDA;
+  // grouped: the P tensor is every expert's weight rows, [experts * N, K]
+  const uint64_t p_rows = expert_offsets ? (uint64_t)experts * N : (uint64_t)prm.rows_p;
+  if (!make_tmap(&tmp, swap ? W->q : A->q, rb, p_rows, 128)) return QG_ERR_CUDA;
   if (A != nullptr) {
     if (!make_tmap(&tmq, swap ? A->q : W->q, rb, (uint64_t)prm.rows_q, (uint32_t)cfg->tile_n))
       return QG_ERR_CUDA;
   } else {
     tmq = tmp;                                 // fused: the kernel writes the Q tiles itself
+  }
+  // grouped: one y index per token tile of any expert.  An expert with c > 0
+  // tokens has ceil(c / tile_n) <= (c - 1) / tile_n + 1 tiles; over at most
+  // a = min(experts, M) such experts that sums to at most
+  // floor((M - a) / tile_n) + a (nondecreasing in the number of experts), so
+  // the grid needs no routing from the host.  CTAs past the last tile exit,
+  // and each costs launch and retire time, so the bound is kept tight.
+  if (expert_offsets) {
+    const int a = std::min(experts, M);
+    tq = (M - a) / cfg->tile_n + a;
   }
   if (tq > 65535) return QG_ERR_UNSUPPORTED;
   const dim3 grid(tp, tq, cfg->split_k);
@@ -479,6 +496,27 @@ qg_status qgemm_run(qg_format f, const qg_operand* A, const qg_operand* W, int M
   return launch_run(f, A, nullptr, 0, nullptr, W, M, N, K, cfg, workspace, Y, ldy, out_kind, stream);
 }
 
+qg_status qgemm_run_grouped(qg_format f, int experts, const int* expert_offsets, const qg_operand* A,
+                            const qg_operand* W, int N, int K, const qg_config* cfg, void* workspace,
+                            size_t ws_bytes, void* Y, int ldy, int out_kind, void* stream) {
+  if (!valid_format(f) || experts <= 0 || !expert_offsets || !A || !W || !aligned(expert_offsets, 4))
+    return QG_ERR_INVALID_ARG;
+  if (experts > qg::kMaxExperts) return QG_ERR_UNSUPPORTED;
+  if (f == QG_NVFP4) return QG_ERR_UNSUPPORTED;           // scale atoms need 128-aligned token tiles
+  if (N <= 0 || N % 128 != 0) return QG_ERR_INVALID_ARG;   // experts' weight rows fill whole 128-row blocks
+  if ((long long)experts * N > 0x7fffffffLL) return QG_ERR_INVALID_ARG;
+  const int M = A->rows;
+  qg_operand Wall = *W;                                    // the operand checks see one expert's rows
+  if (W->rows != experts * N) return QG_ERR_INVALID_ARG;
+  Wall.rows = N;
+  qg_status s = qg::check_run_args(f, A, &Wall, M, N, K, cfg, workspace, ws_bytes, Y, ldy, out_kind);
+  if (s != QG_OK) return s;
+  if (cfg->swap_ab != 1) return QG_ERR_UNSUPPORTED;
+  if (cfg->split_k > 1 && cfg->reduce_mode == qg::kReduceLastCta) return QG_ERR_UNSUPPORTED;
+  return launch_run(f, A, nullptr, 0, nullptr, W, M, N, K, cfg, workspace, Y, ldy, out_kind, stream, experts,
+                    expert_offsets);
+}
+
 qg_status qgemm_run_fused_act(qg_format f, const void* A, int lda, const qg_operand* W, int M, int N,
                               int K, const qg_config* cfg, void* workspace, size_t ws_bytes, void* Y,
                               int ldy, int out_kind, float* act_scale_out, void* stream) {
@@ -497,6 +535,37 @@ qg_status qgemm_default_config(qg_format f, int M, int N, int K, qg_config* out)
   int n = 0;
   if (qgemm_rank_configs(f, M, N, K, out, 1, nullptr, &n) == QG_OK && n == 1) return QG_OK;
   return qg::rule_default_config(f, M, N, K, out);
+}
+
+qg_status qgemm_grouped_default_config(qg_format f, int experts, int T, int N, int K, qg_config* out) {
+  if (!valid_format(f) || experts <= 0 || T <= 0 || N <= 0 || K <= 0 || !out) return QG_ERR_INVALID_ARG;
+  if (f == QG_NVFP4) return QG_ERR_UNSUPPORTED;
+  if (K % k_multiple(f) != 0) return QG_ERR_INVALID_ARG;
+  // T tokens over at most min(experts, T) experts: the launch streams the
+  // weights of the active experts, like one GEMM of active x N rows with the
+  // mean token count per expert
+  const int active = std::min(experts, T);
+  const int m_eff = (T + active - 1) / active;
+  const long long rows = (long long)active * N;
+  if (rows <= (long long)INT32_MAX) {
+    qg_config ranked[256];
+    int n = 0;
+    if (qgemm_rank_configs(f, m_eff, (int)rows, K, ranked, 256, nullptr, &n) == QG_OK)
+      for (int i = 0; i < n; ++i)
+        if (ranked[i].swap_ab == 1 && ranked[i].reduce_mode != 2 &&
+            qg::config_check(f, T, N, K, &ranked[i]) == QG_OK) {
+          *out = ranked[i];
+          return QG_OK;
+        }
+  }
+  qg_config c = {};
+  c.split_k = 1;
+  c.swap_ab = 1;
+  c.tile_n = 16;
+  c.stages = 4;
+  if (qg::config_check(f, T, N, K, &c) != QG_OK) return QG_ERR_UNSUPPORTED;
+  *out = c;
+  return QG_OK;
 }
 
 }  // extern "C"

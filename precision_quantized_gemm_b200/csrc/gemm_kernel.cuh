@@ -89,7 +89,14 @@ struct GemmParams {
   int lda;
   float* act_scale_out;        // optional: the activation scales (per token, or [M, K/128])
   int a_mode;                  // kActTma / kActFused: how the Q (activation) tiles fill
+  // Grouped (mixture-of-experts) launch: tokens sorted by expert, expert e
+  // owning rows [expert_offsets[e], expert_offsets[e + 1]) of A and y, and
+  // weight rows [e * N, (e + 1) * N) of W_q.
+  const int* expert_offsets;   // device, experts + 1 ints
+  int experts;
 };
+
+constexpr int kMaxExperts = 256;
 
 // Phase timestamps (%globaltimer, ns) a traced launch records per CTA.
 enum TraceEvent : int {
@@ -285,7 +292,59 @@ __device__ __forceinline__ void emit(const GemmParams& prm, int r, int c, int m,
       __float2bfloat16_rn(finish_value<FMT>(acc_bits, sa, sw, alpha));
 }
 
-template <int FMT, bool SWAP, int BN, bool FUSED>
+// Grouped launches: the token tile of a CTA.  blockIdx.y enumerates the
+// token tiles of all experts in expert order (ceil(tokens_e / BN) per expert).
+// Lane l owns experts [8 l, 8 l + 8): it sums their tile counts, one warp
+// scan turns the sums into each lane's first tile, the lane whose range holds
+// blockIdx.y walks its eight experts to the one it falls in.  Offsets come
+// from the preceding kernel (routing) and are clamped to [0, M], so a
+// malformed routing never leads to an access outside A or y.  Writes {expert
+// (-1: no tile), first token, tokens} to map.
+template <int BN>
+__device__ __forceinline__ void grouped_tile(const GemmParams& prm, int lane, int* map) {
+  constexpr unsigned kFull = 0xffffffffu;
+  constexpr int kPer = kMaxExperts / 32;
+  const int E = prm.experts;
+  const int y = blockIdx.y;
+  const int e0 = lane * kPer;
+  int ov[kPer + 1];                            // offsets[e0 .. e0 + kPer], past E: offsets[E]
+#pragma unroll
+  for (int j = 0; j <= kPer; ++j)
+    ov[j] = min(max(__ldcg(prm.expert_offsets + min(e0 + j, E)), 0), prm.M);
+  int sum = 0;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) sum += (max(ov[j + 1] - ov[j], 0) + BN - 1) / BN;
+  int incl = sum;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int t = __shfl_up_sync(kFull, incl, d);
+    if (lane >= d) incl += t;
+  }
+  const int excl = incl - sum;
+  const unsigned hit = __ballot_sync(kFull, y >= excl && y < incl);
+  if (hit == 0u) {
+    if (lane == 0) map[0] = -1;
+    return;
+  }
+  if (lane == __ffs(hit) - 1) {
+    int base = excl;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int cnt = max(ov[j + 1] - ov[j], 0);
+      const int t = (cnt + BN - 1) / BN;
+      if (y < base + t) {
+        const int tile = y - base;
+        map[0] = e0 + j;
+        map[1] = ov[j] + tile * BN;
+        map[2] = min(BN, cnt - tile * BN);
+        break;
+      }
+      base += t;
+    }
+  }
+}
+
+template <int FMT, bool SWAP, int BN, bool FUSED, bool GROUPED>
 __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBlocks)
     qgemm_kernel(const __grid_constant__ CUtensorMap tmap_p,
                  const __grid_constant__ CUtensorMap tmap_q, const GemmParams prm) {
@@ -319,7 +378,24 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int p0 = blockIdx.x * 128;
-  const int q0 = blockIdx.y * BN;
+  int q0 = blockIdx.y * BN;
+  // tokens of this CTA are [q0, Mlim); weight rows start at wrow (grouped:
+  // the expert's first row)
+  int Mlim = prm.M;
+  int wrow = 0;
+  if constexpr (GROUPED) {
+    // which expert and tokens this CTA serves depends on the routing of the
+    // preceding kernel: resolved before any set-up, and a CTA without work
+    // leaves at once (all CTAs of a split-K cluster share the tile)
+    __shared__ int gmap[3];
+    griddep_wait();
+    if (warp == 0) grouped_tile<BN>(prm, lane, gmap);
+    __syncthreads();
+    if (gmap[0] < 0 || gmap[2] <= 0) return;
+    q0 = gmap[1];
+    Mlim = gmap[1] + gmap[2];
+    wrow = gmap[0] * prm.N;
+  }
   const int kz = blockIdx.z;
   const int kt_begin = (int)(((long long)kz * prm.kt_total) / prm.split_k);
   const int kt_end = (int)(((long long)(kz + 1) * prm.kt_total) / prm.split_k);
@@ -379,7 +455,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
       const uint32_t off_a = SWAP ? L.q : L.p;
       const uint32_t bytes_w = SWAP ? kPTileBytes : C::kQTileBytes;
       const uint32_t bytes_a = SWAP ? C::kQTileBytes : kPTileBytes;
-      const int row_w = SWAP ? p0 : q0;
+      const int row_w = SWAP ? wrow + p0 : q0;
       const int row_a = SWAP ? q0 : p0;
       // NVFP4 scale atoms: P rows [p0, p0+128) are one 128-row block; Q has
       // one or two blocks (the second only if it holds any row).
@@ -586,7 +662,8 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
     // FP8 / INT8 Swap-AB: the weight (row) scales do not depend on the
     // preceding kernel, so they are staged while it still runs
     if constexpr (C::kRowColScales && SWAP)
-      for (int r = etid; r < 128; r += ET) row_s[r] = (p0 + r < prm.rows_p) ? __ldg(prm.scale_w + p0 + r) : 0.f;
+      for (int r = etid; r < 128; r += ET)
+        row_s[r] = (p0 + r < prm.rows_p) ? __ldg(prm.scale_w + wrow + p0 + r) : 0.f;
     griddep_wait();                            // scales/partials/activations of earlier kernels
     if (a_threads && etid == 0) trace_at(prm, kTrDepWait);
     bool fz_ok = true;
@@ -763,12 +840,12 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
         for (int idx = Mt * nkt + etid; idx < act_rows * nkt; idx += ET) sa_s[idx] = 0.f;
       }
       constexpr int WB = block_weight_blocks<SWAP, BN>();              // weight blocks per tile
-      const int wrow0 = (SWAP ? p0 : q0) / 128;
+      const int wrow0 = (SWAP ? p0 : q0) / 128;                        // block within the weight
       const int nblk = (prm.N + 127) / 128;
       for (int idx = etid; idx < WB * nkt; idx += ET) {
         const int gl = idx / WB, jb = idx % WB;
         const int b = wrow0 + jb;
-        sw_s[idx] = (b < nblk) ? __ldg(prm.scale_w + (size_t)b * G + g0 + gl) : 0.f;
+        sw_s[idx] = (b < nblk) ? __ldg(prm.scale_w + (size_t)(wrow / 128 + b) * G + g0 + gl) : 0.f;
       }
       named_bar_sync(1, ET);
 #pragma unroll
@@ -866,7 +943,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
         else      { r = r_begin + u / (c_count / 8); c = c_begin + (u % (c_count / 8)) * 8; }
         const int m = SWAP ? q0 + c : p0 + r;
         const int n0 = SWAP ? p0 + r : q0 + c;
-        if (m >= prm.M || n0 >= prm.N) continue;
+        if (m >= Mlim || n0 >= prm.N) continue;
         const uint4* src = reinterpret_cast<const uint4*>(otile + tile_index<SWAP, BN>(r, c));
         const uint4 w0 = src[0], w1 = src[1];
         const uint32_t acc8[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
@@ -929,7 +1006,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
       // tiles are mostly padding), token rows < M otherwise.
       const int Sk = prm.split_k;
       const int owner = row / rows_per, rl = row % rows_per;
-      const int cvalid = SWAP ? min(BN, prm.M - q0) : BN;
+      const int cvalid = SWAP ? min(BN, Mlim - q0) : BN;
       const bool rvalid = SWAP || (p0 + row < prm.M);
       if (!epi_phase1) cluster_wait();         // phase 1: every receiver is initialised
       const uint32_t dst = mapa_shared(smem_u32(smem + L.recv) + (uint32_t)kz * slot_bytes, (uint32_t)owner);
@@ -1022,7 +1099,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
             const int c = cbeg + c0 + j;
             const int m = SWAP ? q0 + c : prow;
             const int n = SWAP ? prow : q0 + c;
-            if (m < prm.M && n < prm.N) part[(size_t)kz * MN + (size_t)m * prm.N + n] = v[j];
+            if (m < Mlim && n < prm.N) part[(size_t)kz * MN + (size_t)m * prm.N + n] = v[j];
           }
         }
       }
@@ -1057,7 +1134,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
                     const int c = cbeg + c0 + j;
                     const int m = SWAP ? q0 + c : prow;
                     const int n = SWAP ? prow : q0 + c;
-                    t[dz][j] = (z0 + dz < prm.split_k && m < prm.M && n < prm.N)
+                    t[dz][j] = (z0 + dz < prm.split_k && m < Mlim && n < prm.N)
                                    ? ld_u32_cg(part + (z0 + dz) * MN + (size_t)m * prm.N + n)
                                    : 0u;
                   }
@@ -1073,7 +1150,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
                 const int c = cbeg + c0 + j;
                 const int m = SWAP ? q0 + c : prow;
                 const int n = SWAP ? prow : q0 + c;
-                if (m < prm.M && n < prm.N) emit<FMT, SWAP>(prm, row, c, m, n, acc[j], alpha, row_s, col_s);
+                if (m < Mlim && n < prm.N) emit<FMT, SWAP>(prm, row, c, m, n, acc[j], alpha, row_s, col_s);
               }
             }
           }
@@ -1129,7 +1206,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
           }
           const int m = SWAP ? q0 + c : p0 + r;
           const int n0 = SWAP ? p0 + r : q0 + c;
-          if (m >= prm.M || n0 >= prm.N) continue;
+          if (m >= Mlim || n0 >= prm.N) continue;
           if (prm.out_kind == 1) {
             uint32_t* Yu = reinterpret_cast<uint32_t*>(prm.Y) + (size_t)m * prm.ldy;
             for (int j = 0; j < 8 && n0 + j < prm.N; ++j) Yu[n0 + j] = acc8[j];
@@ -1203,7 +1280,19 @@ __global__ void splitk_reduce_kernel(const GemmParams prm) {
       float sa = 1.f, sw = 1.f;
       if constexpr (FMT == kFP8 || FMT == kINT8) {
         sa = __ldg(prm.scale_a + m);
-        sw = __ldg(prm.scale_w + n);
+        // grouped: row m belongs to the last expert whose first token is <= m
+        // (offsets clamped to [0, M] as in the GEMM kernel)
+        int wrow = 0;
+        if (prm.expert_offsets != nullptr) {
+          int lo = 0, hi = prm.experts - 1;
+          while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (min(max(__ldg(prm.expert_offsets + mid), 0), prm.M) <= m) lo = mid;
+            else hi = mid - 1;
+          }
+          wrow = lo * prm.N;
+        }
+        sw = __ldg(prm.scale_w + wrow + n);
       }
       reinterpret_cast<__nv_bfloat16*>(prm.Y)[(size_t)m * prm.ldy + n] =
           __float2bfloat16_rn(finish_value<FMT>(bits, sa, sw, alpha));

@@ -8,10 +8,10 @@
 namespace qg {
 namespace {
 
-template <int FMT, bool SWAP, int BN, bool FUSED>
+template <int FMT, bool SWAP, int BN, bool FUSED, bool GROUPED>
 cudaError_t launch_one(const CUtensorMap& tp, const CUtensorMap& tq, const GemmParams& prm,
                        dim3 grid, cudaStream_t st, bool pdl) {
-  auto kern = qgemm_kernel<FMT, SWAP, BN, FUSED>;
+  auto kern = qgemm_kernel<FMT, SWAP, BN, FUSED, GROUPED>;
   const int act_tiles = FUSED ? prm.nkt_max : 0;
   size_t smem = smem_bytes<FMT, SWAP, BN>(prm.stages, prm.nkt_max, prm.recv_cols, act_tiles);
   // Every CTA of this kernel that fits on an SM must also fit in its 512 TMEM
@@ -53,15 +53,15 @@ cudaError_t launch_one(const CUtensorMap& tp, const CUtensorMap& tq, const GemmP
   return cudaLaunchKernelEx(&cfg, kern, tp, tq, prm);
 }
 
-template <int FMT, bool SWAP, bool FUSED>
+template <int FMT, bool SWAP, bool FUSED, bool GROUPED = false>
 cudaError_t launch_bn(int bn, const CUtensorMap& tp, const CUtensorMap& tq, const GemmParams& prm,
                       dim3 grid, cudaStream_t st, bool pdl) {
   switch (bn) {
-    case 16: return launch_one<FMT, SWAP, 16, FUSED>(tp, tq, prm, grid, st, pdl);
-    case 32: return launch_one<FMT, SWAP, 32, FUSED>(tp, tq, prm, grid, st, pdl);
-    case 64: return launch_one<FMT, SWAP, 64, FUSED>(tp, tq, prm, grid, st, pdl);
-    case 128: return launch_one<FMT, SWAP, 128, FUSED>(tp, tq, prm, grid, st, pdl);
-    case 256: return launch_one<FMT, SWAP, 256, FUSED>(tp, tq, prm, grid, st, pdl);
+    case 16: return launch_one<FMT, SWAP, 16, FUSED, GROUPED>(tp, tq, prm, grid, st, pdl);
+    case 32: return launch_one<FMT, SWAP, 32, FUSED, GROUPED>(tp, tq, prm, grid, st, pdl);
+    case 64: return launch_one<FMT, SWAP, 64, FUSED, GROUPED>(tp, tq, prm, grid, st, pdl);
+    case 128: return launch_one<FMT, SWAP, 128, FUSED, GROUPED>(tp, tq, prm, grid, st, pdl);
+    case 256: return launch_one<FMT, SWAP, 256, FUSED, GROUPED>(tp, tq, prm, grid, st, pdl);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -116,6 +116,13 @@ size_t smem_for(int bn, int stages, int nkt_max, int recv_cols, int act_tiles) {
 
 cudaError_t QG_LAUNCH_NAME(bool swap, int tile_n, const CUtensorMap& tp, const CUtensorMap& tq,
                            const GemmParams& prm, dim3 grid, cudaStream_t st, bool pdl) {
+  if (prm.expert_offsets != nullptr) {
+    // grouped (mixture-of-experts) launch: Swap-AB, 8-bit formats only
+    if constexpr (QG_FMT != kNVF4) {
+      if (swap && prm.a_mode == kActTma) return launch_bn<QG_FMT, true, false, true>(tile_n, tp, tq, prm, grid, st, pdl);
+    }
+    return cudaErrorInvalidValue;
+  }
   if (prm.a_mode == kActFused) {
     // fused activation quantisation: Swap-AB, 8-bit formats only
     if constexpr (QG_FMT != kNVF4) {

@@ -249,3 +249,49 @@ def test_fused_valid_arguments_reach_the_device_check():
           dict(fmt=qg.QG_FP8_DYNAMIC, cfg=qg.make_config(split_k=1, swap_ab=1, tile_n=32, stages=4))]
     for kw in ok:
         assert _fused(**kw) in (qg.QG_ERR_NO_DEVICE, qg.QG_ERR_UNSUPPORTED)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(fmt=qg.QG_NVFP4), qg.QG_ERR_UNSUPPORTED),
+    (dict(E=0), qg.QG_ERR_INVALID_ARG),
+    (dict(E=300), qg.QG_ERR_UNSUPPORTED),                       # more than 256 experts
+    (dict(offsets=None), qg.QG_ERR_INVALID_ARG),
+    (dict(offsets=FAKE + 2), qg.QG_ERR_INVALID_ARG),
+    (dict(N=200), qg.QG_ERR_INVALID_ARG),                       # experts must fill 128-row blocks
+    (dict(Wrows=4 * 256 + 128), qg.QG_ERR_INVALID_ARG),         # W rows != experts * N
+    (dict(cfg=qg.make_config(split_k=1, swap_ab=0, tile_n=128, stages=4)), qg.QG_ERR_UNSUPPORTED),
+    (dict(cfg=qg.make_config(split_k=2, swap_ab=1, tile_n=16, stages=4, reduce_mode=2), ws=FAKE),
+     qg.QG_ERR_UNSUPPORTED),                                     # last-CTA counters are per tile
+])
+def test_grouped_rejects_bad_arguments_before_any_launch(kw, status):
+    fmt = kw.get("fmt", qg.QG_FP8_DYNAMIC)
+    E, N, K, T = kw.get("E", 4), kw.get("N", 256), 512, 24
+    cfg = kw.get("cfg", qg.make_config(split_k=1, swap_ab=1, tile_n=16, stages=4))
+    W = _op(kw.get("Wrows", E * N), K)
+    st = qg.qgemm_run_grouped(fmt, E, kw.get("offsets", FAKE), _op(T, K), W, N, K, cfg, kw.get("ws", None),
+                              1 << 30, FAKE, N, 0, None)
+    assert st == status
+
+
+@pytest.mark.parametrize("fmt", [qg.QG_FP8_DYNAMIC, qg.QG_W8A8_INT8, qg.QG_BLOCK_FP8])
+@pytest.mark.parametrize("E,T,N,K", [(128, 8, 1536, 2048), (128, 512, 2048, 768), (4, 3, 256, 512),
+                                     (256, 4096, 1024, 4096)])
+def test_grouped_default_config_is_accepted_by_the_grouped_launch(fmt, E, T, N, K):
+    c = qg.qgemm_grouped_default_config(fmt, E, T, N, K)
+    assert c.swap_ab == 1 and c.reduce_mode in (0, 1)
+    assert c.split_k >= 1 and c.split_k & (c.split_k - 1) == 0 and c.tile_n in (16, 32, 64, 128, 256)
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        return                     # the fake pointers below must never reach a launch
+    # the arguments pass every host check of qgemm_run_grouped: only the device is missing here
+    wsb = qg.qgemm_workspace_size(fmt, T, N, K, c)
+    st = qg.qgemm_run_grouped(fmt, E, FAKE, _op(T, K), _op(E * N, K), N, K, c, FAKE if wsb else None, wsb, FAKE,
+                              N, 0, None)
+    assert st == qg.QG_ERR_NO_DEVICE
+
+
+def test_grouped_default_config_rejects_nvfp4_and_bad_sizes():
+    c = qg.qg_config()
+    assert qg.lib().qgemm_grouped_default_config(qg.QG_NVFP4, 8, 8, 256, 512, c) == qg.QG_ERR_UNSUPPORTED
+    assert qg.lib().qgemm_grouped_default_config(qg.QG_FP8_DYNAMIC, 0, 8, 256, 512, c) == qg.QG_ERR_INVALID_ARG
+    assert qg.lib().qgemm_grouped_default_config(qg.QG_FP8_DYNAMIC, 8, 8, 256, 100, c) == qg.QG_ERR_INVALID_ARG
