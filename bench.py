@@ -58,6 +58,8 @@ def parse():
     ap.add_argument("--suite", default=None,
                     help="comma list of per-shape suites to time instead of the step: "
                          "fp8_tiny,int8,block_fp8,nvfp4,sweep,large_m,medium_m,moe (one JSON line per shape)")
+    ap.add_argument("--moe-tokens", default=None, help="comma list of token counts of the moe suite (default: all)")
+    ap.add_argument("--moe-formats", default=None, help="comma list of format ids of the moe suite (default: 0,1,2)")
     return ap.parse_args()
 
 
@@ -493,12 +495,14 @@ def run_moe_suite(args, local):
     gen.manual_seed(0)
     E = MOE_EXPERTS
     results = []
-    for fmt in MOE_FMTS:
+    fmts = [int(x) for x in args.moe_formats.split(",")] if args.moe_formats else MOE_FMTS
+    tokens = [int(x) for x in args.moe_tokens.split(",")] if args.moe_tokens else MOE_TOKENS
+    for fmt in fmts:
         for (N, K) in MOE_NK:
             w = (torch.randn(E * N, K, device=dev, generator=gen) * 0.02).to(torch.bfloat16)
             Wq = qg.quantize_weight(fmt, w)
             del w
-            for T in MOE_TOKENS:
+            for T in tokens:
                 counts = moe_routing(T, seed=1000 + T)
                 rows = int(counts.sum())
                 offs = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
