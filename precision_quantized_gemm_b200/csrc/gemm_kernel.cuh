@@ -418,9 +418,9 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], C::kEpiWarps);
     }
-    // push mode: each of the 128 rows of the owned slices arrives once, from
-    // whichever CTA computed it (split_k CTAs x 128/split_k rows)
-    mbar_init(recv_full, 128);
+    // push mode: one arrival (the receiver's expected byte count); the
+    // senders' asynchronous stores complete the bytes
+    mbar_init(recv_full, 1);
     // fused per-token amax exchange: one arrival per epilogue thread of the cluster
     mbar_init(amax_full, C::kEpiThreads);
     // thread-written activation slice: one arrival per epilogue thread
@@ -1000,16 +1000,25 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
     } else if (cluster_red && C::kPush) {
       // ---- cluster split-K, push: every thread stores its row of this
       // partial straight from registers into the owning CTA's receive slot
-      // `kz` and arrives (release) on that CTA's barrier; each CTA sums the
-      // rows it owns, in split order, into the output tile.  Only real
-      // outputs cross the cluster: token columns < M under Swap-AB (decode
-      // tiles are mostly padding), token rows < M otherwise.
+      // `kz` with asynchronous stores that count their bytes on that CTA's
+      // barrier; each CTA waits for the bytes of the rows it owns and sums
+      // them, in split order, into the output tile.  Only real outputs cross
+      // the cluster: token columns < M under Swap-AB (decode tiles are mostly
+      // padding), token rows < M otherwise.
       const int Sk = prm.split_k;
       const int owner = row / rows_per, rl = row % rows_per;
       const int cvalid = SWAP ? min(BN, Mlim - q0) : BN;
       const bool rvalid = SWAP || (p0 + row < prm.M);
+      if (etid == 0) {
+        // bytes this CTA receives: from each of the Sk CTAs, its owned rows
+        // (Swap-AB: all rows_per; standard: those below M) x cvalid words
+        const int r_own = (int)cluster_ctarank() * rows_per;
+        const int rows_in = SWAP ? rows_per : max(0, min(rows_per, prm.M - p0 - r_own));
+        mbar_arrive_expect_tx(recv_full, (uint32_t)(Sk * rows_in * cvalid * 4));
+      }
       if (!epi_phase1) cluster_wait();         // phase 1: every receiver is initialised
       const uint32_t dst = mapa_shared(smem_u32(smem + L.recv) + (uint32_t)kz * slot_bytes, (uint32_t)owner);
+      const uint32_t rbar = mapa_shared(smem_u32(recv_full), (uint32_t)owner);
 #pragma unroll
       for (int c0 = 0; c0 < NC; c0 += CW) {
         if (cbeg + c0 >= cvalid) break;
@@ -1024,15 +1033,14 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
 #pragma unroll
           for (int j = 0; j < CW; ++j)
             if (cbeg + c0 + j < cvalid)
-              st_dsmem_b32(dst + 4u * (uint32_t)slice_index<SWAP, BN>(rl, cbeg + c0 + j, rows_per), v[j]);
+              st_async_b32(dst + 4u * (uint32_t)slice_index<SWAP, BN>(rl, cbeg + c0 + j, rows_per), v[j], rbar);
         } else if (rvalid) {                   // slice [rl][c]: 16 bytes per store
 #pragma unroll
           for (int j = 0; j < CW; j += 4)
-            st_dsmem_v4(dst + 4u * (uint32_t)slice_index<SWAP, BN>(rl, cbeg + c0 + j, rows_per), v[j], v[j + 1],
-                        v[j + 2], v[j + 3]);
+            st_async_v4(dst + 4u * (uint32_t)slice_index<SWAP, BN>(rl, cbeg + c0 + j, rows_per), v[j], v[j + 1],
+                        v[j + 2], v[j + 3], rbar);
         }
       }
-      mbar_arrive_remote(mapa_shared(smem_u32(recv_full), (uint32_t)owner));
       if (etid == 0) trace_at(prm, kTrSent);
       const bool got = __all_sync(0xffffffffu, mbar_wait_cluster(recv_full, 0, prm.err));
       if (etid == 0) trace_at(prm, kTrRecv);
