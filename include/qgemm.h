@@ -383,14 +383,16 @@ qg_status qgemm_device_error(void);
  * library's kernels (default 1). */
 void qgemm_set_pdl(int enable);
 /* Tracing (debug): while set, every qgemm_run whose grid fits records, per
- * CTA, 12 GPU-clock timestamps (%globaltimer, ns, 64-bit) into the device
+ * CTA, 15 GPU-clock timestamps (%globaltimer, ns, 64-bit) into the device
  * buffer: entry, set-up done, first weight tile issued, dependency wait
  * returned, first stage landed, last MMA committed, accumulator ready, stores
  * done, and for cluster split-K: partial pushed, owned slices received,
  * owned rows reduced; word 11: the MMA issuer saw the last full stage.  In a
  * fused launch (qgemm_run_fused_act) word 3 is the epilogue warps' dependency
- * wait.  CTA c = (z * gridDim.y + y) *
- * gridDim.x + x writes words [12c, 12c+12).
+ * wait and words 12-14 mark the activation slice's local maxima, the
+ * cluster's exchanged maxima and the published codes.  Words not reached
+ * stay as they were.  CTA c = (z * gridDim.y + y) * gridDim.x + x writes
+ * words [15c, 15c+15).
  * Launches whose grid needs more than `bytes` are not traced.  NULL turns
  * tracing off.  Not thread-safe; meant for profiling runs. */
 void qgemm_set_trace(void* device_buffer, size_t bytes);

@@ -112,7 +112,10 @@ enum TraceEvent : int {
   kTrRecv = 9,         // cluster split-K: owned slices received
   kTrReduced = 10,     // cluster split-K: owned rows summed into the output tile
   kTrLastFull = 11,    // MMA issuer saw the last full stage
-  kTraceEvents = 12
+  kTrActLoaded = 12,   // fused: the slice's per-token maxima of this CTA are known
+  kTrActAmax = 13,     // fused: the cluster's maxima exchanged (the scales are known)
+  kTrActReady = 14,    // fused: the codes are published to the tensor core
+  kTraceEvents = 15
 };
 __device__ __forceinline__ void trace_at(const GemmParams& prm, int ev) {
   if (prm.trace != nullptr) {
@@ -644,6 +647,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
     auto publish_act = [&]() {
       fence_proxy_async_smem();
       mbar_arrive(act_ready);
+      if (etid == 0) trace_at(prm, kTrActReady);
     };
     if constexpr (kFusable) {
       if (a_threads) {
@@ -716,6 +720,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
           }
         }
         named_bar_sync(1, ET);
+        if (etid == 0) trace_at(prm, kTrActLoaded);
         // the row amax spans the whole K: the split-K CTAs of the cluster
         // swap their partial maxima (thread etid serves peer etid % split)
         if (cluster_red) {
@@ -728,6 +733,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
           mbar_arrive_remote(mapa_shared(smem_u32(amax_full), z));
           fz_ok = mbar_wait_cluster(amax_full, 0, prm.err);
         }
+        if (etid == 0) trace_at(prm, kTrActAmax);
         if (etid < BN) {
           float am = 0.f;
           if (etid < Mt) {
