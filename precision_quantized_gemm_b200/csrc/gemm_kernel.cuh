@@ -424,8 +424,9 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
     // push mode: one arrival (the receiver's expected byte count); the
     // senders' asynchronous stores complete the bytes
     mbar_init(recv_full, 1);
-    // fused per-token amax exchange: one arrival per epilogue thread of the cluster
-    mbar_init(amax_full, C::kEpiThreads);
+    // fused per-token amax exchange: one arrival (the receiver's expected
+    // byte count); the peers' asynchronous stores complete the bytes
+    mbar_init(amax_full, 1);
     // thread-written activation slice: one arrival per epilogue thread
     mbar_init(act_ready, C::kEpiThreads);
     *flag_abort = 0;
@@ -724,13 +725,15 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
         // the row amax spans the whole K: the split-K CTAs of the cluster
         // swap their partial maxima (thread etid serves peer etid % split)
         if (cluster_red) {
+          const int Sk = prm.split_k;
+          // every CTA of the cluster sends this one its Mt maxima
+          if (etid == 0) mbar_arrive_expect_tx(amax_full, (uint32_t)(Sk * Mt * 4));
           cluster_wait();                      // phase 1: every peer is initialised
           epi_phase1 = true;
-          const int Sk = prm.split_k;
           const uint32_t z = (uint32_t)(etid % Sk);
           const uint32_t dst = mapa_shared(smem_u32(exch + kz * BN), z);
-          for (int r = etid / Sk; r < Mt; r += ET / Sk) st_dsmem_b32(dst + 4u * (uint32_t)r, amax_u[r]);
-          mbar_arrive_remote(mapa_shared(smem_u32(amax_full), z));
+          const uint32_t zbar = mapa_shared(smem_u32(amax_full), z);
+          for (int r = etid / Sk; r < Mt; r += ET / Sk) st_async_b32(dst + 4u * (uint32_t)r, amax_u[r], zbar);
           fz_ok = mbar_wait_cluster(amax_full, 0, prm.err);
         }
         if (etid == 0) trace_at(prm, kTrActAmax);

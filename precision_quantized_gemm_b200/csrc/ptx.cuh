@@ -172,16 +172,6 @@ __device__ __forceinline__ uint32_t lds_u32(uint32_t saddr) {
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(saddr));
   return v;
 }
-// Stores into (possibly another CTA's) shared memory of the cluster.
-__device__ __forceinline__ void st_dsmem_b32(uint32_t dst_cluster, uint32_t v) {
-  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(dst_cluster), "r"(v) : "memory");
-}
-__device__ __forceinline__ void st_dsmem_v4(uint32_t dst_cluster, uint32_t a, uint32_t b, uint32_t c,
-                                            uint32_t d) {
-  asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst_cluster), "r"(a), "r"(b),
-               "r"(c), "r"(d)
-               : "memory");
-}
 // Asynchronous stores into a CTA of the cluster whose completion counts their
 // bytes against that CTA's mbarrier (complete_tx): a wait on the barrier's
 // phase sees the data, with no release by the storing thread.
@@ -195,12 +185,6 @@ __device__ __forceinline__ void st_async_v4(uint32_t dst_cluster, uint32_t a, ui
   asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
                    dst_cluster),
                "r"(a), "r"(b), "r"(c), "r"(d), "r"(bar_cluster)
-               : "memory");
-}
-// Arrive (release, cluster scope) on an mbarrier of a CTA of the cluster:
-// this thread's earlier stores are visible to whoever waits on its phase.
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)
                : "memory");
 }
 __device__ __forceinline__ uint4 ld_dsmem_v4(uint32_t caddr) {

@@ -61,6 +61,50 @@ def test_weight_quant_bit_exact(fmt, N, K):
         np.testing.assert_array_equal(np.asarray(g), np.asarray(ww))
 
 
+def _tie_rows(fmt, rows, K, seed):
+    """bf16 rows whose amax fixes the scale to a power of two and whose other
+    elements sit exactly on, or one bf16 step beside, a rounding tie of the
+    code format (int8: k + 1/2; e4m3: midpoints of normal and subnormal
+    codes), times the scale: every unit needs the quantisers' exact path."""
+    rng = np.random.default_rng(seed)
+    if fmt == qg.QG_W8A8_INT8:
+        ties = np.arange(-127, 127) + 0.5
+        qmax = 127.0
+    else:
+        mids = [(1 + (2 * j + 1) / 16) * 2.0 ** e for e in range(-6, 8) for j in range(8)]
+        mids += [(2 * j + 1) * 2.0 ** -10 for j in range(7)]
+        ties = np.array(mids + [-m for m in mids])
+        qmax = 448.0
+    out = np.empty((rows, K), np.float32)
+    for r in range(rows):
+        scale = 2.0 ** int(rng.integers(-3, 3))
+        v = rng.choice(ties, size=K) * scale
+        nudge = rng.integers(-1, 2, size=K)                 # -1, 0, +1 bf16 steps
+        bits = (v.astype(np.float32).view(np.uint32) >> 16).astype(np.int64) + nudge * (v != 0)
+        v = (bits.astype(np.uint32) << 16).view(np.float32)
+        # the scale is fixed by the format's maximum times the power of two,
+        # once per 128-element group (covers per-row and per-group scales)
+        v[::128] = qmax * scale
+        out[r] = v
+    return (out.view(np.uint32) >> 16).astype(np.uint16)
+
+
+@pytest.mark.parametrize("fmt", [qg.QG_FP8_DYNAMIC, qg.QG_W8A8_INT8, qg.QG_BLOCK_FP8], ids=["fp8", "int8", "block"])
+def test_quant_codes_on_rounding_ties(fmt):
+    a = _tie_rows(fmt, 7, 1024, seed=11)
+    op = qg.quantize_act(fmt, to_dev_bf16(a))
+    for g, w in zip(gpu_codes(fmt, op), oracle_quant(fmt, a, False)):
+        np.testing.assert_array_equal(np.asarray(g), np.asarray(w))
+    w_bits = _tie_rows(fmt, 256, 512, seed=12)
+    if fmt == qg.QG_BLOCK_FP8:                            # one power-of-two scale per 128x128 block
+        w_bits = w_bits.copy()
+        for nb in range(2):
+            w_bits[nb * 128:(nb + 1) * 128] = w_bits[nb * 128]
+    wop = qg.quantize_weight(fmt, to_dev_bf16(w_bits))
+    for g, w in zip(gpu_codes(fmt, wop), oracle_quant(fmt, w_bits, True)):
+        np.testing.assert_array_equal(np.asarray(g), np.asarray(w))
+
+
 def test_act_quant_with_row_stride():
     a, _ = inputs(4, 8, 512)
     big = np.zeros((4, 640), np.uint16)
