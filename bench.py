@@ -58,6 +58,7 @@ def parse():
     ap.add_argument("--suite", default=None,
                     help="comma list of per-shape suites to time instead of the step: "
                          "fp8_tiny,int8,block_fp8,nvfp4,sweep,large_m,medium_m,moe (one JSON line per shape)")
+    ap.add_argument("--only-m", default=None, help="comma list: keep only these token counts of the per-shape suites")
     ap.add_argument("--moe-tokens", default=None, help="comma list of token counts of the moe suite (default: all)")
     ap.add_argument("--moe-formats", default=None, help="comma list of format ids of the moe suite (default: 0,1,2)")
     return ap.parse_args()
@@ -626,6 +627,11 @@ def run_suite(args, names, local):
     results = []
     for name in names:
         for fmt, Ms, NKs in SUITES[name]:
+            if args.only_m:
+                keep = {int(x) for x in args.only_m.split(",")}
+                Ms = [m for m in Ms if m in keep]
+                if not Ms:
+                    continue
             for (N, K) in NKs:
                 w = (torch.randn(N, K, device=dev, generator=gen) * 0.02).to(torch.bfloat16)
                 Wq = qg.quantize_weight(fmt, w)

@@ -872,9 +872,8 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
         // accumulator is small, 32 when it already holds 128 registers
         // (16 columns when 16 warps share the register file)
         constexpr int PB = C::kEpiWarps >= 16 ? 16 : NC >= 128 ? 32 : 64;
-#pragma unroll
-        for (int c0 = 0; c0 < NC; c0 += PB) {
-          uint32_t v[PB];
+        constexpr int NCH = (NC + PB - 1) / PB;
+        auto ld_chunk = [&](int c0, uint32_t (&v)[PB]) {
           if constexpr (NC % 32 == 0 && PB >= 32) {
             tmem_ld32(lane_addr + b * BN + cbeg + c0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
             if constexpr (PB == 64)
@@ -883,7 +882,8 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
           } else {                             // 16-column tiles: stay inside the buffer
             tmem_ld16(lane_addr + b * BN + cbeg + c0, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
           }
-          tmem_ld_wait();
+        };
+        auto fma_chunk = [&](int c0, const uint32_t (&v)[PB]) {
           if (SWAP) {
             const float sw = sw_s[i];
 #pragma unroll
@@ -897,6 +897,32 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
             const uint64_t f2 = pack_f32x2(f, f);
 #pragma unroll
             for (int j = 0; j < PB && c0 + j < NC; j += 2) ffma2(acc2[(c0 + j) / 2], v[j], v[j + 1], f2);
+          }
+        };
+        if constexpr (NCH >= 2 && PB <= 16) {
+          // narrow chunks (16 warps share the register file): the next
+          // chunk's TMEM load is in flight while this chunk's FMAs run
+          uint32_t va[PB], vb[PB];
+          ld_chunk(0, va);
+          tmem_ld_wait();
+#pragma unroll
+          for (int ch = 0; ch < NCH; ch += 2) {
+            if (ch + 1 < NCH) ld_chunk((ch + 1) * PB, vb);
+            fma_chunk(ch * PB, va);
+            if (ch + 1 < NCH) {
+              tmem_ld_wait();
+              if (ch + 2 < NCH) ld_chunk((ch + 2) * PB, va);
+              fma_chunk((ch + 1) * PB, vb);
+              if (ch + 2 < NCH) tmem_ld_wait();
+            }
+          }
+        } else {
+#pragma unroll
+          for (int c0 = 0; c0 < NC; c0 += PB) {
+            uint32_t v[PB];
+            ld_chunk(c0, v);
+            tmem_ld_wait();
+            fma_chunk(c0, v);
           }
         }
         tc_fence_before();
