@@ -466,12 +466,17 @@ class GraphStep:
     ("Helion in the vLLM backend", fourth paragraph: shapes up to
     max_helion_size run under CUDA-graph replay).  Write the input into
     ``A`` (bf16 [M, K]), call ``replay()``, read ``Y`` (bf16 [M, N]).
-    ``fused=True`` captures the one-launch path (qgemm_run_fused_act)."""
+    ``fused=True`` captures the one-launch path (qgemm_run_fused_act).
+    ``host_io=True`` adds pinned host buffers ``A_host`` / ``Y_host`` whose
+    copies to and from the device are captured in the same graph: a replay
+    then moves the step's input in and its result out with no further call
+    (synchronize the stream before reading ``Y_host``)."""
 
     def __init__(self, layer: "Linear", M: int, W: Operand | None = None, cfg: qg_config | None = None,
-                 fused: bool = False):
+                 fused: bool = False, host_io: bool = False):
         torch = _torch()
         self.fused = fused
+        self.host_io = host_io
         dev = layer.Wq.q.device
         self.M, self.N, self.K = M, layer.N, layer.K
         self.fmt = layer.fmt
@@ -484,6 +489,9 @@ class GraphStep:
         self.ws.get(qgemm_workspace_size(self.fmt, M, self.N, self.K, self.cfg))
         self.qws = torch.zeros(max(qgemm_quant_workspace_size(self.fmt, M, self.K), 16), dtype=torch.uint8,
                                device=dev)
+        if host_io:
+            self.A_host = torch.zeros(M, self.K, dtype=torch.bfloat16, pin_memory=True)
+            self.Y_host = torch.empty(M, self.N, dtype=torch.bfloat16, pin_memory=True)
         side = torch.cuda.Stream(device=dev)
         side.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(side):
@@ -492,7 +500,15 @@ class GraphStep:
         torch.cuda.synchronize(dev)
         self.graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(self.graph):
-            self._launch()
+            self._body()
+
+    def _body(self):
+        """The captured work: [input copy in], quantisation + GEMM, [result copy out]."""
+        if self.host_io:
+            self.A.copy_(self.A_host, non_blocking=True)
+        self._launch()
+        if self.host_io:
+            self.Y_host.copy_(self.Y, non_blocking=True)
 
     def _launch(self):
         st = _stream(None)
@@ -510,12 +526,26 @@ class GraphStep:
 
     def replay(self):
         self.graph.replay()
-        return self.Y
+        return self.Y_host if self.host_io else self.Y
+
+
+def capture_steps(steps) -> "torch.cuda.CUDAGraph":
+    """One CUDA graph that runs the given captured steps back to back (as a
+    decode forward runs its layers), so that each step's kernels overlap the
+    previous step's tail through programmatic dependent launch instead of
+    waiting for a graph launch.  The steps keep their own buffers; replay
+    the returned graph instead of the steps one by one."""
+    torch = _torch()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for st in steps:
+            st._body()
+    return g
 
 
 def _linear_capture(self, M: int, W: Operand | None = None, cfg: qg_config | None = None,
-                    fused: bool = False) -> GraphStep:
-    g = GraphStep(self, M, W=W, cfg=cfg, fused=fused)
+                    fused: bool = False, host_io: bool = False) -> GraphStep:
+    g = GraphStep(self, M, W=W, cfg=cfg, fused=fused, host_io=host_io)
     self.graphs[M] = g
     return g
 
