@@ -283,16 +283,19 @@ qg_status tune_impl(void* table, qg_format f, const int* Ms, int nM, const int* 
           std::fclose(lf);
         }
       }
-      // Near-ties (within 3%) go to a configuration whose ring holds every
-      // K tile of its slice: all of its weights are requested at launch, so
-      // it also keeps its time after a graph boundary or a host sync, where
-      // no earlier kernel's tail hides the reload of a stage (steady-state
-      // timing does not see that case).
+      // Near-ties (within 10%) go to a configuration whose ring holds every
+      // K tile of its slice: all of its weights are requested at launch,
+      // before the dependency wait.  It keeps its time after a graph
+      // boundary, a host sync or a neighbouring kernel of another shape,
+      // where no earlier kernel's tail hides the reload of a stage.  The
+      // same-shape loop timed here does not see those cases: INT8 4096^2,
+      // M = 8, a 3-stage ring over 4 K tiles is 6% faster back to back but
+      // makes a decode step of M = 1, 8, 32 1 us slower.
       {
         double tie_us = 1e30;
         for (const auto& t : timed) {
           const int nkt = (kt_of(f, K) + t.second.split_k - 1) / t.second.split_k;
-          if (t.first <= 1.03 * best_us && t.second.stages >= nkt && t.first < tie_us) {
+          if (t.first <= 1.10 * best_us && t.second.stages >= nkt && t.first < tie_us) {
             tie_us = t.first;
             best = t.second;
           }
