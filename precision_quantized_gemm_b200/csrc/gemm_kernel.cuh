@@ -968,9 +968,41 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
     // scales, converts and stores 16-byte vectors along the contiguous
     // dimension of y (channels: r under Swap-AB, c otherwise).
     uint32_t* otile = stage_buf;
+    // Eight consecutive output channels n0 .. n0+7 of output row m (tile
+    // row r / column c): raw accumulators, or scaled, rounded to bf16 and
+    // stored as one 16-byte vector where the row pitch allows it.
+    auto store8 = [&](int r, int c, int m, int n0, const uint32_t (&acc8)[8]) {
+      const bool vec = (prm.ldy % 8) == 0;
+      if (prm.out_kind == 1) {
+        uint32_t* Yu = reinterpret_cast<uint32_t*>(prm.Y) + (size_t)m * prm.ldy;
+        for (int j = 0; j < 8 && n0 + j < prm.N; ++j) Yu[n0 + j] = acc8[j];
+        return;
+      }
+      float y8[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float sa = 1.f, sw = 1.f;
+        if constexpr (FMT == kFP8 || FMT == kINT8) {
+          sa = SWAP ? col_s[c] : row_s[r];
+          sw = SWAP ? row_s[r + j] : col_s[c + j];
+        }
+        y8[j] = finish_value<FMT>(acc8[j], sa, sw, alpha);
+      }
+      __nv_bfloat16* Yb = reinterpret_cast<__nv_bfloat16*>(prm.Y) + (size_t)m * prm.ldy;
+      if (vec && n0 + 8 <= prm.N) {
+        uint32_t p[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(y8[2 * h], y8[2 * h + 1]);
+          p[h] = *reinterpret_cast<const uint32_t*>(&b2);
+        }
+        *reinterpret_cast<uint4*>(Yb + n0) = make_uint4(p[0], p[1], p[2], p[3]);
+      } else {
+        for (int j = 0; j < 8 && n0 + j < prm.N; ++j) Yb[n0 + j] = __float2bfloat16_rn(y8[j]);
+      }
+    };
     auto write_out = [&](int r_begin, int r_count, int c_begin, int c_count) {
       const int units = SWAP ? c_count * (r_count / 8) : r_count * (c_count / 8);
-      const bool vec = (prm.ldy % 8) == 0;
 #pragma unroll 1
       for (int u = etid; u < units; u += ET) {
         int r, c;                              // first of 8 consecutive output channels
@@ -982,33 +1014,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
         const uint4* src = reinterpret_cast<const uint4*>(otile + tile_index<SWAP, BN>(r, c));
         const uint4 w0 = src[0], w1 = src[1];
         const uint32_t acc8[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-        if (prm.out_kind == 1) {
-          uint32_t* Yu = reinterpret_cast<uint32_t*>(prm.Y) + (size_t)m * prm.ldy;
-          for (int j = 0; j < 8 && n0 + j < prm.N; ++j) Yu[n0 + j] = acc8[j];
-          continue;
-        }
-        float y8[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          float sa = 1.f, sw = 1.f;
-          if constexpr (FMT == kFP8 || FMT == kINT8) {
-            sa = SWAP ? col_s[c] : row_s[r];
-            sw = SWAP ? row_s[r + j] : col_s[c + j];
-          }
-          y8[j] = finish_value<FMT>(acc8[j], sa, sw, alpha);
-        }
-        __nv_bfloat16* Yb = reinterpret_cast<__nv_bfloat16*>(prm.Y) + (size_t)m * prm.ldy;
-        if (vec && n0 + 8 <= prm.N) {
-          uint32_t p[4];
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            const __nv_bfloat162 b2 = __floats2bfloat162_rn(y8[2 * h], y8[2 * h + 1]);
-            p[h] = *reinterpret_cast<const uint32_t*>(&b2);
-          }
-          *reinterpret_cast<uint4*>(Yb + n0) = make_uint4(p[0], p[1], p[2], p[3]);
-        } else {
-          for (int j = 0; j < 8 && n0 + j < prm.N; ++j) Yb[n0 + j] = __float2bfloat16_rn(y8[j]);
-        }
+        store8(r, c, m, n0, acc8);
       }
     };
 
@@ -1079,38 +1085,51 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
       if (etid == 0) trace_at(prm, kTrSent);
       const bool got = __all_sync(0xffffffffu, mbar_wait_cluster(recv_full, 0, prm.err));
       if (etid == 0) trace_at(prm, kTrRecv);
-      const uint32_t* __restrict__ recv = reinterpret_cast<const uint32_t*>(smem + L.recv);
-      uint32_t* __restrict__ ot = otile;
       const int r0 = (int)cluster_ctarank() * rows_per;
       const int zstride = rows_per * prm.recv_cols;
-      if (epi_ok && got) {
-        // fixed per-thread row (Swap-AB) or column (standard), stepping over
-        // the other index: no divisions in the loop, loads of later
-        // iterations overlap
-        if (SWAP) {
-          const int rl2 = etid % rows_per, cstep = ET / rows_per;
+      if constexpr (SWAP) {
+        // Swap-AB: a slot holds, per token column, the owned channels
+        // contiguously, so a unit of 8 consecutive channels of one token is
+        // two 16-byte loads per split, summed in split order, scaled and
+        // stored straight to y (no output tile, no barrier before the stores)
+        if (epi_ok && got) {
           const uint32_t recv_s = smem_u32(smem + L.recv);
-#pragma unroll 4
-          for (int c = etid / rows_per; c < cvalid; c += cstep) {
-            uint32_t acc = 0u;
-            for (int z = 0; z < Sk; ++z)
-              acc = add_acc<FMT>(acc, lds_u32(recv_s + 4u * (uint32_t)(z * zstride + c * rows_per + rl2)));
-            ot[tile_index<SWAP, BN>(r0 + rl2, c)] = acc;
+          const int rb = rows_per / 8;
+#pragma unroll 1
+          for (int u = etid; u < cvalid * rb; u += ET) {
+            const int c = u / rb, rl8 = (u - c * rb) * 8;
+            const int m = q0 + c, n0 = p0 + r0 + rl8;
+            if (m >= Mlim || n0 >= prm.N) continue;
+            uint32_t acc8[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+            for (int z = 0; z < Sk; ++z) {
+              const uint32_t a = recv_s + 4u * (uint32_t)(z * zstride + c * rows_per + rl8);
+              const uint4 w0 = lds_v4(a), w1 = lds_v4(a + 16u);
+              const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+              for (int j = 0; j < 8; ++j) acc8[j] = add_acc<FMT>(acc8[j], w[j]);
+            }
+            store8(r0 + rl8, c, m, n0, acc8);
           }
-        } else {
+        }
+        if (etid == 0) trace_at(prm, kTrReduced);
+      } else {
+        if (epi_ok && got) {
+          // fixed per-thread column, stepping over the rows: no divisions
+          // in the loop, loads of later iterations overlap
+          const uint32_t* __restrict__ recv = reinterpret_cast<const uint32_t*>(smem + L.recv);
           const int nrow = max(0, min(rows_per, prm.M - p0 - r0));
           const int c = etid % BN, rstep = ET / BN;
 #pragma unroll 4
           for (int rl2 = etid / BN; rl2 < nrow; rl2 += rstep) {
             uint32_t acc = 0u;
             for (int z = 0; z < Sk; ++z) acc = add_acc<FMT>(acc, recv[z * zstride + rl2 * BN + c]);
-            ot[tile_index<SWAP, BN>(r0 + rl2, c)] = acc;
+            otile[tile_index<SWAP, BN>(r0 + rl2, c)] = acc;
           }
         }
+        named_bar_sync(1, ET);
+        if (etid == 0) trace_at(prm, kTrReduced);
+        if (epi_ok && got) write_out(r0, rows_per, 0, BN);
       }
-      named_bar_sync(1, ET);
-      if (etid == 0) trace_at(prm, kTrReduced);
-      if (epi_ok && got) write_out(r0, rows_per, 0, BN);
     } else if (cluster_red) {
       // ---- cluster split-K, pull: stage the partial in the idle ring; the
       // reduction runs after the cluster barrier below
