@@ -1087,49 +1087,38 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
       if (etid == 0) trace_at(prm, kTrRecv);
       const int r0 = (int)cluster_ctarank() * rows_per;
       const int zstride = rows_per * prm.recv_cols;
-      if constexpr (SWAP) {
-        // Swap-AB: a slot holds, per token column, the owned channels
-        // contiguously, so a unit of 8 consecutive channels of one token is
-        // two 16-byte loads per split, summed in split order, scaled and
-        // stored straight to y (no output tile, no barrier before the stores)
-        if (epi_ok && got) {
-          const uint32_t recv_s = smem_u32(smem + L.recv);
-          const int rb = rows_per / 8;
+      // The owner reduces and stores in one pass: a slot keeps 8 consecutive
+      // output channels contiguous (Swap-AB: per token column, the owned
+      // channels; standard: per owned token row, the tile's channels), so a
+      // unit of 8 channels is two 16-byte loads per split, summed in split
+      // order, scaled and stored to y as one 16-byte vector (no output tile,
+      // no barrier before the stores).
+      if (epi_ok && got) {
+        const uint32_t recv_s = smem_u32(smem + L.recv);
+        const int nrow = SWAP ? cvalid : max(0, min(rows_per, prm.M - p0 - r0));   // slice rows with outputs
+        const int ub = (SWAP ? rows_per : BN) / 8;                                // units per slice row
 #pragma unroll 1
-          for (int u = etid; u < cvalid * rb; u += ET) {
-            const int c = u / rb, rl8 = (u - c * rb) * 8;
-            const int m = q0 + c, n0 = p0 + r0 + rl8;
-            if (m >= Mlim || n0 >= prm.N) continue;
-            uint32_t acc8[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-            for (int z = 0; z < Sk; ++z) {
-              const uint32_t a = recv_s + 4u * (uint32_t)(z * zstride + c * rows_per + rl8);
-              const uint4 w0 = lds_v4(a), w1 = lds_v4(a + 16u);
-              const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        for (int u = etid; u < nrow * ub; u += ET) {
+          const int i = u / ub, j8 = (u - i * ub) * 8;
+          // Swap-AB: i = token column, j8 = first owned channel; standard:
+          // i = owned token row, j8 = first channel of the tile
+          const int r = SWAP ? r0 + j8 : r0 + i;
+          const int c = SWAP ? i : j8;
+          const int m = SWAP ? q0 + i : p0 + r0 + i;
+          const int n0 = SWAP ? p0 + r0 + j8 : q0 + j8;
+          if (m >= Mlim || n0 >= prm.N) continue;
+          uint32_t acc8[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+          for (int z = 0; z < Sk; ++z) {
+            const uint32_t a = recv_s + 4u * (uint32_t)(z * zstride + i * (SWAP ? rows_per : BN) + j8);
+            const uint4 w0 = lds_v4(a), w1 = lds_v4(a + 16u);
+            const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-              for (int j = 0; j < 8; ++j) acc8[j] = add_acc<FMT>(acc8[j], w[j]);
-            }
-            store8(r0 + rl8, c, m, n0, acc8);
+            for (int k = 0; k < 8; ++k) acc8[k] = add_acc<FMT>(acc8[k], w[k]);
           }
+          store8(r, c, m, n0, acc8);
         }
-        if (etid == 0) trace_at(prm, kTrReduced);
-      } else {
-        if (epi_ok && got) {
-          // fixed per-thread column, stepping over the rows: no divisions
-          // in the loop, loads of later iterations overlap
-          const uint32_t* __restrict__ recv = reinterpret_cast<const uint32_t*>(smem + L.recv);
-          const int nrow = max(0, min(rows_per, prm.M - p0 - r0));
-          const int c = etid % BN, rstep = ET / BN;
-#pragma unroll 4
-          for (int rl2 = etid / BN; rl2 < nrow; rl2 += rstep) {
-            uint32_t acc = 0u;
-            for (int z = 0; z < Sk; ++z) acc = add_acc<FMT>(acc, recv[z * zstride + rl2 * BN + c]);
-            otile[tile_index<SWAP, BN>(r0 + rl2, c)] = acc;
-          }
-        }
-        named_bar_sync(1, ET);
-        if (etid == 0) trace_at(prm, kTrReduced);
-        if (epi_ok && got) write_out(r0, rows_per, 0, BN);
       }
+      if (etid == 0) trace_at(prm, kTrReduced);
     } else if (cluster_red) {
       // ---- cluster split-K, pull: stage the partial in the idle ring; the
       // reduction runs after the cluster barrier below

@@ -24,9 +24,9 @@
 //   time   = body + epi   (+ a per-shape constant that ranking ignores)
 //
 // Waves and CTAs per SM follow the launch's shared memory, register budget
-// and TMEM columns.  On the 218 tuned shapes (34,852 candidates) the
-// top-ranked configuration is within 1.084x of the measured best (geomean),
-// the best of the top 8 within 1.012x and of the top 16 within 1.004x (the
+// and TMEM columns.  On the 218 tuned shapes (34870 candidates) the
+// top-ranked configuration is within 1.071x of the measured best (geomean),
+// the best of the top 8 within 1.009x and of the top 16 within 1.003x (the
 // fixed rule it replaced was 1.32x on an earlier 170-shape set).
 #include <algorithm>
 #include <cmath>
@@ -40,17 +40,17 @@ namespace {
 // Fitted constants (B200, 1965 MHz boost, measured HBM 6450.9 GB/s).
 struct Model {
   double hbm_gbs = 6450.9;   // HBM bandwidth (measured copy bandwidth, held fixed)
-  double lat_us = 1.40939;   // load latency under load seen by one CTA's ring
-  double sm_gbs = 130.780;   // per-SM load bandwidth
-  double a0 = 653.480, a1 = 0.803035;  // MMA-loop cycles per K tile: fixed, per tile_n column
-  double a2 = 7.87483, a3 = 0.0;       // Block_FP8 promotion cycles per K tile: per promoted column
+  double lat_us = 1.38161;   // load latency under load seen by one CTA's ring
+  double sm_gbs = 133.412;   // per-SM load bandwidth
+  double a0 = 636.147, a1 = 0.873829;  // MMA-loop cycles per K tile: fixed, per tile_n column
+  double a2 = 6.58675, a3 = 22.4012;   // Block_FP8 promotion cycles per K tile: per promoted column
   double clock_mhz = 1900.0;
-  double e0 = 0.461216;      // epilogue per 16 pushed token columns, µs
-  double e1 = 3.58593;       // cluster split-K exchange, fixed, µs per wave
-  double e2 = 72.4581;       // cluster exchange bandwidth, GB/s per tile
-  double e3 = 4.23571;       // second-pass launch, µs
-  double e4 = 11.4859;       // last-CTA reduction, µs
-  double e5 = 1195.38;       // workspace traffic bandwidth, GB/s
+  double e0 = 0.503163;      // epilogue per 16 pushed token columns, µs
+  double e1 = 2.80164;       // cluster split-K exchange, fixed, µs per wave
+  double e2 = 73.0506;       // cluster exchange bandwidth, GB/s per tile
+  double e3 = 3.95830;       // second-pass launch, µs
+  double e4 = 11.2845;       // last-CTA reduction, µs
+  double e5 = 1180.85;       // workspace traffic bandwidth, GB/s
 };
 const Model kModel;
 

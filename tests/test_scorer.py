@@ -65,8 +65,8 @@ def test_scorer_ranking_against_measured_candidates():
         top16.append(min(t for _, t in scored[:16]) / best)
     geo = lambda xs: math.exp(sum(math.log(x) for x in xs) / len(xs))
     assert len(top1) >= 200
-    assert geo(top1) <= 1.10, geo(top1)          # fitted: 1.084 (the fixed rule it replaced: 1.32)
-    assert geo(top16) <= 1.01, geo(top16)        # fitted: 1.004
-    # worst shape: Block_FP8 M = 128, 5120 x 2048 (a medium-M bucket), whose
-    # best configuration the model ranks outside its top 16 (1.27x)
+    assert geo(top1) <= 1.10, geo(top1)          # fitted: 1.071 (the fixed rule it replaced: 1.32)
+    assert geo(top16) <= 1.01, geo(top16)        # fitted: 1.003
+    # the worst shape's best configuration lies outside the top 16 (fitted:
+    # 1.22x, a medium-M bucket)
     assert max(top16) <= 1.30
