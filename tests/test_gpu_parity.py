@@ -150,6 +150,10 @@ SWAP_CASES = [  # (M, N, K, split_k, tile_n, reduce_mode, stages); reduce 0 clus
     (3, 260, 4096, 16, 16, 2, 4),     # split beyond the cluster limit
     (8, 512, 2048, 4, 16, 0, 2),      # two-stage ring, wrapping twice per CTA
     (1, 384, 4096, 2, 16, 0, 3),      # three-stage ring, ragged wrap
+    (100, 512, 2048, 2, 128, 0, 4),   # wide token tiles: cluster pull reduction
+    (130, 384, 1024, 1, 128, 0, 4),   # two wide token tiles, ragged
+    (64, 256, 1024, 2, 128, 2, 4),    # wide tile, last-CTA reduction
+    (200, 256, 1024, 1, 256, 0, 3),   # widest token tile
 ]
 STD_CASES = [
     (128, 256, 512, 1, 128, 0, 4),
@@ -161,6 +165,7 @@ STD_CASES = [
     (140, 200, 1024, 2, 64, 2, 4),
     (260, 520, 2048, 1, 256, 0, 3),   # wide tile: Block_FP8 promotes with 8 epilogue warps
     (200, 300, 1024, 2, 256, 0, 3),
+    (140, 300, 1024, 2, 128, 2, 4),   # last-CTA reduction of a 128-wide tile
 ]
 
 
