@@ -172,11 +172,6 @@ __device__ __forceinline__ uint4 lds_v4(uint32_t saddr) {
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(saddr));
   return v;
 }
-__device__ __forceinline__ uint32_t lds_u32(uint32_t saddr) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(saddr));
-  return v;
-}
 // Asynchronous stores into a CTA of the cluster whose completion counts their
 // bytes against that CTA's mbarrier (complete_tx): a wait on the barrier's
 // phase sees the data, with no release by the storing thread.
@@ -220,13 +215,6 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
-}
-// Remote shared-memory load (kept after the cluster barrier that published
-// the data: volatile, with a memory clobber).
-__device__ __forceinline__ uint32_t ld_dsmem_u32(uint32_t caddr) {
-  uint32_t v;
-  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(caddr) : "memory");
-  return v;
 }
 
 // ------------------------------------------------------------- tcgen05 --
