@@ -343,7 +343,11 @@ qg_status qgemm_dispatch(const void* table, qg_format f, int M, int N, int K, qg
  * qgemm_run, as a layer with dynamic activations runs them (selection pass),
  * re-times the winner in an independent pass whose step time is what the
  * table records, and rejects any config whose output differs from the
- * default config's.  Shapes already
+ * default config's.  Among configs within 10% of the fastest it picks one
+ * whose ring holds every K tile of its split (all weights requested before
+ * the dependency wait), which keeps its time next to kernels of other shapes
+ * and after graph boundaries, where the same-shape timing loop is blind.
+ * Shapes already
  * present in `table` are skipped (resume).  Synthetic inputs are generated
  * on the device; `budget_s_per_shape` bounds the wall time per shape.
  * NK holds nNK pairs (N, K). */
