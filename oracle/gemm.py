@@ -92,3 +92,25 @@ def split_k_partials(qa, qw, splits: int, acc_fn=acc_e4m3):
 def swap_ab(qa, qw, acc_fn=acc_e4m3):
     """Swap-AB: (W_q . A_q^T)^T, the weight filling the row role."""
     return acc_fn(qw, qa).T
+
+
+def grouped(gemm_fn, qa, sa, qw, sw, offsets, n_per_expert: int, w_rows_per_scale: int = 1):
+    """Mixture-of-experts grouped GEMM ("Helion in the vLLM backend", last
+    paragraph: the MoE backend is the next target): the tokens are sorted by
+    expert, expert e owns token rows [offsets[e], offsets[e + 1]) of A and y
+    and weight rows [e N, (e + 1) N) of the stacked W; its rows of y are the
+    plain GEMM ``gemm_fn`` (one of the four above, taking (qa, sa, qw, sw))
+    of those slices.  ``w_rows_per_scale`` is 1 for per-channel weight scales
+    and 128 for 128x128 block scales (N is then a multiple of 128).  Returns
+    y [T, N] in fp64 values of bf16."""
+    T = qa.shape[0]
+    N = n_per_expert
+    y = np.zeros((T, N), np.float64)
+    for e in range(len(offsets) - 1):
+        r0, r1 = int(offsets[e]), int(offsets[e + 1])
+        if r1 <= r0:
+            continue
+        w0, w1 = e * N, (e + 1) * N
+        s0, s1 = w0 // w_rows_per_scale, w1 // w_rows_per_scale
+        y[r0:r1] = gemm_fn(qa[r0:r1], sa[r0:r1], qw[w0:w1], sw[s0:s1])
+    return y

@@ -10,13 +10,16 @@ import pytest
 import torch
 
 import precision_quantized_gemm_b200 as qg
-from gpu_util import assert_within_tolerance, bf16_to_np, oracle_quant, oracle_y, to_dev_bf16
+from gpu_util import assert_within_tolerance, bf16_to_np, oracle_quant, to_dev_bf16
 import qg_synth
 from oracle import gemm as OG
 
 pytestmark = pytest.mark.gpu
 
 FMTS = [qg.QG_FP8_DYNAMIC, qg.QG_W8A8_INT8, qg.QG_BLOCK_FP8]
+# the oracle's plain GEMM per format and its weight rows per scale
+ORACLE_GEMM = {qg.QG_FP8_DYNAMIC: (OG.fp8_dynamic, 1), qg.QG_W8A8_INT8: (OG.w8a8_int8, 1),
+               qg.QG_BLOCK_FP8: (OG.block_fp8, 128)}
 IDS = {qg.QG_FP8_DYNAMIC: "fp8", qg.QG_W8A8_INT8: "int8", qg.QG_BLOCK_FP8: "block"}
 
 
@@ -86,6 +89,8 @@ def test_grouped_matches_per_expert_runs_and_oracle(case):
     assert torch.equal(y, y_again)
     qa = oracle_quant(fmt, a, False)
     qw = oracle_quant(fmt, w, True)
+    gemm_fn, w_rows_per_scale = ORACLE_GEMM[fmt]
+    ref = OG.grouped(gemm_fn, qa[0], qa[1], qw[0], qw[1], offs, N, w_rows_per_scale)
     ws = qg.Workspace()
     for e in range(E):
         m0, m = int(offs[e]), counts[e]
@@ -97,10 +102,7 @@ def test_grouped_matches_per_expert_runs_and_oracle(case):
         qg.check(qg.qgemm_run(fmt, Ae, We, m, N, K, cfg, wsp, wsb, ye.data_ptr(), N, 0, qg._stream(None)))
         torch.cuda.synchronize()
         assert torch.equal(y[m0:m0 + m], ye), f"expert {e}"
-        qae = (qa[0][m0:m0 + m], qa[1][m0:m0 + m])
-        sw = qw[1][e * N // 128:(e + 1) * N // 128] if fmt == qg.QG_BLOCK_FP8 else qw[1][e * N:(e + 1) * N]
-        qwe = (qw[0][e * N:(e + 1) * N], sw)
-        assert_within_tolerance(bf16_to_np(y[m0:m0 + m]), oracle_y(fmt, qae, qwe), f"{_id(case)} expert {e}")
+        assert_within_tolerance(bf16_to_np(y[m0:m0 + m]), ref[m0:m0 + m], f"{_id(case)} expert {e}")
 
 
 def test_grouped_int8_accumulators_bit_exact():

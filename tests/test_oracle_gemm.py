@@ -203,3 +203,51 @@ def test_block_fp8_reduces_to_fp8_dynamic_with_uniform_scales():
     y_block = G.block_fp8(qa, np.repeat(sa[:, None], 2, 1), qw, np.full((1, 2), sw, np.float32))
     y_dyn = G.fp8_dynamic(qa, sa, qw, np.full(128, sw, np.float32))
     assert np.array_equal(y_block, y_dyn)
+
+
+# ---------------------------------------------------- grouped (MoE) GEMM --
+def test_grouped_with_one_expert_is_the_plain_gemm():
+    a = qg_synth.bf16_matrix(0, 5, 128, 1.0)
+    w = qg_synth.bf16_matrix(1, 12, 128, 0.02)
+    qa, sa = Q.per_row_int8(a)
+    qw, sw = Q.per_row_int8(w)
+    y = G.grouped(G.w8a8_int8, qa, sa, qw, sw, np.array([0, 5]), 12)
+    assert np.array_equal(y, G.w8a8_int8(qa, sa, qw, sw))
+
+
+def test_grouped_brute_force_routing_with_an_empty_expert():
+    # 3 experts x N = 4 channels; tokens 0-1 -> expert 0, none -> expert 1,
+    # tokens 2-4 -> expert 2: every y row uses its own expert's weight rows
+    a = qg_synth.bf16_matrix(0, 5, 64, 1.0)
+    w = qg_synth.bf16_matrix(1, 12, 64, 0.02)
+    qa, sa = Q.per_row_fp8(a)
+    qw, sw = Q.per_row_fp8(w)
+    offsets = np.array([0, 2, 2, 5])
+    expert_of = [0, 0, 2, 2, 2]
+    ref = np.zeros((5, 4))
+    for t in range(5):
+        e = expert_of[t]
+        for n in range(4):
+            s = 0.0
+            for k in range(64):
+                s += F.E4M3_TABLE[qa[t, k]] * F.E4M3_TABLE[qw[e * 4 + n, k]]
+            ref[t, n] = s * float(sa[t]) * float(sw[e * 4 + n])
+    assert np.array_equal(G.grouped(G.fp8_dynamic, qa, sa, qw, sw, offsets, 4), F.bf16_round(ref))
+
+
+def test_grouped_block_scales_follow_the_expert():
+    # Block_FP8 with 128-row weight blocks: swapping the two experts' weights
+    # (rows and block scales) swaps which tokens see which weights
+    a = qg_synth.bf16_matrix(0, 6, 256, 1.0)
+    w = qg_synth.bf16_matrix(1, 256, 256, 0.02)
+    qa, sa = Q.act_groups_fp8(a)
+    qw, sw = Q.weight_blocks_fp8(w)
+    offsets = np.array([0, 4, 6])
+    y = G.grouped(G.block_fp8, qa, sa, qw, sw, offsets, 128, w_rows_per_scale=128)
+    assert np.array_equal(y[:4], G.block_fp8(qa[:4], sa[:4], qw[:128], sw[:1]))
+    assert np.array_equal(y[4:], G.block_fp8(qa[4:], sa[4:], qw[128:], sw[1:]))
+    qw_s = np.concatenate([qw[128:], qw[:128]])
+    sw_s = np.concatenate([sw[1:], sw[:1]])
+    y_s = G.grouped(G.block_fp8, qa, sa, qw_s, sw_s, offsets, 128, w_rows_per_scale=128)
+    assert np.array_equal(y_s[:4], G.block_fp8(qa[:4], sa[:4], qw[128:], sw[1:]))
+    assert not np.array_equal(y_s[:4], y[:4])
