@@ -677,11 +677,26 @@ def run_suite(args, names, local):
                     e1.record()
                     torch.cuda.synchronize()
                     us = 1000.0 * e0.elapsed_time(e1) / (n_rep * reps)
+                    # one eager call on its own (after a sync, events on the
+                    # same stream): the device waits from the first event
+                    # for the host's submission (argument checks, two tensor
+                    # map encodings, the launch), so this is what an eager
+                    # call costs from call to completion, with no neighbour
+                    # to overlap; its weight copy is the next in the
+                    # rotation, last read `copies` calls ago (past 2 x L2)
+                    st = qg._stream(None)
+                    e0.record()
+                    qg.check(qg.qgemm_run(fmt, As[reps % len(As)].c, Ws[reps % copies].c, M, N, K, cfg, wsp, wsb,
+                                          Y.data_ptr(), N, 0, st))
+                    e1.record()
+                    torch.cuda.synchronize()
+                    us_single = 1000.0 * e0.elapsed_time(e1)
                     t_hbm = byts / (hbm * 1e9) * 1e6
                     t_tc = flops / (tensor_peak(fmt, bf16) * 1e12) * 1e6
                     bound = "hbm" if t_hbm >= t_tc else "tensor"
                     frac = max(t_hbm, t_tc) / us
                     rec = {"suite": name, "format": FMT_NAME[fmt], "M": M, "N": N, "K": K, "us": round(us, 3),
+                           "single_launch_us": round(us_single, 3),
                            "GB/s": round(byts / us / 1e3, 1), "TFLOP/s": round(flops / us / 1e6, 2),
                            "bound": bound, "roofline_us": round(max(t_hbm, t_tc), 3),
                            "frac_roofline": round(frac, 4), "config": cfg.as_dict(), "table_hit": hit,
