@@ -87,12 +87,25 @@ def peaks():
     return 6650.0, "fallback"
 
 
+def kernel_source_code(text: str) -> str:
+    """The code of a CUDA source: `//` comments, trailing blanks and empty
+    lines removed (the kernel sources hold no `//` inside a string)."""
+    out = []
+    for line in text.splitlines():
+        line = line.split("//", 1)[0].rstrip()
+        if line:
+            out.append(line)
+    return "\n".join(out) + "\n"
+
+
 def kernel_source_hash():
-    """sha1 of the GEMM kernel sources: ties an ncu traffic figure to the code it measured."""
+    """sha1 of the GEMM kernel code (gemm_kernel.cuh + ptx.cuh, comments
+    ignored): ties an ncu traffic figure to the code it measured."""
     import hashlib
     h = hashlib.sha1()
     for f in ("gemm_kernel.cuh", "ptx.cuh"):
-        h.update(open(os.path.join(ROOT, "precision_quantized_gemm_b200", "csrc", f), "rb").read())
+        with open(os.path.join(ROOT, "precision_quantized_gemm_b200", "csrc", f), encoding="utf-8") as fh:
+            h.update(kernel_source_code(fh.read()).encode())
     return h.hexdigest()[:12]
 
 

@@ -8,12 +8,13 @@
 // (B^T A^T)^T): P = W_q, Q = A_q, so the weight rows fill the 128-row MMA
 // slot and a handful of tokens fill N = 16 or 32.
 //
-// Warp roles (192 threads):
+// Warp roles (64 threads + the epilogue warps):
 //   warp 0      TMA producer: weights first (they do not depend on the
 //               preceding kernel), then griddepcontrol.wait, then activations;
 //               a `stages`-deep ring of 128-byte K tiles in shared memory.
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer.
-//   warps 2..5  epilogue: tcgen05.ld of the fp32/int32 accumulator, scales in
+//   warps 2..   epilogue, 4 warps (Block_FP8 with 128- or 256-wide tiles: 8
+//               or 16): tcgen05.ld of the fp32/int32 accumulator, scales in
 //               fp32, bf16 store, or this CTA's split-K partial.
 // Block_FP8 promotes every 128-wide K group: the MMA writes the group's
 // partial sum into one of NACC TMEM buffers and the epilogue warps fold it
@@ -24,9 +25,17 @@
 // Split-K ("Helion in the vLLM backend", second and third paragraphs): the
 // split_k CTAs of one output tile either form a thread-block cluster and
 // meet in distributed shared memory (no global scratch), or leave partials
-// in a workspace that the last-arriving CTA or a second kernel sums.  Every
-// mode adds the partials in split order, so results are deterministic and
-// identical across modes.
+// in a workspace that the last-arriving CTA or a second kernel sums.  In the
+// cluster, narrow tiles push each row's partial to the CTA that owns it with
+// asynchronous stores that count their bytes on the owner's barrier; the
+// owner sums and stores units of 8 channels in one pass.  Wide tiles stage
+// their partial in the idle ring and the owners pull.  Every mode adds the
+// partials in split order, so results are deterministic and identical
+// across modes.
+//
+// Grouped (mixture-of-experts) launches read device-side expert offsets after
+// the dependency wait; each CTA finds its expert and token tile with a warp
+// scan, and CTAs without a tile leave before any set-up.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>

@@ -46,3 +46,12 @@ def test_moe_routing_picks_distinct_experts_per_token(T):
     assert counts.sum() == T * bench.MOE_TOPK
     assert counts.max() <= T                      # an expert at most once per token
     assert np.array_equal(counts, bench.moe_routing(T, seed=1000 + T))
+
+
+def test_kernel_source_hash_ignores_comments_but_not_code():
+    src = "// header\nint f(int x) {  // doubles\n  return 2 * x;\n}\n\n"
+    same = "int f(int x) {\n\n  return 2 * x;   // twice\n}\n"
+    other = "int f(int x) {\n  return 3 * x;\n}\n"
+    assert bench.kernel_source_code(src) == bench.kernel_source_code(same)
+    assert bench.kernel_source_code(src) != bench.kernel_source_code(other)
+    assert len(bench.kernel_source_hash()) == 12
