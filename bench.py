@@ -5,10 +5,16 @@
 One step is one pass of the whole decode hot path over one batch: for each
 token count M of the W8A8_INT8 decode workload (M in {1, 8, 32}, N = K = 4096,
 per-token int8 activations, per-channel int8 weights, bf16 out) the dynamic
-activation quantiser and the tcgen05 GEMM run as one CUDA-graph replay with
-the configuration the per-shape table dispatches (or the built-in default).
-Weights are quantised once at set-up; the step rotates over enough weight
-copies (more than twice the L2) that every GEMM streams its weights from HBM.
+activation quantiser and the tcgen05 GEMM run with the configuration the
+per-shape table dispatches (or the built-in default).  The timed steps run as
+CUDA graphs of consecutive steps (capture_steps), as a decode forward
+captures its layers.  Weights are quantised once at set-up; the steps rotate
+over enough weight copies (more than twice the L2) that every GEMM streams
+its weights from HBM.
+
+``--suite`` times per-shape GEMMs of the workload families instead (one JSON
+line per shape, plus geomeans); ``--suite moe`` times the grouped
+(mixture-of-experts) launch.
 
 Printed (rank 0, one JSON line): the metric of the workload as whole-job
 algorithmic HBM throughput (GB/s) of the step, per-shape GEMM microseconds and
