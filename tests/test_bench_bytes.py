@@ -55,3 +55,10 @@ def test_kernel_source_hash_ignores_comments_but_not_code():
     assert bench.kernel_source_code(src) == bench.kernel_source_code(same)
     assert bench.kernel_source_code(src) != bench.kernel_source_code(other)
     assert len(bench.kernel_source_hash()) == 12
+
+
+def test_all_cores_oracle_baseline_reassembles_the_single_process_result():
+    # the pool splits each oracle GEMM by output-column blocks; the function
+    # asserts that the blocks reassemble into the single-process result
+    cb = bench.cpu_baseline_all_cores(1)
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] > 0
