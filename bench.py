@@ -270,7 +270,9 @@ def cpu_baseline_all_cores(sample_steps=6):
         def step():
             acts_q = [OQ.per_row_int8(acts[m]) for m in MS]
             jobs = [(int(bounds[i]), int(bounds[i + 1]), acts_q) for i in range(cores)]
-            parts = pool.map(_oracle_block, jobs)
+            # bounded: a stalled worker raises (TimeoutError) instead of
+            # holding the bench; leaving the `with` terminates the pool
+            parts = pool.map_async(_oracle_block, jobs).get(timeout=300)
             return [np.concatenate([p[j] for p in parts], axis=1) for j in range(len(MS))]
         got = step()                                   # warm-up, and the reassembly check
         for j, m in enumerate(MS):
