@@ -124,3 +124,106 @@ def test_nvfp4_static_global_scale():
     a = _act(2, 64, seed=19)
     q, sf, g = Q.nvfp4(a, global_amax=1000.0)
     assert g == np.float32(1000.0) / np.float32(2688.0)
+
+
+# ---------------------------------------------------------------------------
+# Hand-derived rounding decisions.  The reading of the quantisers rounds the
+# fp32 quotient x / s half to even ("Helion in the vLLM backend", first
+# paragraph, names W8A8_INT8; the symmetric int8 recipe rounds to nearest,
+# and the tie rule is the reading stated with the oracle).  Every expected
+# code below is worked out by hand in the comments, not by the oracle.
+
+def _int8_tie_row(scale_num):
+    """One row whose amax is 127 * scale_num, so that s = amax / 127 is
+    exactly scale_num, followed by the values (k + 1/2) * scale_num for
+    k = -127 .. 126 (each a tie of the fp32 quotient x / s)."""
+    ks = np.arange(-127, 127)
+    vals = np.concatenate([[127.0], ks + 0.5]) * scale_num
+    return vals, ks
+
+
+@pytest.mark.parametrize("scale_num", [1.0, 2.0, 0.25])
+def test_int8_ties_round_half_to_even(scale_num):
+    # scale_num = 1: the row [127, -126.5, ..., 126.5]; amax 127 gives
+    # s = 127 / 127 = 1 exactly, and x / s = k + 1/2 is a tie between k and
+    # k + 1.  Half to even picks the even one of the two: 0.5 -> 0,
+    # 1.5 -> 2, 2.5 -> 2, -0.5 -> 0, -1.5 -> -2, 125.5 -> 126, -126.5 -> -126.
+    # Half away from zero would give 1, 2, 3, -1, -2, 126, -127 instead.
+    # scale_num = 2 (amax 254, s = 2) and 0.25 (amax 31.75, s = 0.25): the
+    # same quotients, every value exact in bf16 (at most 8 significant bits).
+    vals, ks = _int8_tie_row(scale_num)
+    a = _bits(vals[None, :])
+    assert np.array_equal(F.bf16_from_bits(a)[0].astype(np.float64), vals)   # exact in bf16
+    q, s = Q.per_row_int8(a)
+    assert s[0] == np.float32(scale_num)
+    want = np.where(ks % 2 == 0, ks, ks + 1)         # the even one of k and k + 1
+    assert q[0, 0] == 127
+    assert np.array_equal(q[0, 1:].astype(np.int64), want)
+    # sign symmetry: -x gives -code at every tie
+    qn, _ = Q.per_row_int8(_bits(-vals[None, :]))
+    assert np.array_equal(qn[0].astype(np.int64), -q[0].astype(np.int64))
+
+
+def test_int8_one_ulp_either_side_of_a_tie():
+    # s = 1 (amax 127).  Around the tie 2.5 the bf16 neighbours are
+    # 2.5 - 2^-6 and 2.5 + 2^-6 (bf16 keeps 8 significant bits, so the
+    # spacing in [2, 4) is 2^-6): they round to 2 and 3, while 2.5 itself
+    # goes to 2.  Around -0.5 (spacing 2^-8 above 0.5 in magnitude, 2^-9
+    # below): -0.5 - 2^-8 goes to -1, -0.5 + 2^-9 to 0, -0.5 itself to 0.
+    # Around 63.5 (spacing 2^-2 in [32, 64)): 63.25 -> 63, 63.5 -> 64,
+    # 63.75 -> 64.
+    vals = np.array([127.0, 2.5 - 2 ** -6, 2.5, 2.5 + 2 ** -6, -0.5 - 2 ** -8, -0.5, -0.5 + 2 ** -9,
+                     63.25, 63.5, 63.75])
+    a = _bits(vals[None, :])
+    assert np.array_equal(F.bf16_from_bits(a)[0].astype(np.float64), vals)
+    q, s = Q.per_row_int8(a)
+    assert s[0] == 1.0
+    assert q[0].tolist() == [127, 2, 2, 3, -1, 0, 0, 63, 64, 64]
+
+
+# NVFP4 hand-worked blocks.  Reading (stated with the oracle): g =
+# amax(tensor) / (448 * 6); block scale code = e4m3_RNE_satfinite((amax_b /
+# 6) / g); code = e2m1_RNE_satfinite(x / (dec(block scale) * g)); code 0
+# wherever the block scale decodes to 0.  e2m1 magnitudes in code order:
+# 0, 0.5, 1, 1.5, 2, 3, 4, 6 (codes 0..7, sign bit 8).  e4m3 codes near 14:
+# 0x56 = 1.110b * 2^3 = 14, 0x57 = 15, 0x58 = 16.
+NVFP4_ROW0 = [6, 5, -5, 3.5, 2.5, 1.75, 1.25, 0.75, 0.25, -0.25, 0, 4.5, 2.75, 1.125, -6, 0.625]
+NVFP4_ROW1 = [87, 70, 49, 35, 24.5, 17.5, 10.5, 3.5, -87, 7, 21, 42, 56, 0, -3.5, 28]
+NVFP4_ROW2 = [6 * 2 ** -10, 2 ** -8, -(2 ** -8), 2 ** -9, 0, 3 * 2 ** -10, -6 * 2 ** -10, 2 ** -10,
+              0, 0, 0, 0, 0, 0, 0, 2 ** -8]
+
+
+def _nvfp4_hand_tensor():
+    return np.array([np.array(NVFP4_ROW0) * 448.0, NVFP4_ROW1, NVFP4_ROW2])
+
+
+def test_nvfp4_hand_worked_blocks():
+    x = _nvfp4_hand_tensor()
+    a = _bits(x)
+    assert np.array_equal(F.bf16_from_bits(a).astype(np.float64), x)   # every value exact in bf16
+    q, sf, g = Q.nvfp4(a)
+    # tensor amax = 6 * 448 = 2688, so g = 2688 / 2688 = 1 exactly.
+    assert g == np.float32(1.0)
+    # Row 0: amax_b = 2688, (2688 / 6) / 1 = 448 -> e4m3 0x7E (448), d = 448
+    # and x / d is the listed multiple exactly.  Codes: 6 -> 7; 5 is the tie
+    # of 4 (code 6, even) and 6 (code 7) -> 6; -5 -> 8 | 6 = 14; 3.5, tie of
+    # 3 (5) and 4 (6) -> 6; 2.5, tie of 2 (4) and 3 (5) -> 4; 1.75, tie of
+    # 1.5 (3) and 2 (4) -> 4; 1.25, tie of 1 (2) and 1.5 (3) -> 2; 0.75, tie
+    # of 0.5 (1) and 1 (2) -> 2; 0.25, tie of 0 (0) and 0.5 (1) -> 0; -0.25
+    # -> -0 = 8 (the sign of x sets the sign bit); 0 -> 0; 4.5 -> 4 (6);
+    # 2.75 -> 3 (5); 1.125 -> 1 (2); -6 -> 15; 0.625 -> 0.5 (1).
+    # Row 1: amax_b = 87, 87 / 6 = 14.5, the tie of 14 (0x56, even mantissa)
+    # and 15 (0x57) -> 0x56, d = 14 (a rounded-up scale would be 15).  x / 14:
+    # 87 -> 6.21.. saturates to 6 (7); 70 -> 5, tie -> 4 (6); 49 -> 3.5 -> 4
+    # (6); 35 -> 2.5 -> 2 (4); 24.5 -> 1.75 -> 2 (4); 17.5 -> 1.25 -> 1 (2);
+    # 10.5 -> 0.75 -> 1 (2); 3.5 -> 0.25 -> 0 (0); -87 -> 15; 7 -> 0.5 (1);
+    # 21 -> 1.5 (3); 42 -> 3 (5); 56 -> 4 (6); 0 -> 0; -3.5 -> -0 (8);
+    # 28 -> 2 (4).
+    # Row 2: amax_b = 6 * 2^-10, (amax_b / 6) / 1 = 2^-10, half of the
+    # smallest e4m3 subnormal 2^-9: the tie of 0 (code 0, even) and 2^-9
+    # (code 1) -> code 0, which decodes to 0, so every element code is 0
+    # (without that rule x / 0 would saturate the non-zero elements to +-6).
+    assert sf[:, 0].tolist() == [0x7E, 0x56, 0x00]
+    assert q[0].tolist() == [7, 6, 14, 6, 4, 4, 2, 2, 0, 8, 0, 6, 5, 2, 15, 1]
+    assert q[1].tolist() == [7, 6, 6, 4, 4, 2, 2, 0, 15, 1, 3, 5, 6, 0, 8, 4]
+    assert q[2].tolist() == [0] * 16
