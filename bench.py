@@ -12,16 +12,22 @@ captures its layers.  Weights are quantised once at set-up; the steps rotate
 over enough weight copies (more than twice the L2) that every GEMM streams
 its weights from HBM.
 
-``--suite`` times per-shape GEMMs of the workload families instead (one JSON
-line per shape, plus geomeans); ``--suite moe`` times the grouped
+After the step, the default run times every configured shape on its own
+(the metric's M <= 32 decode shapes of all four formats, and Block_FP8 at
+M = 4096 and 16384): one CUDA graph of back-to-back GEMMs per shape over
+weight copies totalling more than 2 x L2, giving µs per shape, the fraction of
+roofline per shape and their geomeans (``--no-suite`` skips this phase).
+``--suite`` prints those per-shape lines (and other families, e.g.
+``medium_m``) instead of the step; ``--suite moe`` times the grouped
 (mixture-of-experts) launch.
 
 Printed (rank 0, one JSON line): the metric of the workload as whole-job
 algorithmic HBM throughput (GB/s) of the step, per-shape GEMM microseconds and
-fraction of the HBM roofline, the dominant kernel's roofline object, the CPU
-oracle's throughput on a bounded sample, the end-to-end number through the
-public API with host buffers, clocks sampled during the timed region and the
-count of library kernels launched while timing.
+fraction of the HBM roofline, the geomean over every configured shape, the
+dominant kernel's roofline object, the CPU oracle's throughput on a bounded
+sample, the end-to-end number through the public API with host buffers,
+clocks sampled (NVML) during the timed work and the count of library kernels
+launched while timing.
 
 ``--impl reference`` times the CPU oracle on the same workload (the only
 "reference" that exists: the pages ship no code).  Multi-GPU (torchrun): every
@@ -51,6 +57,17 @@ FMT_INT8 = 1
 MS = (1, 8, 32)
 N = K = 4096
 TABLE = os.path.join(ROOT, "precision_quantized_gemm_b200", "tables", "b200.qgt")
+L2_POLICY = ("inputs larger than L2: every GEMM of the timed steps and of the per-shape phase reads weight "
+             "copies from a rotation of more than 2 x L2 (126 MB), activations too at M >= 4096")
+
+
+def bench_config(world):
+    """The `config` of the bench line, the same dict for both arms."""
+    return {"workload": WORKLOAD, "M": list(MS), "N": N, "K": K, "format": "W8A8_INT8",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU", "l2": L2_POLICY,
+            "per_shape_workloads": "every configured shape: FP8_Dynamic 16x2048x2048; W8A8_INT8 M in {1,8,32} "
+                                   "4096^2; Block_FP8 16 decode shapes; NVFP4 16 shapes; FP8_Dynamic and Block_FP8 "
+                                   "sweep 144 shapes; Block_FP8 M in {4096,16384} 5120^2"}
 
 
 def parse():
@@ -61,6 +78,8 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--table", default=TABLE)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-suite", action="store_true",
+                    help="skip the per-shape phase over every configured shape (the metric's geomean)")
     ap.add_argument("--suite", default=None,
                     help="comma list of per-shape suites to time instead of the step: "
                          "fp8_tiny,int8,block_fp8,nvfp4,sweep,large_m,medium_m,moe (one JSON line per shape)")
@@ -129,48 +148,142 @@ def measured_traffic():
 
 
 # ------------------------------------------------------------- clocks ---
-class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+CLOCK_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+SMI_FIELDS = "clocks.sm,clocks.max.sm,power.draw"
+SMI_REASON_FIELDS = ("clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                     "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = None
+
+def parse_smi_row(line):
+    """One nvidia-smi CSV row (noheader, nounits) of SMI_FIELDS, optionally
+    followed by the four SMI_REASON_FIELDS -> a sample dict, or None."""
+    f = [x.strip() for x in line.split(",")]
+    if len(f) < 3:
+        return None
+    try:
+        sm, mx = float(f[0]), float(f[1])
+    except ValueError:
+        return None
+    try:
+        pw = float(f[2])
+    except ValueError:
+        pw = None
+    reasons = [CLOCK_REASONS[i] for i in range(4) if len(f) >= 7 and f[3 + i].lower() == "active"]
+    return {"sm_mhz": sm, "sm_max_mhz": mx, "power_w": pw, "reasons": reasons}
+
+
+def summarise_clocks(samples, error=None):
+    """Median SM clock of the samples taken under load (the GPU busy, at
+    least half of the largest clock seen), the largest max clock, and every
+    throttle reason any sample reported."""
+    if not samples:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [f"no samples: {error}" if error else "no samples"],
+                "samples": 0}
+    top = max(x["sm_mhz"] for x in samples)
+    load = [x for x in samples if x.get("busy", True) and x["sm_mhz"] >= 0.5 * top] or samples
+    return {"sm_mhz": statistics.median(x["sm_mhz"] for x in load),
+            "sm_max_mhz": max(x["sm_max_mhz"] for x in samples),
+            "reasons": sorted({r for x in samples for r in x["reasons"]}),
+            "samples": len(samples), "samples_under_load": len(load),
+            "power_w_max": max((x["power_w"] for x in samples if x.get("power_w") is not None), default=None)}
+
+
+class Clocks:
+    """Samples the SM clock, power and throttle reasons of this process's GPU
+    every `period` seconds on a host thread while the timed work runs.  NVML
+    (read-only queries) first; where NVML is missing, one-shot nvidia-smi
+    queries.  The GPU is found by its PCI bus id, so the sample is of the
+    device this process uses whatever CUDA_VISIBLE_DEVICES maps."""
+
+    def __init__(self, bus_id, period=0.1):
+        import threading
+        self.bus_id = bus_id
+        self.period = period
+        self.samples = []
+        self.error = None
+        self._stop = threading.Event()
+        self._thread = threading.Thread(target=self._run, daemon=True)
+
+    def _nvml(self):
+        import pynvml as N
+        N.nvmlInit()
+        h = N.nvmlDeviceGetHandleByPciBusId(self.bus_id.encode() if isinstance(self.bus_id, str) else self.bus_id)
+        bits = {"hw_slowdown": N.nvmlClocksEventReasonHwSlowdown,
+                "hw_thermal_slowdown": N.nvmlClocksEventReasonHwThermalSlowdown,
+                "sw_thermal_slowdown": N.nvmlClocksEventReasonSwThermalSlowdown,
+                "sw_power_cap": N.nvmlClocksEventReasonSwPowerCap}
+
+        def one():
+            sm = float(N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM))
+            mx = float(N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM))
+            try:
+                pw = N.nvmlDeviceGetPowerUsage(h) / 1000.0
+            except N.NVMLError:
+                pw = None
+            try:
+                r = N.nvmlDeviceGetCurrentClocksEventReasons(h)
+                reasons = [k for k, b in bits.items() if r & b]
+            except N.NVMLError:
+                reasons = []
+            try:
+                busy = N.nvmlDeviceGetUtilizationRates(h).gpu > 0
+            except N.NVMLError:
+                busy = True
+            return {"sm_mhz": sm, "sm_max_mhz": mx, "power_w": pw, "reasons": reasons, "busy": busy}
+        return one, N.nvmlShutdown
+
+    def _smi(self):
+        def one():
+            r = subprocess.run(["nvidia-smi", "-i", self.bus_id, f"--query-gpu={SMI_FIELDS},{SMI_REASON_FIELDS}",
+                                "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=10)
+            if r.returncode != 0:     # an older driver may lack the reason fields: ask for the clocks alone
+                r = subprocess.run(["nvidia-smi", "-i", self.bus_id, f"--query-gpu={SMI_FIELDS}",
+                                    "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=10)
+            if r.returncode != 0:
+                raise RuntimeError((r.stderr or r.stdout).strip().splitlines()[0][:120])
+            x = parse_smi_row(r.stdout.strip().splitlines()[0])
+            if x is None:
+                raise RuntimeError(f"unparsed nvidia-smi row: {r.stdout.strip()[:120]}")
+            return x
+        return one, lambda: None
+
+    def _run(self):
+        try:
+            one, done = self._nvml()
+        except Exception as exc:                       # no NVML: nvidia-smi queries
+            self.error = f"nvml: {type(exc).__name__}"
+            one, done = self._smi()
+        try:
+            while not self._stop.is_set():
+                t = time.perf_counter()
+                try:
+                    self.samples.append(dict(one(), t=t))
+                except Exception as exc:
+                    self.error = f"{type(exc).__name__}: {exc}"[:160]
+                    if not self.samples:
+                        break
+                self._stop.wait(max(0.0, self.period - (time.perf_counter() - t)))
+        finally:
+            done()
 
     def start(self):
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+        self._thread.start()
+        return self
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        rows = []
-        for line in open(self.path):
-            f = [x.strip() for x in line.split(",")]
-            if len(f) >= 9:
-                rows.append(f)
-        os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        self._stop.set()
+        self._thread.join(timeout=15)
+        return summarise_clocks(self.samples, self.error)
+
+    def window(self, t0, t1):
+        """Summary of the samples taken between perf_counter times t0 and t1."""
+        return summarise_clocks([x for x in self.samples if t0 <= x["t"] <= t1], self.error)
+
+
+def device_bus_id(dev_index):
+    import torch
+    p = torch.cuda.get_device_properties(dev_index)
+    return "%08X:%02X:%02X.0" % (getattr(p, "pci_domain_id", 0), p.pci_bus_id, p.pci_device_id)
 
 
 # ------------------------------------------------------------ helpers ---
@@ -249,7 +362,7 @@ def _oracle_block(job):
     return [OG.w8a8_int8(qa, sa, qw[n0:n1], sw[n0:n1]) for qa, sa in acts_q]
 
 
-def cpu_baseline_all_cores(sample_steps=6):
+def cpu_baseline_all_cores(sample_steps=6, warmup=1):
     """The same oracle step on every host core: a process pool (started with
     spawn, as a CUDA process must) splits each step's three GEMMs over blocks
     of output columns; the activation quantisation runs in this process.  The
@@ -261,7 +374,13 @@ def cpu_baseline_all_cores(sample_steps=6):
     from oracle import gemm as OG
     from oracle import quant as OQ
     avail = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
-    cores = max(1, min(avail, 16))                # bounded: each worker holds the 16 MB of weight codes
+    # each worker holds the 16 MB of weight codes and a step's int64
+    # temporaries (~0.4 GB at most): bounded by the host's memory
+    try:
+        mem = os.sysconf("SC_PAGE_SIZE") * os.sysconf("SC_AVPHYS_PAGES")
+    except (ValueError, OSError):
+        mem = 8 << 30
+    cores = max(1, min(avail, int(mem // (1 << 30)), 64))
     acts = {m: qg_synth.activations(m, K) for m in MS}
     qw, sw = OQ.per_row_int8(qg_synth.weights(N, K))
     bounds = np.linspace(0, N, cores + 1).astype(int)
@@ -277,37 +396,43 @@ def cpu_baseline_all_cores(sample_steps=6):
         got = step()                                   # warm-up, and the reassembly check
         for j, m in enumerate(MS):
             qa, sa = OQ.per_row_int8(acts[m])
-            assert np.array_equal(got[j], OG.w8a8_int8(qa, sa, qw, sw)), "oracle blocks do not reassemble"
+            if not np.array_equal(got[j], OG.w8a8_int8(qa, sa, qw, sw)):
+                raise RuntimeError("oracle column blocks do not reassemble into the single-process result")
+        for _ in range(max(0, warmup - 1)):           # the check above was the first warm-up step
+            step()
         t0 = time.perf_counter()
         for _ in range(sample_steps):
             step()
         dt = (time.perf_counter() - t0) / sample_steps
-    return {"value": step_bytes() / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+    return {"value": step_bytes() / dt / 1e9, "unit": "GB/s", "cores": cores, "host_cores": avail,
+            "kind": "oracle",
             "sample": f"{sample_steps} full steps (3 activation quantisations + 3 exact int64 GEMMs "
                       f"M in {{1,8,32}}, N=K=4096 + bf16 epilogue), weights quantised once; the GEMMs "
                       f"split over {cores} processes by output-column blocks (numpy int64 matmul is "
-                      f"single-threaded; {avail} host cores available, at most 16 used)",
+                      f"single-threaded; {avail} host cores available)",
             "seconds_per_step": dt}
 
 
 # ---------------------------------------------------------- reference ---
 def run_reference(args, world, rank):
+    """The oracle on the host cores, on the same workload, `config`, metric and
+    step count as the GPU arm: `--warmup` untimed steps, then `--steps` timed
+    steps, each one full step of the workload (three activation quantisations
+    and three exact GEMMs)."""
     if rank != 0:
         return
-    steps = max(2, min(args.steps, 4))
-    warm = 1                                   # cpu_baseline_all_cores runs one untimed step first
+    steps = max(1, args.steps)
     single = cpu_baseline(1)
     try:
-        cb = cpu_baseline_all_cores(max(steps, 2))
+        cb = cpu_baseline_all_cores(steps, warmup=max(1, args.warmup))
     except Exception as exc:       # the pool is measurement harness: time the oracle in this process
         cb = dict(cpu_baseline(steps), all_cores_error=f"{type(exc).__name__}: {exc}"[:200])
     line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "GB/s",
-            "n_gpus": args.gpus, "steps": steps, "warmup": warm, "ms_per_step": 1000 * cb["seconds_per_step"],
+            "n_gpus": args.gpus, "steps": steps, "warmup": args.warmup, "ms_per_step": 1000 * cb["seconds_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
-            "data": "synthetic",
-            "config": {"workload": WORKLOAD, "M": list(MS), "N": N, "K": K},
-            "cpu_baseline": {"value": cb["value"], "unit": "GB/s", "cores": cb["cores"], "kind": "oracle",
-                             "sample": cb["sample"]},
+            "data": "synthetic", "config": bench_config(world),
+            "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "host_cores", "kind", "sample",
+                                                  "all_cores_error") if k in cb},
             "cpu_baseline_single_thread": {k: single[k] for k in ("value", "unit", "cores", "kind", "sample")},
             "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -392,9 +517,15 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
 
     # ---- timed region: K full steps
-    clocks = ClockSampler(local)
-    clocks.start()
-    time.sleep(0.3)
+    clocks = Clocks(device_bus_id(local)).start()
+    # Keep the GPU on the same steps for half a second (more untimed warm-up)
+    # so that the clock samples of this window show the conditions the timed
+    # region runs under (the region itself is far shorter than a sample).
+    t_load = time.perf_counter()
+    while time.perf_counter() - t_load < 0.5:
+        for g in timed_graphs:
+            g.replay()
+        torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
@@ -404,6 +535,7 @@ def run_ours(args, world, rank, local):
         g.replay()
     e1.record(stream)
     torch.cuda.synchronize()
+    t_step_end = time.perf_counter()
     barrier(world)
     ms_step = e0.elapsed_time(e1) / args.steps
 
@@ -454,7 +586,18 @@ def run_ours(args, world, rank, local):
                           "config": cfgs[m].as_dict(), "table_hit": hits[m]})
         gemm_total_us += res["gemm"]
         gemm_total_bytes += gb
+    # ---- every configured shape (the metric's M <= 32 decode shapes and the
+    # large-M companion), single GPU only: one graph of back-to-back GEMMs per
+    # shape, dispatched from the same table
+    fam = None
+    if world == 1 and not args.no_suite:
+        fam_results, fam_peaks = time_families(HEADLINE_FAMILIES, dev, table)
+        fam = dict(summarise_families(fam_results), peaks=fam_peaks,
+                   per_shape=[[r["format"], r["M"], r["N"], r["K"], r["us"], r["frac_roofline"], r["bound"]]
+                              for r in fam_results])
+    clk_step = clocks.window(t_load, t_step_end)
     clk = clocks.stop()
+    clk["step_window"] = clk_step
 
     # ---- end to end through the public API with host buffers: per step the
     # three activations are copied in from pinned host memory, the step's
@@ -500,16 +643,16 @@ def run_ours(args, world, rank, local):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step_max, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "M": list(MS), "N": N, "K": K, "format": "W8A8_INT8",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": f"inputs larger than L2: {copies} rotating weight copies "
-                         f"({copies * wbytes / 1e6:.0f} MB > 2 x {l2 / 1e6:.0f} MB L2)",
+        "config": bench_config(world),
+        "method": {"l2": f"{copies} rotating weight copies ({copies * wbytes / 1e6:.0f} MB > 2 x {l2 / 1e6:.0f} MB L2)",
                    "step": "per M: activation quant + GEMM; the K timed steps run as CUDA graphs of up to "
                            f"{chunk} consecutive steps each (qg.capture_steps); e2e: per step copies in from pinned "
                            "host memory, one graph replay, copies out, sync",
+                   "per_shape": "one CUDA graph of back-to-back qgemm_run launches per shape over weight copies "
+                                "totalling more than 2 x L2, 5 replays after a warm one, CUDA events",
                    "table": os.path.relpath(args.table, ROOT) if table is not None else "built-in default"},
         "per_shape": per_shape,
-        "geomean_frac_hbm_roofline": round(geo, 4),
+        "int8_decode_geomean_frac_hbm_roofline": round(geo, 4),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "kernel": "qgemm_kernel<INT8, swap-AB> (all three shapes, launch-weighted)",
@@ -521,6 +664,13 @@ def run_ours(args, world, rank, local):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
     }
+    if fam is not None:
+        # the metric over every configured shape: µs per shape and the
+        # geomean fraction of roofline for M <= 32 (HBM-bound decode shapes),
+        # plus the tensor-bound M >= 4096 shapes
+        line["geomean_frac_roofline_M_le_32"] = round(fam["geomean_frac_roofline_M_le_32"], 4)
+        line["frac_tensor_peak_M_ge_4096"] = round(fam["geomean_frac_roofline_M_ge_4096"], 4)
+        line["shapes"] = fam
     if not args.no_cpu_baseline and world == 1:
         single = cpu_baseline(2)
         line["cpu_baseline_single_thread"] = {k: single[k] for k in ("value", "unit", "cores", "kind", "sample")}
@@ -528,8 +678,8 @@ def run_ours(args, world, rank, local):
             cb = cpu_baseline_all_cores()
         except Exception as exc:   # the pool is measurement harness, not the product path
             cb = dict(single, all_cores_error=f"{type(exc).__name__}: {exc}"[:200])
-        line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample", "all_cores_error")
-                                if k in cb}
+        line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "host_cores", "kind", "sample",
+                                                     "all_cores_error") if k in cb}
     elif world > 1:
         line["cpu_baseline"] = None
     print(json.dumps(line), flush=True)
@@ -695,15 +845,104 @@ def run_moe_suite(args, local):
                       "peaks": {"hbm_gbs": hbm}}), flush=True)
 
 
-def run_suite(args, names, local):
-    import numpy as np
+def rotation(qg, torch, Wq, fmt, rows, K, is_weight, total_min, dev, cap=4096):
+    """Copies of a quantised operand in one pool, enough that their total
+    exceeds `total_min` bytes (so a pass over them streams from HBM): returns
+    (qg_operand structs, pool tensor that owns them)."""
+    qb, sb = Wq.q.numel(), Wq.scale.numel()
+    qs, ss = -(-qb // 256) * 256, -(-sb // 256) * 256
+    per = qs + ss
+    copies = int(max(2, min(cap, -(-total_min // (qb + sb)) + 2)))
+    pool = torch.empty(copies, per, dtype=torch.uint8, device=dev)
+    pool[0, :qb].copy_(Wq.q)
+    pool[0, qs:qs + sb].copy_(Wq.scale)
+    pool[1:].copy_(pool[0].expand(copies - 1, per))
+    base = pool.data_ptr()
+    ops = [qg.qg_operand(base + i * per, base + i * per + qs, Wq.global_scale.data_ptr(), rows, K)
+           for i in range(copies)]
+    return ops, pool
+
+
+def time_shape(qg, torch, dev, fmt, M, N, K, Wq, cfg, l2, hbm, bf16, gen, single=False):
+    """Device time of one qgemm_run of this shape: a CUDA graph of back-to-back
+    launches (programmatic dependent launch on) over weight copies whose
+    total exceeds 2 x L2 (and activation copies for M >= 4096), replayed
+    after one warm replay, CUDA events on the launching stream."""
+    flops = 2.0 * M * N * K
+    byts = shape_bytes(fmt, M, N, K)
+    a = torch.randn(M, K, device=dev, generator=gen).to(torch.bfloat16)
+    A0 = qg.quantize_act(fmt, a)
+    del a
+    large = M >= 4096
+    if large:
+        Wrot, wpool = rotation(qg, torch, Wq, fmt, N, K, True, 2 * l2, dev, cap=16)
+        Arot, apool = rotation(qg, torch, A0, fmt, M, K, False, 2 * l2, dev, cap=16)
+        n = max(len(Wrot), len(Arot))
+    else:
+        Wrot, wpool = rotation(qg, torch, Wq, fmt, N, K, True, 2 * l2, dev)
+        Arot, apool = [A0.c], None
+        n = len(Wrot)
+    ws = qg.Workspace(dev)
+    wsp, wsb = ws.get(qg.qgemm_workspace_size(fmt, M, N, K, cfg))
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    reps = max(n, 8) if not large else 2 * n
+    st = qg._stream(None)
+    qg.check(qg.qgemm_run(fmt, Arot[0], Wrot[0], M, N, K, cfg, wsp, wsb, Y.data_ptr(), N, 0, st))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        st = qg._stream(None)
+        for r in range(reps):
+            qg.check(qg.qgemm_run(fmt, Arot[r % len(Arot)], Wrot[r % len(Wrot)], M, N, K, cfg, wsp, wsb,
+                                  Y.data_ptr(), N, 0, st))
+    g.replay()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    n_rep = 5 if not large else 2
+    e0.record()
+    for _ in range(n_rep):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    us = 1000.0 * e0.elapsed_time(e1) / (n_rep * reps)
+    rec = {}
+    if single:
+        # one eager call on its own (after a sync, events on the same
+        # stream): the device waits from the first event for the host's
+        # submission (argument checks, two tensor map encodings, the launch),
+        # so this is an eager call's cost from call to completion, with no
+        # neighbour to overlap; its weight copy was last read a rotation ago
+        st = qg._stream(None)
+        e0.record()
+        qg.check(qg.qgemm_run(fmt, Arot[reps % len(Arot)], Wrot[reps % len(Wrot)], M, N, K, cfg, wsp, wsb,
+                              Y.data_ptr(), N, 0, st))
+        e1.record()
+        torch.cuda.synchronize()
+        rec["single_launch_us"] = round(1000.0 * e0.elapsed_time(e1), 3)
+    del g, Wrot, wpool, Arot, apool, Y, A0
+    t_hbm = byts / (hbm * 1e9) * 1e6
+    t_tc = flops / (tensor_peak(fmt, bf16) * 1e12) * 1e6
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    frac = max(t_hbm, t_tc) / us
+    return dict({"format": FMT_NAME[fmt], "M": M, "N": N, "K": K, "us": round(us, 3),
+                 "GB/s": round(byts / us / 1e3, 1), "TFLOP/s": round(flops / us / 1e6, 2), "bound": bound,
+                 "roofline_us": round(max(t_hbm, t_tc), 3), "frac_roofline": round(frac, 4),
+                 "config": cfg.as_dict(), "rotating_copies": n}, **rec)
+
+
+def geomean(xs):
+    xs = list(xs)
+    return math.exp(sum(math.log(max(x, 1e-9)) for x in xs) / len(xs)) if xs else None
+
+
+def time_families(names, dev, table, only_m=None, single=False, emit=None):
+    """Per-shape device times of every shape of the named workload families,
+    each with the configuration the table dispatches (or the scored
+    default).  Returns the records; `emit` sees each as it is made."""
     import torch
 
     import precision_quantized_gemm_b200 as qg
 
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    table = qg.Table(args.table) if os.path.exists(args.table) else None
     pk = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
         os.path.join(ROOT, "MEASURED_PEAKS.json")) else {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
     hbm, bf16 = float(pk["hbm_gbs"]), float(pk["bf16_tflops"])
@@ -713,96 +952,62 @@ def run_suite(args, names, local):
     results = []
     for name in names:
         for fmt, Ms, NKs in SUITES[name]:
-            if args.only_m:
-                keep = {int(x) for x in args.only_m.split(",")}
-                Ms = [m for m in Ms if m in keep]
+            if only_m:
+                Ms = [m for m in Ms if m in only_m]
                 if not Ms:
                     continue
             for (N, K) in NKs:
                 w = (torch.randn(N, K, device=dev, generator=gen) * 0.02).to(torch.bfloat16)
                 Wq = qg.quantize_weight(fmt, w)
                 del w
-                wbytes = Wq.q.numel() + Wq.scale.numel()
                 for M in Ms:
-                    flops = 2.0 * M * N * K
-                    byts = shape_bytes(fmt, M, N, K)
-                    # inputs larger than L2: rotate weight copies (and
-                    # activations for large M) past 2 x L2
-                    per_call = wbytes + (M * K if fmt != 3 else M * K // 2)
-                    copies = int(max(1, min(64, (2 * l2) // max(per_call, 1) + 2)))
-                    Ws = [Wq]
-                    for _ in range(copies - 1):
-                        o = qg.Operand(fmt, True, N, K, dev)
-                        o.q.copy_(Wq.q)
-                        o.scale.copy_(Wq.scale)
-                        o.global_scale.copy_(Wq.global_scale)
-                        Ws.append(o)
-                    a = torch.randn(M, K, device=dev, generator=gen).to(torch.bfloat16)
-                    As = [qg.quantize_act(fmt, a) for _ in range(copies if M >= 4096 else 1)]
                     cfg, hit = (table.dispatch(fmt, M, N, K) if table is not None
                                 else (qg.qgemm_default_config(fmt, M, N, K), 0))
-                    ws = qg.Workspace(dev)
-                    wsp, wsb = ws.get(qg.qgemm_workspace_size(fmt, M, N, K, cfg))
-                    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-                    reps = max(2 * copies, 8) if M < 4096 else 2 * copies
-                    st = qg._stream(None)
-                    qg.check(qg.qgemm_run(fmt, As[0].c, Ws[0].c, M, N, K, cfg, wsp, wsb, Y.data_ptr(), N, 0, st))
-                    g = torch.cuda.CUDAGraph()
-                    with torch.cuda.graph(g):
-                        st = qg._stream(None)
-                        for r in range(reps):
-                            qg.check(qg.qgemm_run(fmt, As[r % len(As)].c, Ws[r % copies].c, M, N, K, cfg,
-                                                  wsp, wsb, Y.data_ptr(), N, 0, st))
-                    g.replay()
-                    torch.cuda.synchronize()
-                    e0 = torch.cuda.Event(enable_timing=True)
-                    e1 = torch.cuda.Event(enable_timing=True)
-                    n_rep = 5 if M < 4096 else 2
-                    e0.record()
-                    for _ in range(n_rep):
-                        g.replay()
-                    e1.record()
-                    torch.cuda.synchronize()
-                    us = 1000.0 * e0.elapsed_time(e1) / (n_rep * reps)
-                    # one eager call on its own (after a sync, events on the
-                    # same stream): the device waits from the first event
-                    # for the host's submission (argument checks, two tensor
-                    # map encodings, the launch), so this is what an eager
-                    # call costs from call to completion, with no neighbour
-                    # to overlap; its weight copy is the next in the
-                    # rotation, last read `copies` calls ago (past 2 x L2)
-                    st = qg._stream(None)
-                    e0.record()
-                    qg.check(qg.qgemm_run(fmt, As[reps % len(As)].c, Ws[reps % copies].c, M, N, K, cfg, wsp, wsb,
-                                          Y.data_ptr(), N, 0, st))
-                    e1.record()
-                    torch.cuda.synchronize()
-                    us_single = 1000.0 * e0.elapsed_time(e1)
-                    t_hbm = byts / (hbm * 1e9) * 1e6
-                    t_tc = flops / (tensor_peak(fmt, bf16) * 1e12) * 1e6
-                    bound = "hbm" if t_hbm >= t_tc else "tensor"
-                    frac = max(t_hbm, t_tc) / us
-                    rec = {"suite": name, "format": FMT_NAME[fmt], "M": M, "N": N, "K": K, "us": round(us, 3),
-                           "single_launch_us": round(us_single, 3),
-                           "GB/s": round(byts / us / 1e3, 1), "TFLOP/s": round(flops / us / 1e6, 2),
-                           "bound": bound, "roofline_us": round(max(t_hbm, t_tc), 3),
-                           "frac_roofline": round(frac, 4), "config": cfg.as_dict(), "table_hit": hit,
-                           "rotating_copies": copies}
-                    print(json.dumps(rec), flush=True)
+                    rec = dict({"suite": name}, **time_shape(qg, torch, dev, fmt, M, N, K, Wq, cfg, l2, hbm, bf16,
+                                                              gen, single=single))
+                    rec["table_hit"] = hit
                     results.append(rec)
-                    del g, As, Ws[1:], Y
+                    if emit:
+                        emit(rec)
                     torch.cuda.empty_cache()
-    def geo(xs):
-        return math.exp(sum(math.log(max(x, 1e-9)) for x in xs) / len(xs)) if xs else None
+                del Wq
+    return results, {"hbm_gbs": hbm, "bf16_tflops": bf16,
+                     "note": "fp8/int8 tensor peak = 2 x measured bf16, fp4 = 4 x"}
+
+
+# The families of the headline metric (M <= 32 decode shapes) and its
+# large-M companion: every configured workload.
+HEADLINE_FAMILIES = ["fp8_tiny", "int8", "block_fp8", "nvfp4", "sweep", "large_m"]
+
+
+def summarise_families(results):
     small = [r["frac_roofline"] for r in results if r["M"] <= 32]
     medium = [r["frac_roofline"] for r in results if 32 < r["M"] < 4096]
     large = [r["frac_roofline"] for r in results if r["M"] >= 4096]
-    print(json.dumps({"summary": True, "shapes": len(results), "geomean_frac_roofline_M_le_32": geo(small),
-                      "geomean_frac_roofline_M_33_to_4095": geo(medium),
-                      "geomean_frac_roofline_M_ge_4096": geo(large),
-                      "geomean_frac_roofline_all": geo([r["frac_roofline"] for r in results]),
-                      "peaks": {"hbm_gbs": hbm, "bf16_tflops": bf16,
-                                "note": "fp8/int8 tensor peak = 2 x measured bf16, fp4 = 4 x"}}), flush=True)
+    by_fmt = {}
+    for r in results:
+        if r["M"] <= 32:
+            by_fmt.setdefault(r["format"], []).append(r["frac_roofline"])
+    return {"shapes": len(results), "shapes_M_le_32": len(small),
+            "geomean_frac_roofline_M_le_32": geomean(small),
+            "geomean_frac_roofline_M_33_to_4095": geomean(medium),
+            "geomean_frac_roofline_M_ge_4096": geomean(large),
+            "geomean_frac_roofline_all": geomean(r["frac_roofline"] for r in results),
+            "geomean_frac_roofline_M_le_32_by_format": {k: round(geomean(v), 4) for k, v in by_fmt.items()}}
+
+
+def run_suite(args, names, local):
+    import torch
+
+    import precision_quantized_gemm_b200 as qg
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    table = qg.Table(args.table) if os.path.exists(args.table) else None
+    only = {int(x) for x in args.only_m.split(",")} if args.only_m else None
+    results, peaks_used = time_families(names, dev, table, only_m=only, single=True,
+                                        emit=lambda r: print(json.dumps(r), flush=True))
+    print(json.dumps(dict({"summary": True}, **summarise_families(results), peaks=peaks_used)), flush=True)
 
 
 def main():

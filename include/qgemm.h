@@ -270,7 +270,8 @@ qg_status qgemm_run_fused_act(qg_format f, const void* A, int lda, const qg_oper
  *     rejected with QG_ERR_WORKSPACE before any device work.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     before any stream capture.  A first call on a device made while
+ *     `stream` is being captured is refused with QG_ERR_UNSUPPORTED.
  *   - No cudaMalloc, cudaFree or other allocation is made.  For reduce_mode 2
  *     the tile-counter region is cleared with cudaMemsetAsync on `stream`.
  *   - Every call shares the one array and it keeps the last call's contents:
@@ -383,6 +384,23 @@ const char* qgemm_status_string(qg_status s);
  * that expired; synchronises the device.  Returns QG_OK or
  * QG_ERR_DEVICE_TIMEOUT. */
 qg_status qgemm_device_error(void);
+
+/* Limit of every bounded in-kernel wait of later launches, in ns of the GPU's
+ * %globaltimer (0 restores the default of 200 ms).  On expiry a wait sets the
+ * device error word (QG_ERR_DEVICE_TIMEOUT from qgemm_device_error) and the
+ * kernel leaves its loops, waits (bounded) for its own copies in flight,
+ * frees its TMEM and returns, so the context stays usable.  Host state, not
+ * thread-safe. */
+void qgemm_set_wait_limit(unsigned long long limit_ns);
+
+/* Failure-detection self-test: launches one CTA on `stream` that waits, with
+ * the library's bounded wait and a limit of `limit_ns` (1 ns .. 200 ms), on
+ * an mbarrier nothing arrives on.  The wait expires and sets the device error
+ * word, which the next qgemm_device_error reports (QG_ERR_DEVICE_TIMEOUT) and
+ * clears.  No copy or MMA is in flight, so the kernel returns normally.
+ * QG_ERR_INVALID_ARG for a limit outside that range; QG_ERR_CUDA if the
+ * launch fails. */
+qg_status qgemm_selftest_wait_expiry(unsigned long long limit_ns, void* stream);
 /* Enables (1) or disables (0) programmatic dependent launch for the
  * library's kernels (default 1). */
 void qgemm_set_pdl(int enable);

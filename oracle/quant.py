@@ -18,8 +18,9 @@ formats; the recipes below are the plain readings of those names):
   those of the "FP8 block-scaling GEMM" of TensorRT-LLM issue 16363.
 * NVFP4 (FlashInfer PR 3948, ``mm_fp4 --use_nvfp4``): e2m1 codes with an e4m3
   scale per 16 consecutive K elements and one fp32 tensor scale.  The pages
-  name the format but not its recipe; the reading used here (parity unpinned
-  by the pages, pinned only by the invariants in the tests):
+  name the format but not its recipe; the reading used here (the pages fix
+  no recipe, so this reading is pinned by hand-worked blocks derived from it
+  and by invariants, not by values the pages print):
   g = amax(tensor) / (448 * 6); block scale s_b = e4m3((amax_b / 6) / g);
   code = e2m1(x / (dec(s_b) * g)), and code 0 wherever dec(s_b) == 0.
 
@@ -95,7 +96,7 @@ def nvfp4(x_bits: np.ndarray, global_amax: float | None = None, sf_vec: int = 16
     Returns (codes uint8 [R, K] one e2m1 code per element, block scale codes
     uint8 [R, K/16] e4m3, g fp32 scalar).  ``global_amax`` replaces the
     tensor's own amax when given (a static activation scale).
-    Parity unpinned by the pages: the recipe is this module's reading.
+    The recipe is this module's reading (the pages give none).
     """
     x = bf16_from_bits(x_bits)
     R, K = x.shape

@@ -43,7 +43,7 @@ EXPORTS = [
     "qgemm_table_free", "qgemm_table_size", "qgemm_dispatch", "qgemm_tune", "qgemm_device_error",
     "qgemm_run_noalloc", "qgemm_set_trace", "qgemm_run_fused_act", "qgemm_set_tune_log",
     "qgemm_score_config", "qgemm_rank_configs", "qgemm_tune_ranked", "qgemm_table_validate",
-    "qgemm_run_grouped", "qgemm_grouped_default_config",
+    "qgemm_run_grouped", "qgemm_grouped_default_config", "qgemm_set_wait_limit", "qgemm_selftest_wait_expiry",
 ]
 
 
@@ -110,6 +110,8 @@ def lib() -> ctypes.CDLL:
             "qgemm_dispatch": (c_int, [c_void_p, c_int, c_int, c_int, c_int, POINTER(qg_config), POINTER(c_int)]),
             "qgemm_tune": (c_int, [c_void_p, c_int, POINTER(c_int), c_int, POINTER(c_int), c_int, c_double, c_int]),
             "qgemm_device_error": (c_int, []),
+            "qgemm_set_wait_limit": (None, [ctypes.c_ulonglong]),
+            "qgemm_selftest_wait_expiry": (c_int, [ctypes.c_ulonglong, c_void_p]),
             "qgemm_set_trace": (None, [c_void_p, c_size_t]),
             "qgemm_set_tune_log": (None, [c_char_p]),
             "qgemm_score_config": (c_int, [c_int, c_int, c_int, c_int, POINTER(qg_config), POINTER(c_double)]),
@@ -238,6 +240,17 @@ def qgemm_dispatch(table, fmt, M, N, K):
 
 def qgemm_device_error():
     return lib().qgemm_device_error()
+
+
+def qgemm_set_wait_limit(limit_ns: int):
+    """Limit (ns) of every bounded in-kernel wait of later launches (0: the 200 ms default)."""
+    lib().qgemm_set_wait_limit(int(limit_ns))
+
+
+def qgemm_selftest_wait_expiry(limit_ns: int, stream=None) -> int:
+    """Launches a wait on an mbarrier nothing arrives on, bounded by limit_ns;
+    the next qgemm_device_error() reports QG_ERR_DEVICE_TIMEOUT."""
+    return lib().qgemm_selftest_wait_expiry(int(limit_ns), _stream(stream))
 
 
 def qgemm_set_trace(buf_ptr, nbytes):

@@ -24,6 +24,7 @@ namespace {
 using qg::GemmParams;
 
 bool g_pdl = true;
+unsigned long long g_wait_ns = qg::kWaitLimitNs;   // limit of every in-kernel wait
 unsigned long long* g_trace = nullptr;   // debug phase trace buffer (device)
 size_t g_trace_bytes = 0;
 
@@ -56,6 +57,21 @@ qg_status device_info(DeviceInfo** out) {
   if (!d.sm100) return QG_ERR_UNSUPPORTED;
   *out = &d;
   return QG_OK;
+}
+
+// One mbarrier that nothing arrives on, waited for with the library's own
+// bounded wait: after `limit_ns` the wait gives up and sets the device error
+// word, exactly as a GEMM's wait would.  No copy or MMA is in flight, so the
+// kernel then simply returns.
+__global__ void wait_expiry_kernel(unsigned int* err, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    qg::mbar_init(&bar, 1);
+    qg::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) (void)qg::mbar_wait(&bar, 0, err, limit_ns);
+  __syncthreads();
 }
 
 // ------------------------------------------------------------- TMA maps --
@@ -437,6 +453,7 @@ qg_status launch_run(qg_format f, const qg_operand* A, const void* act, int lda,
   prm.experts = experts;
   prm.expert_offsets = expert_offsets;
   prm.err = d->err;
+  prm.wait_ns = g_wait_ns;
   if (g_trace != nullptr &&
       (size_t)tp * tq * cfg->split_k * qg::kTraceEvents * sizeof(unsigned long long) <= g_trace_bytes)
     prm.trace = g_trace;
@@ -644,6 +661,19 @@ qg_status rule_default_config(qg_format f, int M, int N, int K, qg_config* out) 
 }  // namespace qg
 
 extern "C" {
+
+void qgemm_set_wait_limit(unsigned long long limit_ns) {
+  g_wait_ns = limit_ns > 0 ? limit_ns : qg::kWaitLimitNs;
+}
+
+qg_status qgemm_selftest_wait_expiry(unsigned long long limit_ns, void* stream) {
+  if (limit_ns == 0 || limit_ns > qg::kWaitLimitNs) return QG_ERR_INVALID_ARG;
+  DeviceInfo* d;
+  qg_status s = device_info(&d);
+  if (s != QG_OK) return s;
+  wait_expiry_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(d->err, limit_ns);
+  return cudaGetLastError() == cudaSuccess ? QG_OK : QG_ERR_CUDA;
+}
 
 qg_status qgemm_device_error(void) {
   DeviceInfo* d;

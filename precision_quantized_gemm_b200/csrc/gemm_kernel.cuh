@@ -87,6 +87,7 @@ struct GemmParams {
   unsigned int* counters;      // split-K per-tile arrival counters
   int reduce_mode;             // kReduce*
   unsigned int* err;           // device error word
+  unsigned long long wait_ns;  // limit of every in-kernel wait (ns)
   unsigned long long* trace;   // optional: kTraceEvents timestamps per CTA (ns)
   int nkt_max;                 // most K tiles any split slice holds: ceil(kt_total / split_k)
   int recv_cols;               // cluster push: token columns per receive slot (0: no receive buffer)
@@ -528,7 +529,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
       int st = 0;                              // stage of K tile i; its previous use's phase
       uint32_t ph = 0;
       for (int i = pre; i < nkt; ++i) {
-        if (!mbar_wait(&empty[st], ph, prm.err)) { ok = false; break; }
+        if (!mbar_wait(&empty[st], ph, prm.err, prm.wait_ns)) { ok = false; break; }
         mbar_arrive_expect_tx(&full[st], stage_tx);
         load_w(i, st);
         if (!a_threads) load_a(i, st);
@@ -539,7 +540,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
         *flag_abort = 1;
         // Drain: wait (bounded) until every issued copy has landed.
         for (int i = (issued > S ? issued - S : 0); i < issued; ++i)
-          mbar_wait(&full[i % S], (i / S) & 1, prm.err);
+          mbar_wait(&full[i % S], (i / S) & 1, prm.err, prm.wait_ns);
       }
     }
   } else if (warp == 1) {
@@ -563,15 +564,15 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
       int gb = 0, gr = 0;                      // Block_FP8: group buffer of K tile i, and its round
       bool abort = false;
       for (int i = 0; i < nkt; ++i) {
-        if (!mbar_wait(&full[st], ph, prm.err)) { abort = true; break; }
+        if (!mbar_wait(&full[st], ph, prm.err, prm.wait_ns)) { abort = true; break; }
         if (i == 0) {
-          if (a_threads && !mbar_wait(act_ready, 0, prm.err)) { abort = true; break; }
+          if (a_threads && !mbar_wait(act_ready, 0, prm.err, prm.wait_ns)) { abort = true; break; }
           trace_at(prm, kTrFirstFull);
         }
         if (i == nkt - 1) trace_at(prm, kTrLastFull);
         uint32_t d_t = tmem_base;
         if constexpr (C::kBlock) {
-          if (gr > 0 && !mbar_wait(&tempty[gb], (uint32_t)(gr - 1) & 1u, prm.err)) { abort = true; break; }
+          if (gr > 0 && !mbar_wait(&tempty[gb], (uint32_t)(gr - 1) & 1u, prm.err, prm.wait_ns)) { abort = true; break; }
           d_t = tmem_base + (uint32_t)(gb * BN);
         }
         tc_fence_after();
@@ -743,7 +744,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
           const uint32_t dst = mapa_shared(smem_u32(exch + kz * BN), z);
           const uint32_t zbar = mapa_shared(smem_u32(amax_full), z);
           for (int r = etid / Sk; r < Mt; r += ET / Sk) st_async_b32(dst + 4u * (uint32_t)r, amax_u[r], zbar);
-          fz_ok = mbar_wait_cluster(amax_full, 0, prm.err);
+          fz_ok = mbar_wait_cluster(amax_full, 0, prm.err, prm.wait_ns);
         }
         if (etid == 0) trace_at(prm, kTrActAmax);
         if (etid < BN) {
@@ -871,7 +872,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
       ok = __all_sync(0xffffffffu, fz_ok);
       for (int i = 0; i < nkt && ok; ++i) {
         const int b = i % C::kNAcc;
-        ok = __all_sync(0xffffffffu, mbar_wait(&tfull[b], (i / C::kNAcc) & 1, prm.err));
+        ok = __all_sync(0xffffffffu, mbar_wait(&tfull[b], (i / C::kNAcc) & 1, prm.err, prm.wait_ns));
         if (!ok) break;
         tc_fence_after();
         // acc += p_g * (s_a * s_w): one FMA per element
@@ -939,7 +940,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
         if (lane == 0) mbar_arrive(&tempty[b]);
       }
     } else {
-      ok = __all_sync(0xffffffffu, fz_ok && mbar_wait(acc_full, 0, prm.err));
+      ok = __all_sync(0xffffffffu, fz_ok && mbar_wait(acc_full, 0, prm.err, prm.wait_ns));
       tc_fence_after();
     }
     if (etid == 0) {
@@ -1092,7 +1093,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
         }
       }
       if (etid == 0) trace_at(prm, kTrSent);
-      const bool got = __all_sync(0xffffffffu, mbar_wait_cluster(recv_full, 0, prm.err));
+      const bool got = __all_sync(0xffffffffu, mbar_wait_cluster(recv_full, 0, prm.err, prm.wait_ns));
       if (etid == 0) trace_at(prm, kTrRecv);
       const int r0 = (int)cluster_ctarank() * rows_per;
       const int zstride = rows_per * prm.recv_cols;

@@ -2,6 +2,7 @@
 // Included by exactly one translation unit per format with QG_FMT and
 // QG_LAUNCH_NAME defined.
 #pragma once
+#include "attr_cache.h"
 #include "gemm_kernel.cuh"
 #include "internal.h"
 
@@ -22,12 +23,16 @@ cudaError_t launch_one(const CUtensorMap& tp, const CUtensorMap& tq, const GemmP
   constexpr int kTmemCtas = 512 / Cfg<FMT, BN>::kTmemCols;
   const size_t smem_floor = (size_t)233472 / (kTmemCtas + 1);
   if (smem < smem_floor) smem = smem_floor;
-  static int configured_bytes = 0;
-  if ((int)smem > configured_bytes) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured_bytes = (int)smem;
-  }
+  // the kernel's shared-memory limit is raised per device (the attribute
+  // acts on the current device), once per larger size
+  static GrowOnlyAttr smem_attr;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = static_cast<cudaError_t>(smem_attr.ensure(dev, (int)smem, [&](int bytes) {
+    return static_cast<int>(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  }));
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(Cfg<FMT, BN>::kThreads);

@@ -30,13 +30,19 @@ void* g_scratch_addr[kMaxDevices] = {};
 std::mutex g_mu;
 
 // Device address of the scratch array on the current device, looked up on
-// the first call per device with that device current.
-qg_status scratch_address(void** out) {
+// the first call per device with that device current.  That lookup may load
+// the library's device code, which a stream being captured into a CUDA graph
+// does not allow: a first call on a device made during capture is refused
+// with QG_ERR_UNSUPPORTED (make one call before capturing), not attempted.
+qg_status scratch_address(cudaStream_t stream, void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return QG_ERR_NO_DEVICE;
   if (dev < 0 || dev >= kMaxDevices) return QG_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lk(g_mu);
   if (g_scratch_addr[dev] == nullptr) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return QG_ERR_CUDA;
+    if (cs != cudaStreamCaptureStatusNone) return QG_ERR_UNSUPPORTED;
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return QG_ERR_CUDA;
     g_scratch_addr[dev] = p;
@@ -63,7 +69,7 @@ extern "C" qg_status qgemm_run_noalloc(qg_format f, const qg_operand* A, const q
   if (s0 != QG_OK) return s0;
   void* scratch = nullptr;
   if (need > 0) {
-    qg_status s = scratch_address(&scratch);
+    qg_status s = scratch_address((cudaStream_t)stream, &scratch);
     if (s != QG_OK) return s;
     // The array keeps the previous call's contents.  Partial sums are fully
     // rewritten before they are read; the tile counters of reduce_mode 2 must

@@ -8,8 +8,9 @@
 
 namespace qg {
 
-// Upper bound of any in-kernel wait (ns).  A healthy wait lasts microseconds;
-// past this the kernel records an error and leaves its loops.
+// Default upper bound of an in-kernel wait (ns), passed to the kernels as a
+// parameter.  A healthy wait lasts microseconds; past the limit the kernel
+// records an error and leaves its loops.
 constexpr unsigned long long kWaitLimitNs = 200000000ull;
 
 // Device error word bits (the word itself lives in the host API's
@@ -65,14 +66,15 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 // Bounded wait for phase `parity` of `bar`.  Returns false (and sets the
-// timeout bit of *err) if the limit expired.  A phase that has already
-// completed costs one non-blocking test.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int* err) {
+// timeout bit of *err) once `limit_ns` of %globaltimer have passed.  A phase
+// that has already completed costs one non-blocking test.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int* err,
+                                          unsigned long long limit_ns) {
   if (mbar_test_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       atomicOr(err, kErrWaitTimeout);
       return false;
     }
@@ -81,7 +83,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
 
 // Bounded wait with acquire semantics at cluster scope (pairs with release
 // arrivals from other CTAs of the cluster).
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, unsigned int* err) {
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, unsigned int* err,
+                                                  unsigned long long limit_ns) {
   const unsigned long long t0 = globaltimer();
   while (true) {
     uint32_t ok;
@@ -93,7 +96,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
         : "r"(smem_u32(bar)), "r"(parity)
         : "memory");
     if (ok) return true;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       atomicOr(err, kErrWaitTimeout);
       return false;
     }

@@ -295,3 +295,11 @@ def test_grouped_default_config_rejects_nvfp4_and_bad_sizes():
     assert qg.lib().qgemm_grouped_default_config(qg.QG_NVFP4, 8, 8, 256, 512, c) == qg.QG_ERR_UNSUPPORTED
     assert qg.lib().qgemm_grouped_default_config(qg.QG_FP8_DYNAMIC, 0, 8, 256, 512, c) == qg.QG_ERR_INVALID_ARG
     assert qg.lib().qgemm_grouped_default_config(qg.QG_FP8_DYNAMIC, 8, 8, 256, 100, c) == qg.QG_ERR_INVALID_ARG
+
+
+def test_wait_expiry_selftest_rejects_limits_before_the_device():
+    # checked on the host before any device work (no GPU needed)
+    assert qg.lib().qgemm_selftest_wait_expiry(0, None) == qg.QG_ERR_INVALID_ARG
+    assert qg.lib().qgemm_selftest_wait_expiry(10 ** 9, None) == qg.QG_ERR_INVALID_ARG
+    qg.qgemm_set_wait_limit(5_000_000)
+    qg.qgemm_set_wait_limit(0)

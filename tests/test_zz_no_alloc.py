@@ -53,6 +53,8 @@ def test_noalloc_matches_run_with_workspace(fmt, M, N, K, split, mode):
         torch.cuda.synchronize()
         bad = tolerance_violations(bf16_to_np(y), ref_np)
         assert not bad.any(), f"call {call}: {int(bad.sum())} elements differ from qgemm_run"
+        # the same kernel sums the same partials in the same split order
+        assert torch.equal(y, ref), f"call {call}: not bitwise equal to qgemm_run"
     assert qg.qgemm_device_error() == qg.QG_OK
 
 
