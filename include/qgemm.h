@@ -74,7 +74,7 @@ typedef enum {
                       before bf16 rounding)                                         */
 } qg_out_kind;
 
-/* Kernel configuration: the tunables of the unified kernel. */
+/* Kernel configuration: which kernel runs (variant) and its tunables. */
 typedef struct {
   int32_t split_k;     /* 1, 2, 4, ..., 256: K is cut into split_k slices of whole
                           128-byte K tiles, each reduced by its own CTA            */
@@ -91,7 +91,17 @@ typedef struct {
                           1 = partials in the workspace + a second-pass kernel;
                           2 = partials in the workspace, summed in-kernel by the
                               last-arriving CTA of each tile (tile counters)    */
-  int32_t reserved[3]; /* must be zero                                             */
+  int32_t variant;     /* 0: the tile kernel (tcgen05, the fields above);
+                          1: the decode ("skinny") kernel for FP8_DYNAMIC,
+                          W8A8_INT8 and BLOCK_FP8: warp-level MMAs with register
+                          accumulators, each CTA owning `rows` weight rows over
+                          the whole of K and tile_n (16 or 32) tokens; requires
+                          split_k = 1, swap_ab = 1, reduce_mode = 0, and
+                          `stages` (the ring of 128-byte K tiles, 2..64) a
+                          multiple of 64 / rows                                  */
+  int32_t rows;        /* variant 1: weight rows per CTA, 8, 16, 32 or 64;
+                          variant 0: must be 0                                    */
+  int32_t reserved;    /* must be zero                                            */
 } qg_config;
 
 /* A quantized operand (activations A_q or weights W_q); non-owning views.

@@ -49,19 +49,28 @@ EXPORTS = [
 
 class qg_config(ctypes.Structure):
     _fields_ = [("split_k", c_int32), ("swap_ab", c_int32), ("tile_n", c_int32),
-                ("stages", c_int32), ("reduce_mode", c_int32), ("reserved", c_int32 * 3)]
+                ("stages", c_int32), ("reduce_mode", c_int32), ("variant", c_int32), ("rows", c_int32),
+                ("reserved", c_int32)]
 
     def as_dict(self):
-        return {k: getattr(self, k) for k in ("split_k", "swap_ab", "tile_n", "stages", "reduce_mode")}
+        return {k: getattr(self, k) for k in ("split_k", "swap_ab", "tile_n", "stages", "reduce_mode", "variant",
+                                               "rows")}
 
     def __repr__(self):
         return f"qg_config({self.as_dict()})"
 
 
-def make_config(split_k=1, swap_ab=1, tile_n=16, stages=8, reduce_mode=0) -> qg_config:
+def make_config(split_k=1, swap_ab=1, tile_n=16, stages=8, reduce_mode=0, variant=0, rows=0) -> qg_config:
     c = qg_config()
     c.split_k, c.swap_ab, c.tile_n, c.stages, c.reduce_mode = split_k, swap_ab, tile_n, stages, reduce_mode
+    c.variant, c.rows = variant, rows
     return c
+
+
+def skinny_config(tile_n=16, rows=32, stages=32) -> qg_config:
+    """Configuration of the decode ("skinny") kernel: `rows` weight rows per
+    CTA over the whole of K, `tile_n` tokens, a ring of `stages` K tiles."""
+    return make_config(split_k=1, swap_ab=1, tile_n=tile_n, stages=stages, reduce_mode=0, variant=1, rows=rows)
 
 
 class qg_operand(ctypes.Structure):

@@ -25,6 +25,7 @@ using qg::GemmParams;
 
 bool g_pdl = true;
 unsigned long long g_wait_ns = qg::kWaitLimitNs;   // limit of every in-kernel wait
+bool g_l2_ahead = true;                           // Swap-AB weight prefetch for later CTAs
 unsigned long long* g_trace = nullptr;   // debug phase trace buffer (device)
 size_t g_trace_bytes = 0;
 
@@ -151,7 +152,17 @@ LaunchShape launch_shape(qg_format f, int M, int K, const qg_config* c, bool fus
   return ls;
 }
 
+size_t skinny_smem(qg_format f, const qg_config* c) {
+  switch (f) {
+    case QG_FP8_DYNAMIC: return qg::launch_gemm_fp8_skinny_smem(c->tile_n, c->rows, c->stages);
+    case QG_W8A8_INT8: return qg::launch_gemm_int8_skinny_smem(c->tile_n, c->rows, c->stages);
+    case QG_BLOCK_FP8: return qg::launch_gemm_block_skinny_smem(c->tile_n, c->rows, c->stages);
+    default: return (size_t)1 << 30;
+  }
+}
+
 size_t gemm_smem(qg_format f, int M, int K, const qg_config* c, bool fused) {
+  if (c->variant == 1) return skinny_smem(f, c);
   const LaunchShape ls = launch_shape(f, M, K, c, fused);
   const bool swap = c->swap_ab != 0;
   const int tn = c->tile_n, st = c->stages;
@@ -185,9 +196,26 @@ qg_status check_launch_fit(qg_format f, int M, int K, const qg_config* c, bool f
   return QG_OK;
 }
 
+// The decode ("skinny") kernel: warp-level MMAs, no split-K; K groups of
+// 64 / rows compute warps each take every (64 / rows)-th K tile, so the ring
+// depth is a multiple of that.
+qg_status check_skinny_config(qg_format f, const qg_config* c) {
+  if (f == QG_NVFP4) return QG_ERR_UNSUPPORTED;
+  if (c->split_k != 1 || c->swap_ab != 1 || c->reduce_mode != 0) return QG_ERR_UNSUPPORTED;
+  if (c->tile_n != 16 && c->tile_n != 32) return QG_ERR_UNSUPPORTED;
+  if (c->rows != 8 && c->rows != 16 && c->rows != 32 && c->rows != 64) return QG_ERR_UNSUPPORTED;
+  const int kg = 64 / c->rows;
+  if (c->stages < 2 || c->stages > 64 || c->stages % kg != 0) return QG_ERR_UNSUPPORTED;
+  if (skinny_smem(f, c) > kSmemLimit) return QG_ERR_UNSUPPORTED;
+  return QG_OK;
+}
+
 qg_status check_config(qg_format f, int M, int N, int K, const qg_config* c) {
   if (!c) return QG_ERR_INVALID_ARG;
-  if (c->reserved[0] || c->reserved[1] || c->reserved[2]) return QG_ERR_INVALID_ARG;
+  if (c->reserved) return QG_ERR_INVALID_ARG;
+  if (c->variant != 0 && c->variant != 1) return QG_ERR_INVALID_ARG;
+  if (c->variant == 1) return check_skinny_config(f, c);
+  if (c->rows != 0) return QG_ERR_INVALID_ARG;
   if (!is_pow2(c->split_k) || c->split_k > 256) return QG_ERR_UNSUPPORTED;
   if (c->swap_ab != 0 && c->swap_ab != 1) return QG_ERR_INVALID_ARG;
   if (c->reduce_mode < 0 || c->reduce_mode > 2) return QG_ERR_INVALID_ARG;
@@ -388,7 +416,7 @@ qg_status check_fused_args(qg_format f, const void* A, int lda, const qg_operand
   qg_status s;
   if ((s = check_operand_impl(f, W, N, K)) != QG_OK) return s;
   if ((s = check_config(f, M, N, K, cfg)) != QG_OK) return s;
-  if (cfg->swap_ab != 1) return QG_ERR_UNSUPPORTED;
+  if (cfg->swap_ab != 1 || cfg->variant != 0) return QG_ERR_UNSUPPORTED;
   // the whole activation slice of a CTA is held in shared memory
   if ((s = check_launch_fit(f, M, K, cfg, true)) != QG_OK) return s;
   // a per-token scale spans all of K: split-K slices must meet in a cluster
@@ -440,6 +468,34 @@ qg_status launch_run(qg_format f, const qg_operand* A, const void* act, int lda,
   prm.act_scale_out = act_scale_out;
   int tp, tq;
   tiles_of(cfg, M, N, &tp, &tq);
+  if (cfg->variant == 1) {
+    // decode kernel: CTA (x, y) = weight rows [x rows, (x + 1) rows) x
+    // tokens [y tile_n, (y + 1) tile_n), the whole of K
+    prm.nkt_max = prm.kt_total;
+    prm.err = d->err;
+    prm.wait_ns = g_wait_ns;
+    const int gx = (N + cfg->rows - 1) / cfg->rows, gy = (M + cfg->tile_n - 1) / cfg->tile_n;
+    if (gy > 65535) return QG_ERR_UNSUPPORTED;
+    if (g_trace != nullptr &&
+        (size_t)gx * gy * qg::kTraceEvents * sizeof(unsigned long long) <= g_trace_bytes)
+      prm.trace = g_trace;
+    if (g_l2_ahead) prm.l2_ahead = (gx * gy + 1) / 2;
+    CUtensorMap tw, ta;
+    const uint64_t rb = row_bytes(f, K);
+    if (!make_tmap(&tw, W->q, rb, (uint64_t)N, (uint32_t)cfg->rows)) return QG_ERR_CUDA;
+    if (!make_tmap(&ta, A->q, rb, (uint64_t)M, (uint32_t)cfg->tile_n)) return QG_ERR_CUDA;
+    const dim3 grid(gx, gy, 1);
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e;
+    switch (f) {
+      case QG_FP8_DYNAMIC: e = qg::launch_gemm_fp8_skinny(cfg->tile_n, cfg->rows, tw, ta, prm, grid, st, g_pdl); break;
+      case QG_W8A8_INT8: e = qg::launch_gemm_int8_skinny(cfg->tile_n, cfg->rows, tw, ta, prm, grid, st, g_pdl); break;
+      case QG_BLOCK_FP8: e = qg::launch_gemm_block_skinny(cfg->tile_n, cfg->rows, tw, ta, prm, grid, st, g_pdl); break;
+      default: return QG_ERR_UNSUPPORTED;
+    }
+    if (e != cudaSuccess) return e == cudaErrorInvalidValue ? QG_ERR_UNSUPPORTED : QG_ERR_CUDA;
+    return QG_OK;
+  }
   if (cfg->split_k > 1 && cfg->reduce_mode != qg::kReduceCluster) {
     prm.partial = workspace;
     prm.counters = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(workspace) +
@@ -481,6 +537,14 @@ qg_status launch_run(qg_format f, const qg_operand* A, const void* act, int lda,
   }
   if (tq > 65535) return QG_ERR_UNSUPPORTED;
   const dim3 grid(tp, tq, cfg->split_k);
+  // weight prefetch for the later half of a Swap-AB grid (launch order:
+  // clusters of split_k, else single CTAs); not for grouped launches, whose
+  // weight rows depend on the routing
+  if (swap && !expert_offsets && act == nullptr && g_l2_ahead) {
+    const bool clus = cfg->split_k > 1 && cfg->reduce_mode == qg::kReduceCluster;
+    const long long units = clus ? (long long)tp * tq : (long long)tp * tq * cfg->split_k;
+    prm.l2_ahead = (int)((units + 1) / 2);
+  }
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e;
   switch (f) {
@@ -528,7 +592,7 @@ qg_status qgemm_run_grouped(qg_format f, int experts, const int* expert_offsets,
   Wall.rows = N;
   qg_status s = qg::check_run_args(f, A, &Wall, M, N, K, cfg, workspace, ws_bytes, Y, ldy, out_kind);
   if (s != QG_OK) return s;
-  if (cfg->swap_ab != 1) return QG_ERR_UNSUPPORTED;
+  if (cfg->swap_ab != 1 || cfg->variant != 0) return QG_ERR_UNSUPPORTED;
   if (cfg->split_k > 1 && cfg->reduce_mode == qg::kReduceLastCta) return QG_ERR_UNSUPPORTED;
   return launch_run(f, A, nullptr, 0, nullptr, W, M, N, K, cfg, workspace, Y, ldy, out_kind, stream, experts,
                     expert_offsets);
@@ -569,7 +633,7 @@ qg_status qgemm_grouped_default_config(qg_format f, int experts, int T, int N, i
     int n = 0;
     if (qgemm_rank_configs(f, m_eff, (int)rows, K, ranked, 256, nullptr, &n) == QG_OK)
       for (int i = 0; i < n; ++i)
-        if (ranked[i].swap_ab == 1 && ranked[i].reduce_mode != 2 &&
+        if (ranked[i].variant == 0 && ranked[i].swap_ab == 1 && ranked[i].reduce_mode != 2 &&
             qg::config_check(f, T, N, K, &ranked[i]) == QG_OK) {
           *out = ranked[i];
           return QG_OK;

@@ -104,6 +104,12 @@ struct GemmParams {
   // weight rows [e * N, (e + 1) * N) of W_q.
   const int* expert_offsets;   // device, experts + 1 ints
   int experts;
+  // Weight prefetch into L2 on behalf of a later CTA: the CTA `l2_ahead`
+  // places after this one in launch order (same split slice in a cluster
+  // launch), 0 for none.  CTAs that start while the previous kernel still
+  // holds the SMs stream the weights of those that can only start after it,
+  // so the HBM stays busy across the kernel boundary.
+  int l2_ahead;
 };
 
 constexpr int kMaxExperts = 256;
@@ -519,6 +525,32 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
         load_w(i, i);
         if (i == 0) trace_at(prm, kTrFirstLoad);
       }
+      if constexpr (SWAP && !GROUPED) {
+        if (prm.l2_ahead > 0) {
+          // the weight slice of the CTA l2_ahead places later in launch
+          // order: clusters launch whole (cluster index x + y * gx, the
+          // split slices z inside), plain grids in x, y, z order
+          const int gx = gridDim.x, gy = gridDim.y, gz = gridDim.z;
+          int tx = -1, tz = 0;
+          if (cluster_red) {
+            const int tc = blockIdx.x + gx * blockIdx.y + prm.l2_ahead;
+            if (tc < gx * gy) { tx = tc % gx; tz = kz; }
+          } else {
+            const long long t = (long long)blockIdx.x + (long long)gx * (blockIdx.y + (long long)gy * kz) + prm.l2_ahead;
+            if (t < (long long)gx * gy * gz) { tx = (int)(t % gx); tz = (int)(t / ((long long)gx * gy)); }
+          }
+          if (tx >= 0) {
+            const int t_begin = (int)(((long long)tz * prm.kt_total) / prm.split_k);
+            const int t_end = (int)(((long long)(tz + 1) * prm.kt_total) / prm.split_k);
+            for (int kt = t_begin; kt < t_end; ++kt) {
+              tma_prefetch_l2_2d(map_w, kt * kKTileBytes, tx * 128);
+              if constexpr (C::kNvf4)
+                bulk_prefetch_l2(prm.sf_p + ((size_t)tx * prm.sf_atoms_per_rb + kt * 4) * kSfAtomBytes,
+                                 4 * kSfAtomBytes);
+            }
+          }
+        }
+      }
       if (!a_threads) {                        // activations come from the preceding kernel
         griddep_wait();
         trace_at(prm, kTrDepWait);
@@ -680,6 +712,14 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
       for (int r = etid; r < 128; r += ET)
         row_s[r] = (p0 + r < prm.rows_p) ? __ldg(prm.scale_w + wrow + p0 + r) : 0.f;
     griddep_wait();                            // scales/partials/activations of earlier kernels
+    // push-mode cluster split-K: wait for cluster phase 1 (every receiver's
+    // barriers initialised) now, while the MMAs run, not after the accumulator
+    if constexpr (C::kPush && !kFusable) {
+      if (cluster_red) {
+        cluster_wait();
+        epi_phase1 = true;
+      }
+    }
     if (a_threads && etid == 0) trace_at(prm, kTrDepWait);
     bool fz_ok = true;
     // FP8 / INT8: the remaining per-row scales of this tile (activation
@@ -1118,12 +1158,25 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
           const int n0 = SWAP ? p0 + r0 + j8 : q0 + j8;
           if (m >= Mlim || n0 >= prm.N) continue;
           uint32_t acc8[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-          for (int z = 0; z < Sk; ++z) {
-            const uint32_t a = recv_s + 4u * (uint32_t)(z * zstride + i * (SWAP ? rows_per : BN) + j8);
-            const uint4 w0 = lds_v4(a), w1 = lds_v4(a + 16u);
-            const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+          // every split's two 16-byte loads first, then the sums in split order
+          const uint32_t a0 = recv_s + 4u * (uint32_t)(i * (SWAP ? rows_per : BN) + j8);
+          uint4 wz[kMaxClusterSplit][2];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) acc8[k] = add_acc<FMT>(acc8[k], w[k]);
+          for (int z = 0; z < kMaxClusterSplit; ++z) {
+            if (z < Sk) {
+              const uint32_t a = a0 + 4u * (uint32_t)(z * zstride);
+              wz[z][0] = lds_v4(a);
+              wz[z][1] = lds_v4(a + 16u);
+            }
+          }
+#pragma unroll
+          for (int z = 0; z < kMaxClusterSplit; ++z) {
+            if (z < Sk) {
+              const uint32_t w[8] = {wz[z][0].x, wz[z][0].y, wz[z][0].z, wz[z][0].w,
+                                     wz[z][1].x, wz[z][1].y, wz[z][1].z, wz[z][1].w};
+#pragma unroll
+              for (int k = 0; k < 8; ++k) acc8[k] = add_acc<FMT>(acc8[k], w[k]);
+            }
           }
           store8(r, c, m, n0, acc8);
         }

@@ -5,6 +5,10 @@
 #include "attr_cache.h"
 #include "gemm_kernel.cuh"
 #include "internal.h"
+#include "skinny.cuh"
+
+#define QG_CAT2(a, b) a##b
+#define QG_CAT(a, b) QG_CAT2(a, b)
 
 namespace qg {
 namespace {
@@ -117,7 +121,77 @@ size_t smem_for(int bn, int stages, int nkt_max, int recv_cols, int act_tiles) {
   }
 }
 
+template <int FMT, int TM, int NF>
+cudaError_t launch_skinny_one(const CUtensorMap& tw, const CUtensorMap& ta, const GemmParams& prm, dim3 grid,
+                              cudaStream_t st, bool pdl) {
+  auto kern = qgemm_skinny_kernel<FMT, TM, NF>;
+  const size_t smem = skinny_smem_bytes<FMT, TM, NF>(prm.stages);
+  static GrowOnlyAttr smem_attr;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = static_cast<cudaError_t>(smem_attr.ensure(dev, (int)smem, [&](int bytes) {
+    return static_cast<int>(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  }));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(SkCfg<FMT, TM, NF>::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, tw, ta, prm);
+}
+
+template <int FMT, int TM>
+cudaError_t launch_skinny_rows(int rows, const CUtensorMap& tw, const CUtensorMap& ta, const GemmParams& prm,
+                               dim3 grid, cudaStream_t st, bool pdl) {
+  switch (rows) {
+    case 8: return launch_skinny_one<FMT, TM, 1>(tw, ta, prm, grid, st, pdl);
+    case 16: return launch_skinny_one<FMT, TM, 2>(tw, ta, prm, grid, st, pdl);
+    case 32: return launch_skinny_one<FMT, TM, 4>(tw, ta, prm, grid, st, pdl);
+    case 64: return launch_skinny_one<FMT, TM, 8>(tw, ta, prm, grid, st, pdl);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int FMT, int TM>
+size_t skinny_smem_rows(int rows, int stages) {
+  switch (rows) {
+    case 8: return skinny_smem_bytes<FMT, TM, 1>(stages);
+    case 16: return skinny_smem_bytes<FMT, TM, 2>(stages);
+    case 32: return skinny_smem_bytes<FMT, TM, 4>(stages);
+    case 64: return skinny_smem_bytes<FMT, TM, 8>(stages);
+    default: return (size_t)1 << 30;
+  }
+}
+
 }  // namespace
+
+cudaError_t QG_CAT(QG_LAUNCH_NAME, _skinny)(int tile_n, int rows, const CUtensorMap& tw, const CUtensorMap& ta,
+                                            const GemmParams& prm, dim3 grid, cudaStream_t st, bool pdl) {
+  if constexpr (QG_FMT == kNVF4) {
+    return cudaErrorInvalidValue;
+  } else {
+    if (tile_n == 16) return launch_skinny_rows<QG_FMT, 16>(rows, tw, ta, prm, grid, st, pdl);
+    if (tile_n == 32) return launch_skinny_rows<QG_FMT, 32>(rows, tw, ta, prm, grid, st, pdl);
+    return cudaErrorInvalidValue;
+  }
+}
+
+size_t QG_CAT(QG_LAUNCH_NAME, _skinny_smem)(int tile_n, int rows, int stages) {
+  if constexpr (QG_FMT == kNVF4) {
+    return (size_t)1 << 30;
+  } else {
+    if (tile_n == 16) return skinny_smem_rows<QG_FMT, 16>(rows, stages);
+    if (tile_n == 32) return skinny_smem_rows<QG_FMT, 32>(rows, stages);
+    return (size_t)1 << 30;
+  }
+}
 
 cudaError_t QG_LAUNCH_NAME(bool swap, int tile_n, const CUtensorMap& tp, const CUtensorMap& tq,
                            const GemmParams& prm, dim3 grid, cudaStream_t st, bool pdl) {
@@ -138,9 +212,6 @@ cudaError_t QG_LAUNCH_NAME(bool swap, int tile_n, const CUtensorMap& tp, const C
   return swap ? launch_bn<QG_FMT, true, false>(tile_n, tp, tq, prm, grid, st, pdl)
               : launch_bn<QG_FMT, false, false>(tile_n, tp, tq, prm, grid, st, pdl);
 }
-
-#define QG_CAT2(a, b) a##b
-#define QG_CAT(a, b) QG_CAT2(a, b)
 
 size_t QG_CAT(QG_LAUNCH_NAME, _smem)(int tile_n, bool swap, int stages, int nkt_max, int recv_cols,
                                      int act_tiles) {

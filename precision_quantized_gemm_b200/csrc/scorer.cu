@@ -51,6 +51,11 @@ struct Model {
   double e3 = 3.95830;       // second-pass launch, µs
   double e4 = 11.2845;       // last-CTA reduction, µs
   double e5 = 1180.85;       // workspace traffic bandwidth, GB/s
+  // decode ("skinny") kernel: K-tile cycles of one compute warp, and its
+  // chain after the data (activation wait, K-group sum, stores) relative to
+  // the tile kernel's, µs
+  double s_tile = 40.0;
+  double s_epi = -1.0;
 };
 const Model kModel;
 
@@ -75,7 +80,29 @@ int ctas_per_sm(qg_format f, int M, int K, const qg_config& c) {
   return std::max(1, std::min(std::min(regcap, tmemcap), smemcap));
 }
 
+// The decode kernel: ceil(N / rows) x ceil(M / tile_n) CTAs, each streaming
+// its rows (and tokens) over the whole of K through its ring, eight compute
+// warps in 64 / rows K groups.
+double estimate_skinny_us(qg_format f, int M, int N, int K, const qg_config& c, int sms) {
+  const Model& m = kModel;
+  const double rb = (double)K;
+  const int kt = (int)((rb + 127) / 128);
+  const double ctas = (double)((N + c.rows - 1) / c.rows) * ((M + c.tile_n - 1) / c.tile_n);
+  const size_t smem = qg::config_smem(f, M, K, &c);
+  const int cps = std::max(1, std::min(2, (int)(kSmemPerSm / (smem + 1024))));
+  const double waves = std::ceil(ctas / ((double)sms * cps));
+  const double stage_bytes = (double)(c.rows + c.tile_n) * 128.0;
+  const double inflight = std::min(c.stages, kt) * stage_bytes;
+  const double rate = std::min(inflight / m.lat_us, m.sm_gbs * 1e3 / cps);
+  const double t_stream = stage_bytes * kt / rate;
+  const int kg = 64 / c.rows;
+  const double t_mma = std::ceil((double)kt / kg) * m.s_tile * (c.tile_n / 16) / m.clock_mhz;
+  const double body = std::max((double)N * rb / (m.hbm_gbs * 1e3), waves * std::max(t_stream, t_mma));
+  return body + m.e0 * std::min(M, c.tile_n) / 16.0 + m.s_epi;
+}
+
 double estimate_us(qg_format f, int M, int N, int K, const qg_config& c, int sms) {
+  if (c.variant == 1) return estimate_skinny_us(f, M, N, K, c, sms);
   const Model& m = kModel;
   const double rb = f == QG_NVFP4 ? K / 2.0 : (double)K;
   const int kt = (int)((rb + 127) / 128);
@@ -143,6 +170,39 @@ void candidate_grid(qg_format f, int M, int N, int K, qg_config* out, int max_ou
             }
             ++n;
           }
+    }
+  }
+  // the decode kernel (8-bit formats, up to 32 tokens per CTA): rows per
+  // CTA, and rings of 8, 16, 32 or every K tile (up to 64) rounded to the K
+  // groups
+  if (f != QG_NVFP4 && M <= 64) {
+    const int rows_opts[] = {8, 16, 32, 64};
+    const int ring_opts[] = {8, 16, 32, 64};
+    for (int tm : {16, 32}) {
+      if (tm == 32 && M <= 16) continue;
+      for (int r : rows_opts) {
+        const int kg = 64 / r;
+        int prev = 0;
+        for (int ro : ring_opts) {
+          int st = std::min(ro, ((kt + kg - 1) / kg) * kg);
+          st = std::max(kg, (st / kg) * kg);
+          if (st < 2) st = 2 * kg > 64 ? kg : 2 * kg;
+          if (st == prev) continue;
+          prev = st;
+          if (n < max_out) {
+            qg_config c = {};
+            c.split_k = 1;
+            c.swap_ab = 1;
+            c.tile_n = tm;
+            c.stages = st;
+            c.reduce_mode = 0;
+            c.variant = 1;
+            c.rows = r;
+            out[n] = c;
+          }
+          ++n;
+        }
+      }
     }
   }
   *n_out = n;

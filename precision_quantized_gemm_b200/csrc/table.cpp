@@ -10,9 +10,10 @@
 // FlashInfer PR 3948 ("M bucketing by floor(log2 M)") share one tactic.
 //
 // File format (text, one entry per line):
-//   qgemm-table 1
+//   qgemm-table 2
 //   device <name with spaces replaced by _> sms <count>
-//   <fmt> <M> <N> <K> <split_k> <swap_ab> <tile_n> <stages> <reduce_mode 0..2> <us>
+//   <fmt> <M> <N> <K> <split_k> <swap_ab> <tile_n> <stages> <reduce_mode 0..2> <variant> <rows> <us>
+// Version 1 files (no variant and rows columns: the tile kernel) still load.
 #include <algorithm>
 #include <cstdio>
 #include <cstring>
@@ -42,12 +43,16 @@ struct Table {
 };
 
 constexpr const char* kMagic = "qgemm-table";
-constexpr int kVersion = 1;
+constexpr int kVersion = 2;
 
 bool valid_cfg_fields(const qg_config& c) {
+  if (c.reserved != 0 || (c.variant != 0 && c.variant != 1)) return false;
+  if (c.variant == 1)
+    return c.split_k == 1 && c.swap_ab == 1 && (c.tile_n == 16 || c.tile_n == 32) && c.stages >= 2 &&
+           c.stages <= 64 && c.reduce_mode == 0 && (c.rows == 8 || c.rows == 16 || c.rows == 32 || c.rows == 64);
   return c.split_k >= 1 && c.split_k <= 256 && (c.swap_ab == 0 || c.swap_ab == 1) &&
          c.tile_n >= 16 && c.tile_n <= 256 && c.stages >= 2 && c.stages <= 12 &&
-         c.reduce_mode >= 0 && c.reduce_mode <= 2;
+         c.reduce_mode >= 0 && c.reduce_mode <= 2 && c.rows == 0;
 }
 
 }  // namespace
@@ -92,8 +97,8 @@ qg_status qgemm_table_save(const void* table, const char* path) {
     std::tie(f, N, K, M) = kv.first;
     const qg_config& c = kv.second.cfg;
     char line[256];
-    std::snprintf(line, sizeof(line), "%d %d %d %d %d %d %d %d %d %.4f\n", f, M, N, K, c.split_k,
-                  c.swap_ab, c.tile_n, c.stages, c.reduce_mode, kv.second.us);
+    std::snprintf(line, sizeof(line), "%d %d %d %d %d %d %d %d %d %d %d %.4f\n", f, M, N, K, c.split_k,
+                  c.swap_ab, c.tile_n, c.stages, c.reduce_mode, c.variant, c.rows, kv.second.us);
     out << line;
   }
   return out.good() ? QG_OK : QG_ERR_TABLE_IO;
@@ -105,7 +110,7 @@ qg_status qgemm_table_load(const char* path, void** table) {
   if (!in) return QG_ERR_TABLE_IO;
   std::string magic;
   int version = 0;
-  if (!(in >> magic >> version) || magic != kMagic || version != kVersion) return QG_ERR_TABLE_IO;
+  if (!(in >> magic >> version) || magic != kMagic || version < 1 || version > kVersion) return QG_ERR_TABLE_IO;
   std::string tag, dev, tag2;
   int sms = 0;
   if (!(in >> tag >> dev >> tag2 >> sms) || tag != "device" || tag2 != "sms") return QG_ERR_TABLE_IO;
@@ -120,9 +125,11 @@ qg_status qgemm_table_load(const char* path, void** table) {
     int f, M, N, K;
     qg_config c = {};
     double us = 0;
-    if (!(ls >> f >> M >> N >> K >> c.split_k >> c.swap_ab >> c.tile_n >> c.stages >>
-          c.reduce_mode >> us) ||
-        f < 0 || f > 3 || M <= 0 || N <= 0 || K <= 0 || !valid_cfg_fields(c)) {
+    bool good = static_cast<bool>(ls >> f >> M >> N >> K >> c.split_k >> c.swap_ab >> c.tile_n >> c.stages >>
+                                  c.reduce_mode);
+    if (good && version >= 2) good = static_cast<bool>(ls >> c.variant >> c.rows);
+    if (good) good = static_cast<bool>(ls >> us);
+    if (!good || f < 0 || f > 3 || M <= 0 || N <= 0 || K <= 0 || !valid_cfg_fields(c)) {
       delete t;
       return QG_ERR_TABLE_IO;
     }

@@ -151,9 +151,21 @@ int kt_of(qg_format f, int K) { return (int)(((f == QG_NVFP4 ? K / 2 : K) + 127)
 std::vector<qg_config> candidates(qg_format f, int M, int N, int K, int top_n) {
   int n = 0;
   if (top_n > 0) {
-    std::vector<qg_config> out((size_t)top_n);
-    if (qgemm_rank_configs(f, M, N, K, out.data(), top_n, nullptr, &n) != QG_OK) n = 0;
-    out.resize((size_t)n);
+    // the scorer's top_n, plus the best four of each kernel variant that the
+    // top_n leaves out, so that both kernels are always timed
+    int total = 0;
+    qg::candidate_grid(f, M, N, K, nullptr, 0, &total);
+    std::vector<qg_config> ranked((size_t)std::max(total, 1));
+    if (qgemm_rank_configs(f, M, N, K, ranked.data(), total, nullptr, &n) != QG_OK) n = 0;
+    std::vector<qg_config> out;
+    int per_variant[2] = {0, 0};
+    for (int i = 0; i < n; ++i) {
+      const int v = ranked[i].variant;
+      if (i < top_n || per_variant[v] < 4) {
+        out.push_back(ranked[i]);
+        ++per_variant[v];
+      }
+    }
     return out;
   }
   qg::candidate_grid(f, M, N, K, nullptr, 0, &n);

@@ -78,6 +78,9 @@ def test_default_config_follows_the_swap_rule_and_fills_sms():
     for fmt, M in ((qg.QG_W8A8_INT8, 8), (qg.QG_FP8_DYNAMIC, 1), (qg.QG_BLOCK_FP8, 16)):
         c = qg.qgemm_default_config(fmt, M, 4096, 4096)
         assert c.swap_ab == 1 and c.tile_n <= 32
+        if c.variant == 1:                             # the decode kernel: rows per CTA fill the SMs
+            assert c.split_k == 1 and 74 <= 4096 // c.rows * ((M + c.tile_n - 1) // c.tile_n) <= 4 * 148
+            continue
         assert c.split_k >= 2 and (c.split_k & (c.split_k - 1)) == 0
         assert 74 <= 32 * c.split_k * ((M + c.tile_n - 1) // c.tile_n) <= 2 * 148
         assert c.reduce_mode == 0                      # cluster reduction: no workspace
@@ -135,8 +138,36 @@ def test_run_rejects_bad_arguments_before_any_launch(kw, status):
 
 def test_run_reserved_fields_must_be_zero():
     c = qg.make_config()
-    c.reserved[1] = 7
+    c.reserved = 7
     assert _run(cfg=c) == qg.QG_ERR_INVALID_ARG
+    c = qg.make_config()
+    c.rows = 32                                     # rows belongs to the decode kernel only
+    assert _run(cfg=c) == qg.QG_ERR_INVALID_ARG
+    c = qg.make_config(variant=2)
+    assert _run(cfg=c) == qg.QG_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(tile_n=16, rows=32, stages=32), qg.QG_ERR_NO_DEVICE),     # valid: reaches the device check
+    (dict(tile_n=32, rows=8, stages=16), qg.QG_ERR_NO_DEVICE),
+    (dict(tile_n=64, rows=32, stages=32), qg.QG_ERR_UNSUPPORTED),   # tokens per CTA: 16 or 32
+    (dict(tile_n=16, rows=24, stages=32), qg.QG_ERR_UNSUPPORTED),   # rows: 8, 16, 32, 64
+    (dict(tile_n=16, rows=8, stages=12), qg.QG_ERR_UNSUPPORTED),    # ring depth a multiple of 64/rows
+    (dict(tile_n=16, rows=64, stages=65), qg.QG_ERR_UNSUPPORTED),
+    (dict(tile_n=32, rows=64, stages=20), qg.QG_ERR_UNSUPPORTED),   # 20 x 12 KB: beyond shared memory
+])
+def test_skinny_config_checks(kw, status):
+    c = qg.skinny_config(**kw)
+    assert _run(cfg=c) == status
+    for bad in (dict(split_k=2), dict(swap_ab=0), dict(reduce_mode=1)):
+        c2 = qg.skinny_config(**kw)
+        for k, v in bad.items():
+            setattr(c2, k, v)
+        assert _run(cfg=c2) == qg.QG_ERR_UNSUPPORTED
+
+
+def test_skinny_refuses_nvfp4_and_the_fused_and_grouped_launches():
+    assert _run(fmt=qg.QG_NVFP4, K=1024, cfg=qg.skinny_config()) == qg.QG_ERR_UNSUPPORTED
 
 
 def test_quantize_rejects_bad_arguments():
@@ -184,10 +215,28 @@ def test_table_roundtrip_and_dispatch(tmp_path):
     assert hit == 0
 
 
+def test_table_version1_files_load_as_the_tile_kernel_and_decode_entries_roundtrip(tmp_path):
+    p = tmp_path / "v1.qgt"
+    p.write_text("qgemm-table 1\ndevice x sms 148\n1 8 4096 4096 4 1 16 8 0 3.5\n")
+    c, hit = qg.Table(str(p)).dispatch(qg.QG_W8A8_INT8, 8, 4096, 4096)
+    assert hit == 1 and c.as_dict() == qg.make_config(4, 1, 16, 8, 0).as_dict()
+    t = qg.Table()
+    sk = qg.skinny_config(tile_n=16, rows=32, stages=32)
+    t.put(qg.QG_FP8_DYNAMIC, 1, 4096, 4096, sk, 2.5)
+    q = str(tmp_path / "v2.qgt")
+    t.save(q)
+    assert open(q).readline().split() == ["qgemm-table", "2"]
+    c, hit = qg.Table(q).dispatch(qg.QG_FP8_DYNAMIC, 1, 4096, 4096)
+    assert hit == 1 and c.as_dict() == sk.as_dict()
+
+
 @pytest.mark.parametrize("content", [
     "",
-    "qgemm-table 2\ndevice x sms 148\n",
+    "qgemm-table 3\ndevice x sms 148\n",                                    # unknown version
     "qgemm-table 1\ndevice x sms 148\n1 8 4096 4096 4 1 16 8 0\n",          # missing field
+    "qgemm-table 2\ndevice x sms 148\n1 8 4096 4096 4 1 16 8 0 1.0\n",      # version 2: variant, rows missing
+    "qgemm-table 2\ndevice x sms 148\n1 8 4096 4096 1 1 16 24 0 1 12 1.0\n",  # decode kernel: bad rows
+    "qgemm-table 2\ndevice x sms 148\n1 8 4096 4096 4 1 16 8 0 0 32 1.0\n",   # rows on the tile kernel
     "qgemm-table 1\ndevice x sms 148\n1 8 4096 4096 4 3 16 8 0 1.0\n",      # bad swap
     "qgemm-table 1\ndevice x sms 148\n1 8 4096 4096 4 1 16 8 3 1.0\n",      # bad reduce mode
     "not a table\n",
