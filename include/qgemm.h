@@ -95,12 +95,13 @@ typedef struct {
                           1: the decode ("skinny") kernel for FP8_DYNAMIC,
                           W8A8_INT8 and BLOCK_FP8: warp-level MMAs with register
                           accumulators, each CTA owning `rows` weight rows over
-                          the whole of K and tile_n (16 or 32) tokens; requires
-                          split_k = 1, swap_ab = 1, reduce_mode = 0, and
-                          `stages` (the ring of 128-byte K tiles, 2..64) a
-                          multiple of 64 / rows                                  */
-  int32_t rows;        /* variant 1: weight rows per CTA, 8, 16, 32 or 64;
-                          variant 0: must be 0                                    */
+                          the whole of K and tile_n (8, 16 or 32) tokens;
+                          requires split_k = 1, swap_ab = 1, reduce_mode = 0,
+                          and `stages` (the ring of 128-byte K tiles, 2..64) a
+                          multiple of the K groups of its eight compute warps:
+                          64 / rows (128 / rows for tile_n = 8)                */
+  int32_t rows;        /* variant 1: weight rows per CTA, 8, 16, 32 or 64 (at
+                          least 16 for tile_n = 8); variant 0: must be 0        */
   int32_t reserved;    /* must be zero                                            */
 } qg_config;
 
@@ -383,9 +384,16 @@ qg_status qgemm_tune_ranked(void* table, qg_format f, const int* Ms, int nM, con
                             int top_n, double budget_s_per_shape, int verbose);
 /* Tuning instrumentation: while `path` is set (NULL clears it), qgemm_tune
  * appends one text line per timed candidate to that file:
- *   <fmt> <M> <N> <K> <split_k> <swap_ab> <tile_n> <stages> <reduce_mode> <us>
+ *   <fmt> <M> <N> <K> <split_k> <swap_ab> <tile_n> <stages> <reduce_mode> <variant> <rows> <us>
  * (the selection-pass step time).  Host only; not thread-safe. */
 void qgemm_set_tune_log(const char* path);
+
+/* What the tuner times per candidate: gemm_only = 0 (the default) replays
+ * steps of a linear layer, the dynamic activation quantisation followed by
+ * the GEMM (their overlap through programmatic dependent launch depends on
+ * the configuration); gemm_only = 1 replays back-to-back GEMMs alone, the
+ * per-shape time of the GEMM itself.  Host only; not thread-safe. */
+void qgemm_set_tune_objective(int gemm_only);
 
 /* -------------------------------------------------------------- errors -- */
 

@@ -44,6 +44,7 @@ EXPORTS = [
     "qgemm_run_noalloc", "qgemm_set_trace", "qgemm_run_fused_act", "qgemm_set_tune_log",
     "qgemm_score_config", "qgemm_rank_configs", "qgemm_tune_ranked", "qgemm_table_validate",
     "qgemm_run_grouped", "qgemm_grouped_default_config", "qgemm_set_wait_limit", "qgemm_selftest_wait_expiry",
+    "qgemm_set_tune_objective",
 ]
 
 
@@ -123,6 +124,7 @@ def lib() -> ctypes.CDLL:
             "qgemm_selftest_wait_expiry": (c_int, [ctypes.c_ulonglong, c_void_p]),
             "qgemm_set_trace": (None, [c_void_p, c_size_t]),
             "qgemm_set_tune_log": (None, [c_char_p]),
+            "qgemm_set_tune_objective": (None, [c_int]),
             "qgemm_score_config": (c_int, [c_int, c_int, c_int, c_int, POINTER(qg_config), POINTER(c_double)]),
             "qgemm_rank_configs": (c_int, [c_int, c_int, c_int, c_int, POINTER(qg_config), c_int,
                                            POINTER(c_double), POINTER(c_int)]),
@@ -270,6 +272,11 @@ def qgemm_set_trace(buf_ptr, nbytes):
 def qgemm_set_tune_log(path):
     """Tuning instrumentation: log every timed candidate of qgemm_tune to `path` (None: off)."""
     lib().qgemm_set_tune_log(path.encode() if path else None)
+
+
+def qgemm_set_tune_objective(gemm_only: bool):
+    """Tuner timing: quantise + GEMM steps (False, the default) or GEMMs alone (True)."""
+    lib().qgemm_set_tune_objective(1 if gemm_only else 0)
 
 
 def qgemm_set_pdl(enable: bool):

@@ -196,15 +196,17 @@ qg_status check_launch_fit(qg_format f, int M, int K, const qg_config* c, bool f
   return QG_OK;
 }
 
-// The decode ("skinny") kernel: warp-level MMAs, no split-K; K groups of
-// 64 / rows compute warps each take every (64 / rows)-th K tile, so the ring
-// depth is a multiple of that.
+// The decode ("skinny") kernel: warp-level MMAs, no split-K; the eight
+// compute warps form 64 / rows K groups (128 / rows for tile_n = 8) that take
+// every K-group-th K tile, so the ring depth is a multiple of that.
 qg_status check_skinny_config(qg_format f, const qg_config* c) {
   if (f == QG_NVFP4) return QG_ERR_UNSUPPORTED;
   if (c->split_k != 1 || c->swap_ab != 1 || c->reduce_mode != 0) return QG_ERR_UNSUPPORTED;
-  if (c->tile_n != 16 && c->tile_n != 32) return QG_ERR_UNSUPPORTED;
+  if (c->tile_n != 8 && c->tile_n != 16 && c->tile_n != 32) return QG_ERR_UNSUPPORTED;
   if (c->rows != 8 && c->rows != 16 && c->rows != 32 && c->rows != 64) return QG_ERR_UNSUPPORTED;
-  const int kg = 64 / c->rows;
+  // tile_n = 8: a warp owns 16 weight rows (weights as the 16-row operand)
+  if (c->tile_n == 8 && c->rows < 16) return QG_ERR_UNSUPPORTED;
+  const int kg = (c->tile_n == 8 ? 128 : 64) / c->rows;
   if (c->stages < 2 || c->stages > 64 || c->stages % kg != 0) return QG_ERR_UNSUPPORTED;
   if (skinny_smem(f, c) > kSmemLimit) return QG_ERR_UNSUPPORTED;
   return QG_OK;

@@ -178,6 +178,29 @@ struct Cfg {
   static constexpr bool kPush = BN <= 64;
 };
 
+// Two MMA-issuing threads (Swap-AB FP8_Dynamic / W8A8_INT8 whose ring holds
+// every K tile of the slice): the MMA warp issues the even K tiles into one
+// accumulator and the producer thread, idle once its loads are out, the odd
+// ones into a second; the epilogue adds the two.  At decode sizes one
+// thread's issue of four small MMAs and a commit per K tile is on the
+// critical path, and two threads issue in parallel.  The plain, fused and
+// grouped launches split the same way, so that for one configuration they
+// sum in the same order.
+template <int FMT, bool SWAP, int BN, bool FUSED, bool GROUPED>
+__host__ __device__ constexpr bool dual_issue_able() {
+  return SWAP && (FMT == kFP8 || FMT == kINT8);
+}
+template <int FMT, bool SWAP, int BN, bool FUSED, bool GROUPED>
+__host__ __device__ constexpr int tmem_cols() {
+  using C = Cfg<FMT, BN>;
+  if constexpr (dual_issue_able<FMT, SWAP, BN, FUSED, GROUPED>()) {
+    return 2 * C::kAccCols <= 32 ? 32 : 2 * C::kAccCols <= 64 ? 64 : 2 * C::kAccCols <= 128 ? 128
+           : 2 * C::kAccCols <= 256 ? 256 : 512;
+  } else {
+    return C::kTmemCols;
+  }
+}
+
 // Block_FP8 scales staged per CTA: activation rows x K tiles, then weight
 // blocks x K tiles.
 template <bool SWAP, int BN>
@@ -375,6 +398,8 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
   // kernel carries none of its code.
   constexpr bool kFusable = FUSED && SWAP && FMT != kNVF4;
   constexpr bool fused = kFusable;
+  constexpr bool kDualAble = dual_issue_able<FMT, SWAP, BN, FUSED, GROUPED>();
+  constexpr int kTmemAlloc = tmem_cols<FMT, SWAP, BN, FUSED, GROUPED>();
   constexpr bool a_threads = fused;                    // Q tiles written by the epilogue warps
   const SmemLayout L =
       smem_layout<FMT, SWAP, BN>(prm.stages, prm.nkt_max, prm.recv_cols, a_threads ? prm.nkt_max : 0);
@@ -423,6 +448,8 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
   const bool cluster_red = prm.split_k > 1 && prm.reduce_mode == kReduceCluster;
   bool epi_phase1 = false;                                 // epilogue warps waited cluster phase 1
   const int rows_per = 128 / prm.split_k;                  // cluster mode: rows owned per CTA
+  // two MMA issuers: the ring holds every K tile of the slice (no refills)
+  const bool dual = kDualAble && prm.stages >= nkt && nkt >= 2;
   const uint32_t slot_bytes = 4u * (uint32_t)(rows_per * prm.recv_cols);
 
   if (threadIdx.x == 0) {
@@ -432,7 +459,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    mbar_init(acc_full, 1);
+    mbar_init(acc_full, dual ? 2 : 1);
     for (int i = 0; i < 4; ++i) {
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], C::kEpiWarps);
@@ -449,7 +476,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_alloc(tmem_slot, kTmemAlloc);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -568,6 +595,31 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
         issued = i + 1;
         if (++st == S) { st = 0; ph ^= 1u; }
       }
+      if constexpr (kDualAble) {
+        if (dual) {
+          // second MMA issuer: the odd K tiles into the second accumulator
+          // (every tile has its own stage, filled once: phase 0)
+          const uint64_t dp0 = sdesc_sw128(smem_u32(smem + L.p));
+          const uint64_t dq0 = sdesc_sw128(smem_u32(smem + L.q));
+          const uint32_t d_t = tmem_base + (uint32_t)BN;
+          // fused: the activation tiles are written by the epilogue warps
+          bool issued_all = !a_threads || mbar_wait(act_ready, 0, prm.err, prm.wait_ns);
+          for (int i = 1; i < nkt && issued_all; i += 2) {
+            if (!mbar_wait(&full[i], 0, prm.err, prm.wait_ns)) { issued_all = false; break; }
+            tc_fence_after();
+            const uint64_t dp = dp0 + (uint64_t)((i * kPTileBytes) >> 4);
+            const uint64_t dq = dq0 + (uint64_t)((i * C::kQTileBytes) >> 4);   // stage i, or act tile i
+#pragma unroll
+            for (int s = 0; s < 4; ++s) {
+              const uint32_t accum = (i > 1 || s > 0);
+              if constexpr (FMT == kINT8) mma_i8(d_t, dp + (uint64_t)(2 * s), dq + (uint64_t)(2 * s), C::kIdesc, accum);
+              else mma_f8f6f4(d_t, dp + (uint64_t)(2 * s), dq + (uint64_t)(2 * s), C::kIdesc, accum);
+            }
+          }
+          if (!issued_all) *flag_abort = 1;
+          mma_commit(acc_full);
+        }
+      }
       if (!ok) {
         *flag_abort = 1;
         // Drain: wait (bounded) until every issued copy has landed.
@@ -595,7 +647,9 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
       uint32_t ph = 0;
       int gb = 0, gr = 0;                      // Block_FP8: group buffer of K tile i, and its round
       bool abort = false;
-      for (int i = 0; i < nkt; ++i) {
+      const int istep = dual ? 2 : 1;          // two issuers: this thread takes the even K tiles
+      for (int i = 0; i < nkt; i += istep) {
+        if (dual) st = i;                      // one stage per K tile, phase 0
         if (!mbar_wait(&full[st], ph, prm.err, prm.wait_ns)) { abort = true; break; }
         if (i == 0) {
           if (a_threads && !mbar_wait(act_ready, 0, prm.err, prm.wait_ns)) { abort = true; break; }
@@ -1006,9 +1060,27 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
         for (int j = 0; j < CW; j += 2) unpack_u32x2(acc2[(c0 + j) / 2], v[j], v[j + 1]);
       } else if constexpr (CW == 32) {
         tmem_ld32(lane_addr + cbeg + c0, v);
+        if constexpr (kDualAble) {
+          if (dual) {                          // the second issuer's accumulator
+            uint32_t v2[CW];
+            tmem_ld32(lane_addr + BN + cbeg + c0, v2);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < CW; ++j) v[j] = add_acc<FMT>(v[j], v2[j]);
+          }
+        }
         tmem_ld_wait();
       } else {
         tmem_ld16(lane_addr + cbeg + c0, v);
+        if constexpr (kDualAble) {
+          if (dual) {
+            uint32_t v2[CW];
+            tmem_ld16(lane_addr + BN + cbeg + c0, v2);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < CW; ++j) v[j] = add_acc<FMT>(v[j], v2[j]);
+          }
+        }
         tmem_ld_wait();
       }
     };
@@ -1158,24 +1230,28 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
           const int n0 = SWAP ? p0 + r0 + j8 : q0 + j8;
           if (m >= Mlim || n0 >= prm.N) continue;
           uint32_t acc8[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-          // every split's two 16-byte loads first, then the sums in split order
+          // four splits' two 16-byte loads at a time, then their sums in split order
           const uint32_t a0 = recv_s + 4u * (uint32_t)(i * (SWAP ? rows_per : BN) + j8);
-          uint4 wz[kMaxClusterSplit][2];
 #pragma unroll
-          for (int z = 0; z < kMaxClusterSplit; ++z) {
-            if (z < Sk) {
-              const uint32_t a = a0 + 4u * (uint32_t)(z * zstride);
-              wz[z][0] = lds_v4(a);
-              wz[z][1] = lds_v4(a + 16u);
+          for (int z0 = 0; z0 < kMaxClusterSplit; z0 += 4) {
+            if (z0 >= Sk) break;
+            uint4 wz[4][2];
+#pragma unroll
+            for (int dz = 0; dz < 4; ++dz) {
+              if (z0 + dz < Sk) {
+                const uint32_t a = a0 + 4u * (uint32_t)((z0 + dz) * zstride);
+                wz[dz][0] = lds_v4(a);
+                wz[dz][1] = lds_v4(a + 16u);
+              }
             }
-          }
 #pragma unroll
-          for (int z = 0; z < kMaxClusterSplit; ++z) {
-            if (z < Sk) {
-              const uint32_t w[8] = {wz[z][0].x, wz[z][0].y, wz[z][0].z, wz[z][0].w,
-                                     wz[z][1].x, wz[z][1].y, wz[z][1].z, wz[z][1].w};
+            for (int dz = 0; dz < 4; ++dz) {
+              if (z0 + dz < Sk) {
+                const uint32_t w[8] = {wz[dz][0].x, wz[dz][0].y, wz[dz][0].z, wz[dz][0].w,
+                                       wz[dz][1].x, wz[dz][1].y, wz[dz][1].z, wz[dz][1].w};
 #pragma unroll
-              for (int k = 0; k < 8; ++k) acc8[k] = add_acc<FMT>(acc8[k], w[k]);
+                for (int k = 0; k < 8; ++k) acc8[k] = add_acc<FMT>(acc8[k], w[k]);
+              }
             }
           }
           store8(r, c, m, n0, acc8);
@@ -1291,40 +1367,23 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
         const uint32_t red_s = smem_u32(smem + L.p);
         const float alpha = alpha_of<FMT>(prm);
         // units of 8 consecutive output channels: 2 x 16-byte remote loads per
-        // split, summed in split order, scaled and stored as one 16-byte vector
+        // split, summed in split order, scaled and stored as one 16-byte vector.
+        // Up to four splits: a thread's next unit's loads are in flight with
+        // this unit's (two units per round), so one remote round trip serves two.
         const int units = rows_per * BN / 8;
         const bool vec = (prm.ldy % 8) == 0;
-#pragma unroll 1
-        for (int u = etid; u < units; u += C::kEpiThreads) {
-          int r, c;
+        auto unit_pos = [&](int u, int& r, int& c) {
           if (SWAP) { c = u / (rows_per / 8); r = r0 + (u % (rows_per / 8)) * 8; }
           else      { r = r0 + u / (BN / 8); c = (u % (BN / 8)) * 8; }
-          const uint32_t off = 4u * (uint32_t)red_index<SWAP, BN>(r, c);
-          uint4 t[kMaxClusterSplit][2];
-#pragma unroll
-          for (int z = 0; z < kMaxClusterSplit; ++z) {
-            if (z < Sk) {
-              t[z][0] = ld_dsmem_v4(mapa_shared(red_s + off, (uint32_t)z));
-              t[z][1] = ld_dsmem_v4(mapa_shared(red_s + off + 16u, (uint32_t)z));
-            }
-          }
-          uint32_t acc8[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-#pragma unroll
-          for (int z = 0; z < kMaxClusterSplit; ++z) {
-            if (z < Sk) {
-              const uint32_t w[8] = {t[z][0].x, t[z][0].y, t[z][0].z, t[z][0].w,
-                                     t[z][1].x, t[z][1].y, t[z][1].z, t[z][1].w};
-#pragma unroll
-              for (int j = 0; j < 8; ++j) acc8[j] = add_acc<FMT>(acc8[j], w[j]);
-            }
-          }
+        };
+        auto finish_unit = [&](int r, int c, const uint32_t (&acc8)[8]) {
           const int m = SWAP ? q0 + c : p0 + r;
           const int n0 = SWAP ? p0 + r : q0 + c;
-          if (m >= Mlim || n0 >= prm.N) continue;
+          if (m >= Mlim || n0 >= prm.N) return;
           if (prm.out_kind == 1) {
             uint32_t* Yu = reinterpret_cast<uint32_t*>(prm.Y) + (size_t)m * prm.ldy;
             for (int j = 0; j < 8 && n0 + j < prm.N; ++j) Yu[n0 + j] = acc8[j];
-            continue;
+            return;
           }
           float y8[8];
 #pragma unroll
@@ -1338,15 +1397,78 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
           }
           __nv_bfloat16* Yb = reinterpret_cast<__nv_bfloat16*>(prm.Y) + (size_t)m * prm.ldy;
           if (vec && n0 + 8 <= prm.N) {
-            uint32_t p[4];
+            uint32_t pk[4];
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
               const __nv_bfloat162 b2 = __floats2bfloat162_rn(y8[2 * h], y8[2 * h + 1]);
-              p[h] = *reinterpret_cast<const uint32_t*>(&b2);
+              pk[h] = *reinterpret_cast<const uint32_t*>(&b2);
             }
-            *reinterpret_cast<uint4*>(Yb + n0) = make_uint4(p[0], p[1], p[2], p[3]);
+            *reinterpret_cast<uint4*>(Yb + n0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           } else {
             for (int j = 0; j < 8 && n0 + j < prm.N; ++j) Yb[n0 + j] = __float2bfloat16_rn(y8[j]);
+          }
+        };
+        if (Sk <= 4) {
+          constexpr int kZ = 4;
+#pragma unroll 1
+          for (int u = etid; u < units; u += 2 * C::kEpiThreads) {
+            const int u2 = u + C::kEpiThreads;
+            int r[2], c[2];
+            unit_pos(u, r[0], c[0]);
+            unit_pos(u2 < units ? u2 : u, r[1], c[1]);
+            uint4 t[2][kZ][2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint32_t off = 4u * (uint32_t)red_index<SWAP, BN>(r[h], c[h]);
+#pragma unroll
+              for (int z = 0; z < kZ; ++z) {
+                if (z < Sk) {
+                  t[h][z][0] = ld_dsmem_v4(mapa_shared(red_s + off, (uint32_t)z));
+                  t[h][z][1] = ld_dsmem_v4(mapa_shared(red_s + off + 16u, (uint32_t)z));
+                }
+              }
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              if (h == 1 && u2 >= units) break;
+              uint32_t acc8[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+              for (int z = 0; z < kZ; ++z) {
+                if (z < Sk) {
+                  const uint32_t w[8] = {t[h][z][0].x, t[h][z][0].y, t[h][z][0].z, t[h][z][0].w,
+                                         t[h][z][1].x, t[h][z][1].y, t[h][z][1].z, t[h][z][1].w};
+#pragma unroll
+                  for (int j = 0; j < 8; ++j) acc8[j] = add_acc<FMT>(acc8[j], w[j]);
+                }
+              }
+              finish_unit(r[h], c[h], acc8);
+            }
+          }
+        } else {
+#pragma unroll 1
+          for (int u = etid; u < units; u += C::kEpiThreads) {
+            int r, c;
+            unit_pos(u, r, c);
+            const uint32_t off = 4u * (uint32_t)red_index<SWAP, BN>(r, c);
+            uint4 t[kMaxClusterSplit][2];
+#pragma unroll
+            for (int z = 0; z < kMaxClusterSplit; ++z) {
+              if (z < Sk) {
+                t[z][0] = ld_dsmem_v4(mapa_shared(red_s + off, (uint32_t)z));
+                t[z][1] = ld_dsmem_v4(mapa_shared(red_s + off + 16u, (uint32_t)z));
+              }
+            }
+            uint32_t acc8[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+            for (int z = 0; z < kMaxClusterSplit; ++z) {
+              if (z < Sk) {
+                const uint32_t w[8] = {t[z][0].x, t[z][0].y, t[z][0].z, t[z][0].w,
+                                       t[z][1].x, t[z][1].y, t[z][1].z, t[z][1].w};
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc8[j] = add_acc<FMT>(acc8[j], w[j]);
+              }
+            }
+            finish_unit(r, c, acc8);
           }
         }
       }
@@ -1361,7 +1483,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
   if (threadIdx.x == 0) trace_at(prm, kTrDone);
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::kTmemCols);
+    tmem_dealloc(tmem_base, kTmemAlloc);
   }
 }
 

@@ -24,7 +24,7 @@ cudaError_t launch_one(const CUtensorMap& tp, const CUtensorMap& tq, const GemmP
   // (clustered) grid could wait for good.  At most 512 / kTmemCols CTAs may
   // share an SM, so the shared memory of one is raised to at least
   // 228 KB / (that count + 1).
-  constexpr int kTmemCtas = 512 / Cfg<FMT, BN>::kTmemCols;
+  constexpr int kTmemCtas = 512 / tmem_cols<FMT, SWAP, BN, FUSED, GROUPED>();
   const size_t smem_floor = (size_t)233472 / (kTmemCtas + 1);
   if (smem < smem_floor) smem = smem_floor;
   // the kernel's shared-memory limit is raised per device (the attribute
@@ -151,7 +151,9 @@ template <int FMT, int TM>
 cudaError_t launch_skinny_rows(int rows, const CUtensorMap& tw, const CUtensorMap& ta, const GemmParams& prm,
                                dim3 grid, cudaStream_t st, bool pdl) {
   switch (rows) {
-    case 8: return launch_skinny_one<FMT, TM, 1>(tw, ta, prm, grid, st, pdl);
+    case 8:
+      if constexpr (TM == 8) return cudaErrorInvalidValue;
+      else return launch_skinny_one<FMT, TM, 1>(tw, ta, prm, grid, st, pdl);
     case 16: return launch_skinny_one<FMT, TM, 2>(tw, ta, prm, grid, st, pdl);
     case 32: return launch_skinny_one<FMT, TM, 4>(tw, ta, prm, grid, st, pdl);
     case 64: return launch_skinny_one<FMT, TM, 8>(tw, ta, prm, grid, st, pdl);
@@ -162,7 +164,9 @@ cudaError_t launch_skinny_rows(int rows, const CUtensorMap& tw, const CUtensorMa
 template <int FMT, int TM>
 size_t skinny_smem_rows(int rows, int stages) {
   switch (rows) {
-    case 8: return skinny_smem_bytes<FMT, TM, 1>(stages);
+    case 8:
+      if constexpr (TM == 8) return (size_t)1 << 30;
+      else return skinny_smem_bytes<FMT, TM, 1>(stages);
     case 16: return skinny_smem_bytes<FMT, TM, 2>(stages);
     case 32: return skinny_smem_bytes<FMT, TM, 4>(stages);
     case 64: return skinny_smem_bytes<FMT, TM, 8>(stages);
@@ -177,6 +181,7 @@ cudaError_t QG_CAT(QG_LAUNCH_NAME, _skinny)(int tile_n, int rows, const CUtensor
   if constexpr (QG_FMT == kNVF4) {
     return cudaErrorInvalidValue;
   } else {
+    if (tile_n == 8) return launch_skinny_rows<QG_FMT, 8>(rows, tw, ta, prm, grid, st, pdl);
     if (tile_n == 16) return launch_skinny_rows<QG_FMT, 16>(rows, tw, ta, prm, grid, st, pdl);
     if (tile_n == 32) return launch_skinny_rows<QG_FMT, 32>(rows, tw, ta, prm, grid, st, pdl);
     return cudaErrorInvalidValue;
@@ -187,6 +192,7 @@ size_t QG_CAT(QG_LAUNCH_NAME, _skinny_smem)(int tile_n, int rows, int stages) {
   if constexpr (QG_FMT == kNVF4) {
     return (size_t)1 << 30;
   } else {
+    if (tile_n == 8) return skinny_smem_rows<QG_FMT, 8>(rows, stages);
     if (tile_n == 16) return skinny_smem_rows<QG_FMT, 16>(rows, stages);
     if (tile_n == 32) return skinny_smem_rows<QG_FMT, 32>(rows, stages);
     return (size_t)1 << 30;

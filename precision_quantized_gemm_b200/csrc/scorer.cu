@@ -95,8 +95,8 @@ double estimate_skinny_us(qg_format f, int M, int N, int K, const qg_config& c, 
   const double inflight = std::min(c.stages, kt) * stage_bytes;
   const double rate = std::min(inflight / m.lat_us, m.sm_gbs * 1e3 / cps);
   const double t_stream = stage_bytes * kt / rate;
-  const int kg = 64 / c.rows;
-  const double t_mma = std::ceil((double)kt / kg) * m.s_tile * (c.tile_n / 16) / m.clock_mhz;
+  const int kg = (c.tile_n == 8 ? 128 : 64) / c.rows;
+  const double t_mma = std::ceil((double)kt / kg) * m.s_tile * std::max(1, c.tile_n / 16) / m.clock_mhz;
   const double body = std::max((double)N * rb / (m.hbm_gbs * 1e3), waves * std::max(t_stream, t_mma));
   return body + m.e0 * std::min(M, c.tile_n) / 16.0 + m.s_epi;
 }
@@ -178,10 +178,11 @@ void candidate_grid(qg_format f, int M, int N, int K, qg_config* out, int max_ou
   if (f != QG_NVFP4 && M <= 64) {
     const int rows_opts[] = {8, 16, 32, 64};
     const int ring_opts[] = {8, 16, 32, 64};
-    for (int tm : {16, 32}) {
-      if (tm == 32 && M <= 16) continue;
+    for (int tm : {8, 16, 32}) {
+      if ((tm == 32 && M <= 16) || (tm == 8 && M > 8)) continue;
       for (int r : rows_opts) {
-        const int kg = 64 / r;
+        if (tm == 8 && r < 16) continue;
+        const int kg = (tm == 8 ? 128 : 64) / r;
         int prev = 0;
         for (int ro : ring_opts) {
           int st = std::min(ro, ((kt + kg - 1) / kg) * kg);

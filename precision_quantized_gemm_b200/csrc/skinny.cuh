@@ -34,17 +34,25 @@
 
 namespace qg {
 
+// TM = 16 or 32: the tokens are the MMA's 16-row A operand and the weight
+// rows its 8-column B operand (a warp owns 8 weight rows).  TM = 8 (up to 8
+// tokens): the roles swap, the weight rows fill the 16-row A operand and the
+// tokens the 8 columns (a warp owns 16 weight rows), which halves the MMAs
+// per weight byte when a CTA has at most 8 tokens.
 template <int FMT, int TM, int NF>
 struct SkCfg {
+  static constexpr bool kWA = TM == 8;           // weights as the A operand
   static constexpr int kR = 8 * NF;              // weight rows per CTA
-  static constexpr int kKG = 8 / NF;             // K groups of compute warps
+  static constexpr int kUnits = kWA ? NF / 2 : NF;   // warps per K group
+  static constexpr int kKG = 8 / kUnits;         // K groups of compute warps
   static constexpr int kWarps = 8;               // compute warps
   static constexpr int kThreads = 32 * (kWarps + 1);
-  static constexpr int kMF = TM / 16;            // 16-token fragments
+  static constexpr int kMF = kWA ? 1 : TM / 16;  // A fragments per warp and K step
   static constexpr int kWTile = kR * kKTileBytes;
   static constexpr int kATile = TM * kKTileBytes;
   static constexpr int kStage = kWTile + kATile; // a multiple of 1024 (swizzle atoms)
   static constexpr int kRedBytes = kWarps * kMF * 16 * 8 * 4;
+  static_assert(!kWA || NF >= 2, "weights as A need 16 rows per warp");
 };
 
 // Shared memory of a skinny launch: the ring, one full and one empty barrier
@@ -82,7 +90,7 @@ __global__ void __launch_bounds__(SkCfg<FMT, TM, NF>::kThreads, 1)
     prefetch_tmap(&tmap_a);
     for (int i = 0; i < S; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], NF);              // the NF warps of the slot's K group
+      mbar_init(&empty[i], C::kUnits);       // the warps of the slot's K group
     }
     fence_barrier_init();
   }
@@ -135,8 +143,9 @@ __global__ void __launch_bounds__(SkCfg<FMT, TM, NF>::kThreads, 1)
     }
   } else {
     // ------------------------------------------------------- compute warps
-    const int nf = warp % NF;                  // weight rows [8 nf, 8 nf + 8) of the CTA
-    const int kg = warp / NF;                  // K tiles i with i % KG == kg
+    // weight rows [8 nf, 8 nf + 8) of the CTA (weights as A: [16 nf, 16 nf + 16))
+    const int nf = warp % C::kUnits;
+    const int kg = warp / C::kUnits;           // K tiles i with i % KG == kg
     const int g = lane >> 2, t = lane & 3;     // fragment row group and column pair
     // the activation scales below come from the preceding kernel
     griddep_wait();
@@ -151,10 +160,12 @@ __global__ void __launch_bounds__(SkCfg<FMT, TM, NF>::kThreads, 1)
         for (int j = 0; j < 4; ++j) acc[q][mf][j] = (Acc)0;
     // ldmatrix row addresses (swizzled: the 16-byte chunk c of row r sits at
     // chunk c ^ (r % 8) of its 128-byte row)
-    const int wrow = nf * 8 + (lane & 7);      // weight row of this lane's matrix row
-    const int arow = ((lane >> 3) & 1) * 8 + (lane & 7);   // token row within a 16-token fragment
-    const int achk = lane >> 4;                // A: chunk offset 0 / 1 (bytes 0-15 / 16-31 of a K step)
-    const int wchk = lane >> 3;                // B: chunk offset 0..3 (two K steps)
+    // B operand rows (8; two K steps per ldmatrix.x4): weight rows, or tokens
+    const int brow = (C::kWA ? 0 : nf * 8) + (lane & 7);
+    const int bchk = lane >> 3;                // chunk offset 0..3 (two K steps)
+    // A operand rows (16 per fragment): tokens, or weight rows
+    const int arow = (C::kWA ? nf * 16 : 0) + ((lane >> 3) & 1) * 8 + (lane & 7);
+    const int achk = lane >> 4;                // chunk offset 0 / 1 (bytes 0-15 / 16-31 of a K step)
     const int G = prm.groups;
     for (int i = kg; i < nkt; i += C::kKG) {
       const int st = i % S;
@@ -164,14 +175,19 @@ __global__ void __launch_bounds__(SkCfg<FMT, TM, NF>::kThreads, 1)
         sw = __ldg(prm.scale_w + (size_t)(n0 / 128) * G + i);
 #pragma unroll
         for (int mf = 0; mf < C::kMF; ++mf) {
-          const int mlo = m0 + mf * 16 + g, mhi = mlo + 8;
+          // the tokens of this thread's accumulator elements: rows g, g + 8 of
+          // a 16-token fragment, or columns 2t, 2t + 1 (weights as A)
+          const int mlo = C::kWA ? m0 + 2 * t : m0 + mf * 16 + g;
+          const int mhi = C::kWA ? mlo + 1 : mlo + 8;
           sa_lo[mf] = (mlo < prm.M) ? __ldg(prm.scale_a + (size_t)mlo * G + i) : 0.f;
           sa_hi[mf] = (mhi < prm.M) ? __ldg(prm.scale_a + (size_t)mhi * G + i) : 0.f;
         }
       }
       if (!mbar_wait(&full[st], (uint32_t)((i / S) & 1), prm.err, prm.wait_ns)) { ok = false; break; }
       const uint32_t wt = smem_u32(smem + (size_t)st * C::kStage);
-      const uint32_t at = wt + C::kWTile;
+      const uint32_t tt = wt + C::kWTile;     // the token tile
+      const uint32_t at = C::kWA ? wt : tt;    // the A and B operands' tiles
+      const uint32_t bt = C::kWA ? tt : wt;
       float p[4][C::kMF][4];                   // Block_FP8: this group's partial sums
       if constexpr (FMT == kBLOCK) {
 #pragma unroll
@@ -185,8 +201,8 @@ __global__ void __launch_bounds__(SkCfg<FMT, TM, NF>::kThreads, 1)
       for (int kp = 0; kp < 2; ++kp) {        // pairs of 32-byte K steps
         uint32_t b[4];
         {
-          const int c = 4 * kp + wchk;
-          ldsm_x4(wt + (uint32_t)(wrow * kKTileBytes + ((c ^ (wrow & 7)) << 4)), b[0], b[1], b[2], b[3]);
+          const int c = 4 * kp + bchk;
+          ldsm_x4(bt + (uint32_t)(brow * kKTileBytes + ((c ^ (brow & 7)) << 4)), b[0], b[1], b[2], b[3]);
         }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {         // K step 2 kp + h
@@ -220,10 +236,13 @@ __global__ void __launch_bounds__(SkCfg<FMT, TM, NF>::kThreads, 1)
           float pg[4];
 #pragma unroll
           for (int j = 0; j < 4; ++j) pg[j] = (p[0][mf][j] + p[1][mf][j]) + (p[2][mf][j] + p[3][mf][j]);
-          af[0] = fmaf(pg[0], flo, af[0]);
-          af[1] = fmaf(pg[1], flo, af[1]);
-          af[2] = fmaf(pg[2], fhi, af[2]);
-          af[3] = fmaf(pg[3], fhi, af[3]);
+          // element j: row g (j < 2) or g + 8, column 2t + (j & 1); the token
+          // is the row (tokens as A) or the column (weights as A)
+          const float f0 = flo, f1 = C::kWA ? fhi : flo, f2 = C::kWA ? flo : fhi, f3 = fhi;
+          af[0] = fmaf(pg[0], f0, af[0]);
+          af[1] = fmaf(pg[1], f1, af[1]);
+          af[2] = fmaf(pg[2], f2, af[2]);
+          af[3] = fmaf(pg[3], f3, af[3]);
         }
       }
     }
@@ -253,14 +272,21 @@ __global__ void __launch_bounds__(SkCfg<FMT, TM, NF>::kThreads, 1)
         const int mm = u / NF, nfu = u % NF;
         const int m = m0 + mm, nb = n0 + nfu * 8;
         if (m >= prm.M || nb >= prm.N) continue;
-        const int mf = mm / 16, rr = mm % 16;
         Acc s8[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) s8[j] = (Acc)0;
         for (int k2 = 0; k2 < C::kKG; ++k2) {  // K-group order: deterministic
-          const Acc* rw = red + ((size_t)((k2 * NF + nfu) * C::kMF + mf) * 16 + rr) * 8;
+          if constexpr (C::kWA) {
+            // warp (k2, nfu / 2), fragment rows 8 (nfu % 2) + j, column mm
+            const Acc* rw = red + (size_t)(k2 * C::kUnits + nfu / 2) * 128 + (nfu % 2) * 64 + mm;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) s8[j] += rw[j];
+            for (int j = 0; j < 8; ++j) s8[j] += rw[j * 8];
+          } else {
+            const int mf = mm / 16, rr = mm % 16;
+            const Acc* rw = red + ((size_t)((k2 * NF + nfu) * C::kMF + mf) * 16 + rr) * 8;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) s8[j] += rw[j];
+          }
         }
         if (prm.out_kind == 1) {
           uint32_t* Yu = reinterpret_cast<uint32_t*>(prm.Y) + (size_t)m * prm.ldy;

@@ -35,6 +35,9 @@ namespace {
 
 // Optional log of every timed candidate (qgemm_set_tune_log).
 std::string g_tune_log;
+// What a timed step is (qgemm_set_tune_objective): 0 = the activation
+// quantisation and the GEMM, 1 = the GEMM alone.
+int g_tune_gemm_only = 0;
 
 __global__ void fill_bf16_kernel(__nv_bfloat16* p, size_t n, unsigned long long seed, float amp) {
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
@@ -113,7 +116,7 @@ double time_config(qg_format f, const std::vector<Operand*>& Ws, const Operand& 
   qg_status s = QG_OK;
   qg_operand aop = A.op;
   for (int i = 0; i < calls && s == QG_OK; ++i) {
-    s = qgemm_quantize_act(f, act, M, K, K, nullptr, &aop, qws, qwsb, st);
+    if (!g_tune_gemm_only) s = qgemm_quantize_act(f, act, M, K, K, nullptr, &aop, qws, qwsb, st);
     if (s == QG_OK)
       s = qgemm_run(f, &A.op, &Ws[i % Ws.size()]->op, M, N, K, &c, ws, wsb, Y, N, QG_OUT_BF16, st);
   }
@@ -178,6 +181,8 @@ std::vector<qg_config> candidates(qg_format f, int M, int N, int K, int top_n) {
 
 extern "C" void qgemm_set_tune_log(const char* path) { g_tune_log = path ? path : ""; }
 
+extern "C" void qgemm_set_tune_objective(int gemm_only) { g_tune_gemm_only = gemm_only != 0; }
+
 namespace {
 qg_status tune_impl(void* table, qg_format f, const int* Ms, int nM, const int* NK, int nNK, int top_n,
                     double budget_s_per_shape, int verbose);
@@ -222,7 +227,7 @@ qg_status tune_impl(void* table, qg_format f, const int* Ms, int nM, const int* 
     size_t qb, sb;
     qgemm_operand_bytes(f, 1, N, K, &qb, &sb);
     const size_t wbytes = qb + sb;
-    const int copies = (int)std::min<size_t>(64, 2 * l2 / std::max<size_t>(wbytes, 1) + 2);
+    const int copies = (int)std::min<size_t>(512, 2 * l2 / std::max<size_t>(wbytes, 1) + 2);
     std::vector<Operand> extra(copies - 1);
     std::vector<Operand*> Ws{&W0};
     for (auto& w : extra) {
@@ -290,8 +295,9 @@ qg_status tune_impl(void* table, qg_format f, const int* Ms, int nM, const int* 
       if (!g_tune_log.empty()) {
         if (FILE* lf = std::fopen(g_tune_log.c_str(), "a")) {
           for (const auto& t : timed)
-            std::fprintf(lf, "%d %d %d %d %d %d %d %d %d %.4f\n", (int)f, M, N, K, t.second.split_k,
-                         t.second.swap_ab, t.second.tile_n, t.second.stages, t.second.reduce_mode, t.first);
+            std::fprintf(lf, "%d %d %d %d %d %d %d %d %d %d %d %.4f\n", (int)f, M, N, K, t.second.split_k,
+                         t.second.swap_ab, t.second.tile_n, t.second.stages, t.second.reduce_mode, t.second.variant,
+                         t.second.rows, t.first);
           std::fclose(lf);
         }
       }

@@ -9,8 +9,10 @@ default configuration, select on one graph-timed pass, record an
 independent second pass) over the decode and prefill shapes of the
 quantized linear layers this library serves, and writes the table that
 qgemm_dispatch reads.  ``--top-n N`` times only the analytic scorer's N
-best-ranked configurations per shape (qgemm_tune_ranked); ``--log`` keeps
-every candidate's time (the data fit_scorer.py fits the scorer to).
+best-ranked configurations per shape (qgemm_tune_ranked) plus the best four
+of each kernel variant; ``--log`` keeps every candidate's time (the data
+fit_scorer.py fits the scorer to); ``--objective`` chooses what a timed
+step is (the GEMM alone, the default, or quantisation + GEMM).
 Needs a B200.
 """
 from __future__ import annotations
@@ -52,9 +54,13 @@ def main(argv=None):
     ap.add_argument("--log", default=None, help="append every timed candidate to this file")
     ap.add_argument("--top-n", type=int, default=0,
                     help="time only the analytic scorer's top-N configurations per shape (0: the whole grid)")
+    ap.add_argument("--objective", choices=["gemm", "step"], default="gemm",
+                    help="time each candidate as back-to-back GEMMs (the per-shape metric) or as "
+                         "activation-quantisation + GEMM steps")
     a = ap.parse_args(argv)
     if a.log:
         qg.qgemm_set_tune_log(a.log)
+    qg.qgemm_set_tune_objective(a.objective == "gemm")
     table = qg.Table(a.out) if (a.resume and os.path.exists(a.out)) else qg.Table()
     for name in [s.strip() for s in a.suites.split(",") if s.strip()]:
         for fmt, Ms, NK in SHAPES[name]:

@@ -150,7 +150,10 @@ def test_run_reserved_fields_must_be_zero():
 @pytest.mark.parametrize("kw,status", [
     (dict(tile_n=16, rows=32, stages=32), qg.QG_ERR_NO_DEVICE),     # valid: reaches the device check
     (dict(tile_n=32, rows=8, stages=16), qg.QG_ERR_NO_DEVICE),
-    (dict(tile_n=64, rows=32, stages=32), qg.QG_ERR_UNSUPPORTED),   # tokens per CTA: 16 or 32
+    (dict(tile_n=8, rows=16, stages=8), qg.QG_ERR_NO_DEVICE),      # up to 8 tokens: weights as A
+    (dict(tile_n=8, rows=8, stages=16), qg.QG_ERR_UNSUPPORTED),     # ... needs 16 rows per warp
+    (dict(tile_n=8, rows=32, stages=6), qg.QG_ERR_UNSUPPORTED),     # 4 K groups: ring a multiple of 4
+    (dict(tile_n=64, rows=32, stages=32), qg.QG_ERR_UNSUPPORTED),   # tokens per CTA: 8, 16 or 32
     (dict(tile_n=16, rows=24, stages=32), qg.QG_ERR_UNSUPPORTED),   # rows: 8, 16, 32, 64
     (dict(tile_n=16, rows=8, stages=12), qg.QG_ERR_UNSUPPORTED),    # ring depth a multiple of 64/rows
     (dict(tile_n=16, rows=64, stages=65), qg.QG_ERR_UNSUPPORTED),

@@ -32,8 +32,14 @@ CASES = [  # (M, N, K, tile_n, rows, stages)
     (3, 24, 1024, 16, 32, 2),         # fewer weight rows than one CTA holds
     (2, 640, 8192, 16, 8, 64),        # K groups of 8 warps, deepest ring
     (64, 256, 2048, 32, 16, 8),       # two 32-token tiles
+    # up to 8 tokens per CTA: the weight rows are the 16-row MMA operand
+    (1, 256, 512, 8, 16, 8),
+    (8, 1000, 2048, 8, 32, 8),        # ragged N, 4 K groups
+    (3, 640, 4096, 8, 64, 8),         # 2 K groups, ring of 8 over 32 K tiles
+    (13, 384, 1024, 8, 16, 16),       # two 8-token tiles, the last partial
 ]
-RAGGED_K = [(4, 384, 528, 16, 32, 8), (9, 200, 1040, 16, 8, 8)]   # K % 128 != 0 (8-bit per-row formats)
+RAGGED_K = [(4, 384, 528, 16, 32, 8), (9, 200, 1040, 16, 8, 8),   # K % 128 != 0 (8-bit per-row formats)
+            (5, 272, 656, 8, 16, 8)]
 
 
 def _cases():
