@@ -124,11 +124,12 @@ def kernel_source_code(text: str) -> str:
 
 
 def kernel_source_hash():
-    """sha1 of the GEMM kernel code (gemm_kernel.cuh + ptx.cuh, comments
-    ignored): ties an ncu traffic figure to the code it measured."""
+    """sha1 of the GEMM kernels' code (gemm_kernel.cuh, skinny.cuh and
+    ptx.cuh, comments ignored): ties an ncu traffic figure to the code it
+    measured."""
     import hashlib
     h = hashlib.sha1()
-    for f in ("gemm_kernel.cuh", "ptx.cuh"):
+    for f in ("gemm_kernel.cuh", "skinny.cuh", "ptx.cuh"):
         with open(os.path.join(ROOT, "precision_quantized_gemm_b200", "csrc", f), encoding="utf-8") as fh:
             h.update(kernel_source_code(fh.read()).encode())
     return h.hexdigest()[:12]
@@ -655,7 +656,10 @@ def run_ours(args, world, rank, local):
         "int8_decode_geomean_frac_hbm_roofline": round(geo, 4),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "kernel": "qgemm_kernel<INT8, swap-AB> (all three shapes, launch-weighted)",
+                     "kernel": "the step's three INT8 GEMM launches, launch-weighted (configurations per "
+                               "shape from the table: " + ", ".join(
+                                   f"M={m}: " + ("decode kernel" if cfgs[m].variant == 1 else "tile kernel")
+                                   for m in MS) + ")",
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
                      else "fallback 6650 GB/s"},
         "e2e": {"value": round(world * step_bytes() / (ms_e2e_max * 1e-3) / 1e9, 2), "unit": "GB/s",

@@ -51,11 +51,11 @@ struct Model {
   double e3 = 3.95830;       // second-pass launch, µs
   double e4 = 11.2845;       // last-CTA reduction, µs
   double e5 = 1180.85;       // workspace traffic bandwidth, GB/s
-  // decode ("skinny") kernel: K-tile cycles of one compute warp, and its
-  // chain after the data (activation wait, K-group sum, stores) relative to
-  // the tile kernel's, µs
-  double s_tile = 40.0;
-  double s_epi = -1.0;
+  // decode ("skinny") kernel: K-tile cycles of one compute warp, streaming
+  // rate of one CTA (GB/s), fixed chain (µs)
+  double s_tile = 300.0;
+  double s_cta_gbs = 45.0;
+  double s_chain = 2.3;
 };
 const Model kModel;
 
@@ -81,8 +81,13 @@ int ctas_per_sm(qg_format f, int M, int K, const qg_config& c) {
 }
 
 // The decode kernel: ceil(N / rows) x ceil(M / tile_n) CTAs, each streaming
-// its rows (and tokens) over the whole of K through its ring, eight compute
-// warps in 64 / rows K groups.
+// its rows (and tokens) over the whole of K through its ring; eight compute
+// warps in K groups each take a share of the K tiles.  Calibrated on
+// measured launches of this kernel (per-shape sweeps on one B200): a fixed
+// chain of ~2.3 us (dependency release, activation tiles, the K-group sum,
+// the stores), then the slice streaming at ~45 GB/s per CTA (shared when two
+// CTAs sit on an SM), or the warps' MMA loop, whichever is longer, and never
+// faster than the weights over HBM.
 double estimate_skinny_us(qg_format f, int M, int N, int K, const qg_config& c, int sms) {
   const Model& m = kModel;
   const double rb = (double)K;
@@ -91,14 +96,12 @@ double estimate_skinny_us(qg_format f, int M, int N, int K, const qg_config& c, 
   const size_t smem = qg::config_smem(f, M, K, &c);
   const int cps = std::max(1, std::min(2, (int)(kSmemPerSm / (smem + 1024))));
   const double waves = std::ceil(ctas / ((double)sms * cps));
-  const double stage_bytes = (double)(c.rows + c.tile_n) * 128.0;
-  const double inflight = std::min(c.stages, kt) * stage_bytes;
-  const double rate = std::min(inflight / m.lat_us, m.sm_gbs * 1e3 / cps);
-  const double t_stream = stage_bytes * kt / rate;
+  const double cta_bytes = (double)(c.rows + c.tile_n) * 128.0 * kt;
+  const double t_stream = cta_bytes / (m.s_cta_gbs * 1e3 / cps);
   const int kg = (c.tile_n == 8 ? 128 : 64) / c.rows;
   const double t_mma = std::ceil((double)kt / kg) * m.s_tile * std::max(1, c.tile_n / 16) / m.clock_mhz;
   const double body = std::max((double)N * rb / (m.hbm_gbs * 1e3), waves * std::max(t_stream, t_mma));
-  return body + m.e0 * std::min(M, c.tile_n) / 16.0 + m.s_epi;
+  return m.s_chain + body;
 }
 
 double estimate_us(qg_format f, int M, int N, int K, const qg_config& c, int sms) {

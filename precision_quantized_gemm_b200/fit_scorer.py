@@ -4,7 +4,9 @@
 
 The data is the tuner's log of every timed candidate (``tune_tables.py
 --log``): one line per (format, M, N, K, split_k, swap_ab, tile_n, stages,
-reduce_mode, µs).  The model is the one csrc/scorer.cu evaluates (see the
+reduce_mode, [variant, rows,] µs); the tile kernel's model is fitted to its
+own lines (variant 0; logs from before the decode kernel have no variant
+column).  The model is the one csrc/scorer.cu evaluates (see the
 comment at its top): Little's-law streaming per CTA under per-SM and HBM
 caps, MMA-loop cycles per K tile (Block_FP8: plus promotion cycles per
 column a thread promotes), waves over the SMs, and the split-K
@@ -101,7 +103,14 @@ def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--data", default=os.path.join(HERE, "tables", "b200_candidates.txt"))
     a = ap.parse_args(argv)
-    rows = np.array([[float(x) for x in line.split()] for line in open(a.data) if line.strip()])
+    rows = []
+    for line in open(a.data):
+        v = [float(x) for x in line.split()]
+        if len(v) == 12 and v[9] != 0:         # the decode kernel: not this model
+            continue
+        if len(v) in (10, 12):
+            rows.append(v[:9] + [v[-1]])
+    rows = np.array(rows)
     t = rows[:, 9]
     V = features(rows)
     shapes = collections.defaultdict(list)
