@@ -182,6 +182,43 @@ qg_status qgemm_quantize_act(qg_format f, const void* A, int M, int K, int lda,
 qg_status qgemm_quantize_weight(qg_format f, const void* W, int N, int K, qg_operand* out,
                                 void* workspace, size_t ws_bytes, void* stream);
 
+/* Mixture-of-experts operands for qgemm_run_grouped.
+ *
+ * qgemm_grouped_act_bytes: the `q` and `scale` bytes of the activation
+ * operand of T tokens routed over `experts` experts: those of
+ * qgemm_operand_bytes(f, 0, T, K) except NVFP4, whose block scales take
+ * floor((T - a) / 128) + a 128-row atoms, a = min(experts, T) (every active
+ * expert may open a fresh atom).
+ *
+ * qgemm_quantize_act_grouped: qgemm_quantize_act of bf16 A [T, lda], tokens
+ * sorted by expert, expert e owning rows [expert_offsets[e],
+ * expert_offsets[e + 1]) (DEVICE int32 [experts + 1], read after the wait on
+ * the preceding kernel, clamped to [0, T]).  The 8-bit formats' scales are
+ * per token or token group, so this is qgemm_quantize_act.  NVFP4: one
+ * tensor scale over all T tokens (the activation is one tensor), codes
+ * [T, K/2] as usual, and block scales in the per-expert layout: expert e's
+ * scale rows start at 128 x sum_{e' < e} ceil(c_e' / 128) (c the token
+ * counts), its tokens in order, the rest of its last atom zero, so each
+ * expert's scales are the plain 128x4 tiled layout of its own c_e rows.
+ * out->scale holds qgemm_grouped_act_bytes bytes; out->rows = T.
+ *
+ * qgemm_quantize_weight_grouped: qgemm_quantize_weight of the stacked
+ * weights W bf16 [experts * N, K], N a multiple of 128; out->rows =
+ * experts * N.  The 8-bit formats' per-channel and 128x128-block scales
+ * never cross an expert, so this is qgemm_quantize_weight of the stack.
+ * NVFP4: every expert is quantised as its own tensor (its own tensor scale,
+ * out->global_scale [experts]); its codes and block scales sit at
+ * e x qgemm_operand_bytes(f, 1, N, K) in the stacked buffers.  workspace:
+ * qgemm_quant_workspace_size(f, N, K) bytes, reused by each expert in turn.
+ * experts: 1 ... 256. */
+qg_status qgemm_grouped_act_bytes(qg_format f, int experts, int T, int K, size_t* q_bytes,
+                                  size_t* scale_bytes);
+qg_status qgemm_quantize_act_grouped(qg_format f, int experts, const int* expert_offsets, const void* A,
+                                     int T, int K, int lda, const float* static_amax, qg_operand* out,
+                                     void* workspace, size_t ws_bytes, void* stream);
+qg_status qgemm_quantize_weight_grouped(qg_format f, int experts, const void* W, int N, int K,
+                                        qg_operand* out, void* workspace, size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------ GEMM -- */
 
 /* y = dequant(A_q) . dequant(W_q)^T with configuration `cfg`.
@@ -215,10 +252,14 @@ qg_status qgemm_run(qg_format f, const qg_operand* A, const qg_operand* W, int M
  *                   the preceding kernel of the stream (the routing), so the
  *                   call needs no host copy and can be captured.  Offsets
  *                   outside [0, A->rows] are clamped on the device.
- *   A:  activations of all T = A->rows tokens (quantised as one operand).
+ *   A:  activations of all T = A->rows tokens (quantised as one operand,
+ *       by qgemm_quantize_act_grouped with the same offsets: for NVFP4 its
+ *       block scales are in the per-expert layout that call documents).
  *   W:  all experts' weights stacked, W->rows = experts * N, expert e's rows
  *       at [e * N, (e + 1) * N); per-channel scales [experts * N] or 128x128
- *       block scales [experts * N / 128, K / 128].  N must be a multiple of
+ *       block scales [experts * N / 128, K / 128]; NVFP4: block scales of
+ *       the stacked rows and one tensor scale per expert, global_scale
+ *       [experts] (qgemm_quantize_weight_grouped).  N must be a multiple of
  *       128 (no 128-row block straddles two experts).
  *   Y:  [T, ldy]; cfg: swap_ab = 1 (a decode expert sees few tokens), any
  *       split_k with reduce_mode 0 or 1 (workspace as qgemm_workspace_size(f,
@@ -227,8 +268,9 @@ qg_status qgemm_run(qg_format f, const qg_operand* A, const qg_operand* W, int M
  * T): the most that any routing of T tokens over the experts needs.  A CTA
  * finds its expert and tokens with a warp scan over the offsets and exits if
  * it has none.  Weights are loaded after that lookup (which experts run depends on
- * the routing).  FP8_DYNAMIC, W8A8_INT8 and BLOCK_FP8; NVFP4 returns
- * QG_ERR_UNSUPPORTED (its scale atoms need 128-aligned token tiles). */
+ * the routing).  All four formats; NVFP4 takes tile_n >= 64 unless T <=
+ * tile_n (a token tile's block scales must start at an even 32-row word of
+ * its expert's 128-row scale atom). */
 qg_status qgemm_run_grouped(qg_format f, int experts, const int* expert_offsets, const qg_operand* A,
                             const qg_operand* W, int N, int K, const qg_config* cfg, void* workspace,
                             size_t ws_bytes, void* Y, int ldy, int out_kind, void* stream);
@@ -238,8 +280,8 @@ qg_status qgemm_run_grouped(qg_format f, int experts, const int* expert_offsets,
  * and the launch streams their weights, so the configuration is the
  * scorer's first-ranked one for min(experts, T) * N weight rows and
  * ceil(T / active) tokens among those qgemm_run_grouped accepts (swap_ab = 1,
- * reduce_mode 0 or 1); else split_k 1, tile_n 16, 4 stages.  NVFP4 returns
- * QG_ERR_UNSUPPORTED. */
+ * reduce_mode 0 or 1); else split_k 1, tile_n 16 (NVFP4 with T > 16: 64),
+ * 4 stages. */
 qg_status qgemm_grouped_default_config(qg_format f, int experts, int T, int N, int K, qg_config* out);
 
 /* Activation quantisation fused into the GEMM: y = dequant(quant(A)) .

@@ -114,3 +114,23 @@ def grouped(gemm_fn, qa, sa, qw, sw, offsets, n_per_expert: int, w_rows_per_scal
         s0, s1 = w0 // w_rows_per_scale, w1 // w_rows_per_scale
         y[r0:r1] = gemm_fn(qa[r0:r1], sa[r0:r1], qw[w0:w1], sw[s0:s1])
     return y
+
+
+def grouped_nvfp4(qa, sfa, ga, qw, sfw, gw, offsets, n_per_expert: int):
+    """The grouped GEMM above for NVFP4 operands.  Each expert's weight is a
+    tensor of its own (a mixture-of-experts layer holds one linear layer per
+    expert), so expert e contributes its own tensor scale gw[e]; the
+    activations of all tokens are one tensor with one scale ga.  Expert e's
+    rows of y are nvfp4(qa[r0:r1], sfa[r0:r1], ga, qw[eN:(e+1)N],
+    sfw[eN:(e+1)N], gw[e]).  Returns y [T, N] in fp64 values of bf16."""
+    T = qa.shape[0]
+    N = n_per_expert
+    y = np.zeros((T, N), np.float64)
+    for e in range(len(offsets) - 1):
+        r0, r1 = int(offsets[e]), int(offsets[e + 1])
+        if r1 <= r0:
+            continue
+        w0, w1 = e * N, (e + 1) * N
+        y[r0:r1] = nvfp4(qa[r0:r1], sfa[r0:r1], ga, qw[w0:w1], sfw[w0:w1], gw[e])
+    return y
+

@@ -113,3 +113,19 @@ def nvfp4(x_bits: np.ndarray, global_amax: float | None = None, sf_vec: int = 16
     q = encode_e2m1((xb / d_safe[:, :, None]).astype(F32))
     q = np.where(zero[:, :, None], np.uint8(0), q).reshape(R, K)
     return q, sf, g
+
+
+def nvfp4_experts(w_bits: np.ndarray, experts: int, sf_vec: int = 16):
+    """Stacked mixture-of-experts weights [experts * N, K]: every expert's
+    N rows quantised by ``nvfp4`` as a tensor of its own (its own amax and
+    tensor scale).  Returns (codes [experts * N, K], block scale codes
+    [experts * N, K/16], g float32 [experts])."""
+    R = w_bits.shape[0]
+    assert R % experts == 0
+    N = R // experts
+    parts = [nvfp4(w_bits[e * N:(e + 1) * N], sf_vec=sf_vec) for e in range(experts)]
+    q = np.concatenate([p[0] for p in parts], axis=0)
+    sf = np.concatenate([p[1] for p in parts], axis=0)
+    g = np.array([p[2] for p in parts], dtype=F32)
+    return q, sf, g
+

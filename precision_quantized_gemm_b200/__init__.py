@@ -44,7 +44,8 @@ EXPORTS = [
     "qgemm_run_noalloc", "qgemm_set_trace", "qgemm_run_fused_act", "qgemm_set_tune_log",
     "qgemm_score_config", "qgemm_rank_configs", "qgemm_tune_ranked", "qgemm_table_validate",
     "qgemm_run_grouped", "qgemm_grouped_default_config", "qgemm_set_wait_limit", "qgemm_selftest_wait_expiry",
-    "qgemm_set_tune_objective",
+    "qgemm_set_tune_objective", "qgemm_grouped_act_bytes", "qgemm_quantize_act_grouped",
+    "qgemm_quantize_weight_grouped",
 ]
 
 
@@ -132,6 +133,11 @@ def lib() -> ctypes.CDLL:
                                           c_double, c_int]),
             "qgemm_table_validate": (c_int, [c_void_p, POINTER(c_int), POINTER(c_int), c_int]),
             "qgemm_grouped_default_config": (c_int, [c_int, c_int, c_int, c_int, c_int, POINTER(qg_config)]),
+            "qgemm_grouped_act_bytes": (c_int, [c_int, c_int, c_int, c_int, POINTER(c_size_t), POINTER(c_size_t)]),
+            "qgemm_quantize_act_grouped": (c_int, [c_int, c_int, c_void_p, c_void_p, c_int, c_int, c_int, c_void_p,
+                                                   POINTER(qg_operand), c_void_p, c_size_t, c_void_p]),
+            "qgemm_quantize_weight_grouped": (c_int, [c_int, c_int, c_void_p, c_int, c_int, POINTER(qg_operand),
+                                                      c_void_p, c_size_t, c_void_p]),
             "qgemm_run_grouped": (c_int, [c_int, c_int, c_void_p, POINTER(qg_operand), POINTER(qg_operand), c_int,
                                           c_int, POINTER(qg_config), c_void_p, c_size_t, c_void_p, c_int, c_int,
                                           c_void_p]),
@@ -212,6 +218,27 @@ def qgemm_run_grouped(fmt, experts, offsets_ptr, A: qg_operand, W: qg_operand, N
     """Grouped (mixture-of-experts) GEMM over tokens sorted by expert."""
     return lib().qgemm_run_grouped(fmt, experts, offsets_ptr, ctypes.byref(A), ctypes.byref(W), N, K,
                                    ctypes.byref(cfg), ws_ptr, ws_bytes, Y_ptr, ldy, out_kind, stream)
+
+
+def qgemm_grouped_act_bytes(fmt, experts, T, K):
+    """Bytes of the q and scale buffers of a grouped activation operand."""
+    q, s = c_size_t(), c_size_t()
+    check(lib().qgemm_grouped_act_bytes(fmt, experts, T, K, ctypes.byref(q), ctypes.byref(s)),
+          "qgemm_grouped_act_bytes")
+    return q.value, s.value
+
+
+def qgemm_quantize_act_grouped(fmt, experts, offsets_ptr, A_ptr, T, K, lda, static_amax_ptr, out: qg_operand,
+                               ws_ptr, ws_bytes, stream):
+    """Activation quantisation for a grouped launch (NVFP4: per-expert scale layout)."""
+    return lib().qgemm_quantize_act_grouped(fmt, experts, offsets_ptr, A_ptr, T, K, lda, static_amax_ptr,
+                                            ctypes.byref(out), ws_ptr, ws_bytes, stream)
+
+
+def qgemm_quantize_weight_grouped(fmt, experts, W_ptr, N, K, out: qg_operand, ws_ptr, ws_bytes, stream):
+    """Stacked expert weights (NVFP4: one tensor scale per expert)."""
+    return lib().qgemm_quantize_weight_grouped(fmt, experts, W_ptr, N, K, ctypes.byref(out), ws_ptr, ws_bytes,
+                                               stream)
 
 
 def qgemm_default_config(fmt, M, N, K) -> qg_config:
@@ -352,15 +379,17 @@ def _stream(stream=None):
 
 
 class Operand:
-    """Caller-owned buffers of a quantized operand, allocated with torch."""
+    """Caller-owned buffers of a quantized operand, allocated with torch.
+    ``sizes`` overrides the (q, scale) byte counts and ``n_global`` the number
+    of tensor scales (grouped operands)."""
 
-    def __init__(self, fmt: int, is_weight: bool, rows: int, K: int, device="cuda"):
+    def __init__(self, fmt: int, is_weight: bool, rows: int, K: int, device="cuda", sizes=None, n_global=1):
         torch = _torch()
-        qb, sb = qgemm_operand_bytes(fmt, is_weight, rows, K)
+        qb, sb = sizes or qgemm_operand_bytes(fmt, is_weight, rows, K)
         self.fmt, self.is_weight, self.rows, self.K = fmt, is_weight, rows, K
         self.q = torch.empty(qb, dtype=torch.uint8, device=device)
         self.scale = torch.zeros(sb, dtype=torch.uint8, device=device)
-        self.global_scale = torch.zeros(4, dtype=torch.float32, device=device)
+        self.global_scale = torch.zeros(max(n_global, 4), dtype=torch.float32, device=device)
         self.c = qg_operand(self.q.data_ptr(), self.scale.data_ptr(), self.global_scale.data_ptr(), rows, K)
 
 
@@ -374,6 +403,37 @@ def quantize_act(fmt: int, A, out: Operand | None = None, static_amax=None, stre
     sa = static_amax.data_ptr() if static_amax is not None else None
     check(qgemm_quantize_act(fmt, A.data_ptr(), M, K, A.stride(0), sa, out.c, ws.data_ptr(), wsb,
                              _stream(stream)), "qgemm_quantize_act")
+    out._ws = ws
+    return out
+
+
+def quantize_act_grouped(fmt: int, A, offsets, static_amax=None, stream=None) -> Operand:
+    """Activation quantisation of bf16 A [T, K], tokens sorted by expert
+    (``offsets``: device int32 [experts + 1]), for run_grouped."""
+    torch = _torch()
+    T, K = A.shape
+    experts = offsets.numel() - 1
+    out = Operand(fmt, False, T, K, A.device, sizes=qgemm_grouped_act_bytes(fmt, experts, T, K))
+    wsb = qgemm_quant_workspace_size(fmt, T, K)
+    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=A.device)
+    sa = static_amax.data_ptr() if static_amax is not None else None
+    check(qgemm_quantize_act_grouped(fmt, experts, offsets.data_ptr(), A.data_ptr(), T, K, A.stride(0), sa,
+                                     out.c, ws.data_ptr(), wsb, _stream(stream)), "qgemm_quantize_act_grouped")
+    out._ws = ws
+    return out
+
+
+def quantize_weight_grouped(fmt: int, W, experts: int, stream=None) -> Operand:
+    """Stacked expert weights bf16 [experts * N, K] for run_grouped (NVFP4:
+    each expert its own tensor, one tensor scale per expert)."""
+    torch = _torch()
+    R, K = W.shape
+    N = R // experts
+    out = Operand(fmt, True, R, K, W.device, n_global=experts)
+    wsb = qgemm_quant_workspace_size(fmt, N, K)
+    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=W.device)
+    check(qgemm_quantize_weight_grouped(fmt, experts, W.contiguous().data_ptr(), N, K, out.c, ws.data_ptr(), wsb,
+                                        _stream(stream)), "qgemm_quantize_weight_grouped")
     out._ws = ws
     return out
 

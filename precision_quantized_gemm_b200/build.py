@@ -24,6 +24,7 @@ LIB = os.path.join(PKG, "libqgemm.so")
 INCLUDE = os.path.join(ROOT, "include")
 
 SOURCES = ["api.cu", "quant.cu", "gemm_fp8.cu", "gemm_int8.cu", "gemm_block.cu", "gemm_nvf4.cu",
+           "gemm_nvf4_grouped.cu",
            "tune.cu", "table.cpp", "noalloc.cu", "scorer.cu"]
 HEADERS = ["ptx.cuh", "gemm_kernel.cuh", "gemm_launch.cuh", "internal.h", "quant_math.cuh", "attr_cache.h", "skinny.cuh"]
 

@@ -349,6 +349,41 @@ qg_status qgemm_quantize_act(qg_format f, const void* A, int M, int K, int lda,
   return e == cudaSuccess ? QG_OK : QG_ERR_CUDA;
 }
 
+qg_status qgemm_grouped_act_bytes(qg_format f, int experts, int T, int K, size_t* q_bytes,
+                                  size_t* scale_bytes) {
+  if (experts <= 0) return QG_ERR_INVALID_ARG;
+  if (experts > qg::kMaxExperts) return QG_ERR_UNSUPPORTED;
+  qg_status s = qgemm_operand_bytes(f, 0, T, K, q_bytes, scale_bytes);
+  if (s != QG_OK || f != QG_NVFP4) return s;
+  // every active expert (at most a = min(experts, T)) opens a fresh 128-row
+  // atom: sum_e ceil(c_e / 128) <= floor((T - a) / 128) + a
+  const int a = std::min(experts, T);
+  *scale_bytes = (size_t)((T - a) / 128 + a) * 128 * (size_t)(((K + 255) / 256) * 16);
+  return QG_OK;
+}
+
+qg_status qgemm_quantize_act_grouped(qg_format f, int experts, const int* expert_offsets, const void* A,
+                                     int T, int K, int lda, const float* static_amax, qg_operand* out,
+                                     void* workspace, size_t ws_bytes, void* stream) {
+  if (experts <= 0 || !expert_offsets || !aligned(expert_offsets, 4)) return QG_ERR_INVALID_ARG;
+  if (experts > qg::kMaxExperts) return QG_ERR_UNSUPPORTED;
+  // the 8-bit formats' scales are per token (group): their layout does not
+  // depend on the routing
+  if (f != QG_NVFP4) return qgemm_quantize_act(f, A, T, K, lda, static_amax, out, workspace, ws_bytes, stream);
+  if (!A || T <= 0 || K <= 0 || lda < K) return QG_ERR_INVALID_ARG;
+  if (K % k_multiple(f) != 0 || (lda * 2) % 16 != 0 || !aligned(A, 16)) return QG_ERR_INVALID_ARG;
+  qg_status s = check_quant_out(f, T, K, out);
+  if (s != QG_OK) return s;
+  if (static_amax == nullptr && (ws_bytes < qgemm_quant_workspace_size(f, T, K) || !workspace))
+    return QG_ERR_WORKSPACE;
+  DeviceInfo* d;
+  if ((s = device_info(&d)) != QG_OK) return s;
+  const cudaError_t e = qg::launch_quant_nvfp4(A, T, K, lda, static_amax, out->q, out->scale, out->global_scale,
+                                               (float*)workspace, (cudaStream_t)stream, g_pdl, expert_offsets,
+                                               experts);
+  return e == cudaSuccess ? QG_OK : QG_ERR_CUDA;
+}
+
 qg_status qgemm_quantize_weight(qg_format f, const void* W, int N, int K, qg_operand* out,
                                 void* workspace, size_t ws_bytes, void* stream) {
   if (!valid_format(f) || !W || N <= 0 || K <= 0) return QG_ERR_INVALID_ARG;
@@ -374,6 +409,36 @@ qg_status qgemm_quantize_weight(qg_format f, const void* W, int N, int K, qg_ope
                                  (float*)workspace, st, g_pdl);
   }
   return e == cudaSuccess ? QG_OK : QG_ERR_CUDA;
+}
+
+qg_status qgemm_quantize_weight_grouped(qg_format f, int experts, const void* W, int N, int K,
+                                        qg_operand* out, void* workspace, size_t ws_bytes, void* stream) {
+  if (experts <= 0 || N <= 0 || N % 128 != 0 || !out) return QG_ERR_INVALID_ARG;
+  if (experts > qg::kMaxExperts) return QG_ERR_UNSUPPORTED;
+  if ((long long)experts * N > 0x7fffffffLL) return QG_ERR_INVALID_ARG;
+  // per-row and 128x128-block scales never cross an expert boundary
+  // (N % 128 == 0): the stacked tensor quantises as each expert would
+  if (f != QG_NVFP4) return qgemm_quantize_weight(f, W, experts * N, K, out, workspace, ws_bytes, stream);
+  if (!W || K <= 0 || K % k_multiple(f) != 0 || !aligned(W, 16)) return QG_ERR_INVALID_ARG;
+  qg_status s = check_quant_out(f, experts * N, K, out);
+  if (s != QG_OK) return s;
+  if (ws_bytes < qgemm_quant_workspace_size(f, N, K) || !workspace) return QG_ERR_WORKSPACE;
+  DeviceInfo* d;
+  if ((s = device_info(&d)) != QG_OK) return s;
+  // NVFP4: each expert is its own tensor with its own tensor scale; its
+  // codes, block scales (whole 128-row atoms) and tensor scale sit at
+  // expert x (N rows) in the stacked buffers
+  size_t qb = 0, sb = 0;
+  if ((s = qgemm_operand_bytes(f, 1, N, K, &qb, &sb)) != QG_OK) return s;
+  const __nv_bfloat16* w = static_cast<const __nv_bfloat16*>(W);
+  for (int e = 0; e < experts; ++e) {
+    const cudaError_t err = qg::launch_quant_nvfp4(
+        w + (size_t)e * N * K, N, K, K, nullptr, static_cast<uint8_t*>(out->q) + (size_t)e * qb,
+        static_cast<uint8_t*>(out->scale) + (size_t)e * sb, out->global_scale + e, (float*)workspace,
+        (cudaStream_t)stream, g_pdl);
+    if (err != cudaSuccess) return QG_ERR_CUDA;
+  }
+  return QG_OK;
 }
 
 qg_status check_operand_impl(qg_format f, const qg_operand* o, int rows, int K) {
@@ -542,7 +607,9 @@ qg_status launch_run(qg_format f, const qg_operand* A, const void* act, int lda,
   // weight prefetch for the later half of a Swap-AB grid (launch order:
   // clusters of split_k, else single CTAs); not for grouped launches, whose
   // weight rows depend on the routing
-  if (swap && !expert_offsets && act == nullptr && g_l2_ahead) {
+  // (the kernel indexes the grid in 32 bits: only grids below 2^31 CTAs)
+  if (swap && !expert_offsets && act == nullptr && g_l2_ahead &&
+      (long long)tp * tq * cfg->split_k < 0x7fffffffLL) {
     const bool clus = cfg->split_k > 1 && cfg->reduce_mode == qg::kReduceCluster;
     const long long units = clus ? (long long)tp * tq : (long long)tp * tq * cfg->split_k;
     prm.l2_ahead = (int)((units + 1) / 2);
@@ -585,7 +652,6 @@ qg_status qgemm_run_grouped(qg_format f, int experts, const int* expert_offsets,
   if (!valid_format(f) || experts <= 0 || !expert_offsets || !A || !W || !aligned(expert_offsets, 4))
     return QG_ERR_INVALID_ARG;
   if (experts > qg::kMaxExperts) return QG_ERR_UNSUPPORTED;
-  if (f == QG_NVFP4) return QG_ERR_UNSUPPORTED;           // scale atoms need 128-aligned token tiles
   if (N <= 0 || N % 128 != 0) return QG_ERR_INVALID_ARG;   // experts' weight rows fill whole 128-row blocks
   if ((long long)experts * N > 0x7fffffffLL) return QG_ERR_INVALID_ARG;
   const int M = A->rows;
@@ -622,7 +688,6 @@ qg_status qgemm_default_config(qg_format f, int M, int N, int K, qg_config* out)
 
 qg_status qgemm_grouped_default_config(qg_format f, int experts, int T, int N, int K, qg_config* out) {
   if (!valid_format(f) || experts <= 0 || T <= 0 || N <= 0 || K <= 0 || !out) return QG_ERR_INVALID_ARG;
-  if (f == QG_NVFP4) return QG_ERR_UNSUPPORTED;
   if (K % k_multiple(f) != 0) return QG_ERR_INVALID_ARG;
   // T tokens over at most min(experts, T) experts: the launch streams the
   // weights of the active experts, like one GEMM of active x N rows with the
@@ -644,7 +709,7 @@ qg_status qgemm_grouped_default_config(qg_format f, int experts, int T, int N, i
   qg_config c = {};
   c.split_k = 1;
   c.swap_ab = 1;
-  c.tile_n = 16;
+  c.tile_n = (f == QG_NVFP4 && T > 16) ? 64 : 16;    // NVFP4: narrow tiles only as the sole tile
   c.stages = 4;
   if (qg::config_check(f, T, N, K, &c) != QG_OK) return QG_ERR_UNSUPPORTED;
   *out = c;

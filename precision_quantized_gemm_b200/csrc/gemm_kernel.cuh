@@ -308,9 +308,11 @@ __device__ __forceinline__ uint32_t add_acc(uint32_t a, uint32_t b) {
   else return __float_as_uint(__uint_as_float(a) + __uint_as_float(b));
 }
 
+// NVFP4 tensor-scale product; a grouped launch takes expert e's weight
+// tensor scale g_w[e] (every expert quantised as its own tensor).
 template <int FMT>
-__device__ __forceinline__ float alpha_of(const GemmParams& prm) {
-  if constexpr (FMT == kNVF4) return __ldg(prm.g_a) * __ldg(prm.g_w);
+__device__ __forceinline__ float alpha_of(const GemmParams& prm, int expert = 0) {
+  if constexpr (FMT == kNVF4) return __ldg(prm.g_a) * __ldg(prm.g_w + expert);
   else return 1.f;
 }
 
@@ -341,8 +343,13 @@ __device__ __forceinline__ void emit(const GemmParams& prm, int r, int c, int m,
 // blockIdx.y walks its eight experts to the one it falls in.  Offsets come
 // from the preceding kernel (routing) and are clamped to [0, M], so a
 // malformed routing never leads to an access outside A or y.  Writes {expert
-// (-1: no tile), first token, tokens} to map.
-template <int BN>
+// (-1: no tile), first token, tokens, scale row} to map; the scale row is the
+// tile's first token in the NVFP4 per-expert padded scale layout (every
+// expert's scale rows start on a 128-row atom boundary: expert e's first
+// row is 128 x the sum of ceil(tokens / 128) over the experts before it).
+// With SF, a tile whose scale rows would pass the layout's end (only a
+// malformed, decreasing routing claims that many atoms) gets no tile.
+template <int BN, bool SF>
 __device__ __forceinline__ void grouped_tile(const GemmParams& prm, int lane, int* map) {
   constexpr unsigned kFull = 0xffffffffu;
   constexpr int kPer = kMaxExperts / 32;
@@ -363,6 +370,16 @@ __device__ __forceinline__ void grouped_tile(const GemmParams& prm, int lane, in
     if (lane >= d) incl += t;
   }
   const int excl = incl - sum;
+  // 128-row scale atoms of this lane's experts, and the atoms before them
+  int asum = 0;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) asum += (max(ov[j + 1] - ov[j], 0) + 127) / 128;
+  int aincl = asum;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int t = __shfl_up_sync(kFull, aincl, d);
+    if (lane >= d) aincl += t;
+  }
   const unsigned hit = __ballot_sync(kFull, y >= excl && y < incl);
   if (hit == 0u) {
     if (lane == 0) map[0] = -1;
@@ -370,6 +387,7 @@ __device__ __forceinline__ void grouped_tile(const GemmParams& prm, int lane, in
   }
   if (lane == __ffs(hit) - 1) {
     int base = excl;
+    int abase = aincl - asum;
 #pragma unroll
     for (int j = 0; j < kPer; ++j) {
       const int cnt = max(ov[j + 1] - ov[j], 0);
@@ -379,9 +397,15 @@ __device__ __forceinline__ void grouped_tile(const GemmParams& prm, int lane, in
         map[0] = e0 + j;
         map[1] = ov[j] + tile * BN;
         map[2] = min(BN, cnt - tile * BN);
+        map[3] = abase * 128 + tile * BN;
+        if constexpr (SF) {
+          const int a = min(E, prm.M);
+          if (map[3] + map[2] > ((prm.M - a) / 128 + a) * 128) map[0] = -1;
+        }
         break;
       }
       base += t;
+      abase += (cnt + 127) / 128;
     }
   }
 }
@@ -427,22 +451,28 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
   // the expert's first row)
   int Mlim = prm.M;
   int wrow = 0;
+  int sf_row_q = q0;                           // NVFP4: scale row of the first Q row of the tile
+  int expert = 0;
   if constexpr (GROUPED) {
     // which expert and tokens this CTA serves depends on the routing of the
     // preceding kernel: resolved before any set-up, and a CTA without work
     // leaves at once (all CTAs of a split-K cluster share the tile)
-    __shared__ int gmap[3];
+    __shared__ int gmap[4];
     griddep_wait();
-    if (warp == 0) grouped_tile<BN>(prm, lane, gmap);
+    if (warp == 0) grouped_tile<BN, FMT == kNVF4>(prm, lane, gmap);
     __syncthreads();
     if (gmap[0] < 0 || gmap[2] <= 0) return;
     q0 = gmap[1];
     Mlim = gmap[1] + gmap[2];
     wrow = gmap[0] * prm.N;
+    sf_row_q = gmap[3];
+    expert = gmap[0];
   }
   const int kz = blockIdx.z;
-  const int kt_begin = (int)(((long long)kz * prm.kt_total) / prm.split_k);
-  const int kt_end = (int)(((long long)(kz + 1) * prm.kt_total) / prm.split_k);
+  // split_k is a power of two: slice z is K tiles [z kt / split_k, (z + 1) kt / split_k)
+  const int sk_log2 = __ffs(prm.split_k) - 1;
+  const int kt_begin = (int)(((long long)kz * prm.kt_total) >> sk_log2);
+  const int kt_end = (int)(((long long)(kz + 1) * prm.kt_total) >> sk_log2);
   const int nkt = kt_end - kt_begin;
   if (threadIdx.x == 0) trace_at(prm, kTrEntry);
   const bool cluster_red = prm.split_k > 1 && prm.reduce_mode == kReduceCluster;
@@ -506,7 +536,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
       const int row_a = SWAP ? q0 : p0;
       // NVFP4 scale atoms: P rows [p0, p0+128) are one 128-row block; Q has
       // one or two blocks (the second only if it holds any row).
-      const int sfq_atoms = (C::kSfQAtoms == 2 && q0 + 128 < prm.rows_q) ? 2 : 1;
+      const int sfq_atoms = (C::kSfQAtoms == 2 && q0 + 128 < (GROUPED ? Mlim : prm.rows_q)) ? 2 : 1;
       const uint32_t stage_tx = a_threads ? bytes_w
                                       : kPTileBytes + C::kQTileBytes +
                                             (C::kNvf4 ? (uint32_t)(4 * kSfAtomBytes * (1 + sfq_atoms)) : 0u);
@@ -533,7 +563,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
         tma_load_2d(smem + off_a + st * bytes_a, map_a, &full[st], kt * kKTileBytes, row_a, pol_a);
         if constexpr (C::kNvf4) {
           const uint8_t* sfa = SWAP ? prm.sf_q : prm.sf_p;
-          const int rb = row_a / 128;
+          const int rb = (SWAP ? sf_row_q : row_a) / 128;
           if (SWAP) {
             for (int a = 0; a < sfq_atoms; ++a)
               bulk_load(smem + L.sfq + st * C::kSfQBytes + a * 4 * kSfAtomBytes,
@@ -563,12 +593,13 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
             const int tc = blockIdx.x + gx * blockIdx.y + prm.l2_ahead;
             if (tc < gx * gy) { tx = tc % gx; tz = kz; }
           } else {
-            const long long t = (long long)blockIdx.x + (long long)gx * (blockIdx.y + (long long)gy * kz) + prm.l2_ahead;
-            if (t < (long long)gx * gy * gz) { tx = (int)(t % gx); tz = (int)(t / ((long long)gx * gy)); }
+            // the launch keeps l2_ahead at 0 unless gx * gy * gz fits 31 bits
+            const unsigned t = blockIdx.x + (unsigned)gx * (blockIdx.y + (unsigned)gy * kz) + (unsigned)prm.l2_ahead;
+            if (t < (unsigned)(gx * gy * gz)) { tx = (int)(t % (unsigned)gx); tz = (int)(t / (unsigned)(gx * gy)); }
           }
           if (tx >= 0) {
-            const int t_begin = (int)(((long long)tz * prm.kt_total) / prm.split_k);
-            const int t_end = (int)(((long long)(tz + 1) * prm.kt_total) / prm.split_k);
+            const int t_begin = (int)(((long long)tz * prm.kt_total) >> sk_log2);
+            const int t_end = (int)(((long long)(tz + 1) * prm.kt_total) >> sk_log2);
             for (int kt = t_begin; kt < t_end; ++kt) {
               tma_prefetch_l2_2d(map_w, kt * kKTileBytes, tx * 128);
               if constexpr (C::kNvf4)
@@ -642,7 +673,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
       const uint32_t sfa_t = tmem_base + C::kSfaCol;
       const uint32_t sfb_t = tmem_base + C::kSfbCol;
       // word offset of this CTA's first Q row inside its 128-row SF atom
-      const uint32_t sfb_word = (uint32_t)((q0 % 128) / 32);
+      const uint32_t sfb_word = (uint32_t)((sf_row_q % 128) / 32);
       int st = 0;                              // stage of K tile i, and its full-barrier phase
       uint32_t ph = 0;
       int gb = 0, gr = 0;                      // Block_FP8: group buffer of K tile i, and its round
@@ -1052,7 +1083,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
     const size_t MN = (size_t)prm.M * prm.N;
     uint32_t* part = reinterpret_cast<uint32_t*>(prm.partial);
     uint32_t* stage_buf = reinterpret_cast<uint32_t*>(smem + L.p);   // ring, idle now
-    const float alpha = alpha_of<FMT>(prm);
+    const float alpha = alpha_of<FMT>(prm, expert);
     // Accumulator columns [cbeg + c0, cbeg + c0 + CW) of this thread's row.
     auto load_chunk = [&](int c0, uint32_t (&v)[CW]) {
       if constexpr (C::kBlock) {
@@ -1365,7 +1396,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
         const uint32_t rank = cluster_ctarank();
         const int r0 = (int)rank * rows_per;
         const uint32_t red_s = smem_u32(smem + L.p);
-        const float alpha = alpha_of<FMT>(prm);
+        const float alpha = alpha_of<FMT>(prm, expert);
         // units of 8 consecutive output channels: 2 x 16-byte remote loads per
         // split, summed in split order, scaled and stored as one 16-byte vector.
         // Up to four splits: a thread's next unit's loads are in flight with
@@ -1495,8 +1526,6 @@ __global__ void splitk_reduce_kernel(const GemmParams prm) {
   griddep_launch_dependents();
   const size_t MN = (size_t)prm.M * prm.N;
   const uint32_t* part = reinterpret_cast<const uint32_t*>(prm.partial);
-  float alpha = 1.f;
-  if constexpr (FMT == kNVF4) alpha = __ldg(prm.g_a) * __ldg(prm.g_w);
   for (size_t o = blockIdx.x * (size_t)blockDim.x + threadIdx.x; o < MN;
        o += (size_t)gridDim.x * blockDim.x) {
     const int m = (int)(o / prm.N), n = (int)(o % prm.N);
@@ -1513,25 +1542,25 @@ __global__ void splitk_reduce_kernel(const GemmParams prm) {
     if (prm.out_kind == 1) {
       reinterpret_cast<uint32_t*>(prm.Y)[(size_t)m * prm.ldy + n] = bits;
     } else {
+      // grouped: row m belongs to the last expert whose first token is <= m
+      // (offsets clamped to [0, M] as in the GEMM kernel)
+      int expert = 0;
+      if (prm.expert_offsets != nullptr) {
+        int lo = 0, hi = prm.experts - 1;
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (min(max(__ldg(prm.expert_offsets + mid), 0), prm.M) <= m) lo = mid;
+          else hi = mid - 1;
+        }
+        expert = lo;
+      }
       float sa = 1.f, sw = 1.f;
       if constexpr (FMT == kFP8 || FMT == kINT8) {
         sa = __ldg(prm.scale_a + m);
-        // grouped: row m belongs to the last expert whose first token is <= m
-        // (offsets clamped to [0, M] as in the GEMM kernel)
-        int wrow = 0;
-        if (prm.expert_offsets != nullptr) {
-          int lo = 0, hi = prm.experts - 1;
-          while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (min(max(__ldg(prm.expert_offsets + mid), 0), prm.M) <= m) lo = mid;
-            else hi = mid - 1;
-          }
-          wrow = lo * prm.N;
-        }
-        sw = __ldg(prm.scale_w + wrow + n);
+        sw = __ldg(prm.scale_w + (size_t)expert * prm.N + n);
       }
       reinterpret_cast<__nv_bfloat16*>(prm.Y)[(size_t)m * prm.ldy + n] =
-          __float2bfloat16_rn(finish_value<FMT>(bits, sa, sw, alpha));
+          __float2bfloat16_rn(finish_value<FMT>(bits, sa, sw, alpha_of<FMT>(prm, expert)));
     }
   }
 }

@@ -1,6 +1,9 @@
 // gemm_launch.cuh — host-side launch of one format's GEMM instantiations.
 // Included by exactly one translation unit per format with QG_FMT and
-// QG_LAUNCH_NAME defined.
+// QG_LAUNCH_NAME defined.  A format whose grouped (mixture-of-experts)
+// kernels live in a unit of their own defines QG_GROUPED_OWN_UNIT in the
+// format's unit and QG_GROUPED_ONLY in that second unit (the two compile in
+// parallel).
 #pragma once
 #include "attr_cache.h"
 #include "gemm_kernel.cuh"
@@ -176,6 +179,15 @@ size_t skinny_smem_rows(int rows, int stages) {
 
 }  // namespace
 
+#if !defined(QG_GROUPED_OWN_UNIT) || defined(QG_GROUPED_ONLY)
+// grouped (mixture-of-experts) launch: Swap-AB, activations by TMA
+cudaError_t QG_CAT(QG_LAUNCH_NAME, _grouped)(int tile_n, const CUtensorMap& tp, const CUtensorMap& tq,
+                                             const GemmParams& prm, dim3 grid, cudaStream_t st, bool pdl) {
+  return launch_bn<QG_FMT, true, false, true>(tile_n, tp, tq, prm, grid, st, pdl);
+}
+#endif
+
+#ifndef QG_GROUPED_ONLY
 cudaError_t QG_CAT(QG_LAUNCH_NAME, _skinny)(int tile_n, int rows, const CUtensorMap& tw, const CUtensorMap& ta,
                                             const GemmParams& prm, dim3 grid, cudaStream_t st, bool pdl) {
   if constexpr (QG_FMT == kNVF4) {
@@ -202,10 +214,7 @@ size_t QG_CAT(QG_LAUNCH_NAME, _skinny_smem)(int tile_n, int rows, int stages) {
 cudaError_t QG_LAUNCH_NAME(bool swap, int tile_n, const CUtensorMap& tp, const CUtensorMap& tq,
                            const GemmParams& prm, dim3 grid, cudaStream_t st, bool pdl) {
   if (prm.expert_offsets != nullptr) {
-    // grouped (mixture-of-experts) launch: Swap-AB, 8-bit formats only
-    if constexpr (QG_FMT != kNVF4) {
-      if (swap && prm.a_mode == kActTma) return launch_bn<QG_FMT, true, false, true>(tile_n, tp, tq, prm, grid, st, pdl);
-    }
+    if (swap && prm.a_mode == kActTma) return QG_CAT(QG_LAUNCH_NAME, _grouped)(tile_n, tp, tq, prm, grid, st, pdl);
     return cudaErrorInvalidValue;
   }
   if (prm.a_mode == kActFused) {
@@ -244,5 +253,7 @@ cudaError_t QG_CAT(QG_LAUNCH_NAME, _reduce)(const GemmParams& prm, cudaStream_t 
   cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, splitk_reduce_kernel<QG_FMT>, prm);
 }
+
+#endif  // QG_GROUPED_ONLY
 
 }  // namespace qg

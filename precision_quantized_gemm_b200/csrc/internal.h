@@ -40,7 +40,8 @@ cudaError_t launch_quant_weight_blocks(const void* W, int N, int K, void* q, flo
 int nvfp4_amax_ctas(int R, int K);
 cudaError_t launch_quant_nvfp4(const void* X, int R, int K, int ldx, const float* static_amax,
                                void* q, void* sf, float* gscale, float* partial,
-                               cudaStream_t st, bool pdl);
+                               cudaStream_t st, bool pdl, const int* offsets = nullptr,
+                               int experts = 0);
 
 // GEMM launchers, one per format (each in its own translation unit).
 // Returns cudaErrorInvalidValue for a (swap, tile_n) pair not instantiated.
@@ -51,6 +52,8 @@ cudaError_t launch_quant_nvfp4(const void* X, int R, int K, int ldx, const float
                      int act_tiles);                                                       \
   bool NAME##_cluster_fits(int tile_n, bool swap, int stages, int act_tiles);              \
   cudaError_t NAME##_reduce(const GemmParams& prm, cudaStream_t st, bool pdl);             \
+  cudaError_t NAME##_grouped(int tile_n, const CUtensorMap& tp, const CUtensorMap& tq,     \
+                             const GemmParams& prm, dim3 grid, cudaStream_t st, bool pdl); \
   cudaError_t NAME##_skinny(int tile_n, int rows, const CUtensorMap& tw, const CUtensorMap& ta, \
                             const GemmParams& prm, dim3 grid, cudaStream_t st, bool pdl);     \
   size_t NAME##_skinny_smem(int tile_n, int rows, int stages);

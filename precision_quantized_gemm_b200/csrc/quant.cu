@@ -194,14 +194,38 @@ __global__ void __launch_bounds__(kQThreads) nvfp4_amax_kernel(const __nv_bfloat
   if (threadIdx.x == 0) partial[blockIdx.x] = amax;
 }
 
-// Phase 2: one thread per 16-element block (r, c) of the padded scale
+// Inclusive prefix sum over the block's threads (kQThreads of them).
+__device__ int block_incl_scan(int v, int* warp_tot) {
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, v, d);
+    if (l >= d) v += t;
+  }
+  if (l == 31) warp_tot[w] = v;
+  __syncthreads();
+  for (int j = 0; j < w; ++j) v += warp_tot[j];
+  return v;
+}
+
+// Phase 2: one thread per 16-element block (s, c) of the padded scale
 // matrix [R_pad, C]; writes 8 bytes of codes and one scale byte (0 in the
 // padding).  Every CTA reduces the phase-1 partials itself (deterministic).
+// Grouped layout (offsets != NULL): tokens sorted by expert, and expert e's
+// scale rows start at 128 x (the 128-row atoms of the experts before it), so
+// each expert's first token opens a fresh atom; scale row s holds token
+// offsets[e] + (s - first row of e) of the expert e whose rows contain s, or
+// padding.  Offsets are clamped to [0, R] as the grouped GEMM does.
 __global__ void __launch_bounds__(kQThreads) nvfp4_quant_kernel(
     const __nv_bfloat16* __restrict__ X, int R, int K, int ldx, const float* __restrict__ partial,
     int npartial, const float* __restrict__ static_amax, uint8_t* __restrict__ q,
-    uint8_t* __restrict__ sf, float* __restrict__ gscale, int R_pad, int C) {
+    uint8_t* __restrict__ sf, float* __restrict__ gscale, int R_pad, int C,
+    const int* __restrict__ offsets, int experts) {
   __shared__ float red[32];
+  __shared__ int e_tok[kQThreads];             // grouped: expert's first token
+  __shared__ int e_cnt[kQThreads];             //          its tokens
+  __shared__ int e_row[kQThreads];             //          its first scale row
+  __shared__ int warp_tot[kQThreads / 32];
   // let the next kernel (the GEMM) start streaming its weights now; it
   // waits for this kernel's completion before it reads what we write
   griddep_launch_dependents();
@@ -215,11 +239,38 @@ __global__ void __launch_bounds__(kQThreads) nvfp4_quant_kernel(
   }
   const float g = amax_t > 0.f ? __fdiv_rn(amax_t, 2688.f) : 1.f;
   if (blockIdx.x == 0 && threadIdx.x == 0) *gscale = g;
+  if (offsets != nullptr) {
+    const int t = threadIdx.x;
+    int lo = 0, cnt = 0;
+    if (t < experts) {
+      lo = min(max(__ldg(offsets + t), 0), R);
+      cnt = max(min(max(__ldg(offsets + t + 1), 0), R) - lo, 0);
+    }
+    const int atoms = (cnt + 127) / 128;
+    const int incl = block_incl_scan(atoms, warp_tot);
+    e_tok[t] = lo;
+    e_cnt[t] = cnt;
+    e_row[t] = (incl - atoms) * 128;
+    __syncthreads();
+  }
   const int KS = K / 16;
   const long long total = (long long)R_pad * C;
   for (long long i = blockIdx.x * (long long)kQThreads + threadIdx.x; i < total;
        i += (long long)gridDim.x * kQThreads) {
-    const int r = (int)(i / C), c = (int)(i % C);
+    const int srow = (int)(i / C), c = (int)(i % C);
+    int r = srow;                              // token whose scales sit in row srow
+    if (offsets != nullptr) {
+      // the last expert whose first scale row is <= srow (an empty expert
+      // shares its first row with the next one, which wins)
+      int lo = 0, hi = experts - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (e_row[mid] <= srow) lo = mid;
+        else hi = mid - 1;
+      }
+      const int j = srow - e_row[lo];
+      r = j < e_cnt[lo] ? e_tok[lo] + j : R;
+    }
     uint32_t code = 0;
     if (r < R && c < KS) {
       const uint4* src = reinterpret_cast<const uint4*>(X + (size_t)r * ldx + c * 16);
@@ -243,8 +294,8 @@ __global__ void __launch_bounds__(kQThreads) nvfp4_quant_kernel(
       reinterpret_cast<uint2*>(q + (size_t)r * (K / 2) + c * 8)[0] = packed;
     }
     // 128x4 tiled scale layout
-    const size_t atom = (size_t)(r / 128) * (C / 4) + (c / 4);
-    sf[atom * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + (c % 4)] = (uint8_t)code;
+    const size_t atom = (size_t)(srow / 128) * (C / 4) + (c / 4);
+    sf[atom * 512 + (srow % 32) * 16 + ((srow % 128) / 32) * 4 + (c % 4)] = (uint8_t)code;
   }
 }
 
@@ -304,7 +355,7 @@ int nvfp4_amax_ctas(int R, int K) {
 
 cudaError_t launch_quant_nvfp4(const void* X, int R, int K, int ldx, const float* static_amax,
                                void* q, void* sf, float* gscale, float* partial,
-                               cudaStream_t st, bool pdl) {
+                               cudaStream_t st, bool pdl, const int* offsets, int experts) {
   const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(X);
   int npartial = 0;
   cudaError_t e = cudaSuccess;
@@ -314,7 +365,13 @@ cudaError_t launch_quant_nvfp4(const void* X, int R, int K, int ldx, const float
     e = launch((const void*)nvfp4_amax_kernel, dim3(npartial), dim3(kQThreads), a1, st, pdl);
     if (e != cudaSuccess) return e;
   }
+  // scale rows: whole 128-row atoms; grouped, every active expert (at most
+  // a = min(experts, R)) may open a fresh atom: floor((R - a) / 128) + a atoms
   int R_pad = ((R + 127) / 128) * 128;
+  if (offsets != nullptr) {
+    const int a = experts < R ? experts : R;
+    R_pad = ((R - a) / 128 + a) * 128;
+  }
   int C = ((K + 255) / 256) * 16;
   uint8_t* qq = static_cast<uint8_t*>(q);
   uint8_t* sff = static_cast<uint8_t*>(sf);
@@ -324,7 +381,7 @@ cudaError_t launch_quant_nvfp4(const void* X, int R, int K, int ldx, const float
   const float* pp = partial;
   void* a2[] = {(void*)&x,   (void*)&R,           (void*)&K,  (void*)&ldx,   (void*)&pp,
                 (void*)&npartial, (void*)&static_amax, (void*)&qq, (void*)&sff, (void*)&gscale,
-                (void*)&R_pad, (void*)&C};
+                (void*)&R_pad, (void*)&C, (void*)&offsets, (void*)&experts};
   return launch((const void*)nvfp4_quant_kernel, dim3((unsigned)ctas), dim3(kQThreads), a2, st, pdl);
 }
 

@@ -5,6 +5,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 import precision_quantized_gemm_b200 as qg
@@ -304,6 +305,7 @@ def test_fused_valid_arguments_reach_the_device_check():
 
 
 @pytest.mark.parametrize("kw,status", [
+    # NVFP4: a 16-token tile below row 16 of a scale atom is refused (T = 24 > 16)
     (dict(fmt=qg.QG_NVFP4), qg.QG_ERR_UNSUPPORTED),
     (dict(E=0), qg.QG_ERR_INVALID_ARG),
     (dict(E=300), qg.QG_ERR_UNSUPPORTED),                       # more than 256 experts
@@ -325,13 +327,15 @@ def test_grouped_rejects_bad_arguments_before_any_launch(kw, status):
     assert st == status
 
 
-@pytest.mark.parametrize("fmt", [qg.QG_FP8_DYNAMIC, qg.QG_W8A8_INT8, qg.QG_BLOCK_FP8])
+@pytest.mark.parametrize("fmt", [qg.QG_FP8_DYNAMIC, qg.QG_W8A8_INT8, qg.QG_BLOCK_FP8, qg.QG_NVFP4])
 @pytest.mark.parametrize("E,T,N,K", [(128, 8, 1536, 2048), (128, 512, 2048, 768), (4, 3, 256, 512),
                                      (256, 4096, 1024, 4096)])
 def test_grouped_default_config_is_accepted_by_the_grouped_launch(fmt, E, T, N, K):
     c = qg.qgemm_grouped_default_config(fmt, E, T, N, K)
     assert c.swap_ab == 1 and c.reduce_mode in (0, 1)
     assert c.split_k >= 1 and c.split_k & (c.split_k - 1) == 0 and c.tile_n in (16, 32, 64, 128, 256)
+    if fmt == qg.QG_NVFP4:
+        assert c.tile_n >= 64 or T <= c.tile_n
     torch = pytest.importorskip("torch")
     if torch.cuda.is_available():
         return                     # the fake pointers below must never reach a launch
@@ -342,9 +346,8 @@ def test_grouped_default_config_is_accepted_by_the_grouped_launch(fmt, E, T, N, 
     assert st == qg.QG_ERR_NO_DEVICE
 
 
-def test_grouped_default_config_rejects_nvfp4_and_bad_sizes():
+def test_grouped_default_config_rejects_bad_sizes():
     c = qg.qg_config()
-    assert qg.lib().qgemm_grouped_default_config(qg.QG_NVFP4, 8, 8, 256, 512, c) == qg.QG_ERR_UNSUPPORTED
     assert qg.lib().qgemm_grouped_default_config(qg.QG_FP8_DYNAMIC, 0, 8, 256, 512, c) == qg.QG_ERR_INVALID_ARG
     assert qg.lib().qgemm_grouped_default_config(qg.QG_FP8_DYNAMIC, 8, 8, 256, 100, c) == qg.QG_ERR_INVALID_ARG
 
@@ -355,3 +358,57 @@ def test_wait_expiry_selftest_rejects_limits_before_the_device():
     assert qg.lib().qgemm_selftest_wait_expiry(10 ** 9, None) == qg.QG_ERR_INVALID_ARG
     qg.qgemm_set_wait_limit(5_000_000)
     qg.qgemm_set_wait_limit(0)
+
+
+@pytest.mark.parametrize("E,T,K", [(8, 1, 512), (8, 300, 512), (256, 200, 1024), (4, 4096, 256), (1, 128, 64)])
+def test_grouped_act_bytes_bound_every_routing(E, T, K):
+    # NVFP4: floor((T - a) / 128) + a atoms, a = min(E, T), is the most any
+    # routing of T tokens over E experts needs (brute force over the extremes)
+    q, s = qg.qgemm_grouped_act_bytes(qg.QG_NVFP4, E, T, K)
+    q1, s1 = qg.qgemm_operand_bytes(qg.QG_NVFP4, 0, T, K)
+    C = (K + 255) // 256 * 16
+    a = min(E, T)
+    assert q == q1 and s == ((T - a) // 128 + a) * 128 * C and s >= s1
+    rng = np.random.default_rng(T)
+    worst = 0
+    for counts in ([T] + [0] * (E - 1), [1] * (a - 1) + [T - a + 1] + [0] * (E - a),
+                   rng.multinomial(T, [1 / E] * E)):
+        worst = max(worst, sum((c + 127) // 128 for c in counts))
+    assert worst * 128 * C <= s
+    # the 8-bit formats' scales do not depend on the routing
+    for f in (qg.QG_FP8_DYNAMIC, qg.QG_W8A8_INT8, qg.QG_BLOCK_FP8):
+        if K % 128 == 0 or f != qg.QG_BLOCK_FP8:
+            assert qg.qgemm_grouped_act_bytes(f, E, T, K) == qg.qgemm_operand_bytes(f, 0, T, K)
+
+
+def test_grouped_quantisers_check_arguments_before_the_device():
+    L = qg.lib()
+    T, K, E, N = 24, 512, 4, 256
+    qb, sb = qg.qgemm_grouped_act_bytes(qg.QG_NVFP4, E, T, K)
+    out = _op(T, K)
+    assert L.qgemm_grouped_act_bytes(qg.QG_NVFP4, 0, T, K, None, None) == qg.QG_ERR_INVALID_ARG
+    assert L.qgemm_grouped_act_bytes(qg.QG_NVFP4, 300, T, K, None, None) == qg.QG_ERR_UNSUPPORTED
+    args = lambda **kw: (kw.get("f", qg.QG_NVFP4), kw.get("E", E), kw.get("off", FAKE), kw.get("A", FAKE),
+                         kw.get("T", T), K, kw.get("lda", K), None, kw.get("out", out), FAKE, 1 << 20, None)
+    assert L.qgemm_quantize_act_grouped(*args(off=None)) == qg.QG_ERR_INVALID_ARG
+    assert L.qgemm_quantize_act_grouped(*args(off=FAKE + 2)) == qg.QG_ERR_INVALID_ARG
+    assert L.qgemm_quantize_act_grouped(*args(E=0)) == qg.QG_ERR_INVALID_ARG
+    assert L.qgemm_quantize_act_grouped(*args(E=300)) == qg.QG_ERR_UNSUPPORTED
+    assert L.qgemm_quantize_act_grouped(*args(lda=K - 1)) == qg.QG_ERR_INVALID_ARG
+    assert L.qgemm_quantize_act_grouped(*args(out=_op(T + 1, K))) == qg.QG_ERR_INVALID_ARG
+    assert L.qgemm_quantize_act_grouped(*args(out=_op(T, K, g=0))) == qg.QG_ERR_INVALID_ARG
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        assert L.qgemm_quantize_act_grouped(*args()) == qg.QG_ERR_NO_DEVICE
+        assert L.qgemm_quantize_act_grouped(*args(f=qg.QG_W8A8_INT8)) == qg.QG_ERR_NO_DEVICE
+    W = _op(E * N, K)
+    wargs = lambda **kw: (kw.get("f", qg.QG_NVFP4), kw.get("E", E), FAKE, kw.get("N", N), K, kw.get("out", W),
+                          FAKE, kw.get("wsb", 1 << 20), None)
+    assert L.qgemm_quantize_weight_grouped(*wargs(N=200)) == qg.QG_ERR_INVALID_ARG     # N % 128
+    assert L.qgemm_quantize_weight_grouped(*wargs(E=0)) == qg.QG_ERR_INVALID_ARG
+    assert L.qgemm_quantize_weight_grouped(*wargs(E=300)) == qg.QG_ERR_UNSUPPORTED
+    assert L.qgemm_quantize_weight_grouped(*wargs(out=_op(E * N - 128, K))) == qg.QG_ERR_INVALID_ARG
+    assert L.qgemm_quantize_weight_grouped(*wargs(wsb=0)) == qg.QG_ERR_WORKSPACE
+    if not torch.cuda.is_available():
+        assert L.qgemm_quantize_weight_grouped(*wargs()) == qg.QG_ERR_NO_DEVICE
+

@@ -13,6 +13,7 @@ import precision_quantized_gemm_b200 as qg
 from gpu_util import assert_within_tolerance, bf16_to_np, oracle_quant, to_dev_bf16
 import qg_synth
 from oracle import gemm as OG
+from oracle import quant as OQ
 
 pytestmark = pytest.mark.gpu
 
@@ -119,3 +120,103 @@ def test_grouped_int8_accumulators_bit_exact():
         if m1 > m0:
             np.testing.assert_array_equal(acc[m0:m1].astype(np.int64),
                                           OG.acc_int8(qa[0][m0:m1], qw[0][e * N:(e + 1) * N]))
+
+
+# ------------------------------------------------------------------- NVFP4 --
+# NVFP4 grouped launches: activations quantised with the per-expert scale
+# layout (each expert's block scales start on a 128-row atom), weights one
+# tensor per expert (a tensor scale each).
+NVF4_ROUTINGS = dict(ROUTINGS, big=[300, 0, 129, 5, 200])
+NVF4_CASES = [  # (routing, N, K, split_k, tile_n, reduce_mode, stages)
+    ("sparse", 256, 1024, 1, 16, 0, 4),        # T = 11 <= 16: one tile per expert
+    ("multi-tile", 256, 2048, 1, 64, 0, 4),
+    ("multi-tile", 128, 1024, 2, 64, 1, 4),    # second-pass reduction
+    ("big", 256, 1024, 2, 128, 0, 4),          # experts over 128 tokens: several atoms
+    ("big", 128, 512, 1, 256, 0, 3),           # 256-token tiles: two atoms
+    ("e256", 128, 512, 1, 64, 0, 4),
+]
+
+
+def _nvf4_id(c):
+    return f"nvfp4-{c[0]}-N{c[1]}-K{c[2]}-s{c[3]}-t{c[4]}-r{c[5]}"
+
+
+def _expert_rows(counts):
+    """First scale row of every expert in the per-expert layout."""
+    rows, r = [], 0
+    for c in counts:
+        rows.append(r)
+        r += (c + 127) // 128 * 128
+    return rows, r
+
+
+@pytest.mark.parametrize("case", NVF4_CASES, ids=[_nvf4_id(c) for c in NVF4_CASES])
+def test_grouped_nvfp4_matches_per_expert_runs_and_oracle(case):
+    routing, N, K, sk, tn, rm, st = case
+    fmt = qg.QG_NVFP4
+    counts = NVF4_ROUTINGS[routing]
+    E, T = len(counts), sum(counts)
+    offs = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    a = qg_synth.activations(T, K)
+    w = qg_synth.weights(E * N, K)
+    offsets = torch.from_numpy(offs).cuda()
+    A = qg.quantize_act_grouped(fmt, to_dev_bf16(a), offsets)
+    W = qg.quantize_weight_grouped(fmt, to_dev_bf16(w), E)
+    cfg = qg.make_config(split_k=sk, swap_ab=1, tile_n=tn, stages=st, reduce_mode=rm)
+    y = torch.full((T, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    qg.run_grouped(fmt, A, W, offsets, N, cfg, out=y)
+    y_again = qg.run_grouped(fmt, A, W, offsets, N, cfg)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_again)
+    qa = OQ.nvfp4(a)
+    qw = OQ.nvfp4_experts(w, E)
+    # the tensor scales are the oracle's fp32 quotients
+    assert float(A.global_scale[0]) == float(qa[2])
+    assert np.array_equal(W.global_scale[:E].cpu().numpy(), qw[2])
+    ref = OG.grouped_nvfp4(qa[0], qa[1], qa[2], qw[0], qw[1], qw[2], offs, N)
+    C = (K + 255) // 256 * 16
+    rows, _ = _expert_rows(counts)
+    qbw, sbw = qg.qgemm_operand_bytes(fmt, 1, N, K)
+    ws = qg.Workspace()
+    for e in range(E):
+        m0, m = int(offs[e]), counts[e]
+        if m == 0:
+            continue
+        Ae = qg.qg_operand(A.q.data_ptr() + m0 * K // 2, A.scale.data_ptr() + rows[e] * C,
+                           A.global_scale.data_ptr(), m, K)
+        We = qg.qg_operand(W.q.data_ptr() + e * qbw, W.scale.data_ptr() + e * sbw,
+                           W.global_scale.data_ptr() + 4 * e, N, K)
+        ye = torch.empty(m, N, dtype=torch.bfloat16, device="cuda")
+        wsp, wsb = ws.get(qg.qgemm_workspace_size(fmt, m, N, K, cfg))
+        qg.check(qg.qgemm_run(fmt, Ae, We, m, N, K, cfg, wsp, wsb, ye.data_ptr(), N, 0, qg._stream(None)))
+        torch.cuda.synchronize()
+        assert torch.equal(y[m0:m0 + m], ye), f"expert {e}"
+        assert_within_tolerance(bf16_to_np(y[m0:m0 + m]), ref[m0:m0 + m], f"{_nvf4_id(case)} expert {e}")
+
+
+@pytest.mark.parametrize("routing", ["sparse", "big", "e256"])
+def test_grouped_nvfp4_activation_layout_is_each_experts_plain_layout(routing):
+    # with one static amax, expert e's codes and block scales are bitwise those
+    # of the plain quantiser on its own tokens, placed at its first atom; the
+    # scale rows past the last expert's atoms are zero
+    fmt, K = qg.QG_NVFP4, 512
+    counts = NVF4_ROUTINGS[routing]
+    E, T = len(counts), sum(counts)
+    offs = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    a = to_dev_bf16(qg_synth.activations(T, K))
+    amax = torch.tensor([3.0], dtype=torch.float32, device="cuda")
+    G = qg.quantize_act_grouped(fmt, a, torch.from_numpy(offs).cuda(), static_amax=amax)
+    torch.cuda.synchronize()
+    C = (K + 255) // 256 * 16
+    rows, used = _expert_rows(counts)
+    for e in range(E):
+        m0, m = int(offs[e]), counts[e]
+        if m == 0:
+            continue
+        P = qg.quantize_act(fmt, a[m0:m0 + m], static_amax=amax)
+        torch.cuda.synchronize()
+        assert torch.equal(G.q[m0 * K // 2:(m0 + m) * K // 2], P.q), f"expert {e} codes"
+        nb = P.scale.numel()
+        assert torch.equal(G.scale[rows[e] * C:rows[e] * C + nb], P.scale), f"expert {e} scales"
+        assert float(G.global_scale[0]) == float(P.global_scale[0])
+    assert int(G.scale[used * C:].count_nonzero()) == 0

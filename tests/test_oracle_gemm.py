@@ -254,3 +254,53 @@ def test_grouped_block_scales_follow_the_expert():
     y_s = G.grouped(G.block_fp8, qa, sa, qw_s, sw_s, offsets, 128, w_rows_per_scale=128)
     assert np.array_equal(y_s[:4], G.block_fp8(qa[:4], sa[:4], qw[128:], sw[1:]))
     assert not np.array_equal(y_s[:4], y[:4])
+
+
+def test_grouped_nvfp4_brute_force_with_per_expert_tensor_scales():
+    # 3 experts x N = 4 channels, tokens 0-2 -> expert 0, none -> expert 1,
+    # tokens 3-4 -> expert 2; each y element is summed here token by token,
+    # element by element, with its own expert's block scales and tensor scale
+    a = qg_synth.bf16_matrix(0, 5, 64, 1.0)
+    w = qg_synth.bf16_matrix(1, 12, 64, 0.02)
+    w[8:] = qg_synth.f32_to_bf16_bits(qg_synth.bf16_bits_to_f32(w[8:]) * np.float32(64.0))   # expert 2: other amax
+    qa, sfa, ga = Q.nvfp4(a)
+    qw, sfw, gw = Q.nvfp4_experts(w, 3)
+    offsets = np.array([0, 3, 3, 5])
+    expert_of = [0, 0, 0, 2, 2]
+    ref = np.zeros((5, 4))
+    for t in range(5):
+        e = expert_of[t]
+        for n in range(4):
+            s = 0.0
+            for k in range(64):
+                s += (F.E2M1_TABLE[qa[t, k]] * F.E4M3_TABLE[sfa[t, k // 16]] *
+                      F.E2M1_TABLE[qw[e * 4 + n, k]] * F.E4M3_TABLE[sfw[e * 4 + n, k // 16]])
+            ref[t, n] = s * float(ga) * float(gw[e])
+    y = G.grouped_nvfp4(qa, sfa, ga, qw, sfw, gw, offsets, 4)
+    assert np.array_equal(y, F.bf16_round(ref))
+
+
+def test_nvfp4_experts_scale_each_expert_by_its_own_amax():
+    # expert 1 is expert 0 times 2^5: the same codes and block scales, a
+    # tensor scale 2^5 larger, each tensor scale amax_e / 2688 in fp32
+    # (a single scale over the stack would change expert 0's block scales)
+    w0 = qg_synth.bf16_matrix(3, 16, 64, 0.02)
+    w1 = qg_synth.f32_to_bf16_bits(qg_synth.bf16_bits_to_f32(w0) * np.float32(32.0))
+    q, sf, g = Q.nvfp4_experts(np.concatenate([w0, w1]), 2)
+    assert np.array_equal(q[:16], q[16:]) and np.array_equal(sf[:16], sf[16:])
+    assert g[1] == np.float32(32.0) * g[0]
+    amax0 = np.float32(np.abs(qg_synth.bf16_bits_to_f32(w0)).max())
+    assert g[0] == np.float32(amax0 / np.float32(2688.0))
+    q_all, sf_all, _ = Q.nvfp4(np.concatenate([w0, w1]))
+    assert not np.array_equal(sf_all[:16], sf[:16])
+
+
+def test_grouped_nvfp4_with_one_expert_is_the_plain_gemm():
+    a = qg_synth.bf16_matrix(0, 6, 128, 1.0)
+    w = qg_synth.bf16_matrix(1, 8, 128, 0.02)
+    qa, sfa, ga = Q.nvfp4(a)
+    qw, sfw, gw = Q.nvfp4_experts(w, 1)
+    qw1, sfw1, gw1 = Q.nvfp4(w)
+    assert np.array_equal(qw, qw1) and np.array_equal(sfw, sfw1) and gw[0] == gw1
+    y = G.grouped_nvfp4(qa, sfa, ga, qw, sfw, gw, np.array([0, 6]), 8)
+    assert np.array_equal(y, G.nvfp4(qa, sfa, ga, qw1, sfw1, gw1))
