@@ -475,16 +475,26 @@ def run_ours(args, world, rank, local):
             cfgs[m], hits[m] = qg.qgemm_default_config(FMT_INT8, m, N, K), 0
 
     acts = {m: bf16(qg_synth.activations(m, K)) for m in MS}
-    # one captured step per rotation slot: shape i of step s uses copy (3s+i) % copies
+    # one captured step per rotation slot: shape i of step s uses copy (3s+i) % copies;
+    # a slot's three activations (and results) are views of one buffer, so
+    # that the end-to-end step moves them with one copy each way
     nslots = copies
-    steps_g = []
+    steps_g, slot_in, slot_out = [], [], []
+    rows = sum(MS)
     for s in range(nslots):
         per = []
+        a_all = torch.zeros(rows * K, dtype=torch.bfloat16, device=dev)
+        y_all = torch.empty(rows * N, dtype=torch.bfloat16, device=dev)
+        r0 = 0
         for i, m in enumerate(MS):
-            gs = qg.GraphStep(layer, m, W=Ws[(len(MS) * s + i) % copies], cfg=cfgs[m])
+            gs = qg.GraphStep(layer, m, W=Ws[(len(MS) * s + i) % copies], cfg=cfgs[m],
+                              A=a_all[r0 * K:(r0 + m) * K].view(m, K), Y=y_all[r0 * N:(r0 + m) * N].view(m, N))
             gs.A.copy_(acts[m])
             per.append(gs)
+            r0 += m
         steps_g.append(per)
+        slot_in.append(a_all)
+        slot_out.append(y_all)
     # a single graph per step slot holding the three shapes back to back
     step_graphs = []
     for s in range(nslots):
@@ -601,20 +611,19 @@ def run_ours(args, world, rank, local):
     clk["step_window"] = clk_step
 
     # ---- end to end through the public API with host buffers: per step the
-    # three activations are copied in from pinned host memory, the step's
-    # graph replays, the results are copied out, and the host synchronises.
-    # (Copies captured inside the graph were slower: 113 against 92 us.)
-    host_in = {m: torch.empty(m, K, dtype=torch.bfloat16, pin_memory=True) for m in MS}
-    host_out = {m: torch.empty(m, N, dtype=torch.bfloat16, pin_memory=True) for m in MS}
-    for m in MS:
-        host_in[m].copy_(acts[m].cpu())
+    # three activations are copied in from pinned host memory (one copy: they
+    # are contiguous there and on the device), the step's graph replays, the
+    # results are copied out (one copy), and the host synchronises.
+    # (Copies captured inside the graph were slower: 113 against 92 us with
+    # one copy per shape.)
+    host_in = torch.empty(rows * K, dtype=torch.bfloat16, pin_memory=True)
+    host_out = torch.empty(rows * N, dtype=torch.bfloat16, pin_memory=True)
+    host_in.copy_(torch.cat([acts[m].reshape(-1) for m in MS]).cpu())
 
     def e2e_step(s):
-        for i, m in enumerate(MS):
-            steps_g[s % nslots][i].A.copy_(host_in[m], non_blocking=True)
+        slot_in[s % nslots].copy_(host_in, non_blocking=True)
         step_graphs[s % nslots].replay()
-        for i, m in enumerate(MS):
-            host_out[m].copy_(steps_g[s % nslots][i].Y, non_blocking=True)
+        host_out.copy_(slot_out[s % nslots], non_blocking=True)
         stream.synchronize()
     for s in range(args.warmup):
         e2e_step(s)

@@ -464,6 +464,12 @@ qg_status qgemm_selftest_wait_expiry(unsigned long long limit_ns, void* stream);
 /* Enables (1) or disables (0) programmatic dependent launch for the
  * library's kernels (default 1). */
 void qgemm_set_pdl(int enable);
+/* Enables (1) or disables (0) TMA stores of the output tile (default 1):
+ * launches in the standard orientation (swap_ab = 0) with split_k = 1,
+ * tile_n >= 64 and bf16 output write their tile through a tensor map of y
+ * instead of thread stores (same values, bit for bit).  A switch for
+ * comparison and tests. */
+void qgemm_set_tma_store(int enable);
 /* Tracing (debug): while set, every qgemm_run whose grid fits records, per
  * CTA, 15 GPU-clock timestamps (%globaltimer, ns, 64-bit) into the device
  * buffer: entry, set-up done, first weight tile issued, dependency wait

@@ -45,7 +45,7 @@ EXPORTS = [
     "qgemm_score_config", "qgemm_rank_configs", "qgemm_tune_ranked", "qgemm_table_validate",
     "qgemm_run_grouped", "qgemm_grouped_default_config", "qgemm_set_wait_limit", "qgemm_selftest_wait_expiry",
     "qgemm_set_tune_objective", "qgemm_grouped_act_bytes", "qgemm_quantize_act_grouped",
-    "qgemm_quantize_weight_grouped",
+    "qgemm_quantize_weight_grouped", "qgemm_set_tma_store",
 ]
 
 
@@ -100,6 +100,7 @@ def lib() -> ctypes.CDLL:
         sig = {
             "qgemm_abi_version": (c_int, []),
             "qgemm_set_pdl": (None, [c_int]),
+            "qgemm_set_tma_store": (None, [c_int]),
             "qgemm_status_string": (c_char_p, [c_int]),
             "qgemm_operand_bytes": (c_int, [c_int, c_int, c_int, c_int, POINTER(c_size_t), POINTER(c_size_t)]),
             "qgemm_quant_workspace_size": (c_size_t, [c_int, c_int, c_int]),
@@ -308,6 +309,11 @@ def qgemm_set_tune_objective(gemm_only: bool):
 
 def qgemm_set_pdl(enable: bool):
     lib().qgemm_set_pdl(1 if enable else 0)
+
+
+def qgemm_set_tma_store(enable: bool):
+    """TMA stores of direct standard-orientation output tiles (default on)."""
+    lib().qgemm_set_tma_store(1 if enable else 0)
 
 
 class Table:
@@ -559,10 +565,12 @@ class GraphStep:
     ``host_io=True`` adds pinned host buffers ``A_host`` / ``Y_host`` whose
     copies to and from the device are captured in the same graph: a replay
     then moves the step's input in and its result out with no further call
-    (synchronize the stream before reading ``Y_host``)."""
+    (synchronize the stream before reading ``Y_host``).  ``A`` / ``Y`` may be
+    given: caller-owned contiguous device tensors of those shapes (e.g. views
+    of one buffer shared by several steps, so that one copy fills them all)."""
 
     def __init__(self, layer: "Linear", M: int, W: Operand | None = None, cfg: qg_config | None = None,
-                 fused: bool = False, host_io: bool = False):
+                 fused: bool = False, host_io: bool = False, A=None, Y=None):
         torch = _torch()
         self.fused = fused
         self.host_io = host_io
@@ -571,8 +579,11 @@ class GraphStep:
         self.fmt = layer.fmt
         self.W = W or layer.Wq
         self.cfg = cfg or layer.config(M)
-        self.A = torch.zeros(M, self.K, dtype=torch.bfloat16, device=dev)
-        self.Y = torch.empty(M, self.N, dtype=torch.bfloat16, device=dev)
+        for t, shape in ((A, (M, self.K)), (Y, (M, self.N))):
+            if t is not None and (tuple(t.shape) != shape or t.dtype != torch.bfloat16 or not t.is_contiguous()):
+                raise ValueError(f"GraphStep buffers must be contiguous bf16 {shape}")
+        self.A = A if A is not None else torch.zeros(M, self.K, dtype=torch.bfloat16, device=dev)
+        self.Y = Y if Y is not None else torch.empty(M, self.N, dtype=torch.bfloat16, device=dev)
         self.act = Operand(self.fmt, False, M, self.K, dev)
         self.ws = Workspace(dev)
         self.ws.get(qgemm_workspace_size(self.fmt, M, self.N, self.K, self.cfg))

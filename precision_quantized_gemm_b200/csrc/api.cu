@@ -26,6 +26,7 @@ using qg::GemmParams;
 bool g_pdl = true;
 unsigned long long g_wait_ns = qg::kWaitLimitNs;   // limit of every in-kernel wait
 bool g_l2_ahead = true;                           // Swap-AB weight prefetch for later CTAs
+bool g_tma_store = true;                          // TMA stores of direct standard-orientation tiles
 unsigned long long* g_trace = nullptr;   // debug phase trace buffer (device)
 size_t g_trace_bytes = 0;
 
@@ -108,6 +109,21 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t ro
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The bf16 output y [M, ldy] as a 2D byte tensor of N * 2 bytes per row, read
+// in boxes of 128 rows x 128 bytes (64 channels) with the 128-byte swizzle:
+// the tile-store map of the direct epilogue.
+bool make_tmap_y(CUtensorMap* m, const void* Y, int N, int M, int ldy) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)N * 2, (cuuint64_t)M};
+  cuuint64_t strides[1] = {(cuuint64_t)ldy * 2};
+  cuuint32_t box[2] = {128, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(Y), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -251,6 +267,7 @@ extern "C" {
 int qgemm_abi_version(void) { return QGEMM_ABI_VERSION; }
 
 void qgemm_set_pdl(int enable) { g_pdl = enable != 0; }
+void qgemm_set_tma_store(int enable) { g_tma_store = enable != 0; }
 
 void qgemm_set_trace(void* device_buffer, size_t bytes) {
   g_trace = static_cast<unsigned long long*>(device_buffer);
@@ -581,7 +598,15 @@ qg_status launch_run(qg_format f, const qg_operand* A, const void* act, int lda,
       (size_t)tp * tq * cfg->split_k * qg::kTraceEvents * sizeof(unsigned long long) <= g_trace_bytes)
     prm.trace = g_trace;
 
-  CUtensorMap tmp, tmq;
+  CUtensorMap tmp, tmq, tmy;
+  std::memset(&tmy, 0, sizeof(tmy));
+  // direct standard-orientation tiles of 64 channels or more store bf16
+  // through a tensor map of y (a map that does not encode, e.g. for an
+  // unaligned y, leaves the thread stores)
+  prm.y_tma = 0;
+  if (g_tma_store && !swap && out_kind == 0 && cfg->split_k == 1 && cfg->tile_n >= 64 && act == nullptr &&
+      expert_offsets == nullptr && make_tmap_y(&tmy, Y, N, M, ldy))
+    prm.y_tma = 1;
   const uint64_t rb = row_bytes(f, K);
   // grouped: the P tensor is every expert's weight rows, [experts * N, K]
   const uint64_t p_rows = expert_offsets ? (uint64_t)experts * N : (uint64_t)prm.rows_p;
@@ -617,10 +642,10 @@ qg_status launch_run(qg_format f, const qg_operand* A, const void* act, int lda,
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e;
   switch (f) {
-    case QG_FP8_DYNAMIC: e = qg::launch_gemm_fp8(swap, cfg->tile_n, tmp, tmq, prm, grid, st, g_pdl); break;
-    case QG_W8A8_INT8: e = qg::launch_gemm_int8(swap, cfg->tile_n, tmp, tmq, prm, grid, st, g_pdl); break;
-    case QG_BLOCK_FP8: e = qg::launch_gemm_block(swap, cfg->tile_n, tmp, tmq, prm, grid, st, g_pdl); break;
-    default: e = qg::launch_gemm_nvf4(swap, cfg->tile_n, tmp, tmq, prm, grid, st, g_pdl); break;
+    case QG_FP8_DYNAMIC: e = qg::launch_gemm_fp8(swap, cfg->tile_n, tmp, tmq, tmy, prm, grid, st, g_pdl); break;
+    case QG_W8A8_INT8: e = qg::launch_gemm_int8(swap, cfg->tile_n, tmp, tmq, tmy, prm, grid, st, g_pdl); break;
+    case QG_BLOCK_FP8: e = qg::launch_gemm_block(swap, cfg->tile_n, tmp, tmq, tmy, prm, grid, st, g_pdl); break;
+    default: e = qg::launch_gemm_nvf4(swap, cfg->tile_n, tmp, tmq, tmy, prm, grid, st, g_pdl); break;
   }
   if (e != cudaSuccess) return e == cudaErrorInvalidValue ? QG_ERR_UNSUPPORTED : QG_ERR_CUDA;
   if (cfg->split_k > 1 && cfg->reduce_mode == qg::kReduceSecondPass) {

@@ -110,6 +110,11 @@ struct GemmParams {
   // holds the SMs stream the weights of those that can only start after it,
   // so the HBM stays busy across the kernel boundary.
   int l2_ahead;
+  // Standard orientation, no split, bf16 out, BN >= 64: the epilogue writes
+  // the bf16 tile into the idle ring in boxes of 128 rows x 64 channels with
+  // the 128-byte swizzle and stores them with TMA through the y tensor map
+  // (kernel parameter); 0: 16-byte stores from the threads.
+  int y_tma;
 };
 
 constexpr int kMaxExperts = 256;
@@ -336,6 +341,27 @@ __device__ __forceinline__ void emit(const GemmParams& prm, int r, int c, int m,
       __float2bfloat16_rn(finish_value<FMT>(acc_bits, sa, sw, alpha));
 }
 
+// Scales of the eight consecutive output channels n0 .. n0+7 of tile element
+// (r, c) (FP8_Dynamic, W8A8_INT8): the token's scale sa and the channels'
+// scales sw[0..7], read from the staged copies as two 16-byte vectors when
+// the channel index is a multiple of 8 (it always is in the vector paths).
+template <bool SWAP>
+__device__ __forceinline__ void scales8(const float* row_s, const float* col_s, int r, int c, float& sa,
+                                        float (&sw)[8]) {
+  sa = SWAP ? col_s[c] : row_s[r];
+  const int ch = SWAP ? r : c;
+  const float* s = SWAP ? row_s + r : col_s + c;
+  if ((ch & 7) == 0) {
+    const float4 a = reinterpret_cast<const float4*>(s)[0];
+    const float4 b = reinterpret_cast<const float4*>(s)[1];
+    sw[0] = a.x; sw[1] = a.y; sw[2] = a.z; sw[3] = a.w;
+    sw[4] = b.x; sw[5] = b.y; sw[6] = b.z; sw[7] = b.w;
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) sw[j] = s[j];
+  }
+}
+
 // Grouped launches: the token tile of a CTA.  blockIdx.y enumerates the
 // token tiles of all experts in expert order (ceil(tokens_e / BN) per expert).
 // Lane l owns experts [8 l, 8 l + 8): it sums their tile counts, one warp
@@ -413,7 +439,8 @@ __device__ __forceinline__ void grouped_tile(const GemmParams& prm, int lane, in
 template <int FMT, bool SWAP, int BN, bool FUSED, bool GROUPED>
 __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBlocks)
     qgemm_kernel(const __grid_constant__ CUtensorMap tmap_p,
-                 const __grid_constant__ CUtensorMap tmap_q, const GemmParams prm) {
+                 const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_y,
+                 const GemmParams prm) {
   using C = Cfg<FMT, BN>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -1132,15 +1159,10 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
         return;
       }
       float y8[8];
+      float sa = 1.f, sw[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
+      if constexpr (FMT == kFP8 || FMT == kINT8) scales8<SWAP>(row_s, col_s, r, c, sa, sw);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        float sa = 1.f, sw = 1.f;
-        if constexpr (FMT == kFP8 || FMT == kINT8) {
-          sa = SWAP ? col_s[c] : row_s[r];
-          sw = SWAP ? row_s[r + j] : col_s[c + j];
-        }
-        y8[j] = finish_value<FMT>(acc8[j], sa, sw, alpha);
-      }
+      for (int j = 0; j < 8; ++j) y8[j] = finish_value<FMT>(acc8[j], sa, sw[j], alpha);
       __nv_bfloat16* Yb = reinterpret_cast<__nv_bfloat16*>(prm.Y) + (size_t)m * prm.ldy;
       if (vec && n0 + 8 <= prm.N) {
         uint32_t p[4];
@@ -1154,26 +1176,113 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
         for (int j = 0; j < 8 && n0 + j < prm.N; ++j) Yb[n0 + j] = __float2bfloat16_rn(y8[j]);
       }
     };
+    // A thread takes kUB units per round: their shared-memory reads are all
+    // issued before the first unit is scaled and stored, so that one warp
+    // per TMEM quarter keeps several units in flight.
     auto write_out = [&](int r_begin, int r_count, int c_begin, int c_count) {
-      const int units = SWAP ? c_count * (r_count / 8) : r_count * (c_count / 8);
+      constexpr int kUB = C::kMinBlocks >= 3 ? 2 : 4;
+      const int per = SWAP ? r_count / 8 : c_count / 8;          // units per tile column / row
+      const int units = SWAP ? c_count * per : r_count * per;
 #pragma unroll 1
-      for (int u = etid; u < units; u += ET) {
-        int r, c;                              // first of 8 consecutive output channels
-        if (SWAP) { c = c_begin + u / (r_count / 8); r = r_begin + (u % (r_count / 8)) * 8; }
-        else      { r = r_begin + u / (c_count / 8); c = c_begin + (u % (c_count / 8)) * 8; }
-        const int m = SWAP ? q0 + c : p0 + r;
-        const int n0 = SWAP ? p0 + r : q0 + c;
-        if (m >= Mlim || n0 >= prm.N) continue;
-        const uint4* src = reinterpret_cast<const uint4*>(otile + tile_index<SWAP, BN>(r, c));
-        const uint4 w0 = src[0], w1 = src[1];
-        const uint32_t acc8[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-        store8(r, c, m, n0, acc8);
+      for (int u0 = etid; u0 < units; u0 += kUB * ET) {
+        uint32_t acc8[kUB][8];
+        int rr[kUB], cc[kUB];                  // first of 8 consecutive output channels
+#pragma unroll
+        for (int k = 0; k < kUB; ++k) {
+          const int u = min(u0 + k * ET, units - 1);               // past the end: re-read, never stored
+          if (SWAP) { cc[k] = c_begin + u / per; rr[k] = r_begin + (u % per) * 8; }
+          else      { rr[k] = r_begin + u / per; cc[k] = c_begin + (u % per) * 8; }
+          const uint4* src = reinterpret_cast<const uint4*>(otile + tile_index<SWAP, BN>(rr[k], cc[k]));
+          const uint4 w0 = src[0], w1 = src[1];
+          acc8[k][0] = w0.x; acc8[k][1] = w0.y; acc8[k][2] = w0.z; acc8[k][3] = w0.w;
+          acc8[k][4] = w1.x; acc8[k][5] = w1.y; acc8[k][6] = w1.z; acc8[k][7] = w1.w;
+        }
+#pragma unroll
+        for (int k = 0; k < kUB; ++k) {
+          if (u0 + k * ET >= units) break;
+          const int m = SWAP ? q0 + cc[k] : p0 + rr[k];
+          const int n0 = SWAP ? p0 + rr[k] : q0 + cc[k];
+          if (m < Mlim && n0 < prm.N) store8(rr[k], cc[k], m, n0, acc8[k]);
+        }
       }
     };
 
-    if (!split) {
+    bool tma_out = false;                      // the tile went out through the y tensor map
+    if constexpr (!SWAP && BN >= 64) {
+      if (!split && prm.y_tma && epi_ok) {
+        // ---- direct, TMA store: each thread scales, rounds and writes its
+        // row's channels into 64-channel boxes of 128 rows x 128 bytes (the
+        // ring is idle: every MMA has completed); 16-byte chunk k of row r
+        // of a box sits at chunk k ^ (r % 8), the TMA 128-byte swizzle, so a
+        // quarter warp's eight rows hit eight different bank groups.
+        uint8_t* ybuf = smem + L.p;
+        float sa = 1.f;
+        if constexpr (FMT == kFP8 || FMT == kINT8) sa = row_s[row];
+#pragma unroll
+        for (int c0 = 0; c0 < NC; c0 += CW) {
+          uint32_t v[CW];
+          load_chunk(c0, v);
+#pragma unroll
+          for (int j = 0; j < CW; j += 8) {
+            const int col = cbeg + c0 + j;     // a multiple of 8
+            float sw[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
+            if constexpr (FMT == kFP8 || FMT == kINT8) {
+              const float4 a = reinterpret_cast<const float4*>(col_s + col)[0];
+              const float4 b = reinterpret_cast<const float4*>(col_s + col)[1];
+              sw[0] = a.x; sw[1] = a.y; sw[2] = a.z; sw[3] = a.w;
+              sw[4] = b.x; sw[5] = b.y; sw[6] = b.z; sw[7] = b.w;
+            }
+            uint32_t pk[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const __nv_bfloat162 b2 =
+                  __floats2bfloat162_rn(finish_value<FMT>(v[j + 2 * h], sa, sw[2 * h], alpha),
+                                        finish_value<FMT>(v[j + 2 * h + 1], sa, sw[2 * h + 1], alpha));
+              pk[h] = *reinterpret_cast<const uint32_t*>(&b2);
+            }
+            const uint32_t off = (uint32_t)(col >> 6) * 16384u + (uint32_t)row * 128u +
+                                 ((uint32_t)(((col & 63) >> 3) ^ (row & 7)) << 4);
+            *reinterpret_cast<uint4*>(ybuf + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, ET);
+        if (etid == 0) {
+#pragma unroll
+          for (int b = 0; b < BN / 64; ++b) tma_store_2d(&tmap_y, ybuf + b * 16384, (q0 + b * 64) * 2, p0);
+          bulk_commit();
+          bulk_wait_all();
+        }
+        tma_out = true;
+      }
+    }
+    if (tma_out) {
+    } else if (!split) {
       // ---- direct: accumulator -> tile -> y
-      if (epi_ok) {
+      if constexpr (!C::kBlock && !SWAP && CW == 32 && NC >= 128) {
+        // wide rows: the next 32 columns' TMEM load is in flight while this
+        // chunk goes to the tile
+        if (epi_ok) {
+          auto put = [&](int c0, const uint32_t (&v)[32]) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+              *reinterpret_cast<uint4*>(otile + tile_index<SWAP, BN>(row, cbeg + c0 + j)) =
+                  make_uint4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+          };
+          uint32_t va[32], vb[32];
+          tmem_ld32(lane_addr + cbeg, va);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c0 = 0; c0 < NC; c0 += 64) {
+            tmem_ld32(lane_addr + cbeg + c0 + 32, vb);
+            put(c0, va);
+            tmem_ld_wait();
+            if (c0 + 64 < NC) tmem_ld32(lane_addr + cbeg + c0 + 64, va);
+            put(c0 + 32, vb);
+            if (c0 + 64 < NC) tmem_ld_wait();
+          }
+        }
+      } else if (epi_ok) {
 #pragma unroll
         for (int c0 = 0; c0 < NC; c0 += CW) {
           uint32_t v[CW];
@@ -1417,15 +1526,10 @@ __global__ void __launch_bounds__(Cfg<FMT, BN>::kThreads, Cfg<FMT, BN>::kMinBloc
             return;
           }
           float y8[8];
+          float sa = 1.f, sw[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
+          if constexpr (FMT == kFP8 || FMT == kINT8) scales8<SWAP>(row_s, col_s, r, c, sa, sw);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            float sa = 1.f, sw = 1.f;
-            if constexpr (FMT == kFP8 || FMT == kINT8) {
-              sa = SWAP ? col_s[c] : row_s[r];
-              sw = SWAP ? row_s[r + j] : col_s[c + j];
-            }
-            y8[j] = finish_value<FMT>(acc8[j], sa, sw, alpha);
-          }
+          for (int j = 0; j < 8; ++j) y8[j] = finish_value<FMT>(acc8[j], sa, sw[j], alpha);
           __nv_bfloat16* Yb = reinterpret_cast<__nv_bfloat16*>(prm.Y) + (size_t)m * prm.ldy;
           if (vec && n0 + 8 <= prm.N) {
             uint32_t pk[4];

@@ -17,7 +17,8 @@ namespace qg {
 namespace {
 
 template <int FMT, bool SWAP, int BN, bool FUSED, bool GROUPED>
-cudaError_t launch_one(const CUtensorMap& tp, const CUtensorMap& tq, const GemmParams& prm,
+cudaError_t launch_one(const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap& ty,
+                       const GemmParams& prm,
                        dim3 grid, cudaStream_t st, bool pdl) {
   auto kern = qgemm_kernel<FMT, SWAP, BN, FUSED, GROUPED>;
   const int act_tiles = FUSED ? prm.nkt_max : 0;
@@ -62,18 +63,19 @@ cudaError_t launch_one(const CUtensorMap& tp, const CUtensorMap& tq, const GemmP
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, kern, tp, tq, prm);
+  return cudaLaunchKernelEx(&cfg, kern, tp, tq, ty, prm);
 }
 
 template <int FMT, bool SWAP, bool FUSED, bool GROUPED = false>
-cudaError_t launch_bn(int bn, const CUtensorMap& tp, const CUtensorMap& tq, const GemmParams& prm,
+cudaError_t launch_bn(int bn, const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap& ty,
+                      const GemmParams& prm,
                       dim3 grid, cudaStream_t st, bool pdl) {
   switch (bn) {
-    case 16: return launch_one<FMT, SWAP, 16, FUSED, GROUPED>(tp, tq, prm, grid, st, pdl);
-    case 32: return launch_one<FMT, SWAP, 32, FUSED, GROUPED>(tp, tq, prm, grid, st, pdl);
-    case 64: return launch_one<FMT, SWAP, 64, FUSED, GROUPED>(tp, tq, prm, grid, st, pdl);
-    case 128: return launch_one<FMT, SWAP, 128, FUSED, GROUPED>(tp, tq, prm, grid, st, pdl);
-    case 256: return launch_one<FMT, SWAP, 256, FUSED, GROUPED>(tp, tq, prm, grid, st, pdl);
+    case 16: return launch_one<FMT, SWAP, 16, FUSED, GROUPED>(tp, tq, ty, prm, grid, st, pdl);
+    case 32: return launch_one<FMT, SWAP, 32, FUSED, GROUPED>(tp, tq, ty, prm, grid, st, pdl);
+    case 64: return launch_one<FMT, SWAP, 64, FUSED, GROUPED>(tp, tq, ty, prm, grid, st, pdl);
+    case 128: return launch_one<FMT, SWAP, 128, FUSED, GROUPED>(tp, tq, ty, prm, grid, st, pdl);
+    case 256: return launch_one<FMT, SWAP, 256, FUSED, GROUPED>(tp, tq, ty, prm, grid, st, pdl);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -182,8 +184,9 @@ size_t skinny_smem_rows(int rows, int stages) {
 #if !defined(QG_GROUPED_OWN_UNIT) || defined(QG_GROUPED_ONLY)
 // grouped (mixture-of-experts) launch: Swap-AB, activations by TMA
 cudaError_t QG_CAT(QG_LAUNCH_NAME, _grouped)(int tile_n, const CUtensorMap& tp, const CUtensorMap& tq,
+                                             const CUtensorMap& ty,
                                              const GemmParams& prm, dim3 grid, cudaStream_t st, bool pdl) {
-  return launch_bn<QG_FMT, true, false, true>(tile_n, tp, tq, prm, grid, st, pdl);
+  return launch_bn<QG_FMT, true, false, true>(tile_n, tp, tq, ty, prm, grid, st, pdl);
 }
 #endif
 
@@ -212,20 +215,21 @@ size_t QG_CAT(QG_LAUNCH_NAME, _skinny_smem)(int tile_n, int rows, int stages) {
 }
 
 cudaError_t QG_LAUNCH_NAME(bool swap, int tile_n, const CUtensorMap& tp, const CUtensorMap& tq,
+                           const CUtensorMap& ty,
                            const GemmParams& prm, dim3 grid, cudaStream_t st, bool pdl) {
   if (prm.expert_offsets != nullptr) {
-    if (swap && prm.a_mode == kActTma) return QG_CAT(QG_LAUNCH_NAME, _grouped)(tile_n, tp, tq, prm, grid, st, pdl);
+    if (swap && prm.a_mode == kActTma) return QG_CAT(QG_LAUNCH_NAME, _grouped)(tile_n, tp, tq, ty, prm, grid, st, pdl);
     return cudaErrorInvalidValue;
   }
   if (prm.a_mode == kActFused) {
     // fused activation quantisation: Swap-AB, 8-bit formats only
     if constexpr (QG_FMT != kNVF4) {
-      if (swap) return launch_bn<QG_FMT, true, true>(tile_n, tp, tq, prm, grid, st, pdl);
+      if (swap) return launch_bn<QG_FMT, true, true>(tile_n, tp, tq, ty, prm, grid, st, pdl);
     }
     return cudaErrorInvalidValue;
   }
-  return swap ? launch_bn<QG_FMT, true, false>(tile_n, tp, tq, prm, grid, st, pdl)
-              : launch_bn<QG_FMT, false, false>(tile_n, tp, tq, prm, grid, st, pdl);
+  return swap ? launch_bn<QG_FMT, true, false>(tile_n, tp, tq, ty, prm, grid, st, pdl)
+              : launch_bn<QG_FMT, false, false>(tile_n, tp, tq, ty, prm, grid, st, pdl);
 }
 
 size_t QG_CAT(QG_LAUNCH_NAME, _smem)(int tile_n, bool swap, int stages, int nkt_max, int recv_cols,

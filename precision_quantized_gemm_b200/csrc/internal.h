@@ -47,12 +47,14 @@ cudaError_t launch_quant_nvfp4(const void* X, int R, int K, int ldx, const float
 // Returns cudaErrorInvalidValue for a (swap, tile_n) pair not instantiated.
 #define QG_DECLARE_GEMM_LAUNCH(NAME)                                                      \
   cudaError_t NAME(bool swap, int tile_n, const CUtensorMap& tp, const CUtensorMap& tq,    \
+                   const CUtensorMap& ty,                                                  \
                    const GemmParams& prm, dim3 grid, cudaStream_t st, bool pdl);           \
   size_t NAME##_smem(int tile_n, bool swap, int stages, int nkt_max, int recv_cols,        \
                      int act_tiles);                                                       \
   bool NAME##_cluster_fits(int tile_n, bool swap, int stages, int act_tiles);              \
   cudaError_t NAME##_reduce(const GemmParams& prm, cudaStream_t st, bool pdl);             \
   cudaError_t NAME##_grouped(int tile_n, const CUtensorMap& tp, const CUtensorMap& tq,     \
+                             const CUtensorMap& ty,                                        \
                              const GemmParams& prm, dim3 grid, cudaStream_t st, bool pdl); \
   cudaError_t NAME##_skinny(int tile_n, int rows, const CUtensorMap& tw, const CUtensorMap& ta, \
                             const GemmParams& prm, dim3 grid, cudaStream_t st, bool pdl);     \
