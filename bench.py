@@ -135,17 +135,17 @@ def kernel_source_hash():
     return h.hexdigest()[:12]
 
 
-def measured_traffic():
-    """DRAM bytes per GEMM launch of this workload (read + write, averaged over its
-    three shapes) from the committed ncu summary, or None when the kernel has
-    changed since it was captured."""
+def measured_traffic(key="w8a8_int8_decode_dram_bytes_per_launch"):
+    """DRAM bytes per GEMM launch (read + write) recorded under `key` in the
+    committed ncu summary (default: this workload, averaged over its three
+    shapes), or None when the kernels have changed since the capture."""
     p = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(p):
         return None
     kv = dict(line.split(None, 1) for line in open(p) if line.strip() and not line.startswith("#"))
-    if kv.get("kernel_sources", "").strip() != kernel_source_hash():
+    if kv.get("kernel_sources", "").strip() != kernel_source_hash() or key not in kv:
         return None
-    return float(kv["w8a8_int8_decode_dram_bytes_per_launch"])
+    return float(kv[key])
 
 
 # ------------------------------------------------------------- clocks ---
@@ -604,6 +604,9 @@ def run_ours(args, world, rank, local):
     if world == 1 and not args.no_suite:
         fam_results, fam_peaks = time_families(HEADLINE_FAMILIES, dev, table)
         fam = dict(summarise_families(fam_results), peaks=fam_peaks,
+                   block_fp8_m4096_traffic={"dram_bytes_per_launch": measured_traffic("block_fp8_m4096_dram_bytes_per_launch"),
+                                            "algorithmic_bytes": shape_bytes(2, 4096, 5120, 5120),
+                                            "source": "profiles/traffic.txt (ncu, hash-gated)"},
                    per_shape=[[r["format"], r["M"], r["N"], r["K"], r["us"], r["frac_roofline"], r["bound"]]
                               for r in fam_results])
     clk_step = clocks.window(t_load, t_step_end)
