@@ -94,14 +94,12 @@ typedef struct {
   int32_t variant;     /* 0: the tile kernel (tcgen05, the fields above);
                           1: the decode ("skinny") kernel for FP8_DYNAMIC,
                           W8A8_INT8 and BLOCK_FP8: warp-level MMAs with register
-                          accumulators, each CTA owning `rows` weight rows and
-                          tile_n (8, 16 or 32) tokens over its K slice;
-                          requires swap_ab = 1, reduce_mode = 0, split_k 1, 2,
-                          4 or 8 (the split_k CTAs of a tile form a cluster and
-                          sum their slices through distributed shared memory in
-                          slice order), and `stages` (the ring of 128-byte K
-                          tiles, 2..64) a multiple of the K groups of its eight
-                          compute warps: 64 / rows (128 / rows for tile_n = 8) */
+                          accumulators, each CTA owning `rows` weight rows over
+                          the whole of K and tile_n (8, 16 or 32) tokens;
+                          requires split_k = 1, swap_ab = 1, reduce_mode = 0,
+                          and `stages` (the ring of 128-byte K tiles, 2..64) a
+                          multiple of the K groups of its eight compute warps:
+                          64 / rows (128 / rows for tile_n = 8)                */
   int32_t rows;        /* variant 1: weight rows per CTA, 8, 16, 32 or 64 (at
                           least 16 for tile_n = 8); variant 0: must be 0        */
   int32_t reserved;    /* must be zero                                            */

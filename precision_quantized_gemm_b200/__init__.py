@@ -69,12 +69,10 @@ def make_config(split_k=1, swap_ab=1, tile_n=16, stages=8, reduce_mode=0, varian
     return c
 
 
-def skinny_config(tile_n=16, rows=32, stages=32, split_k=1) -> qg_config:
+def skinny_config(tile_n=16, rows=32, stages=32) -> qg_config:
     """Configuration of the decode ("skinny") kernel: `rows` weight rows per
-    CTA, `tile_n` tokens, a ring of `stages` K tiles; `split_k` (1, 2, 4, 8)
-    CTAs of a cluster share K."""
-    return make_config(split_k=split_k, swap_ab=1, tile_n=tile_n, stages=stages, reduce_mode=0, variant=1,
-                       rows=rows)
+    CTA over the whole of K, `tile_n` tokens, a ring of `stages` K tiles."""
+    return make_config(split_k=1, swap_ab=1, tile_n=tile_n, stages=stages, reduce_mode=0, variant=1, rows=rows)
 
 
 class qg_operand(ctypes.Structure):

@@ -212,14 +212,12 @@ qg_status check_launch_fit(qg_format f, int M, int K, const qg_config* c, bool f
   return QG_OK;
 }
 
-// The decode ("skinny") kernel: warp-level MMAs; split-K only through a
-// cluster (split_k 1, 2, 4 or 8 CTAs along z, at most one per K tile); the
-// eight compute warps form 64 / rows K groups (128 / rows for tile_n = 8) that
-// take every K-group-th K tile, so the ring depth is a multiple of that.
-qg_status check_skinny_config(qg_format f, int K, const qg_config* c) {
+// The decode ("skinny") kernel: warp-level MMAs, no split-K; the eight
+// compute warps form 64 / rows K groups (128 / rows for tile_n = 8) that take
+// every K-group-th K tile, so the ring depth is a multiple of that.
+qg_status check_skinny_config(qg_format f, const qg_config* c) {
   if (f == QG_NVFP4) return QG_ERR_UNSUPPORTED;
-  if (c->swap_ab != 1 || c->reduce_mode != 0) return QG_ERR_UNSUPPORTED;
-  if (!is_pow2(c->split_k) || c->split_k > 8 || c->split_k > kt_total(f, K)) return QG_ERR_UNSUPPORTED;
+  if (c->split_k != 1 || c->swap_ab != 1 || c->reduce_mode != 0) return QG_ERR_UNSUPPORTED;
   if (c->tile_n != 8 && c->tile_n != 16 && c->tile_n != 32) return QG_ERR_UNSUPPORTED;
   if (c->rows != 8 && c->rows != 16 && c->rows != 32 && c->rows != 64) return QG_ERR_UNSUPPORTED;
   // tile_n = 8: a warp owns 16 weight rows (weights as the 16-row operand)
@@ -234,7 +232,7 @@ qg_status check_config(qg_format f, int M, int N, int K, const qg_config* c) {
   if (!c) return QG_ERR_INVALID_ARG;
   if (c->reserved) return QG_ERR_INVALID_ARG;
   if (c->variant != 0 && c->variant != 1) return QG_ERR_INVALID_ARG;
-  if (c->variant == 1) return check_skinny_config(f, K, c);
+  if (c->variant == 1) return check_skinny_config(f, c);
   if (c->rows != 0) return QG_ERR_INVALID_ARG;
   if (!is_pow2(c->split_k) || c->split_k > 256) return QG_ERR_UNSUPPORTED;
   if (c->swap_ab != 0 && c->swap_ab != 1) return QG_ERR_INVALID_ARG;
@@ -555,22 +553,22 @@ qg_status launch_run(qg_format f, const qg_operand* A, const void* act, int lda,
   int tp, tq;
   tiles_of(cfg, M, N, &tp, &tq);
   if (cfg->variant == 1) {
-    // decode kernel: CTA (x, y, z) = weight rows [x rows, (x + 1) rows) x
-    // tokens [y tile_n, (y + 1) tile_n) x split-K slice z
+    // decode kernel: CTA (x, y) = weight rows [x rows, (x + 1) rows) x
+    // tokens [y tile_n, (y + 1) tile_n), the whole of K
     prm.nkt_max = prm.kt_total;
     prm.err = d->err;
     prm.wait_ns = g_wait_ns;
     const int gx = (N + cfg->rows - 1) / cfg->rows, gy = (M + cfg->tile_n - 1) / cfg->tile_n;
     if (gy > 65535) return QG_ERR_UNSUPPORTED;
     if (g_trace != nullptr &&
-        (size_t)gx * gy * cfg->split_k * qg::kTraceEvents * sizeof(unsigned long long) <= g_trace_bytes)
+        (size_t)gx * gy * qg::kTraceEvents * sizeof(unsigned long long) <= g_trace_bytes)
       prm.trace = g_trace;
-    if (g_l2_ahead && cfg->split_k == 1) prm.l2_ahead = (gx * gy + 1) / 2;
+    if (g_l2_ahead) prm.l2_ahead = (gx * gy + 1) / 2;
     CUtensorMap tw, ta;
     const uint64_t rb = row_bytes(f, K);
     if (!make_tmap(&tw, W->q, rb, (uint64_t)N, (uint32_t)cfg->rows)) return QG_ERR_CUDA;
     if (!make_tmap(&ta, A->q, rb, (uint64_t)M, (uint32_t)cfg->tile_n)) return QG_ERR_CUDA;
-    const dim3 grid(gx, gy, cfg->split_k);
+    const dim3 grid(gx, gy, 1);
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e;
     switch (f) {

@@ -200,11 +200,6 @@ __device__ __forceinline__ void st_async_v4(uint32_t dst_cluster, uint32_t a, ui
                "r"(a), "r"(b), "r"(c), "r"(d), "r"(bar_cluster)
                : "memory");
 }
-__device__ __forceinline__ uint32_t ld_dsmem_b32(uint32_t caddr) {
-  uint32_t v;
-  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(caddr) : "memory");
-  return v;
-}
 __device__ __forceinline__ uint4 ld_dsmem_v4(uint32_t caddr) {
   uint4 v;
   asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"

@@ -56,7 +56,6 @@ struct Model {
   double s_tile = 300.0;
   double s_cta_gbs = 45.0;
   double s_chain = 2.3;
-  double s_cluster = 0.6;    // decode kernel split-K: the cluster barriers and remote sums, µs
 };
 const Model kModel;
 
@@ -81,19 +80,19 @@ int ctas_per_sm(qg_format f, int M, int K, const qg_config& c) {
   return std::max(1, std::min(std::min(regcap, tmemcap), smemcap));
 }
 
-// The decode kernel: ceil(N / rows) x ceil(M / tile_n) x split_k CTAs, each
-// streaming its rows (and tokens) over its K slice through its ring; eight
-// compute warps in K groups each take a share of the K tiles.  Calibrated on
+// The decode kernel: ceil(N / rows) x ceil(M / tile_n) CTAs, each streaming
+// its rows (and tokens) over the whole of K through its ring; eight compute
+// warps in K groups each take a share of the K tiles.  Calibrated on
 // measured launches of this kernel (per-shape sweeps on one B200): a fixed
 // chain of ~2.3 us (dependency release, activation tiles, the K-group sum,
 // the stores), then the slice streaming at ~45 GB/s per CTA (shared when two
 // CTAs sit on an SM), or the warps' MMA loop, whichever is longer, and never
-// faster than the weights over HBM; split-K adds the cluster exchange.
+// faster than the weights over HBM.
 double estimate_skinny_us(qg_format f, int M, int N, int K, const qg_config& c, int sms) {
   const Model& m = kModel;
   const double rb = (double)K;
-  const int kt = (int)((rb + 127) / 128 + c.split_k - 1) / c.split_k;   // K tiles per CTA
-  const double ctas = (double)((N + c.rows - 1) / c.rows) * ((M + c.tile_n - 1) / c.tile_n) * c.split_k;
+  const int kt = (int)((rb + 127) / 128);
+  const double ctas = (double)((N + c.rows - 1) / c.rows) * ((M + c.tile_n - 1) / c.tile_n);
   const size_t smem = qg::config_smem(f, M, K, &c);
   const int cps = std::max(1, std::min(2, (int)(kSmemPerSm / (smem + 1024))));
   const double waves = std::ceil(ctas / ((double)sms * cps));
@@ -102,7 +101,7 @@ double estimate_skinny_us(qg_format f, int M, int N, int K, const qg_config& c, 
   const int kg = (c.tile_n == 8 ? 128 : 64) / c.rows;
   const double t_mma = std::ceil((double)kt / kg) * m.s_tile * std::max(1, c.tile_n / 16) / m.clock_mhz;
   const double body = std::max((double)N * rb / (m.hbm_gbs * 1e3), waves * std::max(t_stream, t_mma));
-  return m.s_chain + body + (c.split_k > 1 ? m.s_cluster : 0.0);
+  return m.s_chain + body;
 }
 
 double estimate_us(qg_format f, int M, int N, int K, const qg_config& c, int sms) {
@@ -147,6 +146,7 @@ namespace qg {
 // Swap-AB tiles no wider than twice the token count, standard tiles for at
 // least 64 tokens, rings of 3, 4, 6 or 8 stages, every reduction mode.
 void candidate_grid(qg_format f, int M, int N, int K, qg_config* out, int max_out, int* n_out) {
+  (void)N;
   const int kt = (int)(((f == QG_NVFP4 ? K / 2 : K) + 127) / 128);
   const int tiles_swap[] = {16, 32, 64, 128, 256};
   const int tiles_std[] = {256, 128, 64};
@@ -176,9 +176,8 @@ void candidate_grid(qg_format f, int M, int N, int K, qg_config* out, int max_ou
     }
   }
   // the decode kernel (8-bit formats, up to 32 tokens per CTA): rows per
-  // CTA, cluster split-K (2, 4, 8) while the unsplit grid has fewer CTAs than
-  // SMs, and rings of 8, 16, 32 or every K tile of the slice (up to 64)
-  // rounded to the K groups
+  // CTA, and rings of 8, 16, 32 or every K tile (up to 64) rounded to the K
+  // groups
   if (f != QG_NVFP4 && M <= 64) {
     const int rows_opts[] = {8, 16, 32, 64};
     const int ring_opts[] = {8, 16, 32, 64};
@@ -187,20 +186,16 @@ void candidate_grid(qg_format f, int M, int N, int K, qg_config* out, int max_ou
       for (int r : rows_opts) {
         if (tm == 8 && r < 16) continue;
         const int kg = (tm == 8 ? 128 : 64) / r;
-        const long long ctas = (long long)((N + r - 1) / r) * ((M + tm - 1) / tm);
-        for (int sk = 1; sk <= 8 && sk <= kt; sk *= 2) {
-        if (sk > 1 && ctas >= 148) break;
-        const int kts = (kt + sk - 1) / sk;       // K tiles of a slice
         int prev = 0;
         for (int ro : ring_opts) {
-          int st = std::min(ro, ((kts + kg - 1) / kg) * kg);
+          int st = std::min(ro, ((kt + kg - 1) / kg) * kg);
           st = std::max(kg, (st / kg) * kg);
           if (st < 2) st = 2 * kg > 64 ? kg : 2 * kg;
           if (st == prev) continue;
           prev = st;
           if (n < max_out) {
             qg_config c = {};
-            c.split_k = sk;
+            c.split_k = 1;
             c.swap_ab = 1;
             c.tile_n = tm;
             c.stages = st;
@@ -210,7 +205,6 @@ void candidate_grid(qg_format f, int M, int N, int K, qg_config* out, int max_ou
             out[n] = c;
           }
           ++n;
-        }
         }
       }
     }

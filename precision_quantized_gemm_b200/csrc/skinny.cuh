@@ -27,13 +27,6 @@
 // acc += p_g * (s_a * s_w).  The K groups of warps then meet in shared memory
 // and are summed in K-group order (deterministic); the epilogue applies the
 // scales in fp32 and stores bf16, 8 channels per 16-byte store.
-// Split-K (few weight rows, long K): the split_k CTAs z of one (x, y) form a
-// thread-block cluster along z and take K tiles [z kt / split_k, (z + 1) kt /
-// split_k); each CTA sums its K groups per output unit into a compact
-// partial, the CTAs meet at a cluster barrier, and CTA r of the cluster
-// finishes every split_k-th unit, reading each CTA's partial of it through
-// distributed shared memory (two 16-byte loads per CTA, all in flight
-// together) and adding them in z order.
 #pragma once
 #include <type_traits>
 
@@ -63,13 +56,11 @@ struct SkCfg {
 };
 
 // Shared memory of a skinny launch: the ring, one full and one empty barrier
-// per slot, the K-group reduction area, the CTA's completion word (16 bytes)
-// and its per-unit partials (split-K: TM x NF units of 8 words) (+ alignment
-// slack).
+// per slot, the K-group reduction area (+ alignment slack).
 template <int FMT, int TM, int NF>
 __host__ __device__ constexpr size_t skinny_smem_bytes(int stages) {
   using C = SkCfg<FMT, TM, NF>;
-  return (size_t)stages * C::kStage + 16u * (size_t)stages + (size_t)C::kRedBytes + 16 + 32u * TM * NF + 1024;
+  return (size_t)stages * C::kStage + 16u * (size_t)stages + (size_t)C::kRedBytes + 1024;
 }
 
 template <int FMT, int TM, int NF>
@@ -86,16 +77,11 @@ __global__ void __launch_bounds__(SkCfg<FMT, TM, NF>::kThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * C::kStage);
   uint64_t* empty = full + S;
   Acc* red = reinterpret_cast<Acc*>(empty + S);   // [warp][mf][16 tokens][8 rows]
-  int* done_ok = reinterpret_cast<int*>(red + C::kRedBytes / 4);   // split-K: this CTA's waits all completed
-  Acc* part = red + C::kRedBytes / 4 + 4;        // split-K: [unit][8] K-group sums of this CTA
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * C::kR;
   const int m0 = blockIdx.y * TM;
-  // split-K slice of this CTA (split_k a power of two; 1: all of K)
-  const int Sk = prm.split_k;
-  const int kt_begin = (int)(((long long)blockIdx.z * prm.kt_total) >> (__ffs(Sk) - 1));
-  const int nkt = (int)(((long long)(blockIdx.z + 1) * prm.kt_total) >> (__ffs(Sk) - 1)) - kt_begin;
+  const int nkt = prm.kt_total;
   bool ok = true;                              // this thread's waits all completed
   if (threadIdx.x == 0) trace_at(prm, kTrEntry);
 
@@ -122,7 +108,7 @@ __global__ void __launch_bounds__(SkCfg<FMT, TM, NF>::kThreads, 1)
       const int pre = nkt < S ? nkt : S;
       for (int i = 0; i < pre; ++i) {
         mbar_arrive_expect_tx(&full[i], C::kStage);
-        tma_load_2d(smem + (size_t)i * C::kStage, &tmap_w, &full[i], (kt_begin + i) * kKTileBytes, n0, pol_w);
+        tma_load_2d(smem + (size_t)i * C::kStage, &tmap_w, &full[i], i * kKTileBytes, n0, pol_w);
         if (i == 0) trace_at(prm, kTrFirstLoad);
       }
       if (prm.l2_ahead > 0) {
@@ -130,14 +116,13 @@ __global__ void __launch_bounds__(SkCfg<FMT, TM, NF>::kThreads, 1)
         const long long t = (long long)blockIdx.x + (long long)gridDim.x * blockIdx.y + prm.l2_ahead;
         if (t < (long long)gridDim.x * gridDim.y) {
           const int tn0 = (int)(t % gridDim.x) * C::kR;
-          for (int kt = 0; kt < nkt; ++kt) tma_prefetch_l2_2d(&tmap_w, (kt_begin + kt) * kKTileBytes, tn0);
+          for (int kt = 0; kt < nkt; ++kt) tma_prefetch_l2_2d(&tmap_w, kt * kKTileBytes, tn0);
         }
       }
       griddep_wait();                          // activations come from the preceding kernel
       trace_at(prm, kTrDepWait);
       for (int i = 0; i < pre; ++i)
-        tma_load_2d(smem + (size_t)i * C::kStage + C::kWTile, &tmap_a, &full[i], (kt_begin + i) * kKTileBytes, m0,
-                    pol_a);
+        tma_load_2d(smem + (size_t)i * C::kStage + C::kWTile, &tmap_a, &full[i], i * kKTileBytes, m0, pol_a);
       int issued = pre;
       int st = 0;                              // slot of K tile i; parity of its previous use
       uint32_t ph = 0;
@@ -145,8 +130,8 @@ __global__ void __launch_bounds__(SkCfg<FMT, TM, NF>::kThreads, 1)
         if (!mbar_wait(&empty[st], ph, prm.err, prm.wait_ns)) { ok = false; break; }
         mbar_arrive_expect_tx(&full[st], C::kStage);
         uint8_t* dst = smem + (size_t)st * C::kStage;
-        tma_load_2d(dst, &tmap_w, &full[st], (kt_begin + i) * kKTileBytes, n0, pol_w);
-        tma_load_2d(dst + C::kWTile, &tmap_a, &full[st], (kt_begin + i) * kKTileBytes, m0, pol_a);
+        tma_load_2d(dst, &tmap_w, &full[st], i * kKTileBytes, n0, pol_w);
+        tma_load_2d(dst + C::kWTile, &tmap_a, &full[st], i * kKTileBytes, m0, pol_a);
         issued = i + 1;
         if (++st == S) { st = 0; ph ^= 1u; }
       }
@@ -187,15 +172,15 @@ __global__ void __launch_bounds__(SkCfg<FMT, TM, NF>::kThreads, 1)
       // Block_FP8: this group's scales, loaded while the tile may still be in flight
       float sw = 0.f, sa_lo[C::kMF], sa_hi[C::kMF];
       if constexpr (FMT == kBLOCK) {
-        sw = __ldg(prm.scale_w + (size_t)(n0 / 128) * G + kt_begin + i);
+        sw = __ldg(prm.scale_w + (size_t)(n0 / 128) * G + i);
 #pragma unroll
         for (int mf = 0; mf < C::kMF; ++mf) {
           // the tokens of this thread's accumulator elements: rows g, g + 8 of
           // a 16-token fragment, or columns 2t, 2t + 1 (weights as A)
           const int mlo = C::kWA ? m0 + 2 * t : m0 + mf * 16 + g;
           const int mhi = C::kWA ? mlo + 1 : mlo + 8;
-          sa_lo[mf] = (mlo < prm.M) ? __ldg(prm.scale_a + (size_t)mlo * G + kt_begin + i) : 0.f;
-          sa_hi[mf] = (mhi < prm.M) ? __ldg(prm.scale_a + (size_t)mhi * G + kt_begin + i) : 0.f;
+          sa_lo[mf] = (mlo < prm.M) ? __ldg(prm.scale_a + (size_t)mlo * G + i) : 0.f;
+          sa_hi[mf] = (mhi < prm.M) ? __ldg(prm.scale_a + (size_t)mhi * G + i) : 0.f;
         }
       }
       if (!mbar_wait(&full[st], (uint32_t)((i / S) & 1), prm.err, prm.wait_ns)) { ok = false; break; }
@@ -277,80 +262,30 @@ __global__ void __launch_bounds__(SkCfg<FMT, TM, NF>::kThreads, 1)
   }
   // every thread (the producer warp too) meets here; a thread that gave up on
   // a wait leaves no sum, and then the epilogue stores nothing
-  int all_ok = __syncthreads_and(ok ? 1 : 0);
-  // the K-group sums of unit u (8 consecutive channels nfu of token mm) of
-  // this CTA, in K-group order (deterministic)
-  auto kgroup_sum = [&](int mm, int nfu, Acc (&s8)[8]) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) s8[j] = (Acc)0;
-    for (int k2 = 0; k2 < C::kKG; ++k2) {
-      if constexpr (C::kWA) {
-        // warp (k2, nfu / 2), fragment rows 8 (nfu % 2) + j, column mm
-        const Acc* rw = red + (size_t)(k2 * C::kUnits + nfu / 2) * 128 + (nfu % 2) * 64 + mm;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) s8[j] += rw[j * 8];
-      } else {
-        const Acc* rw = red + ((size_t)((k2 * NF + nfu) * C::kMF + mm / 16) * 16 + mm % 16) * 8;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) s8[j] += rw[j];
-      }
-    }
-  };
-  uint32_t rank = 0;
-  if (Sk > 1) {
-    // this CTA's partial of every unit, then cluster phase 1: every CTA's
-    // partials and completion word are in its shared memory (all threads of
-    // all CTAs take both phases)
-    if (warp < C::kWarps && all_ok) {
-      for (int u = threadIdx.x; u < TM * NF; u += 32 * C::kWarps) {
-        Acc s8[8];
-        kgroup_sum(u / NF, u % NF, s8);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) part[u * 8 + j] = s8[j];
-      }
-    }
-    if (threadIdx.x == 0) *done_ok = all_ok;
-    cluster_sync();
-    rank = cluster_ctarank();
-    for (int z = 0; z < Sk; ++z) all_ok &= (int)ld_dsmem_b32(mapa_shared(smem_u32(done_ok), (uint32_t)z));
-  }
+  const int all_ok = __syncthreads_and(ok ? 1 : 0);
   if (warp < C::kWarps) {
     if (all_ok) {
-      // ---- epilogue: one unit = 8 consecutive channels of one token (split-K:
-      // CTA r of the cluster takes the units u with u % split_k == r)
+      // ---- epilogue: one unit = 8 consecutive channels of one token
       const int etid = threadIdx.x;            // 0 .. 255
       const bool vec = (prm.ldy % 8) == 0;
-      for (int u = etid * Sk + (int)rank; u < TM * NF; u += 32 * C::kWarps * Sk) {
+      for (int u = etid; u < TM * NF; u += 32 * C::kWarps) {
         const int mm = u / NF, nfu = u % NF;
         const int m = m0 + mm, nb = n0 + nfu * 8;
         if (m >= prm.M || nb >= prm.N) continue;
         Acc s8[8];
-        if (Sk == 1) {
-          kgroup_sum(mm, nfu, s8);
-        } else {
-          // every CTA's partial of this unit (all loads in flight), summed in z order
-          uint4 w[8][2];
 #pragma unroll
-          for (int z = 0; z < 8; ++z) {
-            if (z < Sk) {
-              const uint32_t a = mapa_shared(smem_u32(part + u * 8), (uint32_t)z);
-              w[z][0] = ld_dsmem_v4(a);
-              w[z][1] = ld_dsmem_v4(a + 16u);
-            }
-          }
+        for (int j = 0; j < 8; ++j) s8[j] = (Acc)0;
+        for (int k2 = 0; k2 < C::kKG; ++k2) {  // K-group order: deterministic
+          if constexpr (C::kWA) {
+            // warp (k2, nfu / 2), fragment rows 8 (nfu % 2) + j, column mm
+            const Acc* rw = red + (size_t)(k2 * C::kUnits + nfu / 2) * 128 + (nfu % 2) * 64 + mm;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) s8[j] = (Acc)0;
+            for (int j = 0; j < 8; ++j) s8[j] += rw[j * 8];
+          } else {
+            const int mf = mm / 16, rr = mm % 16;
+            const Acc* rw = red + ((size_t)((k2 * NF + nfu) * C::kMF + mf) * 16 + rr) * 8;
 #pragma unroll
-          for (int z = 0; z < 8; ++z) {
-            if (z < Sk) {
-              const uint32_t v[8] = {w[z][0].x, w[z][0].y, w[z][0].z, w[z][0].w,
-                                     w[z][1].x, w[z][1].y, w[z][1].z, w[z][1].w};
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                if constexpr (kInt) s8[j] += (int)v[j];
-                else s8[j] += __uint_as_float(v[j]);
-              }
-            }
+            for (int j = 0; j < 8; ++j) s8[j] += rw[j];
           }
         }
         if (prm.out_kind == 1) {
@@ -386,8 +321,6 @@ __global__ void __launch_bounds__(SkCfg<FMT, TM, NF>::kThreads, 1)
     }
     if (threadIdx.x == 0) trace_at(prm, kTrDone);
   }
-  // cluster phase 2: every remote read is done before any CTA leaves
-  if (Sk > 1) cluster_sync();
 }
 
 }  // namespace qg

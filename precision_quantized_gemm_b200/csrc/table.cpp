@@ -48,8 +48,7 @@ constexpr int kVersion = 2;
 bool valid_cfg_fields(const qg_config& c) {
   if (c.reserved != 0 || (c.variant != 0 && c.variant != 1)) return false;
   if (c.variant == 1)
-    return (c.split_k == 1 || c.split_k == 2 || c.split_k == 4 || c.split_k == 8) && c.swap_ab == 1 &&
-           (c.tile_n == 8 || c.tile_n == 16 || c.tile_n == 32) && c.stages >= 2 &&
+    return c.split_k == 1 && c.swap_ab == 1 && (c.tile_n == 8 || c.tile_n == 16 || c.tile_n == 32) && c.stages >= 2 &&
            c.stages <= 64 && c.reduce_mode == 0 && (c.rows == 8 || c.rows == 16 || c.rows == 32 || c.rows == 64);
   return c.split_k >= 1 && c.split_k <= 256 && (c.swap_ab == 0 || c.swap_ab == 1) &&
          c.tile_n >= 16 && c.tile_n <= 256 && c.stages >= 2 && c.stages <= 12 &&

@@ -79,9 +79,8 @@ def test_default_config_follows_the_swap_rule_and_fills_sms():
     for fmt, M in ((qg.QG_W8A8_INT8, 8), (qg.QG_FP8_DYNAMIC, 1), (qg.QG_BLOCK_FP8, 16)):
         c = qg.qgemm_default_config(fmt, M, 4096, 4096)
         assert c.swap_ab == 1 and c.tile_n <= 32
-        if c.variant == 1:                             # the decode kernel: rows x slices per CTA fill the SMs
-            assert c.split_k in (1, 2, 4, 8) and c.reduce_mode == 0
-            assert 74 <= 4096 // c.rows * ((M + c.tile_n - 1) // c.tile_n) * c.split_k <= 4 * 148
+        if c.variant == 1:                             # the decode kernel: rows per CTA fill the SMs
+            assert c.split_k == 1 and 74 <= 4096 // c.rows * ((M + c.tile_n - 1) // c.tile_n) <= 4 * 148
             continue
         assert c.split_k >= 2 and (c.split_k & (c.split_k - 1)) == 0
         assert 74 <= 32 * c.split_k * ((M + c.tile_n - 1) // c.tile_n) <= 2 * 148
@@ -164,17 +163,11 @@ def test_run_reserved_fields_must_be_zero():
 def test_skinny_config_checks(kw, status):
     c = qg.skinny_config(**kw)
     assert _run(cfg=c) == status
-    # split-K only through a cluster of 2, 4 or 8 CTAs (at most one per K tile)
-    for bad in (dict(split_k=16), dict(split_k=3), dict(split_k=2, reduce_mode=1), dict(swap_ab=0),
-                dict(reduce_mode=1)):
+    for bad in (dict(split_k=2), dict(swap_ab=0), dict(reduce_mode=1)):
         c2 = qg.skinny_config(**kw)
         for k, v in bad.items():
             setattr(c2, k, v)
         assert _run(cfg=c2) == qg.QG_ERR_UNSUPPORTED
-    if status == qg.QG_ERR_NO_DEVICE:
-        for sk in (2, 4, 8):
-            assert _run(K=1024, cfg=qg.skinny_config(**kw, split_k=sk)) == qg.QG_ERR_NO_DEVICE
-        assert _run(K=512, cfg=qg.skinny_config(**kw, split_k=8)) == qg.QG_ERR_UNSUPPORTED   # 4 K tiles
 
 
 def test_skinny_refuses_nvfp4_and_the_fused_and_grouped_launches():

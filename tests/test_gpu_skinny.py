@@ -104,43 +104,3 @@ def test_skinny_in_a_graph_after_the_quantiser():
     for y in outs:
         assert_within_tolerance(bf16_to_np(y), ref, "graph step")
         assert torch.equal(y, outs[0])
-
-
-# cluster split-K: (M, N, K, tile_n, rows, stages, split_k): slices of unequal
-# tile counts, slices shorter than the K groups, every cluster size, both
-# operand roles, ragged N and M
-SPLIT = [
-    (1, 512, 7168, 8, 16, 8, 8),      # 56 K tiles over 8 slices of 7
-    (4, 896, 5120, 8, 16, 8, 4),      # 40 K tiles over 4 slices
-    (16, 1000, 2048, 16, 16, 4, 2),   # ragged N inside a CTA
-    (3, 256, 1152, 16, 32, 2, 8),     # 9 K tiles over 8 slices: 1 or 2 each, fewer than the K groups
-    (32, 640, 4096, 32, 32, 8, 4),
-    (9, 384, 1024, 8, 32, 4, 2),      # two 8-token tiles, the last partial
-]
-SPLIT_ALL = [(f, *c) for f in FMTS for c in SPLIT]
-
-
-def _sid(c):
-    f, M, N, K, tn, rows, st, sk = c
-    return f"{IDS[f]}-M{M}-N{N}-K{K}-t{tn}-r{rows}-s{st}-k{sk}"
-
-
-@pytest.mark.parametrize("case", SPLIT_ALL, ids=[_sid(c) for c in SPLIT_ALL])
-def test_skinny_cluster_split_k(case):
-    fmt, M, N, K, tn, rows, st, sk = case
-    a, w = inputs(M, N, K, edge_rows=True)
-    A = qg.quantize_act(fmt, to_dev_bf16(a))
-    W = qg.quantize_weight(fmt, to_dev_bf16(w))
-    qa, qw = oracle_quant(fmt, a, False), oracle_quant(fmt, w, True)
-    cfg = qg.skinny_config(tile_n=tn, rows=rows, stages=st, split_k=sk)
-    assert qg.qgemm_workspace_size(fmt, M, N, K, cfg) == 0
-    y = qg.run(fmt, A, W, cfg)
-    assert_within_tolerance(bf16_to_np(y), oracle_y(fmt, qa, qw), _sid(case))
-    assert torch.count_nonzero(y[0]).item() == 0
-    assert torch.equal(y, qg.run(fmt, A, W, cfg))                # slices summed in a fixed order
-    if fmt == qg.QG_W8A8_INT8:
-        # integer partials: bit-exact, and the same bits as the unsplit kernel
-        acc = qg.run(fmt, A, W, cfg, out_kind=qg.QG_OUT_ACC)
-        np.testing.assert_array_equal(acc.cpu().numpy().astype(np.int64), OG.acc_int8(qa[0], qw[0]))
-        one = qg.skinny_config(tile_n=tn, rows=rows, stages=st, split_k=1)
-        assert torch.equal(y, qg.run(fmt, A, W, one))
