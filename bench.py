@@ -616,9 +616,8 @@ def run_ours(args, world, rank, local):
     # ---- end to end through the public API with host buffers: per step the
     # three activations are copied in from pinned host memory (one copy: they
     # are contiguous there and on the device), the step's graph replays, the
-    # results are copied out (one copy), and the host synchronises.
-    # (Copies captured inside the graph were slower: 113 against 92 us with
-    # one copy per shape.)
+    # results are copied out (one copy), and the host synchronises.  (The
+    # copies captured inside the step's graph were slower: 75.5 against 66.2 us.)
     host_in = torch.empty(rows * K, dtype=torch.bfloat16, pin_memory=True)
     host_out = torch.empty(rows * N, dtype=torch.bfloat16, pin_memory=True)
     host_in.copy_(torch.cat([acts[m].reshape(-1) for m in MS]).cpu())
@@ -659,8 +658,8 @@ def run_ours(args, world, rank, local):
         "config": bench_config(world),
         "method": {"l2": f"{copies} rotating weight copies ({copies * wbytes / 1e6:.0f} MB > 2 x {l2 / 1e6:.0f} MB L2)",
                    "step": "per M: activation quant + GEMM; the K timed steps run as CUDA graphs of up to "
-                           f"{chunk} consecutive steps each (qg.capture_steps); e2e: per step copies in from pinned "
-                           "host memory, one graph replay, copies out, sync",
+                           f"{chunk} consecutive steps each (qg.capture_steps); e2e: per step one copy in from pinned "
+                           "host memory, one graph replay, one copy out, sync",
                    "per_shape": "one CUDA graph of back-to-back qgemm_run launches per shape over weight copies "
                                 "totalling more than 2 x L2, 5 replays after a warm one, CUDA events",
                    "table": os.path.relpath(args.table, ROOT) if table is not None else "built-in default"},
