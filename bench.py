@@ -740,7 +740,7 @@ def tensor_peak(fmt, bf16_tflops):
 MOE_EXPERTS, MOE_TOPK = 128, 8
 MOE_NK = [(1536, 2048), (2048, 768)]
 MOE_TOKENS = [1, 4, 16, 64]
-MOE_FMTS = [0, 1, 2]
+MOE_FMTS = [0, 1, 2, 3]
 
 
 def moe_routing(T, seed):
@@ -773,28 +773,31 @@ def run_moe_suite(args, local):
     for fmt in fmts:
         for (N, K) in MOE_NK:
             w = (torch.randn(E * N, K, device=dev, generator=gen) * 0.02).to(torch.bfloat16)
-            Wq = qg.quantize_weight(fmt, w)
+            Wq = qg.quantize_weight_grouped(fmt, w, E)   # NVFP4: one tensor scale per expert
             del w
+            qbw, sbw = qg.qgemm_operand_bytes(fmt, 1, N, K)   # one expert's codes / scales
             for T in tokens:
                 counts = moe_routing(T, seed=1000 + T)
                 rows = int(counts.sum())
                 offs = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
                 offsets = torch.from_numpy(offs).to(dev)
                 active = [e for e in range(E) if counts[e] > 0]
-                sb_row = 4 * (K // 128) if fmt == 2 else 4
-                w_bytes = len(active) * (N * K + (4 * (N // 128) * (K // 128) if fmt == 2 else 4 * N))
-                byts = w_bytes + rows * (K + sb_row) + 2 * rows * N
+                # algorithmic bytes: active experts' codes + scales, activations' codes + scales, bf16 y
+                sb_row = 4 * (K // 128) if fmt == 2 else (K // 16 if fmt == 3 else 4)
+                qrow = K // 2 if fmt == 3 else K
+                w_bytes = len(active) * (qbw + (N * K // 16 + 4 if fmt == 3 else sbw))
+                byts = w_bytes + rows * (qrow + sb_row) + 2 * rows * N
                 # rotate weight copies past 2 x L2 so each call streams from HBM
                 copies = int(max(1, min(32, (2 * l2) // max(w_bytes, 1) + 2)))
                 Ws = [Wq]
                 for _ in range(copies - 1):
-                    o = qg.Operand(fmt, True, E * N, K, dev)
+                    o = qg.Operand(fmt, True, E * N, K, dev, n_global=E)
                     o.q.copy_(Wq.q)
                     o.scale.copy_(Wq.scale)
                     o.global_scale.copy_(Wq.global_scale)
                     Ws.append(o)
                 a = torch.randn(rows, K, device=dev, generator=gen).to(torch.bfloat16)
-                A = qg.quantize_act(fmt, a)
+                A = qg.quantize_act_grouped(fmt, a, offsets)   # NVFP4: per-expert scale atoms
                 cfg = qg.qgemm_grouped_default_config(fmt, E, rows, N, K)
                 ws = qg.Workspace(dev)
                 wsp, wsb = ws.get(qg.qgemm_workspace_size(fmt, rows, N, K, cfg))
@@ -811,13 +814,24 @@ def run_moe_suite(args, local):
                 ewsp, ewsb = ews.get(max(qg.qgemm_workspace_size(fmt, int(counts[e]), N, K, ecfg[e])
                                          for e in active))
 
+                # NVFP4: expert e's activation scales start at its first 128-row atom
+                sf_row0, r = {}, 0
+                for e in range(E):
+                    sf_row0[e] = r
+                    r += -(-int(counts[e]) // 128) * 128
+
                 def per_expert(Wo, st):
                     for e in active:
                         m0, m = int(offs[e]), int(counts[e])
-                        s_a = A.scale.data_ptr() + m0 * sb_row
-                        s_w = Wo.scale.data_ptr() + (e * N // 128 * (K // 128) * 4 if fmt == 2 else e * N * 4)
-                        Ae = qg.qg_operand(A.q.data_ptr() + m0 * K, s_a, A.global_scale.data_ptr(), m, K)
-                        We = qg.qg_operand(Wo.q.data_ptr() + e * N * K, s_w, Wo.global_scale.data_ptr(), N, K)
+                        if fmt == 3:
+                            s_a = A.scale.data_ptr() + sf_row0[e] * ((K + 255) // 256 * 16)
+                            g_w = Wo.global_scale.data_ptr() + 4 * e
+                        else:
+                            s_a = A.scale.data_ptr() + m0 * sb_row
+                            g_w = Wo.global_scale.data_ptr()
+                        s_w = Wo.scale.data_ptr() + e * sbw
+                        Ae = qg.qg_operand(A.q.data_ptr() + m0 * qrow, s_a, A.global_scale.data_ptr(), m, K)
+                        We = qg.qg_operand(Wo.q.data_ptr() + e * qbw, s_w, g_w, N, K)
                         qg.check(qg.qgemm_run(fmt, Ae, We, m, N, K, ecfg[e], ewsp, ewsb,
                                               Y.data_ptr() + m0 * N * 2, N, 0, st))
 
