@@ -99,9 +99,18 @@ typedef struct {
                           requires split_k = 1, swap_ab = 1, reduce_mode = 0,
                           and `stages` (the ring of 128-byte K tiles, 2..64) a
                           multiple of the K groups of its eight compute warps:
-                          64 / rows (128 / rows for tile_n = 8)                */
+                          64 / rows (128 / rows for tile_n = 8);
+                          2: the persistent kernel for FP8_DYNAMIC and W8A8_INT8
+                          at large M: one CTA per SM walks the 128 x tile_n
+                          output tiles with two TMEM accumulators, so a tile's
+                          epilogue (bf16 through TMA stores) overlaps the next
+                          tile's MMAs; requires split_k = 1, swap_ab = 0,
+                          reduce_mode = 0, rows = 0, tile_n 128 or 256,
+                          stages 2..12 (capped by shared memory), and bf16
+                          output (QG_ERR_UNSUPPORTED otherwise); y is bitwise
+                          that of variant 0 with the same tile_n              */
   int32_t rows;        /* variant 1: weight rows per CTA, 8, 16, 32 or 64 (at
-                          least 16 for tile_n = 8); variant 0: must be 0        */
+                          least 16 for tile_n = 8); variants 0, 2: must be 0   */
   int32_t reserved;    /* must be zero                                            */
 } qg_config;
 

@@ -26,7 +26,8 @@ INCLUDE = os.path.join(ROOT, "include")
 SOURCES = ["api.cu", "quant.cu", "gemm_fp8.cu", "gemm_int8.cu", "gemm_block.cu", "gemm_nvf4.cu",
            "gemm_nvf4_grouped.cu",
            "tune.cu", "table.cpp", "noalloc.cu", "scorer.cu"]
-HEADERS = ["ptx.cuh", "gemm_kernel.cuh", "gemm_launch.cuh", "internal.h", "quant_math.cuh", "attr_cache.h", "skinny.cuh"]
+HEADERS = ["ptx.cuh", "gemm_kernel.cuh", "gemm_launch.cuh", "internal.h", "quant_math.cuh", "attr_cache.h", "skinny.cuh",
+           "persist.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-std=c++17", "-O3", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",

@@ -8,6 +8,7 @@
 #include "attr_cache.h"
 #include "gemm_kernel.cuh"
 #include "internal.h"
+#include "persist.cuh"
 #include "skinny.cuh"
 
 #define QG_CAT2(a, b) a##b
@@ -166,6 +167,36 @@ cudaError_t launch_skinny_rows(int rows, const CUtensorMap& tw, const CUtensorMa
   }
 }
 
+template <int FMT, int BN>
+cudaError_t launch_persist_one(const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap& ty,
+                               const GemmParams& prm, dim3 grid, cudaStream_t st, bool pdl) {
+  auto kern = qgemm_persist_kernel<FMT, BN>;
+  size_t smem = ps_smem_bytes<FMT, BN>(prm.stages);
+  // at most 512 / (2 BN) CTAs fit an SM's TMEM: the shared memory keeps it so
+  constexpr int kTmemCtas = 512 / PsCfg<FMT, BN>::kTmemCols;
+  const size_t smem_floor = (size_t)233472 / (kTmemCtas + 1);
+  if (smem < smem_floor) smem = smem_floor;
+  static GrowOnlyAttr smem_attr;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = static_cast<cudaError_t>(smem_attr.ensure(dev, (int)smem, [&](int bytes) {
+    return static_cast<int>(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  }));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(PsCfg<FMT, BN>::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, tp, tq, ty, prm);
+}
+
 template <int FMT, int TM>
 size_t skinny_smem_rows(int rows, int stages) {
   switch (rows) {
@@ -201,6 +232,25 @@ cudaError_t QG_CAT(QG_LAUNCH_NAME, _skinny)(int tile_n, int rows, const CUtensor
     if (tile_n == 32) return launch_skinny_rows<QG_FMT, 32>(rows, tw, ta, prm, grid, st, pdl);
     return cudaErrorInvalidValue;
   }
+}
+
+// The persistent kernel (variant 2): FP8_Dynamic and W8A8_INT8, tile_n 128 or 256.
+cudaError_t QG_CAT(QG_LAUNCH_NAME, _persist)(int tile_n, const CUtensorMap& tp, const CUtensorMap& tq,
+                                             const CUtensorMap& ty, const GemmParams& prm, dim3 grid,
+                                             cudaStream_t st, bool pdl) {
+  if constexpr (QG_FMT == kFP8 || QG_FMT == kINT8) {
+    if (tile_n == 128) return launch_persist_one<QG_FMT, 128>(tp, tq, ty, prm, grid, st, pdl);
+    if (tile_n == 256) return launch_persist_one<QG_FMT, 256>(tp, tq, ty, prm, grid, st, pdl);
+  }
+  return cudaErrorInvalidValue;
+}
+
+size_t QG_CAT(QG_LAUNCH_NAME, _persist_smem)(int tile_n, int stages) {
+  if constexpr (QG_FMT == kFP8 || QG_FMT == kINT8) {
+    if (tile_n == 128) return ps_smem_bytes<QG_FMT, 128>(stages);
+    if (tile_n == 256) return ps_smem_bytes<QG_FMT, 256>(stages);
+  }
+  return (size_t)1 << 30;
 }
 
 size_t QG_CAT(QG_LAUNCH_NAME, _skinny_smem)(int tile_n, int rows, int stages) {

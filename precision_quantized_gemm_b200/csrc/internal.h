@@ -58,7 +58,11 @@ cudaError_t launch_quant_nvfp4(const void* X, int R, int K, int ldx, const float
                              const GemmParams& prm, dim3 grid, cudaStream_t st, bool pdl); \
   cudaError_t NAME##_skinny(int tile_n, int rows, const CUtensorMap& tw, const CUtensorMap& ta, \
                             const GemmParams& prm, dim3 grid, cudaStream_t st, bool pdl);     \
-  size_t NAME##_skinny_smem(int tile_n, int rows, int stages);
+  size_t NAME##_skinny_smem(int tile_n, int rows, int stages);                              \
+  cudaError_t NAME##_persist(int tile_n, const CUtensorMap& tp, const CUtensorMap& tq,     \
+                             const CUtensorMap& ty, const GemmParams& prm, dim3 grid,      \
+                             cudaStream_t st, bool pdl);                                   \
+  size_t NAME##_persist_smem(int tile_n, int stages);
 QG_DECLARE_GEMM_LAUNCH(launch_gemm_fp8)
 QG_DECLARE_GEMM_LAUNCH(launch_gemm_int8)
 QG_DECLARE_GEMM_LAUNCH(launch_gemm_block)

@@ -1,0 +1,269 @@
+// persist.cuh — the persistent variant of the quantized GEMM for large M
+// (qg_config.variant = 2): standard orientation, FP8_Dynamic and W8A8_INT8.
+//
+// Why a third kernel: the tile kernel runs one 128 x BN output tile per CTA,
+// so every tile pays the CTA's set-up, the pipeline fill and its epilogue
+// with the tensor core idle (per-CTA stamps at M = 4096, N = K = 5120,
+// 128 x 256 tiles: 13 us of mainloop, then 2.8 us of epilogue and ~1.3 us
+// before the next CTA's first MMA).  Here one CTA per SM walks the tiles
+// t = blockIdx.x, blockIdx.x + gridDim.x, ...; its producer streams the K
+// tiles of consecutive tiles through one continuous ring, and TMEM holds two
+// BN-column accumulators, so the MMAs of tile j + 1 run while the epilogue
+// warps drain tile j (TMEM -> fp32 scales -> bf16 -> 128-byte-swizzled
+// boxes -> TMA store through a tensor map of y).
+//
+// Roles: warp 0 producer (one thread), warp 1 MMA issuer (one thread; also
+// allocates TMEM), warps 2-5 the epilogue (thread = TMEM lane = output row).
+// Barriers: full / empty per ring slot, acc_full / acc_empty per accumulator.
+// Every wait is bounded; a wait that gives up sets the abort word, and every
+// role stops at its next check.  The MMAs of one tile accumulate their K
+// tiles in the same order as the tile kernel's, and the epilogue applies the
+// same fp32 arithmetic, so y is bitwise that of the tile kernel with the
+// same tile_n.
+#pragma once
+#include "gemm_kernel.cuh"
+
+namespace qg {
+
+template <int FMT, int BN>
+struct PsCfg {
+  static constexpr int kThreads = 192;             // producer, MMA, 4 epilogue warps
+  static constexpr int kQTileBytes = BN * kKTileBytes;
+  static constexpr int kStage = kPTileBytes + kQTileBytes;
+  // the bf16 output goes out in slices of up to 128 channels (two boxes of
+  // 64), one slice buffer: a 256-wide tile leaves room for a 4-stage ring
+  static constexpr int kYCols = BN < 128 ? BN : 128;
+  static constexpr int kYBytes = 128 * kYCols * 2;
+  static constexpr int kTmemCols = 2 * BN;         // two accumulators
+  static constexpr uint32_t kIdesc = (FMT == kINT8) ? idesc_i8(BN) : idesc_f8f6f4_e4m3(BN);
+  static_assert(FMT == kFP8 || FMT == kINT8, "persistent kernel: FP8_Dynamic and W8A8_INT8");
+  static_assert(BN == 128 || BN == 256, "persistent kernel: 128- or 256-wide tiles");
+};
+
+// Shared memory: the ring (P tiles, then Q tiles), the y boxes, the channel
+// scales of the tile, the barriers and the TMEM address / abort words
+// (+ alignment slack).
+struct PsLayout {
+  uint32_t p, q, y, cols, bars, misc, total;
+};
+template <int FMT, int BN>
+__host__ __device__ __forceinline__ PsLayout ps_layout(int stages) {
+  using C = PsCfg<FMT, BN>;
+  PsLayout L;
+  L.p = 0;
+  L.q = L.p + (uint32_t)stages * kPTileBytes;
+  L.y = L.q + (uint32_t)stages * C::kQTileBytes;
+  L.cols = L.y + C::kYBytes;
+  L.bars = L.cols + 4u * BN;
+  L.misc = L.bars + 8u * (2u * stages + 4u);
+  L.total = L.misc + 16u;
+  return L;
+}
+template <int FMT, int BN>
+__host__ __device__ constexpr size_t ps_smem_bytes(int stages) {
+  return (size_t)ps_layout<FMT, BN>(stages).total + 1024;
+}
+
+template <int FMT, int BN>
+__global__ void __launch_bounds__(PsCfg<FMT, BN>::kThreads, 1)
+    qgemm_persist_kernel(const __grid_constant__ CUtensorMap tmap_p, const __grid_constant__ CUtensorMap tmap_q,
+                         const __grid_constant__ CUtensorMap tmap_y, const GemmParams prm) {
+  using C = PsCfg<FMT, BN>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int S = prm.stages;
+  const PsLayout L = ps_layout<FMT, BN>(S);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
+  uint64_t* empty = full + S;
+  uint64_t* acc_full = empty + S;              // [2]
+  uint64_t* acc_empty = acc_full + 2;          // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.misc);
+  volatile int* flag_abort = reinterpret_cast<volatile int*>(smem + L.misc + 4);
+  float* col_s = reinterpret_cast<float*>(smem + L.cols);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // tiles: m-tile fastest, so the CTAs of one wave share weight tiles
+  const int tp = (prm.M + 127) / 128, tq = (prm.N + BN - 1) / BN;
+  const int tiles = tp * tq;
+  const int nkt = prm.kt_total;
+
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tmap_p);
+    prefetch_tmap(&tmap_q);
+    prefetch_tmap(&tmap_y);
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);             // one arrival per epilogue warp
+    }
+    *flag_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  if (threadIdx.x == 0) {
+    trace_at(prm, kTrReady);
+    griddep_launch_dependents();
+  }
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      // both operands are re-read by other tiles of the wave: keep them in L2
+      const uint64_t pol = policy_evict_last();
+      griddep_wait();                          // the activations come from the preceding kernel
+      bool ok = true;
+      int issued = 0;                          // K tiles issued over all of this CTA's tiles
+      int st = 0, r = 0;                       // slot of the next K tile, and its round
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+        const int p0 = (t % tp) * 128, q0 = (t / tp) * BN;
+        for (int kt = 0; kt < nkt; ++kt) {
+          // the slot's previous round must have been consumed by the MMAs
+          if (r > 0 && !mbar_wait(&empty[st], (uint32_t)((r - 1) & 1), prm.err, prm.wait_ns)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[st], C::kStage);
+          tma_load_2d(smem + L.p + (size_t)st * kPTileBytes, &tmap_p, &full[st], kt * kKTileBytes, p0, pol);
+          tma_load_2d(smem + L.q + (size_t)st * C::kQTileBytes, &tmap_q, &full[st], kt * kKTileBytes, q0, pol);
+          ++issued;
+          if (++st == S) { st = 0; ++r; }
+        }
+        if (*flag_abort) ok = false;
+      }
+      if (!ok) {
+        *flag_abort = 1;
+        // drain: wait (bounded) until every issued copy has landed
+        for (int g = (issued > S ? issued - S : 0); g < issued; ++g)
+          mbar_wait(&full[g % S], (uint32_t)((g / S) & 1), prm.err, prm.wait_ns);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint64_t dp0 = sdesc_sw128(smem_u32(smem + L.p));
+      const uint64_t dq0 = sdesc_sw128(smem_u32(smem + L.q));
+      int st = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      int j = 0;                               // this CTA's tile count; accumulator j & 1
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++j) {
+        const int ab = j & 1;
+        // the epilogue has read tile j - 2 out of this accumulator
+        if (j >= 2 && !mbar_wait(&acc_empty[ab], (uint32_t)(((j >> 1) - 1) & 1), prm.err, prm.wait_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_t = tmem_base + (uint32_t)(ab * BN);
+        for (int kt = 0; kt < nkt; ++kt) {
+          if (!mbar_wait(&full[st], ph, prm.err, prm.wait_ns)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t dp = dp0 + (uint64_t)((st * kPTileBytes) >> 4);
+          const uint64_t dq = dq0 + (uint64_t)((st * C::kQTileBytes) >> 4);
+#pragma unroll
+          for (int s = 0; s < 4; ++s) {        // 32 bytes of K per MMA
+            const uint32_t accum = (kt > 0 || s > 0);
+            if constexpr (FMT == kINT8) mma_i8(d_t, dp + (uint64_t)(2 * s), dq + (uint64_t)(2 * s), C::kIdesc, accum);
+            else mma_f8f6f4(d_t, dp + (uint64_t)(2 * s), dq + (uint64_t)(2 * s), C::kIdesc, accum);
+          }
+          mma_commit(&empty[st]);
+          if (++st == S) { st = 0; ph ^= 1u; }
+        }
+        if (!ok) break;
+        mma_commit(&acc_full[ab]);
+        if (*flag_abort) ok = false;
+      }
+      if (!ok) *flag_abort = 1;
+    }
+  } else {
+    // --------------------------------------------------------------- epilogue
+    const int quarter = warp & 3;              // TMEM lanes this warp may access
+    const int row = quarter * 32 + lane;       // output row of the tile
+    const int etid = threadIdx.x - 64;         // 0 .. 127
+    const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
+    uint8_t* ybuf = smem + L.y;
+    griddep_wait();                            // the activation scales come from the preceding kernel
+    const float alpha = alpha_of<FMT>(prm);
+    int j = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++j) {
+      const int ab = j & 1;
+      const int p0 = (t % tp) * 128, q0 = (t / tp) * BN;
+      // the tile's channel scales, and the previous tile's boxes read out by its store
+      for (int c = etid; c < BN; c += 128) col_s[c] = (q0 + c < prm.N) ? __ldg(prm.scale_w + q0 + c) : 0.f;
+      if (etid == 0) bulk_wait_read_all();
+      const bool got = mbar_wait(&acc_full[ab], (uint32_t)((j >> 1) & 1), prm.err, prm.wait_ns);
+      if (!__all_sync(0xffffffffu, got)) *flag_abort = 1;
+      named_bar_sync(1, 128);                  // scales staged, boxes free, abort state settled
+      if (*flag_abort) break;
+      tc_fence_after();
+      const float sa = (p0 + row < prm.M) ? __ldg(prm.scale_a + p0 + row) : 0.f;
+#pragma unroll
+      for (int y0 = 0; y0 < BN; y0 += C::kYCols) {   // slices of the tile's channels
+        if (y0 > 0) {                          // the previous slice's boxes read out by its store
+          if (etid == 0) bulk_wait_read_all();
+          named_bar_sync(1, 128);
+        }
+#pragma unroll
+        for (int c0 = y0; c0 < y0 + C::kYCols; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld32(lane_addr + (uint32_t)(ab * BN + c0), v);
+          tmem_ld_wait();
+          if (c0 + 32 == BN) {                 // the accumulator is in registers: free it for tile j + 2
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[ab]);
+          }
+#pragma unroll
+          for (int k = 0; k < 32; k += 8) {
+            const int col = c0 + k;            // a multiple of 8
+            const float4 s0 = reinterpret_cast<const float4*>(col_s + col)[0];
+            const float4 s1 = reinterpret_cast<const float4*>(col_s + col)[1];
+            const float sw[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+            uint32_t pk[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const __nv_bfloat162 b2 =
+                  __floats2bfloat162_rn(finish_value<FMT>(v[k + 2 * h], sa, sw[2 * h], alpha),
+                                        finish_value<FMT>(v[k + 2 * h + 1], sa, sw[2 * h + 1], alpha));
+              pk[h] = *reinterpret_cast<const uint32_t*>(&b2);
+            }
+            // 16-byte chunk (col % 64) / 8 of row `row` of the slice's box, 128-byte swizzle
+            const int lc = col - y0;
+            const uint32_t off = (uint32_t)(lc >> 6) * 16384u + (uint32_t)row * 128u +
+                                 ((uint32_t)(((lc & 63) >> 3) ^ (row & 7)) << 4);
+            *reinterpret_cast<uint4*>(ybuf + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (etid == 0) {
+#pragma unroll
+          for (int b = 0; b < C::kYCols / 64; ++b)
+            tma_store_2d(&tmap_y, ybuf + b * 16384, (q0 + y0 + b * 64) * 2, p0);
+          bulk_commit();
+        }
+      }
+    }
+    if (etid == 0) {
+      bulk_wait_all();                         // every store performed before the CTA ends
+      trace_at(prm, kTrDone);
+    }
+  }
+
+  // ------------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+}  // namespace qg

@@ -106,6 +106,14 @@ double estimate_skinny_us(qg_format f, int M, int N, int K, const qg_config& c, 
 
 double estimate_us(qg_format f, int M, int N, int K, const qg_config& c, int sms) {
   if (c.variant == 1) return estimate_skinny_us(f, M, N, K, c, sms);
+  if (c.variant == 2) {
+    // the persistent kernel: the tile kernel's estimate less the per-tile
+    // set-up and epilogue that the next tile's MMAs hide (a flat 12 %; the
+    // tuner's measurements decide)
+    qg_config t = c;
+    t.variant = 0;
+    return 0.88 * estimate_us(f, M, N, K, t, sms);
+  }
   const Model& m = kModel;
   const double rb = f == QG_NVFP4 ? K / 2.0 : (double)K;
   const int kt = (int)((rb + 127) / 128);
@@ -174,6 +182,24 @@ void candidate_grid(qg_format f, int M, int N, int K, qg_config* out, int max_ou
             ++n;
           }
     }
+  }
+  // the persistent kernel (FP8_Dynamic, W8A8_INT8, at least 256 tokens):
+  // 128- or 256-wide tiles, rings of 3, 4 or 6 stages (as far as they fit)
+  if ((f == QG_FP8_DYNAMIC || f == QG_W8A8_INT8) && M >= 256) {
+    for (int tn : {128, 256})
+      for (int st : {3, 4, 6}) {
+        if (n < max_out) {
+          qg_config c = {};
+          c.split_k = 1;
+          c.swap_ab = 0;
+          c.tile_n = tn;
+          c.stages = st;
+          c.reduce_mode = 0;
+          c.variant = 2;
+          out[n] = c;
+        }
+        ++n;
+      }
   }
   // the decode kernel (8-bit formats, up to 32 tokens per CTA): rows per
   // CTA, and rings of 8, 16, 32 or every K tile (up to 64) rounded to the K

@@ -155,13 +155,13 @@ std::vector<qg_config> candidates(qg_format f, int M, int N, int K, int top_n) {
   int n = 0;
   if (top_n > 0) {
     // the scorer's top_n, plus the best four of each kernel variant that the
-    // top_n leaves out, so that both kernels are always timed
+    // top_n leaves out, so that every kernel is always timed
     int total = 0;
     qg::candidate_grid(f, M, N, K, nullptr, 0, &total);
     std::vector<qg_config> ranked((size_t)std::max(total, 1));
     if (qgemm_rank_configs(f, M, N, K, ranked.data(), total, nullptr, &n) != QG_OK) n = 0;
     std::vector<qg_config> out;
-    int per_variant[2] = {0, 0};
+    int per_variant[3] = {0, 0, 0};
     for (int i = 0; i < n; ++i) {
       const int v = ranked[i].variant;
       if (i < top_n || per_variant[v] < 4) {

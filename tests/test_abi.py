@@ -144,8 +144,28 @@ def test_run_reserved_fields_must_be_zero():
     c = qg.make_config()
     c.rows = 32                                     # rows belongs to the decode kernel only
     assert _run(cfg=c) == qg.QG_ERR_INVALID_ARG
-    c = qg.make_config(variant=2)
+    c = qg.make_config(variant=3)                   # no such kernel
     assert _run(cfg=c) == qg.QG_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(), qg.QG_ERR_NO_DEVICE),                                  # valid: reaches the device check
+    (dict(tile_n=128, stages=4), qg.QG_ERR_NO_DEVICE),
+    (dict(tile_n=64), qg.QG_ERR_UNSUPPORTED),                       # 128- or 256-wide tiles only
+    (dict(stages=13), qg.QG_ERR_UNSUPPORTED),
+    (dict(tile_n=256, stages=5), qg.QG_ERR_UNSUPPORTED),            # 5 x 48 KB + 64 KB of y boxes: beyond smem
+])
+def test_persistent_config_checks(kw, status):
+    c = qg.persist_config(**kw)
+    assert _run(M=512, N=512, cfg=c) == status
+    for bad in (dict(split_k=2), dict(swap_ab=1), dict(reduce_mode=1), dict(rows=16)):
+        c2 = qg.persist_config(**kw)
+        for k, v in bad.items():
+            setattr(c2, k, v)
+        assert _run(M=512, N=512, cfg=c2) == qg.QG_ERR_UNSUPPORTED
+    # Block_FP8 and NVFP4 have no persistent kernel
+    assert _run(fmt=qg.QG_BLOCK_FP8, M=512, N=512, cfg=qg.persist_config()) == qg.QG_ERR_UNSUPPORTED
+    assert _run(fmt=qg.QG_NVFP4, M=512, N=512, cfg=qg.persist_config()) == qg.QG_ERR_UNSUPPORTED
 
 
 @pytest.mark.parametrize("kw,status", [
