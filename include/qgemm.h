@@ -100,11 +100,13 @@ typedef struct {
                           and `stages` (the ring of 128-byte K tiles, 2..64) a
                           multiple of the K groups of its eight compute warps:
                           64 / rows (128 / rows for tile_n = 8);
-                          2: the persistent kernel for FP8_DYNAMIC and W8A8_INT8
-                          at large M: one CTA per SM walks the 128 x tile_n
-                          output tiles with two TMEM accumulators, so a tile's
-                          epilogue (bf16 through TMA stores) overlaps the next
-                          tile's MMAs; requires split_k = 1, swap_ab = 0,
+                          2: the persistent kernel for the 8-bit formats at
+                          large M: one CTA per SM walks the 128 x tile_n
+                          output tiles, so a tile's epilogue (bf16 through TMA
+                          stores) overlaps the next tile's MMAs (FP8_DYNAMIC,
+                          W8A8_INT8: two TMEM accumulators; BLOCK_FP8: the
+                          promotion's group buffers, free once a tile's last
+                          group is promoted); requires split_k = 1, swap_ab = 0,
                           reduce_mode = 0, rows = 0, tile_n 128 or 256,
                           stages 2..12 (capped by shared memory), and bf16
                           output (QG_ERR_UNSUPPORTED otherwise); y is bitwise

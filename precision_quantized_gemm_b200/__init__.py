@@ -70,9 +70,9 @@ def make_config(split_k=1, swap_ab=1, tile_n=16, stages=8, reduce_mode=0, varian
 
 
 def persist_config(tile_n=256, stages=3) -> qg_config:
-    """Configuration of the persistent kernel (FP8_Dynamic, W8A8_INT8; large
-    M): one CTA per SM walks the 128 x tile_n output tiles, two TMEM
-    accumulators overlap a tile's epilogue with the next tile's MMAs."""
+    """Configuration of the persistent kernel (8-bit formats; large M): one
+    CTA per SM walks the 128 x tile_n output tiles, overlapping a tile's
+    epilogue with the next tile's MMAs."""
     return make_config(split_k=1, swap_ab=0, tile_n=tile_n, stages=stages, reduce_mode=0, variant=2)
 
 

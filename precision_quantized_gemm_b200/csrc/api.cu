@@ -177,17 +177,19 @@ size_t skinny_smem(qg_format f, const qg_config* c) {
   }
 }
 
-size_t persist_smem(qg_format f, const qg_config* c) {
+size_t persist_smem(qg_format f, int K, const qg_config* c) {
+  const int nkt = kt_total(f, K);
   switch (f) {
-    case QG_FP8_DYNAMIC: return qg::launch_gemm_fp8_persist_smem(c->tile_n, c->stages);
-    case QG_W8A8_INT8: return qg::launch_gemm_int8_persist_smem(c->tile_n, c->stages);
+    case QG_FP8_DYNAMIC: return qg::launch_gemm_fp8_persist_smem(c->tile_n, c->stages, nkt);
+    case QG_W8A8_INT8: return qg::launch_gemm_int8_persist_smem(c->tile_n, c->stages, nkt);
+    case QG_BLOCK_FP8: return qg::launch_gemm_block_persist_smem(c->tile_n, c->stages, nkt);
     default: return (size_t)1 << 30;
   }
 }
 
 size_t gemm_smem(qg_format f, int M, int K, const qg_config* c, bool fused) {
   if (c->variant == 1) return skinny_smem(f, c);
-  if (c->variant == 2) return persist_smem(f, c);
+  if (c->variant == 2) return persist_smem(f, K, c);
   const LaunchShape ls = launch_shape(f, M, K, c, fused);
   const bool swap = c->swap_ab != 0;
   const int tn = c->tile_n, st = c->stages;
@@ -238,13 +240,13 @@ qg_status check_skinny_config(qg_format f, const qg_config* c) {
 }
 
 // The persistent kernel: the standard orientation without split-K, tiles of
-// 128 or 256 channels, FP8_DYNAMIC and W8A8_INT8 (bf16 output, checked at
-// launch: the tile store needs a tensor map of y).
-qg_status check_persist_config(qg_format f, const qg_config* c) {
-  if (f != QG_FP8_DYNAMIC && f != QG_W8A8_INT8) return QG_ERR_UNSUPPORTED;
+// 128 or 256 channels, FP8_DYNAMIC, W8A8_INT8 and BLOCK_FP8 (bf16 output,
+// checked at launch: the tile store needs a tensor map of y).
+qg_status check_persist_config(qg_format f, int K, const qg_config* c) {
+  if (f != QG_FP8_DYNAMIC && f != QG_W8A8_INT8 && f != QG_BLOCK_FP8) return QG_ERR_UNSUPPORTED;
   if (c->split_k != 1 || c->swap_ab != 0 || c->reduce_mode != 0 || c->rows != 0) return QG_ERR_UNSUPPORTED;
   if (c->tile_n != 128 && c->tile_n != 256) return QG_ERR_UNSUPPORTED;
-  if (c->stages < 2 || c->stages > 12 || persist_smem(f, c) > kSmemLimit) return QG_ERR_UNSUPPORTED;
+  if (c->stages < 2 || c->stages > 12 || persist_smem(f, K, c) > kSmemLimit) return QG_ERR_UNSUPPORTED;
   return QG_OK;
 }
 
@@ -253,7 +255,7 @@ qg_status check_config(qg_format f, int M, int N, int K, const qg_config* c) {
   if (c->reserved) return QG_ERR_INVALID_ARG;
   if (c->variant < 0 || c->variant > 2) return QG_ERR_INVALID_ARG;
   if (c->variant == 1) return check_skinny_config(f, c);
-  if (c->variant == 2) return check_persist_config(f, c);
+  if (c->variant == 2) return check_persist_config(f, K, c);
   if (c->rows != 0) return QG_ERR_INVALID_ARG;
   if (!is_pow2(c->split_k) || c->split_k > 256) return QG_ERR_UNSUPPORTED;
   if (c->swap_ab != 0 && c->swap_ab != 1) return QG_ERR_INVALID_ARG;
@@ -590,9 +592,12 @@ qg_status launch_run(qg_format f, const qg_operand* A, const void* act, int lda,
     if (!make_tmap(&tq, W->q, rb, (uint64_t)N, (uint32_t)cfg->tile_n)) return QG_ERR_CUDA;
     if (!make_tmap_y(&ty, Y, N, M, ldy)) return QG_ERR_UNSUPPORTED;
     cudaStream_t st = (cudaStream_t)stream;
-    cudaError_t e = f == QG_FP8_DYNAMIC
-                        ? qg::launch_gemm_fp8_persist(cfg->tile_n, tp, tq, ty, prm, dim3(ctas), st, g_pdl)
-                        : qg::launch_gemm_int8_persist(cfg->tile_n, tp, tq, ty, prm, dim3(ctas), st, g_pdl);
+    cudaError_t e;
+    switch (f) {
+      case QG_FP8_DYNAMIC: e = qg::launch_gemm_fp8_persist(cfg->tile_n, tp, tq, ty, prm, dim3(ctas), st, g_pdl); break;
+      case QG_W8A8_INT8: e = qg::launch_gemm_int8_persist(cfg->tile_n, tp, tq, ty, prm, dim3(ctas), st, g_pdl); break;
+      default: e = qg::launch_gemm_block_persist(cfg->tile_n, tp, tq, ty, prm, dim3(ctas), st, g_pdl); break;
+    }
     if (e != cudaSuccess) return e == cudaErrorInvalidValue ? QG_ERR_UNSUPPORTED : QG_ERR_CUDA;
     return QG_OK;
   }

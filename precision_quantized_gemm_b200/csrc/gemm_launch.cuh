@@ -5,6 +5,7 @@
 // format's unit and QG_GROUPED_ONLY in that second unit (the two compile in
 // parallel).
 #pragma once
+#include <atomic>
 #include "attr_cache.h"
 #include "gemm_kernel.cuh"
 #include "internal.h"
@@ -197,6 +198,49 @@ cudaError_t launch_persist_one(const CUtensorMap& tp, const CUtensorMap& tq, con
   return cudaLaunchKernelEx(&cfg, kern, tp, tq, ty, prm);
 }
 
+template <int BN>
+cudaError_t launch_persist_block_one(const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap& ty,
+                                     const GemmParams& prm, dim3 grid, cudaStream_t st, bool pdl) {
+  auto kern = qgemm_persist_block_kernel<BN>;
+  if constexpr (PbCfg<BN>::kRegSplit) {
+    // setmaxnreg.inc waits until the new counts fit the CTA's launch
+    // allocation: launch only the build whose count the split was sized for
+    static std::atomic<int> regs{0};
+    int r = regs.load(std::memory_order_relaxed);
+    if (r == 0) {
+      cudaFuncAttributes fa;
+      const cudaError_t e0 = cudaFuncGetAttributes(&fa, kern);
+      if (e0 != cudaSuccess) return e0;
+      r = fa.numRegs;
+      regs.store(r, std::memory_order_relaxed);
+    }
+    if (r != PbCfg<BN>::kRegsLaunch) return cudaErrorInvalidValue;
+  }
+  size_t smem = pb_smem_bytes<BN>(prm.stages, prm.kt_total);
+  // the group buffers take all 512 TMEM columns: one CTA per SM
+  const size_t smem_floor = (size_t)233472 / 2;
+  if (smem < smem_floor) smem = smem_floor;
+  static GrowOnlyAttr smem_attr;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = static_cast<cudaError_t>(smem_attr.ensure(dev, (int)smem, [&](int bytes) {
+    return static_cast<int>(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  }));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(PbCfg<BN>::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, tp, tq, ty, prm);
+}
+
 template <int FMT, int TM>
 size_t skinny_smem_rows(int rows, int stages) {
   switch (rows) {
@@ -234,21 +278,28 @@ cudaError_t QG_CAT(QG_LAUNCH_NAME, _skinny)(int tile_n, int rows, const CUtensor
   }
 }
 
-// The persistent kernel (variant 2): FP8_Dynamic and W8A8_INT8, tile_n 128 or 256.
+// The persistent kernel (variant 2): FP8_Dynamic, W8A8_INT8 and Block_FP8,
+// tile_n 128 or 256.
 cudaError_t QG_CAT(QG_LAUNCH_NAME, _persist)(int tile_n, const CUtensorMap& tp, const CUtensorMap& tq,
                                              const CUtensorMap& ty, const GemmParams& prm, dim3 grid,
                                              cudaStream_t st, bool pdl) {
   if constexpr (QG_FMT == kFP8 || QG_FMT == kINT8) {
     if (tile_n == 128) return launch_persist_one<QG_FMT, 128>(tp, tq, ty, prm, grid, st, pdl);
     if (tile_n == 256) return launch_persist_one<QG_FMT, 256>(tp, tq, ty, prm, grid, st, pdl);
+  } else if constexpr (QG_FMT == kBLOCK) {
+    if (tile_n == 128) return launch_persist_block_one<128>(tp, tq, ty, prm, grid, st, pdl);
+    if (tile_n == 256) return launch_persist_block_one<256>(tp, tq, ty, prm, grid, st, pdl);
   }
   return cudaErrorInvalidValue;
 }
 
-size_t QG_CAT(QG_LAUNCH_NAME, _persist_smem)(int tile_n, int stages) {
+size_t QG_CAT(QG_LAUNCH_NAME, _persist_smem)(int tile_n, int stages, int nkt) {
   if constexpr (QG_FMT == kFP8 || QG_FMT == kINT8) {
     if (tile_n == 128) return ps_smem_bytes<QG_FMT, 128>(stages);
     if (tile_n == 256) return ps_smem_bytes<QG_FMT, 256>(stages);
+  } else if constexpr (QG_FMT == kBLOCK) {
+    if (tile_n == 128) return pb_smem_bytes<128>(stages, nkt);
+    if (tile_n == 256) return pb_smem_bytes<256>(stages, nkt);
   }
   return (size_t)1 << 30;
 }

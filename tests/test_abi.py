@@ -163,9 +163,11 @@ def test_persistent_config_checks(kw, status):
         for k, v in bad.items():
             setattr(c2, k, v)
         assert _run(M=512, N=512, cfg=c2) == qg.QG_ERR_UNSUPPORTED
-    # Block_FP8 and NVFP4 have no persistent kernel
-    assert _run(fmt=qg.QG_BLOCK_FP8, M=512, N=512, cfg=qg.persist_config()) == qg.QG_ERR_UNSUPPORTED
+    # NVFP4 has no persistent kernel; Block_FP8's keeps a share of shared
+    # memory for the tile's scales (more the longer K)
     assert _run(fmt=qg.QG_NVFP4, M=512, N=512, cfg=qg.persist_config()) == qg.QG_ERR_UNSUPPORTED
+    assert _run(fmt=qg.QG_BLOCK_FP8, M=512, N=512, K=5120, cfg=qg.persist_config(256, 3)) == qg.QG_ERR_NO_DEVICE
+    assert _run(fmt=qg.QG_BLOCK_FP8, M=512, N=512, K=65536, cfg=qg.persist_config(256, 3)) == qg.QG_ERR_UNSUPPORTED
 
 
 @pytest.mark.parametrize("kw,status", [

@@ -1,6 +1,7 @@
-"""GPU parity of the persistent kernel (qg_config.variant = 2): FP8_Dynamic and
-W8A8_INT8 in the standard orientation, one CTA per SM walking the 128 x
-tile_n output tiles with two TMEM accumulators.
+"""GPU parity of the persistent kernel (qg_config.variant = 2): the 8-bit
+formats in the standard orientation, one CTA per SM walking the 128 x tile_n
+output tiles (FP8_Dynamic / W8A8_INT8 with two TMEM accumulators, Block_FP8
+with its promotion's group buffers).
 
 Its MMAs accumulate each tile's K tiles in the tile kernel's order and its
 epilogue applies the same fp32 arithmetic, so y is bitwise that of the tile
@@ -25,6 +26,11 @@ CASES = [  # (format, M, N, K, tile_n, stages)
     (qg.QG_FP8_DYNAMIC, 2048, 4096, 1024, 128, 4),    # 512 tiles of 128
     (qg.QG_W8A8_INT8, 129, 392, 272, 128, 2),         # K % 128 != 0: a partial last K tile
     (qg.QG_FP8_DYNAMIC, 520, 1536, 4096, 256, 3),
+    # Block_FP8: promotion into register accumulators, group buffers shared by consecutive tiles
+    (qg.QG_BLOCK_FP8, 300, 640, 1024, 256, 3),
+    (qg.QG_BLOCK_FP8, 2048, 2560, 2048, 256, 3),       # 320 tiles: several per CTA
+    (qg.QG_BLOCK_FP8, 1000, 1152, 512, 128, 3),
+    (qg.QG_BLOCK_FP8, 4096, 5120, 5120, 256, 3),
 ]
 
 
@@ -68,10 +74,10 @@ def test_persistent_refuses_what_it_does_not_cover():
     W = qg.quantize_weight(fmt, to_dev_bf16(w))
     with pytest.raises(qg.QGemmError):                 # raw accumulators: the tile store is bf16 only
         qg.run(fmt, A, W, qg.persist_config(), out_kind=qg.QG_OUT_ACC)
-    Ab = qg.quantize_act(qg.QG_BLOCK_FP8, to_dev_bf16(a))
-    Wb = qg.quantize_weight(qg.QG_BLOCK_FP8, to_dev_bf16(w))
-    with pytest.raises(qg.QGemmError):                 # FP8_Dynamic and W8A8_INT8 only
-        qg.run(qg.QG_BLOCK_FP8, Ab, Wb, qg.persist_config())
+    An = qg.quantize_act(qg.QG_NVFP4, to_dev_bf16(a))
+    Wn = qg.quantize_weight(qg.QG_NVFP4, to_dev_bf16(w))
+    with pytest.raises(qg.QGemmError):                 # the 8-bit formats only
+        qg.run(qg.QG_NVFP4, An, Wn, qg.persist_config())
 
 
 def test_persistent_in_a_graph_after_the_quantiser():
