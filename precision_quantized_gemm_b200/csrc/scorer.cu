@@ -112,9 +112,16 @@ double estimate_us(qg_format f, int M, int N, int K, const qg_config& c, int sms
     // tuner's measurements decide).  Block_FP8's promotion epilogue runs on
     // the same SM as the next tile's MMAs and wins only at some shapes, so
     // there the tile kernel stays the untuned choice.
+    // The base is the tile kernel at the persistent ring's own depth
+    // (256-wide tiles, 4 stages; 3 for Block_FP8), not at c's: with one CTA
+    // per SM the ring alone keeps the loads in flight, and the candidates
+    // below are the rings deep enough for that (128-wide tiles a shade
+    // behind 256-wide ones).
     qg_config t = c;
     t.variant = 0;
-    return (f == QG_BLOCK_FP8 ? 1.02 : 0.88) * estimate_us(f, M, N, K, t, sms);
+    t.tile_n = 256;
+    t.stages = f == QG_BLOCK_FP8 ? 3 : 4;
+    return (f == QG_BLOCK_FP8 ? 1.02 : 0.88) * (c.tile_n == 256 ? 1.0 : 1.03) * estimate_us(f, M, N, K, t, sms);
   }
   const Model& m = kModel;
   const double rb = f == QG_NVFP4 ? K / 2.0 : (double)K;
@@ -185,23 +192,26 @@ void candidate_grid(qg_format f, int M, int N, int K, qg_config* out, int max_ou
           }
     }
   }
-  // the persistent kernel (8-bit formats, at least 256 tokens): 128- or
-  // 256-wide tiles, rings of 3, 4 or 6 stages (as far as they fit)
+  // the persistent kernel (8-bit formats, at least 256 tokens): the rings
+  // that keep about 190 KB of operands in flight per SM (256-wide tiles with
+  // 4 stages, 128-wide with 6; Block_FP8, whose partials and scales take the
+  // rest of shared memory, 256-wide with 3).  Shallower rings measured up to
+  // 1.6x slower at one CTA per SM.
   if (f != QG_NVFP4 && M >= 256) {
-    for (int tn : {128, 256})
-      for (int st : {3, 4, 6}) {
-        if (n < max_out) {
-          qg_config c = {};
-          c.split_k = 1;
-          c.swap_ab = 0;
-          c.tile_n = tn;
-          c.stages = st;
-          c.reduce_mode = 0;
-          c.variant = 2;
-          out[n] = c;
-        }
-        ++n;
+    const int rings[2][2] = {{256, f == QG_BLOCK_FP8 ? 3 : 4}, {128, 6}};
+    for (int r = 0; r < (f == QG_BLOCK_FP8 ? 1 : 2); ++r) {
+      if (n < max_out) {
+        qg_config c = {};
+        c.split_k = 1;
+        c.swap_ab = 0;
+        c.tile_n = rings[r][0];
+        c.stages = rings[r][1];
+        c.reduce_mode = 0;
+        c.variant = 2;
+        out[n] = c;
       }
+      ++n;
+    }
   }
   // the decode kernel (8-bit formats, up to 32 tokens per CTA): rows per
   // CTA, and rings of 8, 16, 32 or every K tile (up to 64) rounded to the K
