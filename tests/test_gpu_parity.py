@@ -166,6 +166,9 @@ STD_CASES = [
     (260, 520, 2048, 1, 256, 0, 3),   # wide tile: Block_FP8 promotes with 8 epilogue warps
     (200, 300, 1024, 2, 256, 0, 3),
     (140, 300, 1024, 2, 128, 2, 4),   # last-CTA reduction of a 128-wide tile
+    (140, 300, 1024, 2, 128, 0, 4),   # cluster pull reduction of a 128-wide tile, ragged M and N
+    (260, 384, 2048, 8, 128, 0, 4),   # pull over eight CTAs, 16 rows owned each
+    (150, 520, 2048, 2, 256, 0, 4),   # 256-wide pull, four-stage ring
 ]
 
 
@@ -236,6 +239,18 @@ def test_split_k_deterministic_and_modes_agree():
           for r in (0, 1, 2, 0, 2)]
     for y in ys[1:]:
         assert torch.equal(ys[0], y)     # fixed split order: every mode, every run, same bits
+
+
+@pytest.mark.parametrize("fmt", [qg.QG_FP8_DYNAMIC, qg.QG_BLOCK_FP8, qg.QG_NVFP4], ids=["fp8", "block", "nvfp4"])
+@pytest.mark.parametrize("sk", [2, 4, 8])
+def test_wide_tile_cluster_reduction_agrees_with_workspace_modes(fmt, sk):
+    # standard orientation, 128-wide tiles: the cluster's pull reduction sums
+    # in the same split order as the two workspace reductions
+    A, W, _, _ = _setup(fmt, 200, 384, 4096)
+    ys = [qg.run(fmt, A, W, qg.make_config(split_k=sk, swap_ab=0, tile_n=128, stages=4, reduce_mode=r))
+          for r in (0, 1, 2)]
+    for y in ys[1:]:
+        assert torch.equal(ys[0], y)
 
 
 def test_swap_and_standard_agree_int8_bitwise():
