@@ -1,5 +1,6 @@
 // persist.cuh — the persistent variant of the quantized GEMM for large M
-// (qg_config.variant = 2): standard orientation, FP8_Dynamic and W8A8_INT8.
+// (qg_config.variant = 2): standard orientation, FP8_Dynamic and W8A8_INT8
+// (qgemm_persist_kernel) and Block_FP8 (qgemm_persist_block_kernel, below).
 //
 // Why a third kernel: the tile kernel runs one 128 x BN output tile per CTA,
 // so every tile pays the CTA's set-up, the pipeline fill and its epilogue
