@@ -124,12 +124,12 @@ def kernel_source_code(text: str) -> str:
 
 
 def kernel_source_hash():
-    """sha1 of the GEMM kernels' code (gemm_kernel.cuh, skinny.cuh and
-    ptx.cuh, comments ignored): ties an ncu traffic figure to the code it
-    measured."""
+    """sha1 of the GEMM kernels' code (gemm_kernel.cuh, skinny.cuh,
+    persist.cuh, pair.cuh and ptx.cuh, comments ignored): ties an ncu
+    traffic figure to the code it measured."""
     import hashlib
     h = hashlib.sha1()
-    for f in ("gemm_kernel.cuh", "skinny.cuh", "ptx.cuh"):
+    for f in ("gemm_kernel.cuh", "skinny.cuh", "persist.cuh", "pair.cuh", "ptx.cuh"):
         with open(os.path.join(ROOT, "precision_quantized_gemm_b200", "csrc", f), encoding="utf-8") as fh:
             h.update(kernel_source_code(fh.read()).encode())
     return h.hexdigest()[:12]

@@ -76,6 +76,13 @@ def persist_config(tile_n=256, stages=3) -> qg_config:
     return make_config(split_k=1, swap_ab=0, tile_n=tile_n, stages=stages, reduce_mode=0, variant=2)
 
 
+def pair_config(tile_n=256, stages=4) -> qg_config:
+    """Configuration of the CTA-pair kernel (Block_FP8, large M): clusters of
+    two CTAs walk 256 x tile_n output tiles (tile_n 128 or 256) with one
+    two-SM MMA per K step."""
+    return make_config(split_k=1, swap_ab=0, tile_n=tile_n, stages=stages, reduce_mode=0, variant=3)
+
+
 def skinny_config(tile_n=16, rows=32, stages=32) -> qg_config:
     """Configuration of the decode ("skinny") kernel: `rows` weight rows per
     CTA over the whole of K, `tile_n` tokens, a ring of `stages` K tiles."""

@@ -187,9 +187,15 @@ size_t persist_smem(qg_format f, int K, const qg_config* c) {
   }
 }
 
+size_t pair_smem(qg_format f, int K, const qg_config* c) {
+  if (f != QG_BLOCK_FP8) return (size_t)1 << 30;
+  return qg::launch_gemm_block_pair_smem(c->tile_n, c->stages, kt_total(f, K));
+}
+
 size_t gemm_smem(qg_format f, int M, int K, const qg_config* c, bool fused) {
   if (c->variant == 1) return skinny_smem(f, c);
   if (c->variant == 2) return persist_smem(f, K, c);
+  if (c->variant == 3) return pair_smem(f, K, c);
   const LaunchShape ls = launch_shape(f, M, K, c, fused);
   const bool swap = c->swap_ab != 0;
   const int tn = c->tile_n, st = c->stages;
@@ -250,12 +256,23 @@ qg_status check_persist_config(qg_format f, int K, const qg_config* c) {
   return QG_OK;
 }
 
+// CTA pairs (variant 3): Block_FP8, standard orientation, 256 x tile_n
+// pair tiles (tile_n 128 or 256), no split.
+qg_status check_pair_config(qg_format f, int K, const qg_config* c) {
+  if (f != QG_BLOCK_FP8) return QG_ERR_UNSUPPORTED;
+  if (c->split_k != 1 || c->swap_ab != 0 || c->reduce_mode != 0 || c->rows != 0) return QG_ERR_UNSUPPORTED;
+  if (c->tile_n != 128 && c->tile_n != 256) return QG_ERR_UNSUPPORTED;
+  if (c->stages < 2 || c->stages > 12 || pair_smem(f, K, c) > kSmemLimit) return QG_ERR_UNSUPPORTED;
+  return QG_OK;
+}
+
 qg_status check_config(qg_format f, int M, int N, int K, const qg_config* c) {
   if (!c) return QG_ERR_INVALID_ARG;
   if (c->reserved) return QG_ERR_INVALID_ARG;
-  if (c->variant < 0 || c->variant > 2) return QG_ERR_INVALID_ARG;
+  if (c->variant < 0 || c->variant > 3) return QG_ERR_INVALID_ARG;
   if (c->variant == 1) return check_skinny_config(f, c);
   if (c->variant == 2) return check_persist_config(f, K, c);
+  if (c->variant == 3) return check_pair_config(f, K, c);
   if (c->rows != 0) return QG_ERR_INVALID_ARG;
   if (!is_pow2(c->split_k) || c->split_k > 256) return QG_ERR_UNSUPPORTED;
   if (c->swap_ab != 0 && c->swap_ab != 1) return QG_ERR_INVALID_ARG;
@@ -598,6 +615,28 @@ qg_status launch_run(qg_format f, const qg_operand* A, const void* act, int lda,
       case QG_W8A8_INT8: e = qg::launch_gemm_int8_persist(cfg->tile_n, tp, tq, ty, prm, dim3(ctas), st, g_pdl); break;
       default: e = qg::launch_gemm_block_persist(cfg->tile_n, tp, tq, ty, prm, dim3(ctas), st, g_pdl); break;
     }
+    if (e != cudaSuccess) return e == cudaErrorInvalidValue ? QG_ERR_UNSUPPORTED : QG_ERR_CUDA;
+    return QG_OK;
+  }
+  if (cfg->variant == 3) {
+    // CTA pairs: clusters of two CTAs (one per SM) walking the 256 x tile_n
+    // output tiles; bf16 output through a tensor map of y
+    if (out_kind != QG_OUT_BF16 || act != nullptr || expert_offsets != nullptr) return QG_ERR_UNSUPPORTED;
+    prm.nkt_max = prm.kt_total;
+    prm.err = d->err;
+    prm.wait_ns = g_wait_ns;
+    const long long tiles = (long long)((M + 255) / 256) * ((N + cfg->tile_n - 1) / cfg->tile_n);
+    const int pairs = (int)std::min<long long>(tiles, (d->sms > 0 ? d->sms : 148) / 2);
+    const int ctas = 2 * pairs;
+    if (g_trace != nullptr && (size_t)ctas * qg::kTraceEvents * sizeof(unsigned long long) <= g_trace_bytes)
+      prm.trace = g_trace;
+    CUtensorMap tp, tq, ty;
+    const uint64_t rb = row_bytes(f, K);
+    if (!make_tmap(&tp, A->q, rb, (uint64_t)M, 128)) return QG_ERR_CUDA;
+    if (!make_tmap(&tq, W->q, rb, (uint64_t)N, (uint32_t)(cfg->tile_n / 2))) return QG_ERR_CUDA;
+    if (!make_tmap_y(&ty, Y, N, M, ldy)) return QG_ERR_UNSUPPORTED;
+    const cudaError_t e =
+        qg::launch_gemm_block_pair(cfg->tile_n, tp, tq, ty, prm, dim3(ctas), (cudaStream_t)stream, g_pdl);
     if (e != cudaSuccess) return e == cudaErrorInvalidValue ? QG_ERR_UNSUPPORTED : QG_ERR_CUDA;
     return QG_OK;
   }

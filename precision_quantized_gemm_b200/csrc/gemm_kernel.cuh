@@ -288,6 +288,19 @@ __device__ __forceinline__ int slice_index(int rl, int c, int rows_per) {
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
+// Named barrier over n threads that returns to every one of them whether
+// any passed `v` true: a decision all of them take the same way (a flag
+// another role may set meanwhile, read once per thread, would not be).
+__device__ __forceinline__ bool named_bar_or(int id, int n, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, %2, %3, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
 
 __device__ __forceinline__ uint32_t ld_u32_cg(const void* p) {
   return __ldcg(reinterpret_cast<const unsigned int*>(p));

@@ -9,6 +9,7 @@
 #include "attr_cache.h"
 #include "gemm_kernel.cuh"
 #include "internal.h"
+#include "pair.cuh"
 #include "persist.cuh"
 #include "skinny.cuh"
 
@@ -241,6 +242,54 @@ cudaError_t launch_persist_block_one(const CUtensorMap& tp, const CUtensorMap& t
   return cudaLaunchKernelEx(&cfg, kern, tp, tq, ty, prm);
 }
 
+// Block_FP8 on CTA pairs (variant 3): clusters of two along x, one CTA per
+// SM (the pair's TMEM takes all 512 columns of each).
+template <int BN>
+cudaError_t launch_pair_block(const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap& ty,
+                              const GemmParams& prm, dim3 grid, cudaStream_t st, bool pdl) {
+  auto kern = qgemm_pair_block_kernel<BN>;
+  {
+    // setmaxnreg.inc waits until the new counts fit the CTA's launch
+    // allocation: launch only the build whose count the split was sized for
+    static std::atomic<int> regs{0};
+    int r = regs.load(std::memory_order_relaxed);
+    if (r == 0) {
+      cudaFuncAttributes fa;
+      const cudaError_t e0 = cudaFuncGetAttributes(&fa, kern);
+      if (e0 != cudaSuccess) return e0;
+      r = fa.numRegs;
+      regs.store(r, std::memory_order_relaxed);
+    }
+    if (r != PpCfg<BN>::kRegsLaunch) return cudaErrorInvalidValue;
+  }
+  size_t smem = pp_smem_bytes<BN>(prm.stages);
+  const size_t smem_floor = (size_t)233472 / 2;
+  if (smem < smem_floor) smem = smem_floor;
+  static GrowOnlyAttr smem_attr;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = static_cast<cudaError_t>(smem_attr.ensure(dev, (int)smem, [&](int bytes) {
+    return static_cast<int>(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  }));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(PpCfg<BN>::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, kern, tp, tq, ty, prm);
+}
+
 template <int FMT, int TM>
 size_t skinny_smem_rows(int rows, int stages) {
   switch (rows) {
@@ -291,6 +340,26 @@ cudaError_t QG_CAT(QG_LAUNCH_NAME, _persist)(int tile_n, const CUtensorMap& tp, 
     if (tile_n == 256) return launch_persist_block_one<256>(tp, tq, ty, prm, grid, st, pdl);
   }
   return cudaErrorInvalidValue;
+}
+
+// Block_FP8 on CTA pairs (variant 3): pair tiles of 256 x 128 or 256 x 256.
+cudaError_t QG_CAT(QG_LAUNCH_NAME, _pair)(int tile_n, const CUtensorMap& tp, const CUtensorMap& tq,
+                                          const CUtensorMap& ty, const GemmParams& prm, dim3 grid,
+                                          cudaStream_t st, bool pdl) {
+  if constexpr (QG_FMT == kBLOCK) {
+    if (tile_n == 128) return launch_pair_block<128>(tp, tq, ty, prm, grid, st, pdl);
+    if (tile_n == 256) return launch_pair_block<256>(tp, tq, ty, prm, grid, st, pdl);
+  }
+  return cudaErrorInvalidValue;
+}
+
+size_t QG_CAT(QG_LAUNCH_NAME, _pair_smem)(int tile_n, int stages, int nkt) {
+  (void)nkt;
+  if constexpr (QG_FMT == kBLOCK) {
+    if (tile_n == 128) return pp_smem_bytes<128>(stages);
+    if (tile_n == 256) return pp_smem_bytes<256>(stages);
+  }
+  return (size_t)1 << 30;
 }
 
 size_t QG_CAT(QG_LAUNCH_NAME, _persist_smem)(int tile_n, int stages, int nkt) {

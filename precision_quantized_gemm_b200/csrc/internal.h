@@ -62,7 +62,11 @@ cudaError_t launch_quant_nvfp4(const void* X, int R, int K, int ldx, const float
   cudaError_t NAME##_persist(int tile_n, const CUtensorMap& tp, const CUtensorMap& tq,     \
                              const CUtensorMap& ty, const GemmParams& prm, dim3 grid,      \
                              cudaStream_t st, bool pdl);                                   \
-  size_t NAME##_persist_smem(int tile_n, int stages, int nkt);
+  size_t NAME##_persist_smem(int tile_n, int stages, int nkt);                              \
+  cudaError_t NAME##_pair(int tile_n, const CUtensorMap& tp, const CUtensorMap& tq,        \
+                          const CUtensorMap& ty, const GemmParams& prm, dim3 grid,         \
+                          cudaStream_t st, bool pdl);                                      \
+  size_t NAME##_pair_smem(int tile_n, int stages, int nkt);
 QG_DECLARE_GEMM_LAUNCH(launch_gemm_fp8)
 QG_DECLARE_GEMM_LAUNCH(launch_gemm_int8)
 QG_DECLARE_GEMM_LAUNCH(launch_gemm_block)

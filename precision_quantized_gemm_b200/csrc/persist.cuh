@@ -201,8 +201,8 @@ __global__ void __launch_bounds__(PsCfg<FMT, BN>::kThreads, 1)
       if (etid == 0) bulk_wait_read_all();
       const bool got = mbar_wait(&acc_full[ab], (uint32_t)((j >> 1) & 1), prm.err, prm.wait_ns);
       if (!__all_sync(0xffffffffu, got)) *flag_abort = 1;
-      named_bar_sync(1, 128);                  // scales staged, boxes free, abort state settled
-      if (*flag_abort) break;
+      // scales staged, boxes free; every epilogue warp takes the same abort decision
+      if (named_bar_or(1, 128, *flag_abort != 0)) break;
       tc_fence_after();
       const float sa = (p0 + row < prm.M) ? __ldg(prm.scale_a + p0 + row) : 0.f;
 #pragma unroll
@@ -456,8 +456,7 @@ __global__ void __launch_bounds__(PbCfg<BN>::kThreads, 1)
         const int b = q0 / 128 + jb;
         sw_s[idx] = (b < nblk) ? __ldg(prm.scale_w + (size_t)b * G + gl) : 0.f;
       }
-      named_bar_sync(1, ET);
-      if (*flag_abort) break;
+      if (named_bar_or(1, ET, *flag_abort != 0)) break;
       uint64_t acc2[NC / 2];
 #pragma unroll
       for (int c = 0; c < NC / 2; ++c) acc2[c] = 0ull;
@@ -511,8 +510,8 @@ __global__ void __launch_bounds__(PbCfg<BN>::kThreads, 1)
         const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(lo), __uint_as_float(hi));
         yb[c] = *reinterpret_cast<const uint32_t*>(&b2);
       }
-      named_bar_sync(1, ET);                   // every warp's promotion done (or given up)
-      if (*flag_abort) break;
+      // every warp's promotion done (or given up); one abort decision for all
+      if (named_bar_or(1, ET, *flag_abort != 0)) break;
       // ---- store from registers, one 128-channel slice at a time
 #pragma unroll
       for (int y0 = 0; y0 < BN; y0 += 128) {

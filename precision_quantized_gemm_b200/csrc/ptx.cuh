@@ -328,6 +328,58 @@ __device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint6
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
 }
+// ---- CTA pairs (cta_group::2): two CTAs of a cluster share one MMA whose
+// 256 rows are split over them (each holds its 128 rows of A and its half
+// of B in shared memory and its 128 rows of D in TMEM); the even CTA of the
+// pair issues it.
+// Both CTAs allocate (one warp each, the same warp index), with the same
+// destination offset in their shared memory.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void mma_f8f6f4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive once on the barrier at the same shared-memory offset in each CTA
+// of `cta_mask` when the pair's previously issued MMAs finish.
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(cta_mask)
+      : "memory");
+}
+// 2D tiled TMA load into this CTA's shared memory whose bytes complete on
+// the barrier of the pair's even CTA (the issuer of the MMAs that read it):
+// `bar_even` is that barrier's shared::cluster address (mapa).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const void* map, uint32_t bar_even, int x, int y,
+                                                 uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(bar_even), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+// Arrive on a barrier of another CTA of the cluster (shared::cluster
+// address), with the default (CTA-scope release) semantics: a cluster-scope
+// release costs a round trip of ~1000 cycles per arrival.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+
 // Arrive on `bar` once all previously issued tcgen05 async ops of this thread finish.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile(
@@ -411,11 +463,11 @@ __device__ __forceinline__ uint64_t sdesc_plain_32x16(uint32_t saddr) {
 }
 
 // Instruction descriptors (dense, K-major A and B, M = 128).
-__host__ __device__ constexpr uint32_t idesc_f8f6f4_e4m3(int n) {
+__host__ __device__ constexpr uint32_t idesc_f8f6f4_e4m3(int n, int m = 128) {
   return (1u << 4)                       // D = f32
          | (0u << 7) | (0u << 10)        // A, B = e4m3
          | ((uint32_t)(n >> 3) << 17)    // N
-         | ((uint32_t)(128 >> 4) << 24); // M
+         | ((uint32_t)(m >> 4) << 24);   // M (256: a CTA pair)
 }
 __host__ __device__ constexpr uint32_t idesc_i8(int n) {
   return (2u << 4)                       // D = s32

@@ -106,6 +106,16 @@ double estimate_skinny_us(qg_format f, int M, int N, int K, const qg_config& c, 
 
 double estimate_us(qg_format f, int M, int N, int K, const qg_config& c, int sms) {
   if (c.variant == 1) return estimate_skinny_us(f, M, N, K, c, sms);
+  if (c.variant == 3) {
+    // CTA pairs (Block_FP8): the 256-wide tile kernel's estimate less the
+    // promotion hand-off that the pair's 256-row MMAs halve per SM (a flat
+    // 12 %; measured 10-27 % at 2048-16384 tokens; the tuner decides)
+    qg_config t = c;
+    t.variant = 0;
+    t.tile_n = 256;
+    t.stages = 3;
+    return 0.88 * estimate_us(f, M, N, K, t, sms);
+  }
   if (c.variant == 2) {
     // the persistent kernel: the tile kernel's estimate less the per-tile
     // set-up and epilogue that the next tile's MMAs hide (a flat 12 %; the
@@ -208,6 +218,25 @@ void candidate_grid(qg_format f, int M, int N, int K, qg_config* out, int max_ou
         c.stages = rings[r][1];
         c.reduce_mode = 0;
         c.variant = 2;
+        out[n] = c;
+      }
+      ++n;
+    }
+  }
+  // CTA pairs (Block_FP8): 256 x 256 pair tiles with rings of 3, 4 or 6
+  // stages, where there are pair tiles for most of the SM pairs (fewer lost
+  // to the tile kernel with split-K: 28-40 tiles measured 4-80 % slower)
+  const long long pair_tiles = (long long)((M + 255) / 256) * ((N + 255) / 256);
+  if (f == QG_BLOCK_FP8 && pair_tiles >= 60) {
+    for (int st : {3, 4, 6}) {
+      if (n < max_out) {
+        qg_config c = {};
+        c.split_k = 1;
+        c.swap_ab = 0;
+        c.tile_n = 256;
+        c.stages = st;
+        c.reduce_mode = 0;
+        c.variant = 3;
         out[n] = c;
       }
       ++n;

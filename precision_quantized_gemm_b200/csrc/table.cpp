@@ -46,7 +46,10 @@ constexpr const char* kMagic = "qgemm-table";
 constexpr int kVersion = 2;
 
 bool valid_cfg_fields(const qg_config& c) {
-  if (c.reserved != 0 || c.variant < 0 || c.variant > 2) return false;
+  if (c.reserved != 0 || c.variant < 0 || c.variant > 3) return false;
+  if (c.variant == 3)
+    return c.split_k == 1 && c.swap_ab == 0 && (c.tile_n == 128 || c.tile_n == 256) && c.stages >= 2 &&
+           c.stages <= 12 && c.reduce_mode == 0 && c.rows == 0;
   if (c.variant == 2)
     return c.split_k == 1 && c.swap_ab == 0 && (c.tile_n == 128 || c.tile_n == 256) && c.stages >= 2 &&
            c.stages <= 12 && c.reduce_mode == 0 && c.rows == 0;

@@ -161,7 +161,7 @@ std::vector<qg_config> candidates(qg_format f, int M, int N, int K, int top_n) {
     std::vector<qg_config> ranked((size_t)std::max(total, 1));
     if (qgemm_rank_configs(f, M, N, K, ranked.data(), total, nullptr, &n) != QG_OK) n = 0;
     std::vector<qg_config> out;
-    int per_variant[3] = {0, 0, 0};
+    int per_variant[4] = {0, 0, 0, 0};
     for (int i = 0; i < n; ++i) {
       const int v = ranked[i].variant;
       if (i < top_n || per_variant[v] < 4) {

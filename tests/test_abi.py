@@ -144,8 +144,31 @@ def test_run_reserved_fields_must_be_zero():
     c = qg.make_config()
     c.rows = 32                                     # rows belongs to the decode kernel only
     assert _run(cfg=c) == qg.QG_ERR_INVALID_ARG
-    c = qg.make_config(variant=3)                   # no such kernel
+    c = qg.make_config(variant=4)                   # no such kernel
     assert _run(cfg=c) == qg.QG_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(), qg.QG_ERR_NO_DEVICE),                                  # valid: reaches the device check
+    (dict(stages=6), qg.QG_ERR_NO_DEVICE),
+    (dict(stages=1), qg.QG_ERR_UNSUPPORTED),
+    (dict(stages=13), qg.QG_ERR_UNSUPPORTED),
+    (dict(stages=8), qg.QG_ERR_NO_DEVICE),                          # 8 x 24 KB + the 32 KB y slice fit
+    (dict(stages=9), qg.QG_ERR_UNSUPPORTED),                        # 9 x 24 KB + 32 KB: beyond smem
+    (dict(tile_n=256, stages=6), qg.QG_ERR_NO_DEVICE),              # 256-wide pair tiles: 32 KB per stage
+    (dict(tile_n=256, stages=7), qg.QG_ERR_UNSUPPORTED),
+])
+def test_pair_config_checks(kw, status):
+    c = qg.pair_config(**({"tile_n": 128} | kw))
+    assert _run(fmt=qg.QG_BLOCK_FP8, M=512, N=512, K=5120, cfg=c) == status
+    for bad in (dict(split_k=2), dict(swap_ab=1), dict(reduce_mode=1), dict(rows=16), dict(tile_n=64)):
+        c2 = qg.pair_config(**({"tile_n": 128} | kw))
+        for k, v in bad.items():
+            setattr(c2, k, v)
+        assert _run(fmt=qg.QG_BLOCK_FP8, M=512, N=512, K=5120, cfg=c2) == qg.QG_ERR_UNSUPPORTED
+    # only Block_FP8 runs on CTA pairs
+    for fmt in (qg.QG_FP8_DYNAMIC, qg.QG_W8A8_INT8, qg.QG_NVFP4):
+        assert _run(fmt=fmt, M=512, N=512, K=5120, cfg=qg.pair_config(128)) == qg.QG_ERR_UNSUPPORTED
 
 
 @pytest.mark.parametrize("kw,status", [
