@@ -111,16 +111,19 @@ typedef struct {
                           stages 2..12 (capped by shared memory), and bf16
                           output (QG_ERR_UNSUPPORTED otherwise); y is bitwise
                           that of variant 0 with the same tile_n;
-                          3: BLOCK_FP8 on CTA pairs at large M: clusters of
-                          two CTAs (one per SM) walk output tiles of 256
-                          tokens x 128 channels; each CTA loads its 128 token
-                          rows and 64 of the weight rows, the even CTA issues
-                          one cta_group::2 MMA (M = 256) per K step, and each
-                          CTA promotes its own rows through four 128-column
-                          TMEM group buffers; requires split_k = 1,
-                          swap_ab = 0, reduce_mode = 0, rows = 0, tile_n 128,
-                          stages 2..12 (capped by shared memory), and bf16
-                          output (QG_ERR_UNSUPPORTED otherwise)              */
+                          3: BLOCK_FP8 on CTA pairs at medium and large M:
+                          clusters of two CTAs (one per SM) walk output
+                          tiles of 256 tokens x tile_n channels; each CTA
+                          loads its 128 token rows and tile_n / 2 of the
+                          weight rows, the even CTA issues one cta_group::2
+                          MMA (M = 256) per K step, and each CTA promotes its
+                          own rows through 512 / tile_n TMEM group buffers;
+                          requires split_k = 1, swap_ab = 0, reduce_mode = 0,
+                          rows = 0, tile_n 128 or 256, stages 2..12 (capped
+                          by shared memory), bf16 output and an output row
+                          pitch of a multiple of 8 elements
+                          (QG_ERR_UNSUPPORTED otherwise); y is bitwise that
+                          of variant 0 with the same tile_n                  */
   int32_t rows;        /* variant 1: weight rows per CTA, 8, 16, 32 or 64 (at
                           least 16 for tile_n = 8); variants 0, 2, 3: 0       */
   int32_t reserved;    /* must be zero                                            */

@@ -279,9 +279,26 @@ def test_table_version1_files_load_as_the_tile_kernel_and_decode_entries_roundtr
     assert hit == 1 and c.as_dict() == sk.as_dict()
 
 
+def test_table_roundtrips_persistent_and_pair_entries(tmp_path):
+    t = qg.Table()
+    t.put(qg.QG_FP8_DYNAMIC, 2048, 4096, 4096, qg.persist_config(256, 4), 29.3)
+    t.put(qg.QG_BLOCK_FP8, 4096, 5120, 5120, qg.pair_config(256, 4), 132.9)
+    t.put(qg.QG_BLOCK_FP8, 1024, 4096, 4096, qg.pair_config(128, 6), 30.0)
+    q = str(tmp_path / "v2.qgt")
+    t.save(q)
+    t2 = qg.Table(q)
+    for fmt, M, N, K, cfg in [(qg.QG_FP8_DYNAMIC, 2048, 4096, 4096, qg.persist_config(256, 4)),
+                              (qg.QG_BLOCK_FP8, 4096, 5120, 5120, qg.pair_config(256, 4)),
+                              (qg.QG_BLOCK_FP8, 1024, 4096, 4096, qg.pair_config(128, 6))]:
+        c, hit = t2.dispatch(fmt, M, N, K)
+        assert hit == 1 and c.as_dict() == cfg.as_dict()
+
+
 @pytest.mark.parametrize("content", [
     "",
     "qgemm-table 3\ndevice x sms 148\n",                                    # unknown version
+    "qgemm-table 2\ndevice x sms 148\n2 4096 5120 5120 1 0 64 4 0 3 0 1.0\n",  # CTA pairs: 128 or 256 wide
+    "qgemm-table 2\ndevice x sms 148\n2 4096 5120 5120 1 0 256 4 0 4 0 1.0\n", # no variant 4
     "qgemm-table 1\ndevice x sms 148\n1 8 4096 4096 4 1 16 8 0\n",          # missing field
     "qgemm-table 2\ndevice x sms 148\n1 8 4096 4096 4 1 16 8 0 1.0\n",      # version 2: variant, rows missing
     "qgemm-table 2\ndevice x sms 148\n1 8 4096 4096 1 1 16 24 0 1 12 1.0\n",  # decode kernel: bad rows

@@ -49,6 +49,31 @@ def test_ranking_is_valid_sorted_and_the_default(fmt, M, N, K):
     assert [c.as_dict() for c, _ in again] == [c.as_dict() for c, _ in ranked]
 
 
+def _variants(fmt, M, N, K):
+    ranked = qg.qgemm_rank_configs(fmt, M, N, K, max_out=4096)
+    return collections.Counter(c.variant for c, _ in ranked), ranked
+
+
+def test_large_m_candidates_per_kernel():
+    # persistent rings deep enough for one CTA per SM: 256 x 4 and 128 x 6
+    # for FP8_Dynamic / W8A8_INT8, 256 x 3 for Block_FP8; CTA pairs (256 x 256
+    # tiles, rings of 3, 4, 6) for Block_FP8 only, and only with at least 60
+    # pair tiles
+    for fmt in (qg.QG_FP8_DYNAMIC, qg.QG_W8A8_INT8):
+        v, ranked = _variants(fmt, 4096, 5120, 5120)
+        assert v[3] == 0
+        assert sorted((c.tile_n, c.stages) for c, _ in ranked if c.variant == 2) == [(128, 6), (256, 4)]
+    v, ranked = _variants(qg.QG_BLOCK_FP8, 4096, 5120, 5120)
+    assert sorted((c.tile_n, c.stages) for c, _ in ranked if c.variant == 2) == [(256, 3)]
+    assert sorted((c.tile_n, c.stages) for c, _ in ranked if c.variant == 3) == [(256, 3), (256, 4), (256, 6)]
+    assert qg.qgemm_default_config(qg.QG_BLOCK_FP8, 4096, 5120, 5120).variant == 3
+    # 4 x 16 = 64 pair tiles: offered; 2 x 16 = 32: not
+    assert _variants(qg.QG_BLOCK_FP8, 1024, 4096, 4096)[0][3] == 3
+    assert _variants(qg.QG_BLOCK_FP8, 512, 4096, 4096)[0][3] == 0
+    assert _variants(qg.QG_NVFP4, 4096, 5120, 5120)[0][2] == 0
+    assert _variants(qg.QG_NVFP4, 4096, 5120, 5120)[0][3] == 0
+
+
 def test_scoring_an_invalid_config_returns_its_status():
     with pytest.raises(qg.QGemmError) as e:
         qg.qgemm_score_config(1, 8, 4096, 4096, qg.make_config(split_k=3))
