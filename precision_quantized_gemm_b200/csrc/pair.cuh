@@ -20,7 +20,8 @@
 // Roles: warp 0 of each CTA loads its own operand halves; their bytes
 // complete on the even CTA's ring barrier.  Warp 1 of each CTA allocates the
 // pair's TMEM; warp 1 of the even CTA issues the MMAs (M = 256) and commits
-// them to the ring and group barriers of both CTAs.  Warps 4-11 of each CTA
+// them to the ring and group barriers of both CTAs (warps 0-3, the role
+// warpgroup, run on 40 registers).  Warps 4-19 of each CTA (104 registers)
 // promote their own 128 TMEM lanes (= token rows), acc += p_g * (s_a * s_w)
 // with fma.rn.f32x2 as the tile kernel does, and arrive on the even CTA's
 // buffer-free barrier.  The pairs walk the tiles persistently (tile t =
