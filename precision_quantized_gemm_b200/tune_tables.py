@@ -40,8 +40,10 @@ SHAPES = {
               (qg.QG_BLOCK_FP8, [1, 2, 4, 8, 16, 32], SWEEP_NK)],
     "large_m": [(qg.QG_BLOCK_FP8, [4096, 16384], [(5120, 5120)])],
     # medium token counts (prefill chunks, batched decode): the buckets between
-    # decode and large M
-    "medium_m": [(qg.QG_FP8_DYNAMIC, MEDIUM_M, MEDIUM_NK), (qg.QG_BLOCK_FP8, MEDIUM_M, MEDIUM_NK)],
+    # decode and large M, and the 4096-token bucket above them (where the
+    # persistent and CTA-pair kernels compete with the tile kernel)
+    "medium_m": [(qg.QG_FP8_DYNAMIC, MEDIUM_M + [4096], MEDIUM_NK), (qg.QG_BLOCK_FP8, MEDIUM_M + [4096], MEDIUM_NK),
+                 (qg.QG_W8A8_INT8, [256, 512, 1024, 2048, 4096], MEDIUM_NK)],
 }
 
 
